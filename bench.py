@@ -1,0 +1,429 @@
+#!/usr/bin/env python3
+"""Benchmark: effective weight GB/s of the small-M quantized matmul on B200.
+
+Metric (MLX issue #4720, "To Reproduce"): weight bytes per call = N*K*bits/8 + N*(K/g)*4
+(packed codes + one fp16 scale and bias per group), divided by the time per call, with the
+weight copies rotated so that they do not sit in L2.
+
+Workload: the q/o projection verify shapes, K = N = 4096, 4-bit, group 64, fp16 x and W
+~ N(0,1), M in {1, 4, 5, 6}.  27 weight sets (255 MB, twice the 126 MB L2) are rotated, so
+every call streams its weights from HBM.  One step = one call per weight set for each M
+(108 calls).  Weights and x are resident in HBM before the timed region; the step is
+captured once in a CUDA graph and replayed (an eager-launch figure is reported beside it).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  With --gpus N > 1 (under torchrun), each rank runs the same
+per-GPU work on its own GPU (independent problems, no collective on the data path: weak
+scaling); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "effective weight GB/s (and % of HBM roofline) per shape vs M=1..64, 1×B200"
+WORKLOAD = "qo"
+BENCH_MS = (1, 4, 5, 6)
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--breakdown-out", default="", help="also write the per-M breakdown JSON here")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------- distributed
+def init_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------- helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, enabled: bool):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"qmm_clocks_{os.getpid()}.csv")
+        try:  # the UUID names the physical GPU whatever CUDA_VISIBLE_DEVICES says
+            gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            gpu_id = str(device_index)
+        if enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={gpu_id}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            except Exception:
+                self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                             "hw": parts[5], "hwt": parts[6], "swt": parts[7], "pcap": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            if r["hw"].lower() == "active":
+                reasons.add("hw_slowdown")
+            if r["hwt"].lower() == "active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"].lower() == "active":
+                reasons.add("sw_thermal_slowdown")
+            if r["pcap"].lower() == "active":
+                reasons.add("sw_power_cap")
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------------------- our arm
+def setup_workload(dev):
+    import bit_quantized_gemm_qmm_b200 as q
+    from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS, w_input, x_input
+    wl = WORKLOADS[WORKLOAD]
+    weights = []
+    for i in range(wl.sets):
+        w = w_input(wl.N, wl.K, wl.dtype, i, wl.w_sigma).to(dev)
+        weights.append(q.quantize(w, wl.bits, wl.group))
+        del w
+    xs = {M: x_input(M, wl.K, wl.dtype).to(dev) for M in BENCH_MS}
+    ys = {M: torch.empty((M, wl.N), dtype=wl.dtype, device=dev) for M in BENCH_MS}
+    plans = {}
+    for M in BENCH_MS:
+        p = q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype)
+        p.flags |= q.PLAN_STATIC_WEIGHTS  # weights are written once, before any timed call
+        plans[M] = p
+    torch.cuda.synchronize()
+    return wl, weights, xs, ys, plans
+
+
+def run_ours(args, rank, world):
+    import bit_quantized_gemm_qmm_b200 as q
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q.lib()  # loud failure if the CUDA library is missing
+    wl, weights, xs, ys, plans = setup_workload(dev)
+    wbytes = wl.weight_bytes()
+    calls_per_step = len(BENCH_MS) * len(weights)
+    step_wbytes = wbytes * calls_per_step
+    step_algo_bytes = sum((wbytes + 2 * M * wl.K + 2 * M * wl.N) * len(weights) for M in BENCH_MS)
+
+    def step(Ms=BENCH_MS):
+        for M in Ms:
+            x, y, p = xs[M], ys[M], plans[M]
+            for (P, S, B) in weights:
+                q.qmm(x, P, S, B, wl.bits, wl.group, out=y, plan=p)
+
+    stream = torch.cuda.current_stream(dev)
+    # eager warm-up, then one CUDA graph per step (and one per M for the breakdown)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    graphs = {}
+    for key, Ms in [("all", BENCH_MS)] + [(M, (M,)) for M in BENCH_MS]:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(Ms)
+        graphs[key] = g
+    for _ in range(max(3, args.warmup)):
+        graphs["all"].replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K graph replays of the step
+    clocks = ClockSampler(dev.index, not args.no_clocks)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        graphs["all"].replay()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    t_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_per_step = t_ms / args.steps
+    value = step_wbytes * world / (ms_per_step * 1e-3) / 1e9
+    achieved = step_algo_bytes / (ms_per_step * 1e-3) / 1e9  # per GPU: the only kernel in the step
+
+    # ---- eager figure (same calls, launched one by one)
+    reps = max(10, args.steps // 20)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    eager_ms = e0.elapsed_time(e1) / reps
+    eager_value = step_wbytes / (eager_ms * 1e-3) / 1e9
+
+    # ---- per-M breakdown (graph replays)
+    peak, peak_kind = measured_peaks()
+    breakdown = {}
+    reps_m = max(20, args.steps // 4)
+    for M in BENCH_MS:
+        for _ in range(3):
+            graphs[M].replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps_m):
+            graphs[M].replay()
+        e1.record(stream)
+        e1.synchronize()
+        per_call_ms = e0.elapsed_time(e1) / reps_m / len(weights)
+        gbs = wbytes / (per_call_ms * 1e-3) / 1e9
+        breakdown[f"M={M}"] = {"gbs": round(gbs, 1), "us_per_call": round(per_call_ms * 1e3, 3),
+                               "frac_of_measured": round(gbs / peak, 4),
+                               "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                               "plan": plans[M].as_dict()}
+
+    # ---- end-to-end through the public API with host buffers
+    e2e = run_e2e(wl, weights, plans, dev, max(5, args.steps // 100))
+
+    del graphs
+    torch.cuda.synchronize()
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 (fp16 dequantized weights x fp16 activations, fp32 accumulation)",
+        "data": "synthetic (seeded N(0,1) fp16 x and W, quantized by the library)",
+        "config": {"workload": "qo: K=4096 N=4096 4-bit g64 fp16, M in {1,4,5,6}",
+                   "weight_sets": len(weights), "calls_per_step": calls_per_step,
+                   "weight_bytes_per_call": wbytes,
+                   "l2": f"rotated weight sets totalling {len(weights) * wbytes / 1e6:.0f} MB > 126 MB L2",
+                   "launch": "CUDA graph replay of the step", "eager_value_gbs": round(eager_value, 2),
+                   "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(),
+                     "peak_kind": peak_kind, "kernel": "qmm_mma_kernel",
+                     "algorithmic_bytes_per_launch": "weight bytes + 2*M*K (x) + 2*M*N (y)"},
+        "breakdown": breakdown,
+        "e2e": e2e,
+        "gpu_launches": calls_per_step * args.steps,
+    }
+    if clk:
+        out["clocks"] = clk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, budget_s=12.0)
+    if rank == 0:
+        if args.breakdown_out:
+            with open(args.breakdown_out, "w") as f:
+                json.dump(out, f, indent=1)
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(wl, weights, plans, dev, steps):
+    """Each call: pinned host x -> device, qmm through the Python API, y -> pinned host."""
+    import bit_quantized_gemm_qmm_b200 as q
+    from bit_quantized_gemm_qmm_b200.inputs import x_input
+    hx = {M: x_input(M, wl.K, wl.dtype).pin_memory() for M in BENCH_MS}
+    hy = {M: torch.empty((M, wl.N), dtype=wl.dtype).pin_memory() for M in BENCH_MS}
+    dx = {M: torch.empty((M, wl.K), dtype=wl.dtype, device=dev) for M in BENCH_MS}
+    dy = {M: torch.empty((M, wl.N), dtype=wl.dtype, device=dev) for M in BENCH_MS}
+    stream = torch.cuda.current_stream(dev)
+
+    def one_step():
+        for M in BENCH_MS:
+            for (P, S, B) in weights:
+                dx[M].copy_(hx[M], non_blocking=True)
+                q.qmm(dx[M], P, S, B, wl.bits, wl.group, out=dy[M], plan=plans[M])
+                hy[M].copy_(dy[M], non_blocking=True)
+        stream.synchronize()
+
+    one_step()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one_step()
+    dt = (time.perf_counter() - t0) / steps
+    h2d = sum(2 * M * wl.K for M in BENCH_MS) * len(weights)
+    d2h = sum(2 * M * wl.N for M in BENCH_MS) * len(weights)
+    value = wl.weight_bytes() * len(BENCH_MS) * len(weights) / dt / 1e9
+    return {"value": round(value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(dt * 1e3, 4), "api": "bit_quantized_gemm_qmm_b200.qmm (C ABI qmm_ex)"}
+
+
+def traffic_per_launch():
+    """DRAM bytes per launch from the committed ncu capture, if the kernel source still
+    matches the one that was profiled (else null)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        d = json.load(open(path))
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(os.path.join(ROOT, "bit_quantized_gemm_qmm_b200", "csrc"))):
+        h.update(open(os.path.join(ROOT, "bit_quantized_gemm_qmm_b200", "csrc", name), "rb").read())
+    if d.get("csrc_sha256") != h.hexdigest():
+        return None
+    return d.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def _oracle_inputs(wl, rows: int):
+    """Oracle-quantized first `rows` rows of weight set 0 and the x of each M (numpy)."""
+    import numpy as np
+
+    import oracle
+    from bit_quantized_gemm_qmm_b200.inputs import w_rows, x_input
+    oracle.build()
+    w = w_rows(wl.K, wl.dtype, 0, wl.w_sigma, 0, rows).view(torch.int16).numpy().view(np.uint16)
+    pq = oracle.quantize(w, wl.bits, wl.group, wl.dtype == torch.bfloat16)
+    xs = {M: x_input(M, wl.K, wl.dtype).view(torch.int16).numpy().view(np.uint16) for M in BENCH_MS}
+    return pq, xs
+
+
+def _oracle_pass(wl, pq, xs, rows: int) -> float:
+    import oracle
+    p, s, b = pq
+    t0 = time.perf_counter()
+    for M in BENCH_MS:
+        oracle.qmm(xs[M], p[:rows], s[:rows], b[:rows], wl.K, wl.bits, wl.group, wl.dtype == torch.bfloat16)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, budget_s: float = 12.0):
+    """The CPU oracle as it stands, on the host cores: whole calls (all N rows of one weight
+    set) for every M, repeated for about `budget_s` seconds."""
+    cores = int(os.environ.get("OMP_NUM_THREADS", host_cores()))
+    pq, xs = _oracle_inputs(wl, wl.N)
+    t_total, passes = 0.0, 0
+    while passes == 0 or t_total < budget_s:
+        t_total += _oracle_pass(wl, pq, xs, wl.N)
+        passes += 1
+    nbytes = passes * len(BENCH_MS) * wl.weight_bytes()
+    return {"value": round(nbytes / t_total / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{passes} pass(es) of one full call per M in {list(BENCH_MS)} on weight set 0 "
+                      f"({t_total:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle, as it stands, on the same workload, metric and unit.
+    Each step is one call per M on a row sample of weight set 0, sized so that all steps
+    take about two minutes."""
+    if rank != 0:
+        return
+    from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS
+    wl = WORKLOADS[WORKLOAD]
+    cores = int(os.environ.get("OMP_NUM_THREADS", host_cores()))
+    pq, xs = _oracle_inputs(wl, wl.N)
+    t_full = _oracle_pass(wl, pq, xs, wl.N)
+    rows = int(min(wl.N, max(64, wl.N * (120.0 / max(1, args.steps + args.warmup)) / max(t_full, 1e-6))))
+    for _ in range(args.warmup):
+        _oracle_pass(wl, pq, xs, rows)
+    t_total = 0.0
+    for _ in range(args.steps):
+        t_total += _oracle_pass(wl, pq, xs, rows)
+    row_bytes = wl.weight_bytes() / wl.N
+    value = round(args.steps * len(BENCH_MS) * rows * row_bytes / t_total / 1e9, 4)
+    sample = f"{rows} of {wl.N} rows of weight set 0, one call per M in {list(BENCH_MS)} per step"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_total * 1e3 / max(1, args.steps), 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+           "data": "synthetic (seeded N(0,1) fp16 x and W)",
+           "config": {"workload": "qo: K=4096 N=4096 4-bit g64 fp16, M in {1,4,5,6}"},
+           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world = init_dist(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

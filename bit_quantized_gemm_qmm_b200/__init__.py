@@ -1,1 +1,221 @@
-"""placeholder"""
+"""Python binding of the B200 small-M affine-quantized matmul library (libqmm_b200.so).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels behind the C ABI
+declared in ``include/qmm.h``.  PyTorch provides device memory and the current stream.  There
+is no CPU fallback: if the shared library is missing, every call raises ``QmmUnavailable``.
+
+    packed, scales, biases = quantize(w, bits=4, group=64)     # w: [N,K] fp16/bf16 on cuda
+    y = qmm(x, packed, scales, biases, bits=4, group=64)       # x: [M,K], y: [M,N], M <= 64
+    w_hat = dequantize(packed, scales, biases, K, bits=4, group=64, dtype=torch.float16)
+
+Operation (MLX issue #4720, "To Reproduce": quantized_matmul(x, *w, transpose=True)):
+y[m,n] = sum_k x[m,k] * (s[n,k/g] * q[n,k] + b[n,k/g]).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqmm_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "qmm.h")
+
+QMM_OK, QMM_ERR_INVALID_ARG, QMM_ERR_UNSUPPORTED, QMM_ERR_CUDA = 0, 1, 2, 3
+QMM_F16, QMM_BF16 = 0, 1
+KERNEL_AUTO, KERNEL_MMA, KERNEL_TC = 0, 1, 2
+PLAN_PDL, PLAN_STATIC_WEIGHTS = 1, 2
+
+
+class QmmUnavailable(RuntimeError):
+    """The compiled library is not present (build it with __graft_entry__.build())."""
+
+
+class QmmError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"qmm status {status}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("split", ctypes.c_int32), ("warps", ctypes.c_int32),
+                ("flags", ctypes.c_uint32), ("reserved", ctypes.c_int32 * 4)]
+
+    def as_dict(self):
+        return {"kernel": self.kernel, "split": self.split, "warps": self.warps, "flags": self.flags}
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqmm_b200.so (in-tree).  Raises QmmUnavailable if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise QmmUnavailable(f"{LIB_PATH} is missing; run __graft_entry__.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I, U = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int
+    L.qmm_packed_words.argtypes = [I64, I64, I]
+    L.qmm_packed_words.restype = ctypes.c_size_t
+    L.qmm_group_count.argtypes = [I64, I64, I]
+    L.qmm_group_count.restype = ctypes.c_size_t
+    L.qmm_quantize.argtypes = [P, U, I64, I64, I, I, P, P, P, P]
+    L.qmm_quantize.restype = I
+    L.qmm_dequantize.argtypes = [P, P, P, I64, I64, I, I, U, P, P]
+    L.qmm_dequantize.restype = I
+    L.qmm.argtypes = [P, P, P, P, P, I64, I64, I64, I, I, U, P]
+    L.qmm.restype = I
+    L.qmm_ex.argtypes = [P, P, P, P, P, I64, I64, I64, I, I, U, ctypes.POINTER(Plan), P]
+    L.qmm_ex.restype = I
+    L.qmm_plan_default.argtypes = [I64, I64, I64, I, I, U, ctypes.POINTER(Plan)]
+    L.qmm_plan_default.restype = I
+    L.qmm_status_string.argtypes = [I]
+    L.qmm_status_string.restype = ctypes.c_char_p
+    L.qmm_last_error.argtypes = []
+    L.qmm_last_error.restype = ctypes.c_char_p
+    L.qmm_version.argtypes = []
+    L.qmm_version.restype = I
+    _lib = L
+    return L
+
+
+def _check(status: int) -> None:
+    if status != QMM_OK:
+        L = lib()
+        raise QmmError(status, f"{L.qmm_status_string(status).decode()}: {L.qmm_last_error().decode()}")
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float16:
+        return QMM_F16
+    if dt == torch.bfloat16:
+        return QMM_BF16
+    raise ValueError(f"unsupported activation/weight dtype {dt} (fp16 or bf16)")
+
+
+def _stream(dev: torch.device) -> int:
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(*ts: torch.Tensor) -> torch.device:
+    dev = ts[0].device
+    for t in ts:
+        if t.device.type != "cuda" or t.device != dev:
+            raise ValueError("all tensors must be on the same CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    return dev
+
+
+def packed_words(N: int, K: int, bits: int) -> int:
+    return int(lib().qmm_packed_words(N, K, bits))
+
+
+def weight_bytes(N: int, K: int, bits: int, group: int) -> int:
+    """Bytes per call that the metric counts: packed codes + one fp16 scale and bias per group."""
+    return N * K * bits // 8 + N * (K // group) * 4
+
+
+def quantize(w: torch.Tensor, bits: int, group: int):
+    """W[N,K] (fp16/bf16, cuda) -> (packed int32 [N,K*bits/32], scales fp16 [N,K/g], biases fp16)."""
+    if w.dim() != 2:
+        raise ValueError("w must be [N, K]")
+    dev = _need_cuda(w)
+    N, K = w.shape
+    L = lib()
+    if K % group:
+        raise ValueError("K must be a multiple of group")
+    packed = torch.empty((N, K * bits // 32), dtype=torch.int32, device=dev)
+    scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    biases = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    _check(L.qmm_quantize(_ptr(w), _dtype_code(w.dtype), N, K, bits, group, _ptr(packed),
+                          _ptr(scales), _ptr(biases), _stream(dev)))
+    return packed, scales, biases
+
+
+def dequantize(packed: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor, K: int, bits: int,
+               group: int, dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None):
+    dev = _need_cuda(packed, scales, biases)
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((N, K), dtype=dtype, device=dev)
+    _check(lib().qmm_dequantize(_ptr(packed), _ptr(scales), _ptr(biases), N, K, bits, group,
+                                _dtype_code(out.dtype), _ptr(out), _stream(dev)))
+    return out
+
+
+def plan_default(M: int, N: int, K: int, bits: int, group: int, dtype: torch.dtype) -> Plan:
+    p = Plan()
+    _check(lib().qmm_plan_default(M, N, K, bits, group, _dtype_code(dtype), ctypes.byref(p)))
+    return p
+
+
+def make_plan(kernel: int = KERNEL_AUTO, split: int = 0, warps: int = 0, flags: int = PLAN_PDL) -> Plan:
+    p = Plan()
+    p.kernel, p.split, p.warps, p.flags = kernel, split, warps, flags
+    return p
+
+
+def qmm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+        bits: int, group: int, out: torch.Tensor | None = None, plan: Plan | None = None):
+    """y[M,N] = x[M,K] . dequant(packed, scales, biases)^T on the current CUDA stream."""
+    if x.dim() != 2 or packed.dim() != 2:
+        raise ValueError("x must be [M, K] and packed [N, K*bits/32]")
+    dev = _need_cuda(x, packed, scales, biases)
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 32 != K * bits:
+        raise ValueError(f"packed has {packed.shape[1]} words per row; K={K} at {bits} bits needs {K * bits // 32}")
+    if out is None:
+        out = torch.empty((M, N), dtype=x.dtype, device=dev)
+    elif out.shape != (M, N) or out.dtype != x.dtype:
+        raise ValueError("out must be [M, N] with x's dtype")
+    L = lib()
+    if plan is None:
+        st = L.qmm(_ptr(x), _ptr(packed), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, bits, group,
+                   _dtype_code(x.dtype), _stream(dev))
+    else:
+        st = L.qmm_ex(_ptr(x), _ptr(packed), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, bits, group,
+                      _dtype_code(x.dtype), ctypes.byref(plan), _stream(dev))
+    _check(st)
+    return out
+
+
+def declared_symbols() -> list[str]:
+    """Function names declared in include/qmm.h (what the library must export)."""
+    import re
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\*?\s+\**(qmm[A-Za-z0-9_]*)\s*\(",
+                                 text, flags=re.M)))
+
+
+@dataclass
+class QuantizedWeight:
+    """A quantized [N, K] weight resident on the device."""
+    packed: torch.Tensor
+    scales: torch.Tensor
+    biases: torch.Tensor
+    N: int
+    K: int
+    bits: int
+    group: int
+
+    @classmethod
+    def from_dense(cls, w: torch.Tensor, bits: int, group: int) -> "QuantizedWeight":
+        p, s, b = quantize(w, bits, group)
+        return cls(p, s, b, w.shape[0], w.shape[1], bits, group)
+
+    def nbytes(self) -> int:
+        return weight_bytes(self.N, self.K, self.bits, self.group)
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None, plan: Plan | None = None):
+        return qmm(x, self.packed, self.scales, self.biases, self.bits, self.group, out=out, plan=plan)

@@ -1,0 +1,242 @@
+// qmm_api.cu -- the C ABI: argument validation, the per-shape dispatch table, launches.
+//
+// Entry points and their contracts are documented in include/qmm.h.  Every check happens
+// on the host before anything is launched; there is no fallback path: a shape or format the
+// kernels do not handle returns QMM_ERR_UNSUPPORTED.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "qmm_internal.h"
+
+namespace qmm_impl {
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+qmm_status fail(qmm_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+qmm_status fail(qmm_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+qmm_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(QMM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool bits_ok(int bits) { return bits == 4 || bits == 6 || bits == 8; }
+bool group_ok(int group) { return group == 32 || group == 64 || group == 128; }
+
+// Shared format/size checks.  Sizes are bounded so every element index fits the kernels'
+// 32-bit row/column arithmetic (row offsets are 64-bit).
+qmm_status check_format(int64_t N, int64_t K, int bits, int group) {
+    if (!bits_ok(bits)) return fail(QMM_ERR_UNSUPPORTED, "bits=%d (supported: 4, 6, 8)", bits);
+    if (!group_ok(group)) return fail(QMM_ERR_UNSUPPORTED, "group=%d (supported: 32, 64, 128)", group);
+    if (N < 0 || K < 0) return fail(QMM_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
+    if (K % group) return fail(QMM_ERR_INVALID_ARG, "K=%lld is not a multiple of group=%d", (long long)K, group);
+    if (N > (int64_t(1) << 30) || K > (int64_t(1) << 24))
+        return fail(QMM_ERR_UNSUPPORTED, "N=%lld or K=%lld too large", (long long)N, (long long)K);
+    return QMM_OK;
+}
+
+constexpr int kNumSM = 148;
+constexpr int kMaxM = 64;
+
+int ceil_div(int64_t a, int64_t b) { return int((a + b - 1) / b); }
+int round_up(int64_t a, int64_t b) { return int((a + b - 1) / b * b); }
+
+// Dispatch table for the MMA kernel: 8-token tiles, warps per block, K split, x staging.
+MmaConfig mma_config(int64_t M, int64_t N, int64_t K, int bits, int warps_req, int split_req) {
+    MmaConfig c;
+    c.mt = M > 0 ? ceil_div(M, 8) : 1;
+    c.warps = warps_req ? warps_req : (N <= 2048 ? 4 : 8);
+    const int KS = bits == 8 ? 64 : 128;
+    const int pfks = 4 * KS;
+    const int R = 16 * c.warps;
+    const int ctas_n = ceil_div(N, R);
+    int split = split_req;
+    if (!split) {
+        const int target = 2 * kNumSM;  // two resident blocks per SM
+        split = (target + ctas_n / 2) / ctas_n;
+        if (split < 1) split = 1;
+        if (split > 8) split = 8;
+        const int min_slice = 512;      // keep at least a few steps per warp
+        while (split > 1 && K / split < min_slice) --split;
+    }
+    int kslice = round_up(ceil_div(K, split), 128);
+    if (kslice < 128) kslice = 128;
+    c.kslice = kslice;
+    c.split = ceil_div(K, kslice);
+    if (c.split < 1) c.split = 1;
+    const int xmax = int(64 * 1024 / (16 * c.mt)) / pfks * pfks;
+    const int xneed = round_up(kslice, pfks);
+    c.xchunk = xneed < xmax ? xneed : xmax;
+    c.pdl = true;
+    c.static_weights = false;
+    return c;
+}
+
+qmm_status validate_qmm(const void* x, const uint32_t* packed, const uint16_t* scales,
+                        const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K,
+                        int bits, int group, qmm_dtype dtype) {
+    qmm_status s = check_format(N, K, bits, group);
+    if (s != QMM_OK) return s;
+    if (dtype != QMM_F16 && dtype != QMM_BF16) return fail(QMM_ERR_INVALID_ARG, "dtype=%d", int(dtype));
+    if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M=%lld", (long long)M);
+    if (M > kMaxM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %d", (long long)M, kMaxM);
+    if (M == 0 || N == 0) return QMM_OK;
+    if (!y) return fail(QMM_ERR_INVALID_ARG, "y is null");
+    if (!aligned(y, 16)) return fail(QMM_ERR_INVALID_ARG, "y must be 16-byte aligned");
+    if (K == 0) return QMM_OK;
+    if (!x || !packed || !scales || !biases) return fail(QMM_ERR_INVALID_ARG, "null input pointer");
+    if (!aligned(x, 16) || !aligned(packed, 16))
+        return fail(QMM_ERR_INVALID_ARG, "x and packed must be 16-byte aligned");
+    if (!aligned(scales, 2) || !aligned(biases, 2))
+        return fail(QMM_ERR_INVALID_ARG, "scales and biases must be 2-byte aligned");
+    return QMM_OK;
+}
+
+qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, const qmm_plan* in,
+                        qmm_plan* out, MmaConfig* mc) {
+    qmm_plan p;
+    memset(&p, 0, sizeof(p));
+    if (in) p = *in;
+    if (p.kernel == QMM_KERNEL_AUTO) p.kernel = QMM_KERNEL_MMA;
+    if (p.kernel != QMM_KERNEL_MMA)
+        return fail(QMM_ERR_UNSUPPORTED, "kernel %d is not available in this build", p.kernel);
+    if (p.split < 0 || p.split > 16) return fail(QMM_ERR_INVALID_ARG, "split=%d (1..16)", p.split);
+    if (p.warps != 0 && p.warps != 4 && p.warps != 8)
+        return fail(QMM_ERR_INVALID_ARG, "warps=%d (4 or 8)", p.warps);
+    if (p.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS))
+        return fail(QMM_ERR_INVALID_ARG, "unknown plan flags 0x%x", p.flags);
+    const bool defaults = in == nullptr;
+    MmaConfig c = mma_config(M, N, K, bits, p.warps, p.split);
+    if (!defaults) {
+        c.pdl = (p.flags & QMM_PLAN_PDL) != 0;
+        c.static_weights = (p.flags & QMM_PLAN_STATIC_WEIGHTS) != 0;
+    }
+    if (mma_smem_bytes(c) > kMmaMaxSmem)
+        return fail(QMM_ERR_UNSUPPORTED, "plan needs %zu bytes of shared memory", mma_smem_bytes(c));
+    p.warps = c.warps;
+    p.split = c.split;
+    p.flags = (c.pdl ? QMM_PLAN_PDL : 0u) | (c.static_weights ? QMM_PLAN_STATIC_WEIGHTS : 0u);
+    if (out) *out = p;
+    if (mc) *mc = c;
+    return QMM_OK;
+}
+
+}  // namespace
+}  // namespace qmm_impl
+
+using namespace qmm_impl;
+
+extern "C" {
+
+size_t qmm_packed_words(int64_t N, int64_t K, int bits) {
+    if (!bits_ok(bits) || N < 0 || K < 0 || (K * bits) % 32) return 0;
+    return size_t(N) * size_t(K * bits / 32);
+}
+
+size_t qmm_group_count(int64_t N, int64_t K, int group) {
+    if (!group_ok(group) || N < 0 || K < 0 || K % group) return 0;
+    return size_t(N) * size_t(K / group);
+}
+
+qmm_status qmm_quantize(const void* w, qmm_dtype w_dtype, int64_t N, int64_t K, int bits,
+                        int group, uint32_t* packed, uint16_t* scales, uint16_t* biases,
+                        void* stream) {
+    qmm_status s = check_format(N, K, bits, group);
+    if (s != QMM_OK) return s;
+    if (w_dtype != QMM_F16 && w_dtype != QMM_BF16) return fail(QMM_ERR_INVALID_ARG, "w_dtype=%d", int(w_dtype));
+    if (N == 0 || K == 0) return QMM_OK;
+    if (!w || !packed || !scales || !biases) return fail(QMM_ERR_INVALID_ARG, "null pointer");
+    if (!aligned(w, 2) || !aligned(packed, 4) || !aligned(scales, 2) || !aligned(biases, 2))
+        return fail(QMM_ERR_INVALID_ARG, "misaligned pointer");
+    cudaError_t e = launch_quantize(w, w_dtype == QMM_BF16, N, K, bits, group, packed, scales,
+                                    biases, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm_quantize launch");
+}
+
+qmm_status qmm_dequantize(const uint32_t* packed, const uint16_t* scales,
+                          const uint16_t* biases, int64_t N, int64_t K, int bits, int group,
+                          qmm_dtype out_dtype, void* w_out, void* stream) {
+    qmm_status s = check_format(N, K, bits, group);
+    if (s != QMM_OK) return s;
+    if (out_dtype != QMM_F16 && out_dtype != QMM_BF16)
+        return fail(QMM_ERR_INVALID_ARG, "out_dtype=%d", int(out_dtype));
+    if (N == 0 || K == 0) return QMM_OK;
+    if (!w_out || !packed || !scales || !biases) return fail(QMM_ERR_INVALID_ARG, "null pointer");
+    if (!aligned(w_out, 2) || !aligned(packed, 4) || !aligned(scales, 2) || !aligned(biases, 2))
+        return fail(QMM_ERR_INVALID_ARG, "misaligned pointer");
+    cudaError_t e = launch_dequantize(packed, scales, biases, N, K, bits, group,
+                                      out_dtype == QMM_BF16, w_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm_dequantize launch");
+}
+
+qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group, qmm_dtype dtype,
+                            qmm_plan* plan) {
+    qmm_status s = check_format(N, K, bits, group);
+    if (s != QMM_OK) return s;
+    if (dtype != QMM_F16 && dtype != QMM_BF16) return fail(QMM_ERR_INVALID_ARG, "dtype=%d", int(dtype));
+    if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M");
+    if (M > kMaxM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %d", (long long)M, kMaxM);
+    if (!plan) return fail(QMM_ERR_INVALID_ARG, "plan is null");
+    return resolve_plan(M, N, K, bits, nullptr, plan, nullptr);
+}
+
+qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
+                  const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+                  int group, qmm_dtype dtype, const qmm_plan* plan, void* stream) {
+    qmm_status s = validate_qmm(x, packed, scales, biases, y, M, N, K, bits, group, dtype);
+    if (s != QMM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M == 0 || N == 0) return QMM_OK;
+    if (K == 0) {
+        cudaError_t e = cudaMemsetAsync(y, 0, size_t(M) * size_t(N) * 2, st);
+        return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm zero fill");
+    }
+    MmaConfig c;
+    s = resolve_plan(M, N, K, bits, plan, nullptr, &c);
+    if (s != QMM_OK) return s;
+    QmmArgs a;
+    a.x = static_cast<const uint16_t*>(x);
+    a.packed = packed;
+    a.scales = scales;
+    a.biases = biases;
+    a.y = static_cast<uint16_t*>(y);
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.bits = bits;
+    a.group = group;
+    a.is_bf16 = dtype == QMM_BF16;
+    cudaError_t e = launch_mma(a, c, st);
+    return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm launch");
+}
+
+qmm_status qmm(const void* x, const uint32_t* packed, const uint16_t* scales,
+               const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+               int group, qmm_dtype dtype, void* stream) {
+    return qmm_ex(x, packed, scales, biases, y, M, N, K, bits, group, dtype, nullptr, stream);
+}
+
+const char* qmm_status_string(qmm_status status) {
+    switch (status) {
+        case QMM_OK: return "ok";
+        case QMM_ERR_INVALID_ARG: return "invalid argument";
+        case QMM_ERR_UNSUPPORTED: return "unsupported shape or format";
+        case QMM_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+const char* qmm_last_error(void) { return g_last_error; }
+
+int qmm_version(void) { return 100; }
+
+}  // extern "C"

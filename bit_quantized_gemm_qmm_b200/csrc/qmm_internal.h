@@ -1,0 +1,47 @@
+// qmm_internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qmm.h"
+
+namespace qmm_impl {
+
+// Arguments of one qmm launch after validation (device pointers, sizes, format).
+struct QmmArgs {
+    const uint16_t* x;
+    const uint32_t* packed;
+    const uint16_t* scales;
+    const uint16_t* biases;
+    uint16_t* y;
+    int64_t M, N, K;
+    int bits, group;
+    int is_bf16;
+};
+
+// Fully resolved launch configuration of the MMA kernel.
+struct MmaConfig {
+    int mt;        // 8-token column tiles (M <= 8*mt)
+    int warps;     // warps per block, each owning 16 weight rows
+    int split;     // K slices = cluster size along grid.y
+    int kslice;    // K elements per slice (multiple of 128)
+    int xchunk;    // K elements of x staged in shared memory at a time
+    bool pdl;
+    bool static_weights;
+};
+
+cudaError_t launch_quantize(const void* w, int is_bf16, int64_t N, int64_t K, int bits,
+                            int group, uint32_t* packed, uint16_t* scales, uint16_t* biases,
+                            cudaStream_t stream);
+cudaError_t launch_dequantize(const uint32_t* packed, const uint16_t* scales,
+                              const uint16_t* biases, int64_t N, int64_t K, int bits, int group,
+                              int out_bf16, void* w_out, cudaStream_t stream);
+
+// Shared-memory bytes the MMA kernel needs for a configuration.
+size_t mma_smem_bytes(const MmaConfig& c);
+// Largest dynamic shared memory the MMA kernel is allowed to request.
+constexpr size_t kMmaMaxSmem = 100 * 1024;
+cudaError_t launch_mma(const QmmArgs& a, const MmaConfig& c, cudaStream_t stream);
+
+}  // namespace qmm_impl

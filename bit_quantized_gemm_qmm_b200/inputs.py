@@ -19,6 +19,9 @@ X_SEED = 1
 W_SEED_BASE = 1000
 
 
+ROW_BLOCK = 256  # weight rows drawn per generator seed
+
+
 def randn(shape, sigma: float, dtype: torch.dtype, seed: int) -> torch.Tensor:
     """CPU tensor: N(0, sigma^2) drawn in fp32 from a seeded generator, rounded to dtype."""
     g = torch.Generator("cpu").manual_seed(int(seed))
@@ -29,8 +32,23 @@ def x_input(M: int, K: int, dtype: torch.dtype, seed: int = X_SEED, sigma: float
     return randn((M, K), sigma, dtype, seed)
 
 
+def w_rows(K: int, dtype: torch.dtype, set_index: int, sigma: float, row_start: int, row_end: int) -> torch.Tensor:
+    """Rows [row_start, row_end) of weight set `set_index`.  Rows come in blocks of ROW_BLOCK,
+    each block from its own seed, so any subset of rows can be drawn without the others."""
+    out = []
+    b0, b1 = row_start // ROW_BLOCK, (row_end + ROW_BLOCK - 1) // ROW_BLOCK
+    for blk in range(b0, b1):
+        seed = (W_SEED_BASE + set_index) * 1_000_003 + blk
+        rows = randn((ROW_BLOCK, K), sigma, dtype, seed)
+        lo = max(row_start - blk * ROW_BLOCK, 0)
+        hi = min(row_end - blk * ROW_BLOCK, ROW_BLOCK)
+        out.append(rows[lo:hi])
+    return torch.cat(out) if out else torch.empty((0, K), dtype=dtype)
+
+
 def w_input(N: int, K: int, dtype: torch.dtype, set_index: int = 0, sigma: float = 1.0) -> torch.Tensor:
-    return randn((N, K), sigma, dtype, W_SEED_BASE + set_index)
+    """Weight set `set_index`, [N, K]."""
+    return w_rows(K, dtype, set_index, sigma, 0, N)
 
 
 @dataclass(frozen=True)

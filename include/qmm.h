@@ -1,0 +1,148 @@
+/*
+ * qmm.h -- C ABI of the B200 (sm_100a) small-M affine-quantized matmul library.
+ *
+ * The operation, after the pages this library restates:
+ *   - "[BUG] qmm_splitk is chosen over qmm_nax on M5 for N=4096 projections M=16-64"
+ *     (ml-explore/mlx issue #4720), section "To Reproduce": W[N,K] is quantized per group
+ *     into (packed codes, scales, biases) and applied as quantized_matmul(x, *w,
+ *     transpose=True), i.e.  y[m,n] = sum_k x[m,k] * (s[n,k/g] * q[n,k] + b[n,k/g]);
+ *     the benchmark there counts N*K*bits/8 + N*(K/g)*4 weight bytes per call.
+ *   - "What Are NAX Verify Kernels ...", section "Supported Data Formats and Quantization
+ *     Schemes": 4-, 6- and 8-bit affine codes, group sizes 32/64/128, fp16 or bf16
+ *     activations.
+ *   - "How the NAX Verify Kernel Path Improves Decode Performance in MTPLX": the small-M
+ *     ("verify", M = 4..6 and up to 64) shapes this library is built for.
+ *
+ * Data layout (all arrays row-major and contiguous, owned by the caller):
+ *   W       [N, K]        fp16 or bf16
+ *   packed  [N, K*bits/32] uint32.  Per row, code k occupies bits [bits*k, bits*k+bits) of a
+ *                          little-endian bit stream and word j holds stream bits
+ *                          [32j, 32j+32); 6-bit codes therefore fill 3 words per 16 codes.
+ *   scales  [N, K/group]  fp16 (raw IEEE binary16 bits in uint16)
+ *   biases  [N, K/group]  fp16
+ *   x       [M, K]        fp16 or bf16 (dtype)
+ *   y       [M, N]        same dtype as x
+ *
+ * Quantization scheme (min/max affine, the plainest reading of "affine" on the pages; every
+ * step in IEEE fp32 with round-to-nearest-even and no fused operations):
+ *   lo = min w, hi = max w over the group;  s = RNE_fp16((hi - lo) / (2^bits - 1));
+ *   b = RNE_fp16(lo);  q = 0 if s == 0, else clamp(rint((w - b) / s), 0, 2^bits - 1).
+ * Dequantization: d = RN_fp32(s*q + b) (one rounding), then RNE to the output dtype.
+ * Weights must be finite with |w| <= 65504 (scale and bias are fp16).
+ *
+ * Pointers passed to the compute entry points are DEVICE pointers (cudaMalloc or any other
+ * device-accessible allocation).  `stream` is a cudaStream_t passed as void* (NULL = legacy
+ * default stream).  Every call is asynchronous on `stream`; the returned status covers
+ * argument validation and launch errors only, so a fault inside a kernel surfaces at the
+ * next synchronizing CUDA call.  On any non-OK status nothing has been launched, except
+ * QMM_ERR_CUDA, which reports a launch that the CUDA runtime rejected.
+ * qmm_last_error() returns a human-readable detail for the calling thread's last failure.
+ */
+#ifndef QMM_B200_H
+#define QMM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QMM_OK = 0,
+    QMM_ERR_INVALID_ARG = 1,  /* null pointer, negative size, K % group != 0, misalignment  */
+    QMM_ERR_UNSUPPORTED = 2,  /* bits not in {4,6,8}, group not in {32,64,128}, M > 64, ... */
+    QMM_ERR_CUDA = 3,         /* the CUDA runtime rejected a launch or a device query        */
+} qmm_status;
+
+typedef enum { QMM_F16 = 0, QMM_BF16 = 1 } qmm_dtype;
+
+/* Number of uint32 words of `packed` for an [N, K] matrix at `bits` (0 if unsupported). */
+size_t qmm_packed_words(int64_t N, int64_t K, int bits);
+
+/* Number of fp16 entries in `scales` (and in `biases`) for an [N, K] matrix (0 if invalid). */
+size_t qmm_group_count(int64_t N, int64_t K, int group);
+
+/*
+ * qmm_quantize -- W[N,K] (w_dtype) -> packed codes, fp16 scales and biases, with the scheme
+ * above.  Bit-exact with the CPU restatement of the same steps.  Offline (not on the timed
+ * path).  Alignment: all pointers at least 4-byte aligned.
+ */
+qmm_status qmm_quantize(const void* w, qmm_dtype w_dtype, int64_t N, int64_t K, int bits,
+                        int group, uint32_t* packed, uint16_t* scales, uint16_t* biases,
+                        void* stream);
+
+/*
+ * qmm_dequantize -- packed codes, scales, biases -> W_out[N,K] in out_dtype, element by
+ * element RNE_out(RN_fp32(s*q + b)).  Bit-exact.
+ */
+qmm_status qmm_dequantize(const uint32_t* packed, const uint16_t* scales,
+                          const uint16_t* biases, int64_t N, int64_t K, int bits, int group,
+                          qmm_dtype out_dtype, void* w_out, void* stream);
+
+/*
+ * qmm -- y[M,N] = x[M,K] . dequant(packed, scales, biases)^T for 0 <= M <= 64.
+ * Arithmetic: codes are dequantized to fp16 (s*q + b with one rounding), bf16 activations
+ * are converted to fp16 after an exact power-of-two rescale chosen per thread block so that
+ * no value overflows, products are accumulated in fp32 on the tensor cores, and the result
+ * is rounded once to the output dtype.  Split-K partial sums are combined in a fixed order,
+ * so the result is bitwise reproducible run to run.  M == 0 or N == 0 is a no-op; K == 0
+ * writes zeros.  Alignment: x, packed and y 16-byte aligned; scales and biases 2-byte.
+ * The kernel may read `packed`, `scales` and `biases` before earlier work on `stream` has
+ * finished only when the plan sets QMM_PLAN_STATIC_WEIGHTS (see qmm_ex); qmm() never does.
+ * Thread safety: calls from different host threads or on different streams are safe.
+ */
+qmm_status qmm(const void* x, const uint32_t* packed, const uint16_t* scales,
+               const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+               int group, qmm_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Plans: which kernel, tile and K split the dispatch table picks for a shape, and a way to
+ * run a specific one (used by the benchmark and the profiling evidence for each choice).
+ */
+enum {
+    QMM_KERNEL_AUTO = 0,   /* let the dispatch table decide                                 */
+    QMM_KERNEL_MMA = 1,    /* warp-per-16-row tile, register-streamed codes, mma.sync       */
+    QMM_KERNEL_TC = 2,     /* swap-AB tcgen05 tile: 128 weight rows x M tokens, TMEM accum   */
+};
+
+enum {
+    QMM_PLAN_PDL = 1u << 0,            /* launch with programmatic dependent launch          */
+    QMM_PLAN_STATIC_WEIGHTS = 1u << 1, /* weights are not written by earlier stream work:
+                                          prefetch them before waiting on the previous kernel */
+};
+
+typedef struct {
+    int32_t kernel;   /* QMM_KERNEL_*                                                       */
+    int32_t split;    /* number of K slices (thread-block cluster size along K), 1..16      */
+    int32_t warps;    /* warps per block for QMM_KERNEL_MMA (4 or 8); ignored otherwise     */
+    uint32_t flags;   /* QMM_PLAN_* bits                                                     */
+    int32_t reserved[4];
+} qmm_plan;
+
+/* Fill *plan with the dispatch table's choice for this shape (QMM_OK), or report why the
+ * shape is unsupported.  Sizes as for qmm(). */
+qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group,
+                            qmm_dtype dtype, qmm_plan* plan);
+
+/* qmm() with an explicit plan (NULL = the default plan).  Fields left at 0 take the default
+ * (kernel AUTO, split chosen by the table, ...).  An invalid plan returns
+ * QMM_ERR_INVALID_ARG and launches nothing. */
+qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
+                  const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+                  int group, qmm_dtype dtype, const qmm_plan* plan, void* stream);
+
+/* Static description of a status code. */
+const char* qmm_status_string(qmm_status status);
+
+/* Detail message of the calling thread's last non-OK status ("" if none). */
+const char* qmm_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int qmm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMM_B200_H */

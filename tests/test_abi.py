@@ -1,0 +1,95 @@
+"""Host-only checks of the C ABI: the library loads, exports every function declared in
+include/qmm.h, and rejects bad arguments before launching anything (no GPU needed: every call
+here fails validation, so no kernel or CUDA API call is reached)."""
+import ctypes
+import subprocess
+
+import pytest
+
+import bit_quantized_gemm_qmm_b200 as q
+
+
+@pytest.fixture(scope="module")
+def L():
+    import __graft_entry__  # noqa: F401  (repo root on sys.path via conftest)
+    from bit_quantized_gemm_qmm_b200 import _build
+    _build.build()
+    return q.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = q.declared_symbols()
+    assert {"qmm", "qmm_quantize", "qmm_dequantize"} <= set(declared)
+    out = subprocess.run(["nm", "-D", "--defined-only", q.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [s for s in declared if s not in exported]
+    assert not missing, missing
+    for s in declared:
+        assert hasattr(L, s)
+
+
+def test_sizes(L):
+    assert q.packed_words(4096, 4096, 4) == 4096 * 512
+    assert q.packed_words(4096, 4096, 6) == 4096 * 768
+    assert q.packed_words(10, 128, 8) == 10 * 32
+    assert L.qmm_packed_words(10, 128, 5) == 0
+    assert L.qmm_group_count(10, 128, 64) == 20
+    assert L.qmm_group_count(10, 100, 64) == 0
+
+
+def _qmm(L, M=4, N=64, K=128, bits=4, group=64, dtype=0, ptr=16, y=16, scales=16):
+    return L.qmm(ptr, ptr, scales, scales, y, M, N, K, bits, group, dtype, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=5), q.QMM_ERR_UNSUPPORTED),
+    (dict(bits=3), q.QMM_ERR_UNSUPPORTED),
+    (dict(group=16), q.QMM_ERR_UNSUPPORTED),
+    (dict(group=256), q.QMM_ERR_UNSUPPORTED),
+    (dict(M=65), q.QMM_ERR_UNSUPPORTED),
+    (dict(M=-1), q.QMM_ERR_INVALID_ARG),
+    (dict(N=-5), q.QMM_ERR_INVALID_ARG),
+    (dict(K=96), q.QMM_ERR_INVALID_ARG),          # not a multiple of 64
+    (dict(dtype=7), q.QMM_ERR_INVALID_ARG),
+    (dict(ptr=0), q.QMM_ERR_INVALID_ARG),         # null x / packed
+    (dict(y=0), q.QMM_ERR_INVALID_ARG),
+    (dict(ptr=8), q.QMM_ERR_INVALID_ARG),         # 8-byte aligned only
+    (dict(y=24), q.QMM_ERR_INVALID_ARG),
+    (dict(scales=1), q.QMM_ERR_INVALID_ARG),
+])
+def test_qmm_rejects_before_launch(L, kw, status):
+    assert _qmm(L, **kw) == status
+    assert L.qmm_last_error()
+
+
+def test_empty_shapes_are_noops(L):
+    # M == 0 or N == 0 returns before touching any pointer or the device
+    assert _qmm(L, M=0, ptr=0, y=0, scales=0) == q.QMM_OK
+    assert _qmm(L, N=0, ptr=0, y=0, scales=0) == q.QMM_OK
+
+
+def test_quantize_dequantize_reject(L):
+    assert L.qmm_quantize(16, 0, 4, 128, 7, 64, 16, 16, 16, None) == q.QMM_ERR_UNSUPPORTED
+    assert L.qmm_quantize(16, 0, 4, 100, 4, 64, 16, 16, 16, None) == q.QMM_ERR_INVALID_ARG
+    assert L.qmm_quantize(0, 0, 4, 128, 4, 64, 16, 16, 16, None) == q.QMM_ERR_INVALID_ARG
+    assert L.qmm_quantize(16, 3, 4, 128, 4, 64, 16, 16, 16, None) == q.QMM_ERR_INVALID_ARG
+    assert L.qmm_dequantize(16, 16, 16, 4, 128, 4, 48, 0, 16, None) == q.QMM_ERR_UNSUPPORTED
+    assert L.qmm_dequantize(16, 16, 16, 4, 128, 4, 64, 0, 0, None) == q.QMM_ERR_INVALID_ARG
+    assert L.qmm_quantize(0, 0, 0, 128, 4, 64, 0, 0, 0, None) == q.QMM_OK  # N == 0
+
+
+def test_plans(L):
+    p = q.plan_default(4, 4096, 4096, 4, 64, __import__("torch").float16)
+    assert p.kernel in (q.KERNEL_MMA, q.KERNEL_TC) and 1 <= p.split <= 16
+    bad = q.make_plan(split=17)
+    assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(bad), None) == q.QMM_ERR_INVALID_ARG
+    bad = q.make_plan(warps=3)
+    assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(bad), None) == q.QMM_ERR_INVALID_ARG
+    bad = q.make_plan(flags=1 << 7)
+    assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(bad), None) == q.QMM_ERR_INVALID_ARG
+
+
+def test_status_strings(L):
+    for s in range(4):
+        assert L.qmm_status_string(s)
+    assert L.qmm_version() >= 100
