@@ -48,6 +48,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--breakdown-out", default="", help="also write the per-M breakdown JSON here")
+    ap.add_argument("--sweep", default="", help="write a per-configuration, per-M GB/s sweep to this "
+                    "JSON file instead of running the headline benchmark")
+    ap.add_argument("--sweep-configs", default="qo,down,gateup_6b,gateup_8b,kv_6b,kv_8b,lmhead")
+    ap.add_argument("--sweep-ms", default="1-64", help="e.g. 1-64 or 1,4,16")
+    ap.add_argument("--sweep-plan", default="", help="kernel:split:warps override, e.g. 1:4:8")
     return ap.parse_args()
 
 
@@ -411,11 +416,88 @@ def run_reference(args, rank, world):
     print(json.dumps(out), flush=True)
 
 
+def _parse_ms(spec: str):
+    out = []
+    for part in spec.split(","):
+        if "-" in part:
+            a, b = part.split("-")
+            out.extend(range(int(a), int(b) + 1))
+        elif part:
+            out.append(int(part))
+    return out
+
+
+def run_sweep(args):
+    """GB/s per (configuration, M): one CUDA graph of one call per rotated weight set,
+    replayed; per-call time = graph time / sets."""
+    import bit_quantized_gemm_qmm_b200 as q
+    from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS, w_input, x_input
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peak, peak_kind = measured_peaks()
+    results = {"peak_gbs": peak, "peak_kind": peak_kind, "configs": {}}
+    stream = torch.cuda.current_stream(dev)
+    for name in args.sweep_configs.split(","):
+        wl = WORKLOADS[name]
+        weights = []
+        for i in range(wl.sets):
+            w = w_input(wl.N, wl.K, wl.dtype, i, wl.w_sigma).to(dev)
+            weights.append(q.quantize(w, wl.bits, wl.group))
+            del w
+        torch.cuda.synchronize()
+        wbytes = wl.weight_bytes()
+        rows = {}
+        for M in _parse_ms(args.sweep_ms):
+            x = x_input(M, wl.K, wl.dtype).to(dev)
+            y = torch.empty((M, wl.N), dtype=wl.dtype, device=dev)
+            if args.sweep_plan:
+                kern, split, warps = (int(v) for v in args.sweep_plan.split(":"))
+                plan = q.make_plan(kernel=kern, split=split, warps=warps,
+                                   flags=q.PLAN_PDL | q.PLAN_STATIC_WEIGHTS)
+            else:
+                plan = q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype)
+                plan.flags |= q.PLAN_STATIC_WEIGHTS
+            for (P, S, B) in weights:
+                q.qmm(x, P, S, B, wl.bits, wl.group, out=y, plan=plan)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for (P, S, B) in weights:
+                    q.qmm(x, P, S, B, wl.bits, wl.group, out=y, plan=plan)
+            reps = max(3, int(2e9 / (wbytes * len(weights))))  # ~2 GB streamed per timing
+            for _ in range(3):
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            best = float("inf")
+            for _ in range(3):
+                torch.cuda.synchronize()
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+                e1.synchronize()
+                best = min(best, e0.elapsed_time(e1) / reps / len(weights))
+            gbs = wbytes / (best * 1e-3) / 1e9
+            rows[M] = {"gbs": round(gbs, 1), "us": round(best * 1e3, 3), "frac": round(gbs / peak, 4),
+                       "frac_nominal": round(gbs / NOMINAL_HBM_GBS, 4), "plan": plan.as_dict()}
+            del g
+        results["configs"][name] = {"N": wl.N, "K": wl.K, "bits": wl.bits, "group": wl.group,
+                                    "dtype": str(wl.dtype), "sets": wl.sets, "weight_bytes": wbytes,
+                                    "M": rows}
+        del weights
+        torch.cuda.empty_cache()
+        print(f"[sweep] {name}: " + " ".join(f"{m}:{r['gbs']:.0f}" for m, r in rows.items()),
+              file=sys.stderr, flush=True)
+    with open(args.sweep, "w") as f:
+        json.dump(results, f, indent=1)
+
+
 def main():
     args = parse()
     rank, world = init_dist(args)
     try:
-        if args.impl == "reference":
+        if args.sweep:
+            run_sweep(args)
+        elif args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world)
