@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.qmm_last_error.restype = ctypes.c_char_p
     L.qmm_version.argtypes = []
     L.qmm_version.restype = I
+    L.qmm_device_errors.argtypes = [P]
+    L.qmm_device_errors.restype = I
     _lib = L
     return L
 
@@ -188,6 +190,13 @@ def qmm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, biases: tor
                       _dtype_code(x.dtype), ctypes.byref(plan), _stream(dev))
     _check(st)
     return out
+
+
+def device_errors() -> int:
+    """Read and clear the current device's kernel error word (0 = no pipeline timeout)."""
+    v = ctypes.c_uint32(0)
+    _check(lib().qmm_device_errors(ctypes.byref(v)))
+    return int(v.value)
 
 
 def declared_symbols() -> list[str]:

@@ -101,32 +101,84 @@ qmm_status validate_qmm(const void* x, const uint32_t* packed, const uint16_t* s
     return QMM_OK;
 }
 
-qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, const qmm_plan* in,
-                        qmm_plan* out, MmaConfig* mc) {
+// Smallest M for which the dispatch table prefers the tensor-core kernel.
+constexpr int kTcMinM = 9;
+
+struct Resolved {
+    int kernel;
+    MmaConfig mma;
+    TcConfig tc;
+};
+
+TcConfig tc_config(int64_t M, int64_t N, int64_t K, int bits, int split_req) {
+    TcConfig c;
+    c.mp = int((M + 15) / 16 * 16);
+    if (c.mp < 16) c.mp = 16;
+    const int tiles = ceil_div(N, 128);
+    const int nst = ceil_div(K, 128);
+    int split = split_req;
+    if (!split) {
+        const int target = 2 * kNumSM;
+        split = (target + tiles / 2) / tiles;
+        if (split < 1) split = 1;
+        if (split > 8) split = 8;
+        while (split > 1 && nst / split < 2) --split;
+    }
+    if (split > nst) split = nst;
+    c.stages_per_split = ceil_div(nst, split);
+    c.ring = tc_ring_for(bits, c.mp);
+    c.pdl = true;
+    c.static_weights = false;
+    return c;
+}
+
+qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, const qmm_plan* in,
+                        const void* scales, const void* biases, qmm_plan* out, Resolved* r) {
     qmm_plan p;
     memset(&p, 0, sizeof(p));
     if (in) p = *in;
-    if (p.kernel == QMM_KERNEL_AUTO) p.kernel = QMM_KERNEL_MMA;
-    if (p.kernel != QMM_KERNEL_MMA)
-        return fail(QMM_ERR_UNSUPPORTED, "kernel %d is not available in this build", p.kernel);
+    if (p.kernel != QMM_KERNEL_AUTO && p.kernel != QMM_KERNEL_MMA && p.kernel != QMM_KERNEL_TC)
+        return fail(QMM_ERR_INVALID_ARG, "kernel=%d", p.kernel);
     if (p.split < 0 || p.split > 16) return fail(QMM_ERR_INVALID_ARG, "split=%d (1..16)", p.split);
     if (p.warps != 0 && p.warps != 4 && p.warps != 8)
         return fail(QMM_ERR_INVALID_ARG, "warps=%d (4 or 8)", p.warps);
     if (p.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS))
         return fail(QMM_ERR_INVALID_ARG, "unknown plan flags 0x%x", p.flags);
+    const bool tc_ok = tc_supported(M, N, K, bits, group) && aligned(scales, 4) && aligned(biases, 4);
+    if (p.kernel == QMM_KERNEL_AUTO) p.kernel = (tc_ok && M >= kTcMinM) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
+    if (p.kernel == QMM_KERNEL_TC && !tc_ok)
+        return fail(QMM_ERR_UNSUPPORTED,
+                    "tensor-core kernel needs K >= 128, an even number of groups per row, a 16-byte "
+                    "multiple of packed bytes per row and 4-byte aligned scales/biases");
     const bool defaults = in == nullptr;
-    MmaConfig c = mma_config(M, N, K, bits, p.warps, p.split);
+    Resolved res;
+    res.kernel = p.kernel;
+    bool pdl = true, stat = false;
     if (!defaults) {
-        c.pdl = (p.flags & QMM_PLAN_PDL) != 0;
-        c.static_weights = (p.flags & QMM_PLAN_STATIC_WEIGHTS) != 0;
+        pdl = (p.flags & QMM_PLAN_PDL) != 0;
+        stat = (p.flags & QMM_PLAN_STATIC_WEIGHTS) != 0;
     }
-    if (mma_smem_bytes(c) > kMmaMaxSmem)
-        return fail(QMM_ERR_UNSUPPORTED, "plan needs %zu bytes of shared memory", mma_smem_bytes(c));
-    p.warps = c.warps;
-    p.split = c.split;
-    p.flags = (c.pdl ? QMM_PLAN_PDL : 0u) | (c.static_weights ? QMM_PLAN_STATIC_WEIGHTS : 0u);
+    if (p.kernel == QMM_KERNEL_MMA) {
+        MmaConfig c = mma_config(M, N, K, bits, p.warps, p.split);
+        c.pdl = pdl;
+        c.static_weights = stat;
+        if (mma_smem_bytes(c) > kMmaMaxSmem)
+            return fail(QMM_ERR_UNSUPPORTED, "plan needs %zu bytes of shared memory", mma_smem_bytes(c));
+        p.warps = c.warps;
+        p.split = c.split;
+        res.mma = c;
+    } else {
+        TcConfig c = tc_config(M, N, K, bits, p.split);
+        c.pdl = pdl;
+        c.static_weights = stat;
+        if (c.ring < 2) return fail(QMM_ERR_UNSUPPORTED, "tensor-core plan does not fit shared memory");
+        p.warps = 10;
+        p.split = ceil_div(ceil_div(K, 128), c.stages_per_split);
+        res.tc = c;
+    }
+    p.flags = (pdl ? QMM_PLAN_PDL : 0u) | (stat ? QMM_PLAN_STATIC_WEIGHTS : 0u);
     if (out) *out = p;
-    if (mc) *mc = c;
+    if (r) *r = res;
     return QMM_OK;
 }
 
@@ -186,7 +238,9 @@ qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group
     if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M");
     if (M > kMaxM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %d", (long long)M, kMaxM);
     if (!plan) return fail(QMM_ERR_INVALID_ARG, "plan is null");
-    return resolve_plan(M, N, K, bits, nullptr, plan, nullptr);
+    // the default plan assumes 4-byte aligned scales and biases (any allocation is)
+    return resolve_plan(M, N, K, bits, group, nullptr, reinterpret_cast<const void*>(16),
+                        reinterpret_cast<const void*>(16), plan, nullptr);
 }
 
 qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
@@ -200,8 +254,8 @@ qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
         cudaError_t e = cudaMemsetAsync(y, 0, size_t(M) * size_t(N) * 2, st);
         return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm zero fill");
     }
-    MmaConfig c;
-    s = resolve_plan(M, N, K, bits, plan, nullptr, &c);
+    Resolved r;
+    s = resolve_plan(M, N, K, bits, group, plan, scales, biases, nullptr, &r);
     if (s != QMM_OK) return s;
     QmmArgs a;
     a.x = static_cast<const uint16_t*>(x);
@@ -215,7 +269,7 @@ qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
     a.bits = bits;
     a.group = group;
     a.is_bf16 = dtype == QMM_BF16;
-    cudaError_t e = launch_mma(a, c, st);
+    cudaError_t e = r.kernel == QMM_KERNEL_TC ? launch_tc(a, r.tc, st) : launch_mma(a, r.mma, st);
     return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm launch");
 }
 
@@ -236,6 +290,15 @@ const char* qmm_status_string(qmm_status status) {
 }
 
 const char* qmm_last_error(void) { return g_last_error; }
+
+qmm_status qmm_device_errors(uint32_t* bits) {
+    if (!bits) return fail(QMM_ERR_INVALID_ARG, "bits is null");
+    unsigned v = 0;
+    cudaError_t e = tc_read_and_clear_errors(&v);
+    if (e != cudaSuccess) return cuda_fail(e, "qmm_device_errors");
+    *bits = v;
+    return QMM_OK;
+}
 
 int qmm_version(void) { return 100; }
 

@@ -132,6 +132,14 @@ qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
                   const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                   int group, qmm_dtype dtype, const qmm_plan* plan, void* stream);
 
+/* Read and clear the current device's kernel error word (synchronizes with the device).
+ * Bit 0: a tensor-core kernel block gave up waiting on one of its pipeline barriers (a wait
+ * that should finish in microseconds ran for about two seconds).  That block then dropped
+ * its work, drained its own copies in flight, released its tensor memory and exited rather
+ * than hang; its part of y is not valid.  Returns QMM_OK and *bits = 0 when nothing went
+ * wrong. */
+qmm_status qmm_device_errors(uint32_t* bits);
+
 /* Static description of a status code. */
 const char* qmm_status_string(qmm_status status);
 
