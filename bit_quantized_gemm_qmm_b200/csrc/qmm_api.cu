@@ -101,8 +101,15 @@ qmm_status validate_qmm(const void* x, const uint32_t* packed, const uint16_t* s
     return QMM_OK;
 }
 
-// Smallest M for which the dispatch table prefers the tensor-core kernel.
-constexpr int kTcMinM = 9;
+// Dispatch between the two kernels, from the measured per-shape sweeps (bench.py --sweep; the
+// crossovers are recorded in the profiles): the tensor-core kernel wins for wide N at every M
+// and for large weight matrices from M = 9 up; on the 4096-wide and narrower projections the
+// warp-tile kernel keeps the lead to M = 32.
+bool prefer_tc(int64_t M, int64_t N, int64_t K) {
+    if (N >= 8192 && N * K <= (int64_t(1) << 27)) return true;  // gate/up-like: wide N, moderate size
+    if (N * K >= (int64_t(1) << 25)) return M >= 9;             // >= 32M codes (down, LM head)
+    return M >= 33;
+}
 
 struct Resolved {
     int kernel;
@@ -114,19 +121,26 @@ TcConfig tc_config(int64_t M, int64_t N, int64_t K, int bits, int split_req) {
     TcConfig c;
     c.mp = int((M + 15) / 16 * 16);
     if (c.mp < 16) c.mp = 16;
+    c.ring = tc_ring_for(bits, c.mp);
     const int tiles = ceil_div(N, 128);
-    const int nst = ceil_div(K, 128);
+    const int nst = ceil_div(K, tc_kc(bits));
     int split = split_req;
     if (!split) {
-        const int target = 2 * kNumSM;
-        split = (target + tiles / 2) / tiles;
-        if (split < 1) split = 1;
-        if (split > 8) split = 8;
-        while (split > 1 && nst / split < 2) --split;
+        // Largest K split (<= 8, >= 2 stages per block) whose whole grid is resident at once;
+        // a second, mostly empty wave would double the time of these short kernels.
+        split = 1;
+        for (int s = 8; s >= 2; --s) {
+            if (nst / s < 2) continue;
+            int clusters = tc_max_active_clusters(bits, c.mp, c.ring, s);
+            if (clusters <= 0) clusters = kNumSM / s;  // no device to ask: one block per SM
+            if (tiles <= clusters) {
+                split = s;
+                break;
+            }
+        }
     }
     if (split > nst) split = nst;
     c.stages_per_split = ceil_div(nst, split);
-    c.ring = tc_ring_for(bits, c.mp);
     c.pdl = true;
     c.static_weights = false;
     return c;
@@ -140,12 +154,10 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
     if (p.kernel != QMM_KERNEL_AUTO && p.kernel != QMM_KERNEL_MMA && p.kernel != QMM_KERNEL_TC)
         return fail(QMM_ERR_INVALID_ARG, "kernel=%d", p.kernel);
     if (p.split < 0 || p.split > 16) return fail(QMM_ERR_INVALID_ARG, "split=%d (1..16)", p.split);
-    if (p.warps != 0 && p.warps != 4 && p.warps != 8)
-        return fail(QMM_ERR_INVALID_ARG, "warps=%d (4 or 8)", p.warps);
     if (p.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS))
         return fail(QMM_ERR_INVALID_ARG, "unknown plan flags 0x%x", p.flags);
     const bool tc_ok = tc_supported(M, N, K, bits, group) && aligned(scales, 4) && aligned(biases, 4);
-    if (p.kernel == QMM_KERNEL_AUTO) p.kernel = (tc_ok && M >= kTcMinM) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
+    if (p.kernel == QMM_KERNEL_AUTO) p.kernel = (tc_ok && prefer_tc(M, N, K)) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
     if (p.kernel == QMM_KERNEL_TC && !tc_ok)
         return fail(QMM_ERR_UNSUPPORTED,
                     "tensor-core kernel needs K >= 128, an even number of groups per row, a 16-byte "
@@ -159,6 +171,8 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
         stat = (p.flags & QMM_PLAN_STATIC_WEIGHTS) != 0;
     }
     if (p.kernel == QMM_KERNEL_MMA) {
+        if (p.warps != 0 && p.warps != 4 && p.warps != 8)
+            return fail(QMM_ERR_INVALID_ARG, "warps=%d (4 or 8)", p.warps);
         MmaConfig c = mma_config(M, N, K, bits, p.warps, p.split);
         c.pdl = pdl;
         c.static_weights = stat;
@@ -172,8 +186,8 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
         c.pdl = pdl;
         c.static_weights = stat;
         if (c.ring < 2) return fail(QMM_ERR_UNSUPPORTED, "tensor-core plan does not fit shared memory");
-        p.warps = 10;
-        p.split = ceil_div(ceil_div(K, 128), c.stages_per_split);
+        p.warps = 18;
+        p.split = ceil_div(ceil_div(K, tc_kc(bits)), c.stages_per_split);
         res.tc = c;
     }
     p.flags = (pdl ? QMM_PLAN_PDL : 0u) | (stat ? QMM_PLAN_STATIC_WEIGHTS : 0u);

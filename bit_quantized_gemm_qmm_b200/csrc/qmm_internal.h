@@ -47,16 +47,18 @@ cudaError_t launch_mma(const QmmArgs& a, const MmaConfig& c, cudaStream_t stream
 // Fully resolved launch configuration of the tensor-core (tcgen05) kernel.
 struct TcConfig {
     int mp;               // MMA N: M rounded up to 16, 32, 48 or 64
-    int stages_per_split; // K stages of 128 per block
+    int stages_per_split; // K stages (tc_kc(bits) elements each) per block
     int ring;             // shared-memory pipeline stages
     bool pdl;
     bool static_weights;
 };
-constexpr int kTcMaxSmem = 110 * 1024;
+constexpr int kTcMaxSmem = 200 * 1024;
 bool tc_supported(int64_t M, int64_t N, int64_t K, int bits, int group);
 int tc_ring_for(int bits, int mp);
+int tc_kc(int bits);  // K elements per pipeline stage
 size_t tc_smem_bytes(int bits, int mp, int ring);
 cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream);
 cudaError_t tc_read_and_clear_errors(unsigned* out);
+int tc_max_active_clusters(int bits, int mp, int ring, int split);
 
 }  // namespace qmm_impl

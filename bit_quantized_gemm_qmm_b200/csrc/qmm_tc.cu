@@ -7,18 +7,22 @@
 // The issue's point is that small-M calls must reach the tensor path ("qmm_nax") instead of a
 // split-K CUDA-core kernel.  On B200 that path is tcgen05 with the weights as the MMA's M
 // dimension (128 rows of W per block) and the tokens as its N dimension (M padded to MP =
-// 16/32/48/64):
-//   warp 0       TMA producer: packed-code tiles [128 rows x 128 codes] and fp16 x tiles
-//                [MP x 64] (128-byte swizzle) into an S-stage shared-memory ring;
-//   warp 1       MMA issuer: tcgen05.mma kind::f16, A from tensor memory, B = x from shared
-//                memory, D (fp32, 128 lanes x MP columns) in tensor memory;
-//   warps 2..9   dequantizers: one thread per weight row, half a stage each; codes ->
-//                fp16 (s*q + b, one rounding) -> tcgen05.st into an A buffer in tensor
-//                memory; after the K loop they read D back and write y.
-// Scales and biases are fetched per thread with cp.async a few stages ahead.  K may be split
-// across a thread-block cluster; partial tiles are summed over DSMEM in rank order.  Every
-// mbarrier wait is bounded: on timeout the block records an error, drains its own copies and
-// frees its tensor memory instead of hanging.
+// 16/32/48/64).  Two kernels per call:
+//   xprep   one block per token row: fp16 copy of x (bf16 rows rescaled by an exact power of
+//           two so none overflows fp16), written straight into the 128-byte-swizzled tile
+//           layout the MMA reads, one contiguous [MP x KC] tile per K stage;
+//   qmm_tc  warp 0      producer: per stage one TMA box of packed codes [128 rows x 128 B] and
+//                       one bulk copy of the stage's x tile into an S-stage ring;
+//           warp 1      MMA issuer: tcgen05.mma kind::f16, A from tensor memory, B = x from
+//                       shared memory, D (fp32, 128 lanes x MP columns) in tensor memory;
+//           warps 2-17  dequantizers, four per tensor-memory lane quadrant: one thread per
+//                       weight row and quarter stage; codes -> fp16 (s*q + b, one rounding)
+//                       -> tcgen05.st into an A buffer; afterwards they read D and write y.
+// Few, large copies keep the copy engine's per-request cost off the critical path (a 2D box
+// costs about the same whether it moves 2 KB or 16 KB).  Scales and biases are fetched per
+// thread with cp.async a few stages ahead.  K may be split across a thread-block cluster;
+// partial tiles are summed over DSMEM in rank order.  Every mbarrier wait is bounded: on
+// timeout the block records an error, drains its own copies and frees its tensor memory.
 #include <cooperative_groups.h>
 #include <cuda.h>
 
@@ -37,32 +41,79 @@ namespace qmm_impl {
 // qmm_device_errors().
 __device__ unsigned int g_tc_error = 0;
 
+#ifdef QMM_TC_TRACE
+// Pipeline trace of block (0,0) for performance analysis (built only with -DQMM_TC_TRACE):
+// g_tc_trace[event * 256 + stage] = %globaltimer at that event.
+__device__ unsigned long long g_tc_trace[16 * 256];
+__device__ unsigned long long g_tc_blocks[4096 * 8];  // per block: start, end, smid, nstages, clk0, clk1
+__device__ __forceinline__ unsigned long long gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void tc_trace(int ev, int i) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && i < 256) g_tc_trace[ev * 256 + i] = gtimer();
+}
+__device__ __forceinline__ void tc_trace_block(int which, unsigned long long v) {
+    const int b = blockIdx.y * gridDim.x + blockIdx.x;
+    if (b < 4096) g_tc_blocks[b * 8 + which] = v;
+}
+#define TC_TRACE(ev, i) tc_trace(ev, i)
+#define TC_TRACE_BLOCK(which, v) tc_trace_block(which, v)
+#else
+#define TC_TRACE(ev, i) ((void)0)
+#define TC_TRACE_BLOCK(which, v) ((void)0)
+#endif
+
 namespace {
 
 using namespace sm100;
 
-constexpr int TC_ROWS = 128;                 // MMA M: weight rows per block
-constexpr int TC_KC = 128;                   // K per pipeline stage
-constexpr int TC_NDQ = 8;                    // dequantizer warps (two per TMEM lane quadrant)
-constexpr int TC_THREADS = (2 + TC_NDQ) * 32;
-constexpr int TC_SPF = 4;                    // stages of scales in flight per thread
-constexpr int TC_NA = 3;                     // A buffers in tensor memory
-constexpr int TC_TMEM_COLS = 256;            // D: cols [0,64); A buffer a: cols [64+64a, 128+64a)
+constexpr int TC_ROWS = 128;                     // MMA M: weight rows per block
+constexpr int TC_NMMA = 4;                       // MMA issuer warps, one accumulator each
+constexpr int TC_NDQ = 16;                       // dequantizer warps (four per TMEM lane quadrant)
+constexpr int TC_DQ0 = 1 + TC_NMMA;              // first dequantizer warp
+constexpr int TC_THREADS = (TC_DQ0 + TC_NDQ) * 32;  // 672
+constexpr int TC_SPF = 4;                        // stages of scales in flight per thread
+constexpr int TC_TMEM_COLS = 512;
 constexpr long long TC_TIMEOUT_CYCLES = 4000000000LL;  // ~2 s at 2 GHz
 
-template <int BITS> struct TcFmt {
-    static constexpr int ROW_BYTES = TC_KC * BITS / 8;       // 64 / 96 / 128
-    static constexpr int W_BYTES = TC_ROWS * ROW_BYTES;      // 8 / 12 / 16 KB
+// Tensor memory: TC_NMMA accumulators of MP columns each at columns [0, TC_NMMA*MP), then the
+// A buffers (KC/2 columns each).
+template <int BITS, int MP> struct TcFmt {
+    static constexpr int KC = BITS == 8 ? 128 : 256;        // K per stage
+    static constexpr int ROW_BYTES = KC * BITS / 8;          // 128 / 192 / 128 bytes per row
+    static constexpr int W_BYTES = TC_ROWS * ROW_BYTES;      // 16 / 24 / 16 KB per stage
+    static constexpr int U = KC / 4;                         // codes per dequant thread per stage
+    static constexpr int COLS = U / 2;                       // A columns per thread
+    static constexpr int A_COLS = KC / 2;                    // A buffer columns
+    static constexpr int ACC_COLS = TC_NMMA * MP;
+    static constexpr int NA_RAW = (TC_TMEM_COLS - ACC_COLS) / A_COLS;
+    static constexpr int NA = NA_RAW > 4 ? 4 : NA_RAW;
+    static_assert(NA >= 2, "tensor memory too small for double-buffered A");
 };
+
+__host__ __device__ constexpr int tc_na(int bits, int mp) {
+    return ((TC_TMEM_COLS - TC_NMMA * mp) / ((bits == 8 ? 128 : 256) / 2)) > 4
+               ? 4
+               : ((TC_TMEM_COLS - TC_NMMA * mp) / ((bits == 8 ? 128 : 256) / 2));
+}
+
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}" : "=r"(pred));
+    return pred != 0;
+}
 
 struct TcParams {
     const uint16_t* scales;
     const uint16_t* biases;
     uint16_t* y;
+    const uint16_t* xt;   // x as fp16 stage tiles [nstages_k][MP x KC], 128-byte swizzled
     const int* xexp;      // per-token exponent E_m (x was scaled by 2^-E_m), or null
     int M, N, K, G, gshift;
     int stages_per_split; // K stages per block
-    int nstages_k;        // ceil(K / TC_KC)
+    int nstages_k;        // ceil(K / KC)
     int split;
     int out_bf16;
     int static_w;
@@ -74,43 +125,44 @@ struct TcSmemLayout {
     int x_off, w_off, sc_off, bar_off, total;
 };
 
-__host__ __device__ inline TcSmemLayout tc_layout(int mp, int w_bytes, int ring) {
+__host__ __device__ inline TcSmemLayout tc_layout(int x_stage, int w_bytes, int ring, int na) {
     TcSmemLayout L;
     L.ring = ring;
-    L.x_stage = mp * 256;  // two 64-column swizzle atoms of MP rows x 128 B
+    L.x_stage = x_stage;
     L.w_stage = w_bytes;
     L.x_off = 0;
     L.w_off = L.x_off + ring * L.x_stage;
     L.sc_off = L.w_off + ring * L.w_stage;
     L.bar_off = L.sc_off + TC_SPF * TC_NDQ * 32 * 8;
-    L.total = L.bar_off + 8 * (2 * ring + 2 * TC_NA + 1) + 16;
+    L.total = L.bar_off + 8 * (2 * ring + 2 * na + 1) + 16;
     return L;
 }
 
 __device__ __forceinline__ void set_error(unsigned bit) { atomicOr(&g_tc_error, bit); }
 
 // ---------------------------------------------------------------- dequantization into A
-// One thread: half a stage of one row (64 codes) -> 32 fp16x2 columns of the A buffer.
+// One thread: U codes of one row (a quarter stage) -> U/2 fp16x2 columns of the A buffer, in
+// natural K order (column j = codes 2j, 2j+1).  s_pair/b_pair: fp16 pair holding the scale
+// (bias) of the thread's groups; two_groups: the U codes span two groups (lo half, hi half).
 template <int BITS>
-__device__ __forceinline__ void dequant_half(uint32_t w_row_base, int row, int half, uint32_t s_pair,
-                                             uint32_t b_pair, int gsel_shift, uint32_t (&out)[32]) {
-    // s/b for the first and second 32 codes (they differ only for group 32)
+__device__ __forceinline__ void dequant_quarter(uint32_t w_row, int row, int quarter, uint32_t s_pair,
+                                                uint32_t b_pair, int two_groups, int sel,
+                                                uint32_t (&out)[TcFmt<BITS, 16>::COLS]) {
     uint32_t s_lo, b_lo, s_hi, b_hi;
-    if (gsel_shift < 0) {  // group 32: s_pair = (s[g0], s[g0+1])
+    if (two_groups) {
         s_lo = __byte_perm(s_pair, 0u, 0x1010u); s_hi = __byte_perm(s_pair, 0u, 0x3232u);
         b_lo = __byte_perm(b_pair, 0u, 0x1010u); b_hi = __byte_perm(b_pair, 0u, 0x3232u);
-    } else {               // one group: pick half `gsel_shift` (0 or 1) of the aligned pair
-        const uint32_t sel = gsel_shift ? 0x3232u : 0x1010u;
-        s_lo = s_hi = __byte_perm(s_pair, 0u, sel);
-        b_lo = b_hi = __byte_perm(b_pair, 0u, sel);
+    } else {
+        const uint32_t ps = sel ? 0x3232u : 0x1010u;
+        s_lo = s_hi = __byte_perm(s_pair, 0u, ps);
+        b_lo = b_hi = __byte_perm(b_pair, 0u, ps);
     }
     if constexpr (BITS == 4) {
-        // 64-byte rows in the 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r>>1)&3).
-        const int sw = (row >> 1) & 3;
+        // 128-byte rows, 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r & 7).
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
-            const uint4 v = lds_v4(w_row_base + uint32_t((c ^ sw) << 4));
+            const int c = 2 * quarter + cc;
+            const uint4 v = lds_v4(w_row + uint32_t((c ^ (row & 7)) << 4));
             const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
             const uint32_t s2 = cc ? s_hi : s_lo, b2 = cc ? b_hi : b_lo;
 #pragma unroll
@@ -125,30 +177,27 @@ __device__ __forceinline__ void dequant_half(uint32_t w_row_base, int row, int h
             }
         }
     } else if constexpr (BITS == 8) {
-        // 128-byte rows in the 128-byte swizzle: chunk c of row r sits at c ^ (r & 7).
-        const int sw = row & 7;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            const int c = 4 * half + cc;
-            const uint4 v = lds_v4(w_row_base + uint32_t((c ^ sw) << 4));
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * quarter + cc;
+            const uint4 v = lds_v4(w_row + uint32_t((c ^ (row & 7)) << 4));
             const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-            const uint32_t s2 = cc < 2 ? s_lo : s_hi, b2 = cc < 2 ? b_lo : b_hi;
 #pragma unroll
             for (int wi = 0; wi < 4; ++wi) {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const uint32_t h = __byte_perm(wd[wi], 0x64646464u, j ? 0x4342u : 0x4140u);
                     const uint32_t q = hfma2(h, kOnes, kMinus1024x2);
-                    out[cc * 8 + wi * 2 + j] = hfma2(q, s2, b2);
+                    out[cc * 8 + wi * 2 + j] = hfma2(q, s_lo, b_lo);
                 }
             }
         }
     } else {
-        // 96-byte rows, no swizzle; the thread's 48 bytes are 4 triplets of 16 codes.
+        // 192-byte rows, no swizzle; the thread's 48 bytes are 4 triplets of 16 codes.
         uint32_t wd[12];
 #pragma unroll
         for (int cc = 0; cc < 3; ++cc) {
-            const uint4 v = lds_v4(w_row_base + uint32_t(half * 48 + cc * 16));
+            const uint4 v = lds_v4(w_row + uint32_t(quarter * 48 + cc * 16));
             wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
         }
 #pragma unroll
@@ -169,25 +218,34 @@ __device__ __forceinline__ void dequant_half(uint32_t w_row_base, int row, int h
 
 // ---------------------------------------------------------------- the kernel
 template <int BITS, int MP>
-__global__ void __launch_bounds__(TC_THREADS, 2)
-    qmm_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
-                  const TcParams p) {
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    qmm_tc_kernel(const __grid_constant__ CUtensorMap wmap, const TcParams p) {
+    using F = TcFmt<BITS, MP>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int W_BYTES = TcFmt<BITS>::W_BYTES;
-    const TcSmemLayout L = tc_layout(MP, W_BYTES, p.ring);
+    constexpr int XS = MP * F::KC * 2;  // bytes of one stage's x tile
+    const TcSmemLayout L = tc_layout(XS, F::W_BYTES, p.ring, F::NA);
     const int S = L.ring;
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar_full = sbase + L.bar_off;              // [S]
     const uint32_t bar_empty = bar_full + 8 * S;               // [S]
     const uint32_t bar_afull = bar_empty + 8 * S;              // [NA]
-    const uint32_t bar_aempty = bar_afull + 8 * TC_NA;         // [NA]
-    const uint32_t bar_acc = bar_aempty + 8 * TC_NA;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.bar_off + 8 * (2 * S + 2 * TC_NA + 1));
+    const uint32_t bar_aempty = bar_afull + 8 * F::NA;         // [NA]
+    const uint32_t bar_acc = bar_aempty + 8 * F::NA;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.bar_off + 8 * (2 * S + 2 * F::NA + 1));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) TC_TRACE(9, 0);
+#ifdef QMM_TC_TRACE
+    if (threadIdx.x == 0) {
+        unsigned smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        TC_TRACE_BLOCK(0, gtimer());
+        TC_TRACE_BLOCK(2, smid);
+        TC_TRACE_BLOCK(4, clock64());
+    }
+#endif
     const int n0 = blockIdx.x * TC_ROWS;
     const int st0 = blockIdx.y * p.stages_per_split;
     const int nst = min(p.stages_per_split, p.nstages_k - st0);
@@ -195,17 +253,16 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(bar_full + 8 * i, 1);
-            mbar_init(bar_empty + 8 * i, TC_NDQ + 1);
+            mbar_init(bar_empty + 8 * i, TC_NDQ + TC_NMMA);
         }
-        for (int i = 0; i < TC_NA; ++i) {
+        for (int i = 0; i < F::NA; ++i) {
             mbar_init(bar_afull + 8 * i, TC_NDQ);
-            mbar_init(bar_aempty + 8 * i, 1);
+            mbar_init(bar_aempty + 8 * i, TC_NMMA);
         }
-        mbar_init(bar_acc, 1);
+        mbar_init(bar_acc, TC_NMMA);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&wmap);
-        prefetch_tensormap(&xmap);
     }
     if (warp == 0) {
         tmem_alloc(smem_addr(tmem_holder), TC_TMEM_COLS);
@@ -214,7 +271,6 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    grid_dependents_launch();  // the next kernel on the stream may start its own prologue
     const uint32_t tmem = *tmem_holder;
     // Everything except the producer's first code tiles depends on earlier kernels; the
     // producer waits after issuing those tiles, everyone else waits here.  Deadlines start
@@ -225,24 +281,21 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            constexpr int WCOLS = TC_KC * BITS / 32;
-            const uint32_t stage_tx = uint32_t(W_BYTES + L.x_stage);
-            int issued = 0;
+            constexpr int WCOLS = F::ROW_BYTES / 4;
+            const uint32_t stage_tx = uint32_t(F::W_BYTES + XS);
+            const uint8_t* xt = reinterpret_cast<const uint8_t*>(p.xt);
             const int pre = p.static_w ? min(S, nst) : 0;
             // codes of the first stages do not depend on earlier kernels when weights are static
             for (int i = 0; i < pre; ++i) {
+                TC_TRACE(0, i);
                 mbar_arrive_expect_tx(bar_full + 8 * i, stage_tx);
-                tma_load_2d(sbase + L.w_off + i * L.w_stage, &wmap, bar_full + 8 * i,
-                            (st0 + i) * WCOLS, n0);
+                tma_load_2d(sbase + L.w_off + i * L.w_stage, &wmap, bar_full + 8 * i, (st0 + i) * WCOLS, n0);
             }
             grid_dependency_wait();
             deadline = clock64() + TC_TIMEOUT_CYCLES;
-            for (int i = 0; i < pre; ++i) {
-                const uint32_t xs = sbase + L.x_off + i * L.x_stage;
-                tma_load_2d(xs, &xmap, bar_full + 8 * i, (st0 + i) * TC_KC, 0);
-                tma_load_2d(xs + MP * 128, &xmap, bar_full + 8 * i, (st0 + i) * TC_KC + 64, 0);
-            }
-            issued = pre;
+            for (int i = 0; i < pre; ++i)
+                bulk_load(sbase + L.x_off + i * L.x_stage, xt + size_t(st0 + i) * XS, XS, bar_full + 8 * i);
+            int issued = pre;
             for (int i = pre; i < nst; ++i) {
                 const int s = i % S;
                 if (i >= S && !mbar_wait(bar_empty + 8 * s, ((i / S) & 1) ^ 1, deadline)) {
@@ -251,12 +304,10 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
                     break;
                 }
                 if (*abort_flag) break;
+                TC_TRACE(0, i);
                 mbar_arrive_expect_tx(bar_full + 8 * s, stage_tx);
-                tma_load_2d(sbase + L.w_off + s * L.w_stage, &wmap, bar_full + 8 * s,
-                            (st0 + i) * WCOLS, n0);
-                const uint32_t xs = sbase + L.x_off + s * L.x_stage;
-                tma_load_2d(xs, &xmap, bar_full + 8 * s, (st0 + i) * TC_KC, 0);
-                tma_load_2d(xs + MP * 128, &xmap, bar_full + 8 * s, (st0 + i) * TC_KC + 64, 0);
+                tma_load_2d(sbase + L.w_off + s * L.w_stage, &wmap, bar_full + 8 * s, (st0 + i) * WCOLS, n0);
+                bulk_load(sbase + L.x_off + s * L.x_stage, xt + size_t(st0 + i) * XS, XS, bar_full + 8 * s);
                 issued = i + 1;
             }
             // drain: every issued stage's copy must land before the block may exit
@@ -264,46 +315,60 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
             for (int i = max(0, issued - S); i < issued; ++i)
                 if (!mbar_wait(bar_full + 8 * (i % S), (i / S) & 1, drain_deadline)) set_error(1u);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16_f32(TC_ROWS, MP);
-            for (int i = 0; i < nst; ++i) {
-                const int s = i % S, a = i % TC_NA;
-                if (!mbar_wait(bar_full + 8 * s, (i / S) & 1, deadline) ||
-                    !mbar_wait(bar_afull + 8 * a, (i / TC_NA) & 1, deadline)) {
+    } else if (warp < TC_DQ0) {
+        // ------------------------------------------------------------ MMA issuers
+        // Warp j issues the K16 steps kk = j, j+4, ... of every stage into its own accumulator
+        // D_j (columns [j*MP, (j+1)*MP)); the whole warp runs the loop so descriptors stay
+        // warp-uniform, one elected lane issues.  Several issuers keep the tensor core fed:
+        // a single one can put an MMA in flight only every ~100 cycles.
+        const int j = warp - 1;
+        constexpr uint32_t idesc = idesc_f16_f32(TC_ROWS, MP);
+        const uint32_t dcol = tmem + uint32_t(j * MP);
+        for (int i = 0; i < nst; ++i) {
+            const int s = i % S, a = i % F::NA;
+            const bool got_full = mbar_wait(bar_full + 8 * s, (i / S) & 1, deadline);
+            if (j == 0 && lane == 0) TC_TRACE(10, i);
+            if (!got_full || !mbar_wait(bar_afull + 8 * a, (i / F::NA) & 1, deadline)) {
+                if (lane == 0) {
                     set_error(1u);
                     *abort_flag = 1;
-                    break;
                 }
-                tc_fence_after();
-                const uint32_t xs = sbase + L.x_off + s * L.x_stage;
-                const uint32_t acol = tmem + 64 + 64 * a;
+                break;
+            }
+            tc_fence_after();
+            if (j == 0 && lane == 0) TC_TRACE(1, i);
+            const uint32_t xs = sbase + L.x_off + s * L.x_stage;
+            const uint32_t acol = tmem + F::ACC_COLS + F::A_COLS * a;
+            if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < TC_KC / 16; ++kk) {
+                for (int kk = j; kk < F::KC / 16; kk += TC_NMMA) {
                     const uint64_t bdesc = smem_desc_sw128(xs + (kk >> 2) * (MP * 128) + (kk & 3) * 32, 1024);
-                    umma_f16_ts(tmem, acol + kk * 8, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    umma_f16_ts(dcol, acol + kk * 8, bdesc, idesc, (i > 0 || kk > j) ? 1u : 0u);
                 }
                 umma_commit(bar_empty + 8 * s);
                 umma_commit(bar_aempty + 8 * a);
             }
-            umma_commit(bar_acc);  // fires once every MMA issued above has completed
+            __syncwarp();
+            if (j == 0 && lane == 0) TC_TRACE(2, i);
         }
+        if (elect_one()) umma_commit(bar_acc);  // fires once every MMA issued above has completed
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ dequantizers
         const int q = warp & 3;                  // TMEM lane quadrant this warp may access
-        const int half = (warp - 2) >> 2;        // which 64 codes of the stage
+        const int quarter = (warp - TC_DQ0) >> 2;  // which quarter of the stage's codes
         const int row = q * 32 + lane;           // weight row within the block
         const int n = n0 + row;
-        const int dq = threadIdx.x - 64;         // 0..255
+        const int dq = threadIdx.x - TC_DQ0 * 32;  // 0..511
         const uint32_t sc_base = sbase + L.sc_off + uint32_t(dq) * 8;
         const uint32_t lane_bits = uint32_t(q * 32) << 16;
-        const int gsel = p.gshift == 5 ? -1 : 0;
+        const int group = 1 << p.gshift;
+        const int two_groups = F::U > group ? 1 : 0;
 
         auto issue_scales = [&](int i) {
             const int slot = i % TC_SPF;
             const uint32_t dst = sc_base + uint32_t(slot) * (TC_NDQ * 32 * 8);
-            const int k = (st0 + i) * TC_KC + half * 64;
+            const int k = (st0 + i) * F::KC + quarter * F::U;
             const int gi = (k >> p.gshift) & ~1;
             const bool ok = i < nst && n < p.N && k < p.K;
             const int64_t off = ok ? int64_t(n) * p.G + gi : 0;
@@ -314,76 +379,90 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
 #pragma unroll
         for (int i = 0; i < TC_SPF; ++i) issue_scales(i);
 
-        bool aborted = false;
         for (int i = 0; i < nst; ++i) {
-            const int s = i % S, a = i % TC_NA;
+            const int s = i % S, a = i % F::NA;
             if (!mbar_wait(bar_full + 8 * s, (i / S) & 1, deadline)) {
                 set_error(1u);
                 *abort_flag = 1;
-                aborted = true;
                 break;
             }
+            if (warp == TC_DQ0 && lane == 0) TC_TRACE(3, i);
             cp_async_wait<TC_SPF - 1>();
-            const int slot = i % TC_SPF;
-            const uint32_t sp = sc_base + uint32_t(slot) * (TC_NDQ * 32 * 8);
+            const uint32_t sp = sc_base + uint32_t(i % TC_SPF) * (TC_NDQ * 32 * 8);
             uint32_t s_pair, b_pair;
             asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(s_pair), "=r"(b_pair) : "r"(sp));
-            const int k = (st0 + i) * TC_KC + half * 64;
-            const int gshift_sel = gsel < 0 ? -1 : ((k >> p.gshift) & 1);
-            uint32_t vals[32];
-            dequant_half<BITS>(sbase + L.w_off + s * L.w_stage + row * TcFmt<BITS>::ROW_BYTES, row, half,
-                               s_pair, b_pair, gshift_sel, vals);
+            const int k = (st0 + i) * F::KC + quarter * F::U;
+            uint32_t vals[F::COLS];
+            dequant_quarter<BITS>(sbase + L.w_off + s * L.w_stage + row * F::ROW_BYTES, row, quarter, s_pair,
+                                  b_pair, two_groups, (k >> p.gshift) & 1, vals);
             __syncwarp();
+            if (warp == TC_DQ0 && lane == 0) TC_TRACE(4, i);
             if (lane == 0) mbar_arrive(bar_empty + 8 * s);   // codes of stage s consumed
             issue_scales(i + TC_SPF);
-            if (i >= TC_NA && !mbar_wait(bar_aempty + 8 * a, ((i / TC_NA) & 1) ^ 1, deadline)) {
+            if (i >= F::NA && !mbar_wait(bar_aempty + 8 * a, ((i / F::NA) & 1) ^ 1, deadline)) {
                 set_error(1u);
                 *abort_flag = 1;
-                aborted = true;
                 break;
             }
             tc_fence_after();
-            tmem_st_32x32b_x32(tmem + lane_bits + 64 + 64 * a + half * 32, vals);
+            const uint32_t taddr = tmem + lane_bits + F::ACC_COLS + F::A_COLS * a + quarter * F::COLS;
+            if constexpr (F::COLS == 32) {
+                tmem_st_32x32b_x32(taddr, vals);
+            } else {
+                tmem_st_32x32b_x16(taddr, vals);
+            }
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
+            if (warp == TC_DQ0 && lane == 0) TC_TRACE(6, i);
             if (lane == 0) mbar_arrive(bar_afull + 8 * a);
         }
         cp_async_wait<0>();
-        (void)aborted;
     }
 
     // ---------------------------------------------------------------- epilogue
+    // D = sum of the TC_NMMA accumulators, each [128 lanes x MP columns] fp32, added in a fixed
+    // order; 8-column chunk c is read by dequant warp quarter c % 4.
     __syncwarp();
-    float acc[MP / 2];
-    const bool dq_warp = warp >= 2;
-    const int q = warp & 3, half = dq_warp ? (warp - 2) >> 2 : 0;
+    constexpr int NCH = MP / 8;               // 8-column chunks
+    constexpr int CPW = (NCH + 3) / 4;        // chunks per dequant warp (max)
+    float acc[CPW][8];
+    const bool dq_warp = warp >= TC_DQ0;
+    const int q = warp & 3, quarter = dq_warp ? (warp - TC_DQ0) >> 2 : 0;
     const int row = q * 32 + lane;
     const int n = n0 + row;
-    bool have_acc = false;
     if (dq_warp) {
-        // wait until every MMA of this block has completed (bounded)
         const long long d2 = clock64() + TC_TIMEOUT_CYCLES;
-        have_acc = mbar_wait(bar_acc, 0, d2);
+        const bool have_acc = mbar_wait(bar_acc, 0, d2);
+        if (warp == TC_DQ0 && lane == 0) TC_TRACE(8, 0);
         if (!have_acc) set_error(1u);
         tc_fence_after();
-        if (have_acc && *abort_flag == 0) {
+        const bool ok = have_acc && *abort_flag == 0;
 #pragma unroll
-            for (int c = 0; c < MP / 16; ++c) {
-                uint32_t v[8];
-                tmem_ld_32x32b_x8(tmem + (uint32_t(q * 32) << 16) + half * (MP / 2) + 8 * c, v);
-                tc_wait_ld();
+        for (int cw = 0; cw < CPW; ++cw) {
+            const int c = quarter + 4 * cw;
+            if (c < NCH) {
+                float sum[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[8 * c + j] = __uint_as_float(v[j]);
+                for (int jj = 0; jj < 8; ++jj) sum[jj] = 0.f;
+                if (ok) {
+#pragma unroll
+                    for (int d = 0; d < TC_NMMA; ++d) {
+                        uint32_t v[8];
+                        tmem_ld_32x32b_x8(tmem + (uint32_t(q * 32) << 16) + uint32_t(d * MP + 8 * c), v);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj) sum[jj] += __uint_as_float(v[jj]);
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int m = 8 * c + jj;
+                    float val = sum[jj];
+                    if (p.xexp && m < p.M) val *= exp2i(p.xexp[m]);
+                    acc[cw][jj] = val;
+                }
             }
-        } else {
-#pragma unroll
-            for (int j = 0; j < MP / 2; ++j) acc[j] = 0.f;
-        }
-#pragma unroll
-        for (int j = 0; j < MP / 2; ++j) {
-            const int m = half * (MP / 2) + j;
-            if (p.xexp && m < p.M) acc[j] *= exp2i(p.xexp[m]);
         }
     }
     tc_fence_before();
@@ -392,11 +471,18 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
     if (p.split == 1) {
         if (dq_warp && n < p.N) {
 #pragma unroll
-            for (int j = 0; j < MP / 2; ++j) {
-                const int m = half * (MP / 2) + j;
-                if (m < p.M)
-                    p.y[int64_t(m) * p.N + n] = p.out_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]))
-                                                           : __half_as_ushort(__float2half_rn(acc[j]));
+            for (int cw = 0; cw < CPW; ++cw) {
+                const int c = quarter + 4 * cw;
+                if (c < NCH) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int m = 8 * c + j;
+                        if (m < p.M)
+                            p.y[int64_t(m) * p.N + n] = p.out_bf16
+                                                            ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[cw][j]))
+                                                            : __half_as_ushort(__float2half_rn(acc[cw][j]));
+                    }
+                }
             }
         }
     } else {
@@ -404,7 +490,13 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
         float* red = reinterpret_cast<float*>(smem);
         if (dq_warp) {
 #pragma unroll
-            for (int j = 0; j < MP / 2; ++j) red[(half * (MP / 2) + j) * TC_ROWS + row] = acc[j];
+            for (int cw = 0; cw < CPW; ++cw) {
+                const int c = quarter + 4 * cw;
+                if (c < NCH) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) red[(8 * c + j) * TC_ROWS + row] = acc[cw][j];
+                }
+            }
         }
         cg::cluster_group cluster = cg::this_cluster();
         cluster.sync();
@@ -425,49 +517,71 @@ __global__ void __launch_bounds__(TC_THREADS, 2)
     }
 
     // ---------------------------------------------------------------- teardown
+#ifdef QMM_TC_TRACE
+    if (threadIdx.x == 0) {
+        TC_TRACE_BLOCK(1, gtimer());
+        TC_TRACE_BLOCK(3, nst);
+        TC_TRACE_BLOCK(5, clock64());
+    }
+#endif
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, TC_TMEM_COLS);
     }
 }
 
-// ---------------------------------------------------------------- bf16 activations
-// One block per token row m: E_m = max(0, e - 141) where max|x[m,:]| < 2^(e-126), then
-// x16[m,k] = fp16(x[m,k] * 2^-E_m) (exact scaling; fp16 holds every bf16 significand).
-__global__ void __launch_bounds__(256) xprep_bf16_kernel(const uint16_t* __restrict__ x,
-                                                         uint16_t* __restrict__ x16, int* __restrict__ xexp,
-                                                         int K) {
+// ---------------------------------------------------------------- activations -> stage tiles
+// One block per padded token row m (MP blocks).  Writes x'[stage][m][k] (fp16) in the layout
+// the MMA reads: per stage, KC/64 swizzle atoms of [MP rows x 128 B], 16-byte chunk c of row m
+// at chunk c ^ (m & 7).  Rows m >= M and columns k >= K are zero.  bf16 rows are scaled by
+// 2^-E_m, E_m = max(0, e - 141) where max|x[m,:]| < 2^(e-126), so every value fits fp16.
+template <int KC>
+__global__ void __launch_bounds__(256) xprep_kernel(const uint16_t* __restrict__ x, int M, int K, int is_bf16,
+                                                    int MP, int nst, uint16_t* __restrict__ xt,
+                                                    int* __restrict__ xexp) {
     __shared__ float red[8];
-    grid_dependency_wait();
     grid_dependents_launch();
+    grid_dependency_wait();
     const int m = blockIdx.x;
     const uint16_t* xr = x + int64_t(m) * K;
-    float amax = 0.f;
-    for (int k = threadIdx.x * 8; k < K; k += 256 * 8) {
-        const uint4 v = ldg_nc_v4(xr + k);
-        const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+    int E = 0;
+    if (is_bf16 && m < M) {
+        float amax = 0.f;
+        for (int k = threadIdx.x * 8; k < K; k += 256 * 8) {
+            const uint4 v = ldg_nc_v4(xr + k);
+            const uint32_t r[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            amax = fmaxf(amax, fmaxf(fabsf(bf16lo_to_f32(r[i])), fabsf(bf16hi_to_f32(r[i]))));
+            for (int i = 0; i < 4; ++i)
+                amax = fmaxf(amax, fmaxf(fabsf(bf16lo_to_f32(r[i])), fabsf(bf16hi_to_f32(r[i]))));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+        __syncthreads();
+        float a = red[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+        const int eb = int(__float_as_uint(a) >> 23) & 0xFF;
+        E = eb > 141 ? eb - 141 : 0;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-    __syncthreads();
-    float a = red[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
-    const int eb = int(__float_as_uint(a) >> 23) & 0xFF;
-    const int E = eb > 141 ? eb - 141 : 0;
-    if (threadIdx.x == 0) xexp[m] = E;
+    if (threadIdx.x == 0 && m < M && xexp) xexp[m] = E;
     const float sc = exp2i(-E);
-    for (int k = threadIdx.x * 8; k < K; k += 256 * 8) {
-        uint4 v = ldg_nc_v4(xr + k);
-        v.x = f32x2_to_f16x2(bf16lo_to_f32(v.x) * sc, bf16hi_to_f32(v.x) * sc);
-        v.y = f32x2_to_f16x2(bf16lo_to_f32(v.y) * sc, bf16hi_to_f32(v.y) * sc);
-        v.z = f32x2_to_f16x2(bf16lo_to_f32(v.z) * sc, bf16hi_to_f32(v.z) * sc);
-        v.w = f32x2_to_f16x2(bf16lo_to_f32(v.w) * sc, bf16hi_to_f32(v.w) * sc);
-        *reinterpret_cast<uint4*>(x16 + int64_t(m) * K + k) = v;
+    const int nchunks = nst * (KC / 8);
+    for (int u = threadIdx.x; u < nchunks; u += 256) {
+        const int k = u * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (m < M && k < K) {
+            v = ldg_nc_v4(xr + k);
+            if (is_bf16) {
+                v.x = f32x2_to_f16x2(bf16lo_to_f32(v.x) * sc, bf16hi_to_f32(v.x) * sc);
+                v.y = f32x2_to_f16x2(bf16lo_to_f32(v.y) * sc, bf16hi_to_f32(v.y) * sc);
+                v.z = f32x2_to_f16x2(bf16lo_to_f32(v.z) * sc, bf16hi_to_f32(v.z) * sc);
+                v.w = f32x2_to_f16x2(bf16lo_to_f32(v.w) * sc, bf16hi_to_f32(v.w) * sc);
+            }
+        }
+        const int st = k / KC, kk = k % KC, atom = kk / 64, c = (kk % 64) / 8;
+        const int64_t off = int64_t(st) * MP * KC + int64_t(atom) * MP * 64 + int64_t(m) * 64 + ((c ^ (m & 7)) * 8);
+        *reinterpret_cast<uint4*>(xt + off) = v;
     }
 }
 
@@ -503,43 +617,40 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void
 }
 
 // ---------------------------------------------------------------- host: workspace
-// fp16 copy of bf16 activations plus the per-token exponents, one buffer per (device,
-// stream), grown on demand and never freed while the library is loaded (a captured graph may
-// still hold a pointer to an older one).
-struct WsKey {
-    int dev;
-    cudaStream_t st;
-    bool operator==(const WsKey& o) const { return dev == o.dev && st == o.st; }
-};
-struct WsHash {
-    size_t operator()(const WsKey& k) const { return std::hash<void*>()(k.st) ^ size_t(k.dev) * 0x9E3779B97F4A7C15ull; }
-};
-std::mutex g_ws_mu;
-std::unordered_map<WsKey, std::pair<void*, size_t>, WsHash> g_ws;
-
-cudaError_t workspace(cudaStream_t st, size_t bytes, void** out) {
+// The fp16 copy of bf16 activations (and their per-token exponents) lives in stream-ordered
+// memory from a pool the library owns, one per device: allocated on the call's stream before
+// the two kernels and released on the same stream after them.  This is safe for concurrent
+// calls on different streams and is recorded as allocation nodes when the stream is being
+// captured into a CUDA graph.  The pool keeps freed memory cached (no release threshold).
+cudaError_t device_pool(cudaMemPool_t* out) {
+    static std::mutex mu;
+    static std::unordered_map<int, cudaMemPool_t> pools;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    std::lock_guard<std::mutex> lk(g_ws_mu);
-    auto& slot = g_ws[WsKey{dev, st}];
-    if (slot.second >= bytes) {
-        *out = slot.first;
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = pools.find(dev);
+    if (it != pools.end()) {
+        *out = it->second;
         return cudaSuccess;
     }
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    e = cudaStreamIsCapturing(st, &cs);
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool;
+    e = cudaMemPoolCreate(&pool, &props);
     if (e != cudaSuccess) return e;
-    if (cs != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
-    void* p = nullptr;
-    e = cudaMalloc(&p, bytes);
+    uint64_t keep = ~uint64_t(0);
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
     if (e != cudaSuccess) return e;
-    slot = {p, bytes};  // the previous buffer is deliberately kept alive
-    *out = p;
+    pools[dev] = pool;
+    *out = pool;
     return cudaSuccess;
 }
 
-using TcKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const TcParams);
+using TcKernelFn = void (*)(const CUtensorMap, const TcParams);
 
 template <int BITS>
 TcKernelFn pick_tc_mp(int mp) {
@@ -559,19 +670,23 @@ TcKernelFn pick_tc(int bits, int mp) {
     return nullptr;
 }
 
-int w_bytes_for(int bits) { return TC_ROWS * (TC_KC * bits / 8); }
+int kc_for(int bits) { return bits == 8 ? 128 : 256; }
+int w_bytes_for(int bits) { return TC_ROWS * (kc_for(bits) * bits / 8); }
+int na_for(int bits, int mp) { return tc_na(bits, mp); }
 
 }  // namespace
 
 bool tc_supported(int64_t M, int64_t N, int64_t K, int bits, int group) {
-    if (M < 1 || M > 64 || N < 1 || K < TC_KC) return false;
+    if (M < 1 || M > 64 || N < 1 || K < 128) return false;
     if ((K / group) % 2) return false;              // scale pairs are fetched 4 bytes at a time
     if ((K * bits / 8) % 16) return false;          // TMA row pitch of the packed codes
     return true;
 }
 
+int tc_kc(int bits) { return kc_for(bits); }
+
 int tc_ring_for(int bits, int mp) {
-    const int per = mp * 256 + w_bytes_for(bits);
+    const int per = mp * kc_for(bits) * 2 + w_bytes_for(bits);
     const int budget = kTcMaxSmem - TC_SPF * TC_NDQ * 32 * 8 - 1024 - 256;
     int ring = budget / per;
     if (ring > 8) ring = 8;
@@ -579,74 +694,77 @@ int tc_ring_for(int bits, int mp) {
 }
 
 size_t tc_smem_bytes(int bits, int mp, int ring) {
-    const TcSmemLayout L = tc_layout(mp, w_bytes_for(bits), ring);
-    size_t red = size_t(mp) * TC_ROWS * 4;
-    size_t body = size_t(L.total) > red ? size_t(L.total) : red;
+    const TcSmemLayout L = tc_layout(mp * kc_for(bits) * 2, w_bytes_for(bits), ring, na_for(bits, mp));
+    const size_t red = size_t(mp) * TC_ROWS * 4;
+    const size_t body = size_t(L.total) > red ? size_t(L.total) : red;
     return body + 1024;  // alignment slack
 }
 
 cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) {
     TcKernelFn fn = pick_tc(a.bits, c.mp);
     if (!fn) return cudaErrorInvalidValue;
-    const void* xsrc = a.x;
-    const int* xexp = nullptr;
-    if (a.is_bf16) {
-        void* ws = nullptr;
-        const size_t xbytes = size_t(a.M) * size_t(a.K) * 2;
-        const size_t need = ((xbytes + 255) & ~size_t(255)) + 64 * sizeof(int);
-        cudaError_t e = workspace(stream, need, &ws);
-        if (e != cudaSuccess) return e;
-        uint16_t* x16 = static_cast<uint16_t*>(ws);
-        int* ex = reinterpret_cast<int*>(static_cast<char*>(ws) + ((xbytes + 255) & ~size_t(255)));
-        cudaLaunchConfig_t pc = {};
-        pc.gridDim = dim3(unsigned(a.M), 1, 1);
-        pc.blockDim = dim3(256, 1, 1);
-        pc.stream = stream;
-        cudaLaunchAttribute pa[1];
-        pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        pa[0].val.programmaticStreamSerializationAllowed = 1;
-        pc.attrs = pa;
-        pc.numAttrs = c.pdl ? 1 : 0;
-        e = cudaLaunchKernelEx(&pc, xprep_bf16_kernel, a.x, x16, ex, int(a.K));
-        if (e != cudaSuccess) return e;
-        xsrc = x16;
-        xexp = ex;
-    }
+    const int KC = kc_for(a.bits);
+    const int nst_k = int((a.K + KC - 1) / KC);
 
-    CUtensorMap wmap, xmap;
+    // stage tiles of x (fp16) and the per-token exponents, in stream-ordered scratch memory
+    cudaMemPool_t pool;
+    cudaError_t e = device_pool(&pool);
+    if (e != cudaSuccess) return e;
+    const size_t xt_bytes = size_t(nst_k) * size_t(c.mp) * size_t(KC) * 2;
+    void* ws = nullptr;
+    e = cudaMallocFromPoolAsync(&ws, xt_bytes + 64 * sizeof(int), pool, stream);
+    if (e != cudaSuccess) return e;
+    auto finish = [&](cudaError_t err) {
+        cudaError_t f = cudaFreeAsync(ws, stream);  // after everything enqueued above
+        return err == cudaSuccess ? f : err;
+    };
+    uint16_t* xt = static_cast<uint16_t*>(ws);
+    int* xexp = a.is_bf16 ? reinterpret_cast<int*>(static_cast<char*>(ws) + xt_bytes) : nullptr;
+
+    cudaLaunchAttribute pdl_attr;
+    pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3(unsigned(c.mp), 1, 1);
+    pc.blockDim = dim3(256, 1, 1);
+    pc.stream = stream;
+    pc.attrs = &pdl_attr;
+    pc.numAttrs = c.pdl ? 1 : 0;
+    e = KC == 256 ? cudaLaunchKernelEx(&pc, xprep_kernel<256>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
+                  : cudaLaunchKernelEx(&pc, xprep_kernel<128>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp);
+    if (e != cudaSuccess) return finish(e);
+
+    CUtensorMap wmap;
     const uint64_t KW = uint64_t(a.K) * a.bits / 32;
-    const CUtensorMapSwizzle wsw = a.bits == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                 : a.bits == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
     if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
-                     uint32_t(TC_KC * a.bits / 32), TC_ROWS, wsw))
-        return cudaErrorInvalidValue;
-    if (!make_map_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xsrc, uint64_t(a.K), uint64_t(a.M), 64,
-                     uint32_t(c.mp), CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
+                     uint32_t(KC * a.bits / 32), TC_ROWS, wsw))
+        return finish(cudaErrorInvalidValue);
 
     TcParams p;
     p.scales = a.scales;
     p.biases = a.biases;
     p.y = a.y;
+    p.xt = xt;
     p.xexp = xexp;
     p.M = int(a.M);
     p.N = int(a.N);
     p.K = int(a.K);
     p.G = int(a.K / a.group);
     p.gshift = a.group == 32 ? 5 : a.group == 64 ? 6 : 7;
-    p.nstages_k = int((a.K + TC_KC - 1) / TC_KC);
+    p.nstages_k = nst_k;
     p.stages_per_split = c.stages_per_split;
-    p.split = (p.nstages_k + c.stages_per_split - 1) / c.stages_per_split;
+    p.split = (nst_k + c.stages_per_split - 1) / c.stages_per_split;
     p.out_bf16 = a.is_bf16;
     p.static_w = c.static_weights ? 1 : 0;
     p.ring = c.ring;
 
     const size_t smem = tc_smem_bytes(a.bits, c.mp, c.ring);
-    cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (err != cudaSuccess) return err;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return finish(e);
     if (p.split > 8) {
-        err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (err != cudaSuccess) return err;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return finish(e);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned((a.N + TC_ROWS - 1) / TC_ROWS), unsigned(p.split), 1);
@@ -662,15 +780,60 @@ cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) 
         attrs[na].val.clusterDim.z = 1;
         ++na;
     }
-    if (c.pdl) {
-        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attrs[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
+    if (c.pdl) attrs[na++] = pdl_attr;
     cfg.attrs = attrs;
     cfg.numAttrs = unsigned(na);
-    return cudaLaunchKernelEx(&cfg, fn, wmap, xmap, p);
+    return finish(cudaLaunchKernelEx(&cfg, fn, wmap, p));
 }
+
+// How many clusters of `split` blocks of this kernel can be resident at once (0 if the query
+// fails, e.g. without a device).  Cached per (device, bits, mp, ring, split).
+int tc_max_active_clusters(int bits, int mp, int ring, int split) {
+    static std::mutex mu;
+    static std::unordered_map<uint64_t, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const uint64_t key = (uint64_t(dev) << 40) | (uint64_t(bits) << 32) | (uint64_t(mp) << 16) |
+                         (uint64_t(ring) << 8) | uint64_t(split);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) return it->second;
+    }
+    TcKernelFn fn = pick_tc(bits, mp);
+    int n = 0;
+    if (fn) {
+        const size_t smem = tc_smem_bytes(bits, mp, ring);
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) == cudaSuccess &&
+            (split <= 8 || cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(1, unsigned(split), 1);
+            cfg.blockDim = dim3(TC_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr;
+            attr.id = cudaLaunchAttributeClusterDimension;
+            attr.val.clusterDim.x = 1;
+            attr.val.clusterDim.y = unsigned(split);
+            attr.val.clusterDim.z = 1;
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) n = 0;
+        }
+        cudaGetLastError();  // a failed query must not leave a sticky error behind
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    cache[key] = n;
+    return n;
+}
+
+#ifdef QMM_TC_TRACE
+extern "C" cudaError_t qmm_tc_trace_read(unsigned long long* host16x256) {
+    return cudaMemcpyFromSymbol(host16x256, g_tc_trace, sizeof(g_tc_trace));
+}
+extern "C" cudaError_t qmm_tc_trace_blocks(unsigned long long* host4096x8) {
+    return cudaMemcpyFromSymbol(host4096x8, g_tc_blocks, sizeof(g_tc_blocks));
+}
+#endif
 
 cudaError_t tc_read_and_clear_errors(unsigned* out) {
     unsigned v = 0, zero = 0;

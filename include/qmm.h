@@ -82,12 +82,18 @@ qmm_status qmm_dequantize(const uint32_t* packed, const uint16_t* scales,
 
 /*
  * qmm -- y[M,N] = x[M,K] . dequant(packed, scales, biases)^T for 0 <= M <= 64.
- * Arithmetic: codes are dequantized to fp16 (s*q + b with one rounding), bf16 activations
- * are converted to fp16 after an exact power-of-two rescale chosen per thread block so that
- * no value overflows, products are accumulated in fp32 on the tensor cores, and the result
- * is rounded once to the output dtype.  Split-K partial sums are combined in a fixed order,
- * so the result is bitwise reproducible run to run.  M == 0 or N == 0 is a no-op; K == 0
- * writes zeros.  Alignment: x, packed and y 16-byte aligned; scales and biases 2-byte.
+ * Arithmetic: codes are dequantized to fp16 (s*q + b with one rounding); bf16 activations
+ * are converted to fp16 after an exact power-of-two rescale (per thread block on the
+ * warp-tile kernel, per token on the tensor-core kernel) chosen so that no value overflows;
+ * products are accumulated in fp32 on the tensor cores and the result is rounded once to the
+ * output dtype.  Split-K partial sums are combined in a fixed order, so the result is
+ * bitwise reproducible run to run.  M == 0 or N == 0 is a no-op; K == 0 writes zeros.
+ * Alignment: x, packed and y 16-byte aligned; scales and biases 2-byte (4-byte alignment is
+ * needed for the tensor-core kernel, which the dispatcher otherwise avoids).
+ * Scratch memory: the tensor-core kernel stages x in a small buffer (about 2*64*K bytes) taken
+ * on `stream` from a memory pool the library owns (cudaMallocFromPoolAsync) and released on
+ * the same stream after the call; this is also valid while the stream is being captured into
+ * a CUDA graph.
  * The kernel may read `packed`, `scales` and `biases` before earlier work on `stream` has
  * finished only when the plan sets QMM_PLAN_STATIC_WEIGHTS (see qmm_ex); qmm() never does.
  * Thread safety: calls from different host threads or on different streams are safe.
@@ -115,7 +121,8 @@ enum {
 typedef struct {
     int32_t kernel;   /* QMM_KERNEL_*                                                       */
     int32_t split;    /* number of K slices (thread-block cluster size along K), 1..16      */
-    int32_t warps;    /* warps per block for QMM_KERNEL_MMA (4 or 8); ignored otherwise     */
+    int32_t warps;    /* warps per block: 4 or 8 for QMM_KERNEL_MMA (0 = default); the      
+                         tensor-core kernel always uses 18 and ignores this field           */
     uint32_t flags;   /* QMM_PLAN_* bits                                                     */
     int32_t reserved[4];
 } qmm_plan;

@@ -83,7 +83,7 @@ def test_plans(L):
     assert p.kernel in (q.KERNEL_MMA, q.KERNEL_TC) and 1 <= p.split <= 16
     bad = q.make_plan(split=17)
     assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(bad), None) == q.QMM_ERR_INVALID_ARG
-    bad = q.make_plan(warps=3)
+    bad = q.make_plan(kernel=q.KERNEL_MMA, warps=3)
     assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(bad), None) == q.QMM_ERR_INVALID_ARG
     bad = q.make_plan(flags=1 << 7)
     assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(bad), None) == q.QMM_ERR_INVALID_ARG

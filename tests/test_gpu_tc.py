@@ -95,3 +95,24 @@ def test_tc_deterministic_and_back_to_back(oracle_mod):
     assert all(torch.equal(ys[0], y) for y in ys[1:])
     op, os_, ob = oracle_quantize(oracle_mod, w2.cpu(), 4, 64)
     check_close(y2, oracle_qmm(oracle_mod, y1.cpu(), op, os_, ob, K, 4, 64), torch.float16, "chained")
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_tc_inside_cuda_graph(oracle_mod, dtype):
+    """Captured on a side stream (torch.cuda.graph) and replayed: the bf16 path's stream-ordered
+    workspace must work inside capture."""
+    M, N, K = 24, 512, 1024
+    w = w_input(N, K, dtype, 4, 0.02)
+    op, os_, ob = oracle_quantize(oracle_mod, w, 4, 64)
+    P, S, B = to_device_weights(op, os_, ob)
+    x = x_input(M, K, dtype).cuda()
+    y = torch.empty((M, N), dtype=dtype, device="cuda")
+    plan = q.make_plan(kernel=q.KERNEL_TC, flags=q.PLAN_PDL | q.PLAN_STATIC_WEIGHTS)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        q.qmm(x, P, S, B, 4, 64, out=y, plan=plan)
+    y.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    check_close(y, oracle_qmm(oracle_mod, x.cpu(), op, os_, ob, K, 4, 64), dtype, "graph")
