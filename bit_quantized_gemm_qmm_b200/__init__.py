@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.qmm_version.restype = I
     L.qmm_device_errors.argtypes = [P]
     L.qmm_device_errors.restype = I
+    L.qmm_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, I, I, U, P]
+    L.qmm_noalloc.restype = I
     _lib = L
     return L
 

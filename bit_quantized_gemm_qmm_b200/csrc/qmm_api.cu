@@ -293,6 +293,41 @@ qmm_status qmm(const void* x, const uint32_t* packed, const uint16_t* scales,
     return qmm_ex(x, packed, scales, biases, y, M, N, K, bits, group, dtype, nullptr, stream);
 }
 
+qmm_status qmm_noalloc(const void* x, const uint32_t* packed, const uint16_t* scales,
+                       const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+                       int group, qmm_dtype dtype, void* stream) {
+    qmm_status s = validate_qmm(x, packed, scales, biases, y, M, N, K, bits, group, dtype);
+    if (s != QMM_OK) return s;
+    if (M == 0 || N == 0 || K == 0)
+        return fail(QMM_ERR_UNSUPPORTED, "qmm_noalloc needs M, N, K > 0 (use qmm for empty shapes)");
+    if (!tc_supported(M, N, K, bits, group) || !aligned(scales, 4) || !aligned(biases, 4))
+        return fail(QMM_ERR_UNSUPPORTED,
+                    "qmm_noalloc runs only the tensor-core kernel: K >= 128, an even number of groups "
+                    "per row, a 16-byte multiple of packed bytes per row, 4-byte aligned scales/biases");
+    const size_t need = tc_noalloc_need(M, K, bits);
+    if (need > tc_noalloc_capacity())
+        return fail(QMM_ERR_UNSUPPORTED,
+                    "qmm_noalloc scratch limit: this call needs %zu bytes of staged activations, the "
+                    "fixed array holds %zu (K rounded up to the stage size x M rounded up to 16 x 2)",
+                    need, tc_noalloc_capacity());
+    TcConfig c = tc_config(M, N, K, bits, 0);
+    if (c.ring < 2) return fail(QMM_ERR_UNSUPPORTED, "tensor-core plan does not fit shared memory");
+    QmmArgs a;
+    a.x = static_cast<const uint16_t*>(x);
+    a.packed = packed;
+    a.scales = scales;
+    a.biases = biases;
+    a.y = static_cast<uint16_t*>(y);
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.bits = bits;
+    a.group = group;
+    a.is_bf16 = dtype == QMM_BF16;
+    cudaError_t e = launch_tc_noalloc(a, c, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm_noalloc launch");
+}
+
 const char* qmm_status_string(qmm_status status) {
     switch (status) {
         case QMM_OK: return "ok";

@@ -60,5 +60,9 @@ size_t tc_smem_bytes(int bits, int mp, int ring);
 cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream);
 cudaError_t tc_read_and_clear_errors(unsigned* out);
 int tc_max_active_clusters(int bits, int mp, int ring, int split);
+// Tensor-core path with scratch in a fixed device array (qmm_noalloc).
+size_t tc_noalloc_need(int64_t M, int64_t K, int bits);
+size_t tc_noalloc_capacity();
+cudaError_t launch_tc_noalloc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream);
 
 }  // namespace qmm_impl

@@ -845,3 +845,133 @@ cudaError_t tc_read_and_clear_errors(unsigned* out) {
 }
 
 }  // namespace qmm_impl
+
+// ==========================================================================================
+// Tensor-core path with its scratch in a fixed device array (entry point qmm_noalloc).
+//
+// For callers that must not allocate device memory during a call, such as a serving loop
+// under a fixed memory budget that reserves every byte at start-up, or code running where
+// an allocation would add a device-wide synchronization it cannot afford.  The fp16 x tiles
+// and per-token exponents live in one file-scope array per device instead of pool memory.
+// Every call on a device reuses that array; calls whose kernels overlap on the GPU (for
+// instance on two streams at once) race on it.  Each call rewrites all of the scratch it
+// reads (padding rows and columns included), so nothing needs clearing between calls.
+// ==========================================================================================
+namespace qmm_impl {
+namespace {
+
+constexpr size_t kNoAllocXBytes = size_t(2) << 20;        // fp16 x tiles: up to 2 MiB
+constexpr size_t kNoAllocBytes = kNoAllocXBytes + 256;     // + 64 per-token exponents
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch for each device, looked up once with that device
+// current (the host-side symbol is only a handle, not a device address).
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t tc_noalloc_need(int64_t M, int64_t K, int bits) {
+    const int64_t KC = kc_for(bits);
+    const int64_t mp = (M + 15) / 16 * 16;
+    return size_t((K + KC - 1) / KC * KC) * size_t(mp < 16 ? 16 : mp) * 2;
+}
+
+size_t tc_noalloc_capacity() { return kNoAllocXBytes; }
+
+cudaError_t launch_tc_noalloc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) {
+    TcKernelFn fn = pick_tc(a.bits, c.mp);
+    if (!fn) return cudaErrorInvalidValue;
+    const int KC = kc_for(a.bits);
+    const int nst_k = int((a.K + KC - 1) / KC);
+    const size_t xt_bytes = size_t(nst_k) * size_t(c.mp) * size_t(KC) * 2;
+    if (xt_bytes > kNoAllocXBytes) return cudaErrorInvalidValue;
+    void* ws = nullptr;
+    cudaError_t e = noalloc_scratch(&ws);
+    if (e != cudaSuccess) return e;
+    uint16_t* xt = static_cast<uint16_t*>(ws);
+    int* xexp = a.is_bf16 ? reinterpret_cast<int*>(static_cast<char*>(ws) + kNoAllocXBytes) : nullptr;
+
+    cudaLaunchAttribute pdl_attr;
+    pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3(unsigned(c.mp), 1, 1);
+    pc.blockDim = dim3(256, 1, 1);
+    pc.stream = stream;
+    pc.attrs = &pdl_attr;
+    pc.numAttrs = c.pdl ? 1 : 0;
+    e = KC == 256 ? cudaLaunchKernelEx(&pc, xprep_kernel<256>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
+                  : cudaLaunchKernelEx(&pc, xprep_kernel<128>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp);
+    if (e != cudaSuccess) return e;
+
+    CUtensorMap wmap;
+    const uint64_t KW = uint64_t(a.K) * a.bits / 32;
+    const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
+                     uint32_t(KC * a.bits / 32), TC_ROWS, wsw))
+        return cudaErrorInvalidValue;
+
+    TcParams p;
+    p.scales = a.scales;
+    p.biases = a.biases;
+    p.y = a.y;
+    p.xt = xt;
+    p.xexp = xexp;
+    p.M = int(a.M);
+    p.N = int(a.N);
+    p.K = int(a.K);
+    p.G = int(a.K / a.group);
+    p.gshift = a.group == 32 ? 5 : a.group == 64 ? 6 : 7;
+    p.nstages_k = nst_k;
+    p.stages_per_split = c.stages_per_split;
+    p.split = (nst_k + c.stages_per_split - 1) / c.stages_per_split;
+    p.out_bf16 = a.is_bf16;
+    p.static_w = c.static_weights ? 1 : 0;
+    p.ring = c.ring;
+
+    const size_t smem = tc_smem_bytes(a.bits, c.mp, c.ring);
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    if (p.split > 8) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned((a.N + TC_ROWS - 1) / TC_ROWS), unsigned(p.split), 1);
+    cfg.blockDim = dim3(TC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    if (p.split > 1) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = unsigned(p.split);
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (c.pdl) attrs[na++] = pdl_attr;
+    cfg.attrs = attrs;
+    cfg.numAttrs = unsigned(na);
+    return cudaLaunchKernelEx(&cfg, fn, wmap, p);
+}
+
+}  // namespace qmm_impl

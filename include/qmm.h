@@ -139,6 +139,31 @@ qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
                   const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                   int group, qmm_dtype dtype, const qmm_plan* plan, void* stream);
 
+/*
+ * qmm_noalloc -- qmm() on the tensor-core kernel without allocating anything.  The pages have
+ * no counterpart to this call; it exists for callers that must not allocate device memory
+ * during a call: a serving loop that reserves all of its memory at start-up and runs under
+ * a fixed budget, or code for which an allocation's possible device-wide synchronization is
+ * not acceptable.  Where qmm() takes its activation staging buffer from a stream-ordered
+ * pool, this call uses one fixed array compiled into the library: 2 MiB + 256 bytes of
+ * device memory that every GPU which loads the library holds until the process exits.
+ *   - Limit: the staged activations, roundup(K, 256) * roundup(M, 16) * 2 bytes for 4- and
+ *     6-bit codes (roundup(K, 128) for 8-bit), must fit in 2 MiB (for example K <= 16384
+ *     at M = 64); larger calls return QMM_ERR_UNSUPPORTED with the sizes in qmm_last_error.
+ *   - Shapes: only those the tensor-core kernel takes (K >= 128, an even number of groups
+ *     per row, a 16-byte multiple of packed bytes per row, 4-byte aligned scales and biases;
+ *     M, N, K > 0); others return QMM_ERR_UNSUPPORTED and launch nothing.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before capturing any stream.
+ *   - All calls on a device share the array and it keeps the last call's contents; every
+ *     call rewrites all of it that it reads, so nothing needs clearing.  Calls whose kernels
+ *     overlap on the GPU (for example on two streams at once) race on it: serialize them.
+ * Arguments, layouts, results and errors are otherwise those of qmm().
+ */
+qmm_status qmm_noalloc(const void* x, const uint32_t* packed, const uint16_t* scales,
+                       const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
+                       int group, qmm_dtype dtype, void* stream);
+
 /* Read and clear the current device's kernel error word (synchronizes with the device).
  * Bit 0: a tensor-core kernel block gave up waiting on one of its pipeline barriers (a wait
  * that should finish in microseconds ran for about two seconds).  That block then dropped
