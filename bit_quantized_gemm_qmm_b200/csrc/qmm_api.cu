@@ -51,8 +51,9 @@ int ceil_div(int64_t a, int64_t b) { return int((a + b - 1) / b); }
 int round_up(int64_t a, int64_t b) { return int((a + b - 1) / b * b); }
 
 // Dispatch table for the MMA kernel: 8-token tiles, warps per block, K split, x staging.
-MmaConfig mma_config(int64_t M, int64_t N, int64_t K, int bits, int warps_req, int split_req) {
+MmaConfig mma_config(int64_t M, int64_t N, int64_t K, int bits, int group, int warps_req, int split_req) {
     MmaConfig c;
+    c.group = group;
     c.mt = M > 0 ? ceil_div(M, 8) : 1;
     c.warps = warps_req ? warps_req : (N <= 2048 ? 4 : 8);
     const int KS = bits == 8 ? 64 : 128;
@@ -173,7 +174,7 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
     if (p.kernel == QMM_KERNEL_MMA) {
         if (p.warps != 0 && p.warps != 4 && p.warps != 8)
             return fail(QMM_ERR_INVALID_ARG, "warps=%d (4 or 8)", p.warps);
-        MmaConfig c = mma_config(M, N, K, bits, p.warps, p.split);
+        MmaConfig c = mma_config(M, N, K, bits, group, p.warps, p.split);
         c.pdl = pdl;
         c.static_weights = stat;
         if (mma_smem_bytes(c) > kMmaMaxSmem)

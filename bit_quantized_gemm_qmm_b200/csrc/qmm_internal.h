@@ -27,6 +27,7 @@ struct MmaConfig {
     int split;     // K slices = cluster size along grid.y
     int kslice;    // K elements per slice (multiple of 128)
     int xchunk;    // K elements of x staged in shared memory at a time
+    int group;     // quantization group (the staged group sums depend on it)
     bool pdl;
     bool static_weights;
 };
@@ -39,6 +40,7 @@ cudaError_t launch_dequantize(const uint32_t* packed, const uint16_t* scales,
                               int out_bf16, void* w_out, cudaStream_t stream);
 
 // Shared-memory bytes the MMA kernel needs for a configuration.
+int mma_gpad(const MmaConfig& c);
 size_t mma_smem_bytes(const MmaConfig& c);
 // Largest dynamic shared memory the MMA kernel is allowed to request.
 constexpr size_t kMmaMaxSmem = 100 * 1024;

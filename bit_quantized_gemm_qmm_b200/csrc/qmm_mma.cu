@@ -15,11 +15,16 @@
 //   * C (16 x 8)  = y^T, fp32 in registers, MT tiles of 8 tokens (M <= 8*MT).
 // Packed codes stream straight from HBM into registers with 128-bit (4/8-bit) or 64-bit
 // (6-bit) loads, PF steps ahead; no shared memory or barrier touches the weight stream.
-// Within each MMA the K order is free, so each lane takes 4 *consecutive* codes per MMA and
-// x is read in its natural order.  Codes become fp16 with byte permutes and the exponent
-// trick (1024 + q is exact in fp16), then w = s*q + b in one fp16 fma, the same single
-// rounding as RNE_fp16(s*q + b).  bf16 activations are rescaled by an exact power of two
-// per block (so none overflows fp16) and converted once while staged in shared memory.
+//
+// Arithmetic.  Per group, sum_k x_k (s q_k + b) = sum_k x_k (s q_k) + b X with X = sum_k x_k
+// (the bias factored out of the group).  The tensor cores take A = RN_fp16(s q): a code is dropped into the
+// mantissa of an fp16 "magic" constant M with one AND/OR, giving M + q exactly, and
+// fma(M + q, s, -M s) = s q with a single rounding (M s is exact while |s| < 64; a step with
+// a larger scale takes sub-then-mul instead).  Within an MMA the K order is free, so each
+// format pairs the codes that one AND can reach (4-bit: codes i and i+4 of a word) and x is
+// staged in shared memory in the same order.  The b X term runs as one more MMA per eight
+// groups, with X split into fp16 hi + lo parts.  bf16 activations are rescaled by an exact
+// power of two per block (so none overflows fp16) and converted once while staged.
 // K may be split across the blocks of a thread-block cluster; partial sums are combined
 // over distributed shared memory in rank order, so results are deterministic.
 #include <cooperative_groups.h>
@@ -32,13 +37,16 @@ namespace cg = cooperative_groups;
 namespace qmm_impl {
 namespace {
 
-// Codes per lane per row per step (U) and the 32-bit words they occupy (NREG).
+// Per format: U codes per lane per row per step (one K-span of a lane), NREG 32-bit words
+// holding them, UN codes per staging unit (the block the K permutation acts on).  A step
+// covers KS = 4*U codes of K (the four lanes of a row side by side).
 template <int BITS> struct Fmt;
-template <> struct Fmt<4> { static constexpr int U = 32, NREG = 4; };  // 16 bytes
-template <> struct Fmt<6> { static constexpr int U = 32, NREG = 6; };  // 24 bytes
-template <> struct Fmt<8> { static constexpr int U = 16, NREG = 4; };  // 16 bytes
+template <> struct Fmt<4> { static constexpr int U = 32, NREG = 4, UN = 8; };   // 16 bytes
+template <> struct Fmt<6> { static constexpr int U = 32, NREG = 6, UN = 16; };  // 24 bytes
+template <> struct Fmt<8> { static constexpr int U = 16, NREG = 4, UN = 8; };   // 16 bytes
 
-constexpr int PF = 4;  // steps of codes in flight per lane
+constexpr int PF = 4;    // steps of codes in flight per lane
+constexpr int XPAD = 4;  // 16-byte chunks of padding after each staged x row
 
 struct Params {
     const uint16_t* x;
@@ -49,145 +57,157 @@ struct Params {
     int M, N, K;
     int G;        // groups per row
     int KW;       // words per row
+    int group;
     int gshift;   // log2(group)
     int is_bf16;
     int kslice;   // K elements per split
-    int xchunk;   // K elements of x per staging pass (multiple of PF * KS)
+    int xchunk;   // K elements of x per staging pass (multiple of PF * KS and of group)
+    int gpad;     // group slots per staged row of group sums (multiple of 8)
     int split;
     int static_w;
 };
 
-// x tile in shared memory: [8*MT rows][xchunk] fp16, 16-byte chunks XOR-swizzled so that the
-// B-fragment reads (8 lanes of a phase = 2 rows x 4 lanes) hit 8 distinct bank groups.
-__device__ __forceinline__ uint32_t x_chunk_addr(uint32_t base, int rowbytes, int m, int c) {
-    const int phys = c ^ (((c >> 3) & 1) << 1) ^ (m & 1);
-    return base + uint32_t(m * rowbytes + (phys << 4));
+// fp16x2 constants of the code -> value conversion.  A code q placed in mantissa bits
+// [o, o+n) of an fp16 whose exponent makes bit o worth 1 reads as M + q exactly, where
+// M = 2^(10-o): 1024 for o = 0, 256 for o = 2, 64 for o = 4.
+constexpr uint32_t kM1024x2 = 0x64006400u;   // (1024, 1024)
+constexpr uint32_t kM64x2 = 0x54005400u;     // (64, 64)
+constexpr uint32_t kM1024_256 = 0x5C006400u; // (lo 1024, hi 256)
+constexpr uint32_t kM64_1024 = 0x64005400u;  // (lo 64, hi 1024)
+constexpr uint32_t kN1024x2 = 0xE400E400u;   // (-1024, -1024)
+constexpr uint32_t kN64x2 = 0xD400D400u;     // (-64, -64)
+constexpr uint32_t kN1024_256 = 0xDC00E400u; // (lo -1024, hi -256)
+constexpr uint32_t kN64_1024 = 0xE400D400u;  // (lo -64, hi -1024)
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Per-row constants of one step: S = (s, s) and the offsets -M*s for the two magic layouts
+// the format uses.  All are exact while |s| < 64 (then 1024*s is a finite fp16).
+struct RowConst {
+    uint32_t S, NA, NB;
+};
+
+template <int BITS>
+__device__ __forceinline__ RowConst row_const(uint32_t sbits) {
+    RowConst r;
+    r.S = __byte_perm(sbits, 0u, 0x1010u);
+    if constexpr (BITS == 6) {
+        r.NA = hmul2(r.S, kN1024_256);
+        r.NB = hmul2(r.S, kN64_1024);
+    } else {
+        r.NA = hmul2(r.S, kN1024x2);
+        r.NB = hmul2(r.S, kN64x2);
+    }
+    return r;
+}
+
+// s*q for the two codes held in v = M + q (per half): one rounding of the exact product.
+template <bool SAFE>
+__device__ __forceinline__ uint32_t scaled(uint32_t v, uint32_t magic, uint32_t S, uint32_t N) {
+    if constexpr (SAFE) return hmul2(hsub2(v, magic), S);  // |s| >= 64: -M*s would overflow
+    else return hfma2(v, S, N);                            // s*(M+q) - M*s
 }
 
 // ---------------------------------------------------------------- loads of one step
 template <int BITS>
-__device__ __forceinline__ void load_step(const Params& p, bool v0, bool v1, int64_t woff0,
-                                          int64_t woff1, int64_t goff0, int64_t goff1, int k,
-                                          bool valid, uint32_t (&w)[2][Fmt<BITS>::NREG],
-                                          uint32_t (&sb)[2]) {
-    constexpr int NREG = Fmt<BITS>::NREG;
+__device__ __forceinline__ void load_codes(const uint32_t* wp, uint32_t (&w)[Fmt<BITS>::NREG]) {
+    if constexpr (BITS == 6) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const bool ok = valid && (r == 0 ? v0 : v1);
-        const int64_t woff = r == 0 ? woff0 : woff1;
-        const int64_t goff = r == 0 ? goff0 : goff1;
-        if (ok) {
-            if constexpr (BITS == 6) {
-                const uint32_t* src = p.packed + woff + (k >> 5) * 6;
-#pragma unroll
-                for (int i = 0; i < 3; ++i) {
-                    uint2 v = ldg_nc_v2(src + 2 * i);
-                    w[r][2 * i] = v.x;
-                    w[r][2 * i + 1] = v.y;
-                }
-            } else {
-                const uint4 v = ldg_stream_v4(p.packed + woff + (k * BITS >> 5));
-                w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
-            }
-            const int64_t gi = goff + (k >> p.gshift);
-            sb[r] = ldg_nc_u16(p.scales + gi) | (ldg_nc_u16(p.biases + gi) << 16);
-        } else {
-#pragma unroll
-            for (int i = 0; i < NREG; ++i) w[r][i] = 0u;
-            sb[r] = 0u;  // s = b = 0 -> the dequantized weight is exactly 0
+        for (int i = 0; i < 3; ++i) {
+            const uint2 v = ldg_nc_v2(wp + 2 * i);
+            w[2 * i] = v.x;
+            w[2 * i + 1] = v.y;
         }
+    } else {
+        const uint4 v = ldg_stream_v4(wp);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
     }
 }
 
-// ---------------------------------------------------------------- dequant helpers
-// Pair (code 2j, code 2j+1) of a 4-bit word -> fp16x2 (s*q + b).
-__device__ __forceinline__ uint32_t dq4_pair(uint32_t w, int j, uint32_t s2, uint32_t b2) {
-    const uint32_t t = __byte_perm(w, 0u, 0x4040u | uint32_t(j) | (uint32_t(j) << 8));
-    const uint32_t h = (t & 0x00F0000Fu) | kMagic1024x2;   // (1024 + lo, 1024 + 16*hi)
-    const uint32_t q = hfma2(h, kOneSixteenth, kMinus1024_64);  // (lo, hi), exact
-    return hfma2(q, s2, b2);
-}
-
-// Pair (byte 2j, byte 2j+1) of an 8-bit word -> fp16x2.
-__device__ __forceinline__ uint32_t dq8_pair(uint32_t w, int j, uint32_t s2, uint32_t b2) {
-    const uint32_t h = __byte_perm(w, 0x64646464u, j == 0 ? 0x4140u : 0x4342u);  // 1024 + q
-    const uint32_t q = hfma2(h, kOnes, kMinus1024x2);
-    return hfma2(q, s2, b2);
-}
-
-// 12-bit field (code 2j at bits 0..5, code 2j+1 at bits 6..11) -> fp16x2.
-__device__ __forceinline__ uint32_t dq6_field(uint32_t f, uint32_t s2, uint32_t b2) {
-    const uint32_t h = (f & 0x3Fu) | ((f << 10) & 0x3F0000u) | kMagic1024x2;
-    const uint32_t q = hfma2(h, kOnes, kMinus1024x2);
-    return hfma2(q, s2, b2);
-}
-
 // ---------------------------------------------------------------- one step of MMAs
-// w[r][...] : codes of rows g (r=0) and g+8 (r=1), U consecutive codes starting at the lane's
-// span.  cbase: index of the lane's first 16-byte x chunk within the staged tile.
-template <int BITS, int MT>
+// w[r]: the lane's U codes of rows g (r=0) and g+8 (r=1); C[r]: their step constants.
+// xa: shared address of the lane's first staged x chunk of this step for token row g;
+// xmt: byte distance between 8-token tiles.  Each MMA takes two code pairs per row; the
+// staged x of the lane's K-span is stored in exactly that pair order.
+template <int BITS, int MT, bool SAFE>
 __device__ __forceinline__ void compute_step(const uint32_t (&w)[2][Fmt<BITS>::NREG],
-                                             const uint32_t (&sb)[2], uint32_t xs, int rowbytes,
-                                             int g, int cbase, float (&acc)[MT][4]) {
-    const uint32_t s2_0 = __byte_perm(sb[0], 0u, 0x1010u), b2_0 = __byte_perm(sb[0], 0u, 0x3232u);
-    const uint32_t s2_1 = __byte_perm(sb[1], 0u, 0x1010u), b2_1 = __byte_perm(sb[1], 0u, 0x3232u);
+                                             const RowConst (&C)[2], uint32_t xa, uint32_t xmt,
+                                             float (&acc)[MT][4]) {
     if constexpr (BITS == 4) {
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {  // one word = 8 codes = 2 MMAs = one x chunk
-            uint32_t a0[4], a1[4];
+        for (int j = 0; j < 4; ++j) {  // word j: codes 8j..8j+7, pairs (0,4) (1,5) (2,6) (3,7)
+            uint32_t a[2][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                a0[j] = dq4_pair(w[0][wi], j, s2_0, b2_0);
-                a1[j] = dq4_pair(w[1][wi], j, s2_1, b2_1);
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t v = w[r][j], v8 = v >> 8;
+                a[r][0] = scaled<SAFE>((v & 0x000F000Fu) | kM1024x2, kM1024x2, C[r].S, C[r].NA);
+                a[r][1] = scaled<SAFE>((v & 0x00F000F0u) | kM64x2, kM64x2, C[r].S, C[r].NB);
+                a[r][2] = scaled<SAFE>((v8 & 0x000F000Fu) | kM1024x2, kM1024x2, C[r].S, C[r].NA);
+                a[r][3] = scaled<SAFE>((v8 & 0x00F000F0u) | kM64x2, kM64x2, C[r].S, C[r].NB);
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const uint4 xb = lds_v4(x_chunk_addr(xs, rowbytes, g + 8 * mt, cbase + wi));
-                mma_16816(acc[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
-                mma_16816(acc[mt], a0[2], a1[2], a0[3], a1[3], xb.z, xb.w);
+                const uint4 xb = lds_v4(xa + j * 64 + mt * xmt);
+                mma_16816(acc[mt], a[0][0], a[1][0], a[0][1], a[1][1], xb.x, xb.y);
+                mma_16816(acc[mt], a[0][2], a[1][2], a[0][3], a[1][3], xb.z, xb.w);
             }
         }
     } else if constexpr (BITS == 8) {
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {  // two words = 8 codes = 2 MMAs = one x chunk
-            uint32_t a0[4], a1[4];
+        for (int j = 0; j < 2; ++j) {  // words 2j, 2j+1: codes 8j..8j+7 in natural pairs
+            uint32_t a[2][4];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                a0[2 * h] = dq8_pair(w[0][2 * jj + h], 0, s2_0, b2_0);
-                a0[2 * h + 1] = dq8_pair(w[0][2 * jj + h], 1, s2_0, b2_0);
-                a1[2 * h] = dq8_pair(w[1][2 * jj + h], 0, s2_1, b2_1);
-                a1[2 * h + 1] = dq8_pair(w[1][2 * jj + h], 1, s2_1, b2_1);
+            for (int r = 0; r < 2; ++r) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t v = w[r][2 * j + h];
+                    a[r][2 * h] = scaled<SAFE>(__byte_perm(v, 0x64646464u, 0x4140u), kM1024x2, C[r].S, C[r].NA);
+                    a[r][2 * h + 1] = scaled<SAFE>(__byte_perm(v, 0x64646464u, 0x4342u), kM1024x2, C[r].S, C[r].NA);
+                }
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const uint4 xb = lds_v4(x_chunk_addr(xs, rowbytes, g + 8 * mt, cbase + jj));
-                mma_16816(acc[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
-                mma_16816(acc[mt], a0[2], a1[2], a0[3], a1[3], xb.z, xb.w);
+                const uint4 xb = lds_v4(xa + j * 64 + mt * xmt);
+                mma_16816(acc[mt], a[0][0], a[1][0], a[0][1], a[1][1], xb.x, xb.y);
+                mma_16816(acc[mt], a[0][2], a[1][2], a[0][3], a[1][3], xb.z, xb.w);
             }
         }
     } else {  // BITS == 6: two triplets of words, 16 codes each
 #pragma unroll
-        for (int tr = 0; tr < 2; ++tr) {
-            uint32_t a0[8], a1[8];
+        for (int t = 0; t < 2; ++t) {
+            uint32_t a[2][8];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                const uint32_t A = w[r][3 * tr], B = w[r][3 * tr + 1], C = w[r][3 * tr + 2];
-                const uint32_t f[8] = {A, A >> 12, __funnelshift_r(A, B, 24), B >> 4,
-                                       B >> 16, __funnelshift_r(B, C, 28), C >> 8, C >> 20};
-                const uint32_t s2 = r == 0 ? s2_0 : s2_1, b2 = r == 0 ? b2_0 : b2_1;
+                const uint32_t A = w[r][3 * t], B = w[r][3 * t + 1], Cw = w[r][3 * t + 2];
+                // code i sits at bits 6i..6i+5 of the 96-bit triplet.  Each shifted word holds
+                // a pair at (bits 0-5, bits 18-23) -> magic (1024, 256), or at (bits 4-9,
+                // bits 16-21) -> magic (64, 1024).
+                const uint32_t fa[6] = {A, A >> 6, __funnelshift_r(A, B, 12), B >> 4,
+                                        __funnelshift_r(B, Cw, 10), __funnelshift_r(B, Cw, 16)};
+                const uint32_t fb[2] = {Cw >> 4, Cw >> 10};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) (r == 0 ? a0 : a1)[j] = dq6_field(f[j], s2, b2);
+                for (int i = 0; i < 6; ++i)
+                    a[r][i] = scaled<SAFE>((fa[i] & 0x00FC003Fu) | kM1024_256, kM1024_256, C[r].S, C[r].NA);
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    a[r][6 + i] = scaled<SAFE>((fb[i] & 0x003F03F0u) | kM64_1024, kM64_1024, C[r].S, C[r].NB);
             }
 #pragma unroll
-            for (int jc = 0; jc < 2; ++jc) {
+            for (int h = 0; h < 2; ++h) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
-                    const uint4 xb =
-                        lds_v4(x_chunk_addr(xs, rowbytes, g + 8 * mt, cbase + 2 * tr + jc));
-                    mma_16816(acc[mt], a0[4 * jc], a1[4 * jc], a0[4 * jc + 1], a1[4 * jc + 1],
-                              xb.x, xb.y);
-                    mma_16816(acc[mt], a0[4 * jc + 2], a1[4 * jc + 2], a0[4 * jc + 3],
-                              a1[4 * jc + 3], xb.z, xb.w);
+                    const uint4 xb = lds_v4(xa + (2 * t + h) * 64 + mt * xmt);
+                    mma_16816(acc[mt], a[0][4 * h], a[1][4 * h], a[0][4 * h + 1], a[1][4 * h + 1], xb.x, xb.y);
+                    mma_16816(acc[mt], a[0][4 * h + 2], a[1][4 * h + 2], a[0][4 * h + 3], a[1][4 * h + 3], xb.z, xb.w);
                 }
             }
         }
@@ -195,27 +215,94 @@ __device__ __forceinline__ void compute_step(const uint32_t (&w)[2][Fmt<BITS>::N
 }
 
 // ---------------------------------------------------------------- x staging
-// Stage x[0:8*MT, kc : kc + xchunk) as fp16 (zero outside [0,M) x [kc, kend)).
-template <int MT, int NTHREADS>
-__device__ __forceinline__ void stage_x(const Params& p, uint32_t xs, int kc, int kend,
+// Position, within the lane's staged K-span, of each code of a staging unit: the MMA pair
+// order of compute_step.  4-bit: word pairs (i, i+4); 6-bit: the triplet pairs
+// (0,3) (1,4) (2,5) (6,9) (7,10) (8,11) (12,14) (13,15); 8-bit: natural order.
+template <int BITS>
+__host__ __device__ constexpr int perm_src(int i) {
+    if (BITS == 4) return (i & 1) ? 4 + (i >> 1) : (i >> 1);  // 0 4 1 5 2 6 3 7
+    if (BITS == 6) {
+        constexpr int t[16] = {0, 3, 1, 4, 2, 5, 6, 9, 7, 10, 8, 11, 12, 14, 13, 15};
+        return t[i];
+    }
+    return i;
+}
+
+// Stage x[0:8*MT, kc : kc + xchunk) as fp16 (zero outside [0,M) x [kc, kend)) in the lane
+// layout: row m, step s, lane span c, chunk j at 16-byte chunk m*RS + s*(KS/8) + 4j + c
+// (RS = xchunk/8 + XPAD), codes in pair order.  Also the per-group sums X of the same
+// (scaled) values, times 2^-7 so any group of fp16 values stays finite, as fp16 (hi, lo)
+// with X*2^-7 = hi + lo to about 2^-22 relative: xg[m*gpad + group] = (hi, lo).
+template <int BITS, int MT, int NTHREADS>
+__device__ __forceinline__ void stage_x(const Params& p, uint32_t xs, uint32_t xg, int kc, int kend,
                                         float xscale) {
-    const int cpr = p.xchunk >> 3;  // 16-byte chunks per row
-    const int rowbytes = p.xchunk * 2;
-    const int total = 8 * MT * cpr;
-    for (int u = threadIdx.x; u < total; u += NTHREADS) {
-        const int m = u / cpr, c = u - m * cpr;
-        const int k = kc + 8 * c;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    using F = Fmt<BITS>;
+    constexpr int UN = F::UN, KS = 4 * F::U, UPS = KS / UN;  // units per step
+    constexpr int UPL = F::U / UN;                            // units per lane span
+    const int upr = p.xchunk / UN;                            // units per row
+    const int total = 8 * MT * upr;                           // a multiple of 32
+    const int RS = p.xchunk / 8 + XPAD;
+    const int upg = p.group / UN;                             // units per group
+    for (int u0 = 0; u0 < total; u0 += NTHREADS) {
+        const int u = u0 + int(threadIdx.x);
+        if (u0 + int(threadIdx.x & ~31u) >= total) break;     // whole warps only
+        const int m = u / upr, kk = u - m * upr;
+        const int k = kc + kk * UN;
+        float f[UN];
         if (m < p.M && k < kend) {
-            v = ldg_nc_v4(p.x + int64_t(m) * p.K + k);
-            if (p.is_bf16) {
-                v.x = f32x2_to_f16x2(bf16lo_to_f32(v.x) * xscale, bf16hi_to_f32(v.x) * xscale);
-                v.y = f32x2_to_f16x2(bf16lo_to_f32(v.y) * xscale, bf16hi_to_f32(v.y) * xscale);
-                v.z = f32x2_to_f16x2(bf16lo_to_f32(v.z) * xscale, bf16hi_to_f32(v.z) * xscale);
-                v.w = f32x2_to_f16x2(bf16lo_to_f32(v.w) * xscale, bf16hi_to_f32(v.w) * xscale);
+            const uint16_t* src = p.x + int64_t(m) * p.K + k;
+#pragma unroll
+            for (int h = 0; h < UN / 8; ++h) {
+                const uint4 v = ldg_nc_v4(src + 8 * h);
+                const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (p.is_bf16) {
+                        f[8 * h + 2 * i] = bf16lo_to_f32(r[i]) * xscale;
+                        f[8 * h + 2 * i + 1] = bf16hi_to_f32(r[i]) * xscale;
+                    } else {
+                        const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
+                        f[8 * h + 2 * i] = t.x;
+                        f[8 * h + 2 * i + 1] = t.y;
+                    }
+                }
             }
+        } else {
+#pragma unroll
+            for (int i = 0; i < UN; ++i) f[i] = 0.f;
         }
-        sts_v4(x_chunk_addr(xs, rowbytes, m, c), v);
+        // group sum over the upg consecutive lanes holding one group
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < UN; ++i) sum += f[i];
+        for (int o = 1; o < upg; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if ((kk & (upg - 1)) == 0) {
+            const float X = sum * 0.0078125f;
+            const __half hi = __float2half_rn(X);
+            const __half lo = __float2half_rn(X - __half2float(hi));
+            const uint32_t pk = uint32_t(__half_as_ushort(hi)) | (uint32_t(__half_as_ushort(lo)) << 16);
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(m * p.gpad + kk / upg) * 4u), "r"(pk));
+        }
+        // permuted fp16 chunks
+        const int s = kk / UPS, wu = kk - s * UPS;
+        const int c = wu / UPL, t = wu - c * UPL;
+#pragma unroll
+        for (int h = 0; h < UN / 8; ++h) {
+            const int j = t * (UN / 8) + h;
+            uint4 o;
+            uint32_t* ov = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                ov[i] = f32x2_to_f16x2(f[perm_src<BITS>(8 * h + 2 * i)], f[perm_src<BITS>(8 * h + 2 * i + 1)]);
+            sts_v4(xs + uint32_t(m * RS + s * (KS / 8) + 4 * j + c) * 16u, o);
+        }
+    }
+    // group slots past this pass's groups read as zero
+    const int npg = p.xchunk / p.group;
+    const int extra = p.gpad - npg;
+    for (int e = threadIdx.x; e < 8 * MT * extra; e += NTHREADS) {
+        const int m = e / extra, gi = npg + (e - m * extra);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(m * p.gpad + gi) * 4u), "r"(0u));
     }
 }
 
@@ -246,23 +333,32 @@ __device__ __forceinline__ int bf16_block_exponent(const Params& p, int kb, int 
 }
 
 // ---------------------------------------------------------------- the kernel
+// y[m, n] = sum_k x[m,k] * (s*q + b) is computed as sum_k x[m,k] * RN_fp16(s*q)
+//           + sum_groups b * X[m, group] (X = sum of x over the group), both on the tensor
+// cores with fp32 accumulation.
 template <int BITS, int MT, int NWARP>
 __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int U = Fmt<BITS>::U, NREG = Fmt<BITS>::NREG, KS = 4 * U;
+    using F = Fmt<BITS>;
+    constexpr int U = F::U, NREG = F::NREG, KS = 4 * U;
+    constexpr int WPS = KS * BITS / 32;  // words per row per step
     constexpr int NTHREADS = NWARP * 32;
     constexpr int R = 16 * NWARP;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
+    const int g = lane >> 2, c = lane & 3;
     const int k_begin = blockIdx.y * p.kslice;
     const int k_end = min(p.K, k_begin + p.kslice);
     const int nsteps = (k_end - k_begin + KS - 1) / KS;
     const int rbase = blockIdx.x * R + warp * 16;
     const int r0 = rbase + g, r1 = rbase + g + 8;
-    const bool v0 = r0 < p.N, v1 = r1 < p.N;
-    const int64_t woff0 = int64_t(r0) * p.KW, woff1 = int64_t(r1) * p.KW;
-    const int64_t goff0 = int64_t(r0) * p.G, goff1 = int64_t(r1) * p.G;
+    // rows past N read row N-1 (always valid); their results are never stored
+    const int rr0 = min(r0, p.N - 1), rr1 = min(r1, p.N - 1);
+    const int kl = k_begin + c * U;  // first code of the lane's span at step 0
+    const uint32_t* wp0 = p.packed + int64_t(rr0) * p.KW + (kl * BITS >> 5);
+    const uint32_t* wp1 = p.packed + int64_t(rr1) * p.KW + (kl * BITS >> 5);
+    const uint16_t* sp0 = p.scales + int64_t(rr0) * p.G;
+    const uint16_t* sp1 = p.scales + int64_t(rr1) * p.G;
 
     uint32_t wb[PF][2][NREG];
     uint32_t sb[PF][2];
@@ -270,42 +366,87 @@ __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(cons
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 
+    // A lane span past k_end gets scale 0 (its stale codes then contribute exactly 0).
+    auto load = [&](uint32_t (&w)[2][NREG], uint32_t (&sbits)[2], int step) {
+        const int k = kl + step * KS;
+        if (step < nsteps && k < k_end) {
+            load_codes<BITS>(wp0 + step * WPS, w[0]);
+            load_codes<BITS>(wp1 + step * WPS, w[1]);
+            sbits[0] = ldg_nc_u16(sp0 + (k >> p.gshift));
+            sbits[1] = ldg_nc_u16(sp1 + (k >> p.gshift));
+        } else {
+            sbits[0] = sbits[1] = 0u;
+        }
+    };
+
     // Codes and scales never depend on the previous kernel when the caller says so; then
     // the first PF steps are requested before waiting for it.
     if (!p.static_w) grid_dependency_wait();
 #pragma unroll
-    for (int s = 0; s < PF; ++s) {
-        const int k = k_begin + s * KS + t * U;
-        load_step<BITS>(p, v0, v1, woff0, woff1, goff0, goff1, k, s < nsteps && k < k_end, wb[s],
-                        sb[s]);
-    }
+    for (int s = 0; s < PF; ++s) load(wb[s], sb[s], s);
     if (p.static_w) grid_dependency_wait();
     grid_dependents_launch();
 
     const int E = p.is_bf16 ? bf16_block_exponent<NTHREADS>(p, k_begin, k_end) : 0;
     const float xscale = exp2i(-E);
+    const int RS = p.xchunk / 8 + XPAD;
     const uint32_t xs = smem_addr(smem);
-    const int rowbytes = p.xchunk * 2;
+    const uint32_t xg = xs + uint32_t(8 * MT * RS * 16);
+    const uint32_t xmt = uint32_t(8 * RS * 16);
+    const uint32_t xlane = xs + uint32_t(g * RS + c) * 16u;
 
     int step_base = 0;
     for (int kc = k_begin; kc < k_end; kc += p.xchunk) {
         const int csteps = (min(p.xchunk, k_end - kc) + KS - 1) / KS;
         __syncthreads();
-        stage_x<MT, NTHREADS>(p, xs, kc, k_end, xscale);
+        stage_x<BITS, MT, NTHREADS>(p, xs, xg, kc, k_end, xscale);
         __syncthreads();
         for (int s0 = 0; s0 < csteps; s0 += PF) {
 #pragma unroll
             for (int slot = 0; slot < PF; ++slot) {
                 const int cs = s0 + slot;
                 if (cs < csteps) {
-                    compute_step<BITS, MT>(wb[slot], sb[slot], xs, rowbytes, g,
-                                           (cs * KS + t * U) >> 3, acc);
-                    const int ns = step_base + cs + PF;
-                    const int k = k_begin + ns * KS + t * U;
-                    load_step<BITS>(p, v0, v1, woff0, woff1, goff0, goff1, k,
-                                    ns < nsteps && k < k_end, wb[slot], sb[slot]);
+                    RowConst C[2] = {row_const<BITS>(sb[slot][0]), row_const<BITS>(sb[slot][1])};
+                    const bool big = ((sb[slot][0] & 0x7FFFu) >= 0x5400u) | ((sb[slot][1] & 0x7FFFu) >= 0x5400u);
+                    const uint32_t xa = xlane + uint32_t(cs * KS * 2);
+                    if (__any_sync(0xffffffffu, big))
+                        compute_step<BITS, MT, true>(wb[slot], C, xa, xmt, acc);
+                    else
+                        compute_step<BITS, MT, false>(wb[slot], C, xa, xmt, acc);
+                    load(wb[slot], sb[slot], step_base + cs + PF);
                 }
             }
+        }
+        // bias term of this pass's groups: y += b * X, X = 2^7 * (hi + lo)
+        {
+            const int pg0 = (kc - 0) >> p.gshift;
+            const int npg = (min(p.xchunk, k_end - kc)) >> p.gshift;
+            const uint16_t* bp0 = p.biases + int64_t(rr0) * p.G + pg0;
+            const uint16_t* bp1 = p.biases + int64_t(rr1) * p.G + pg0;
+            float t[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) t[mt][0] = t[mt][1] = t[mt][2] = t[mt][3] = 0.f;
+            for (int gi = 0; gi < npg; gi += 8) {
+                const int ga = gi + c, gb = gi + c + 4;
+                const uint32_t b0a = ga < npg ? ldg_nc_u16(bp0 + ga) : 0u;
+                const uint32_t b1a = ga < npg ? ldg_nc_u16(bp1 + ga) : 0u;
+                const uint32_t b0b = gb < npg ? ldg_nc_u16(bp0 + gb) : 0u;
+                const uint32_t b1b = gb < npg ? ldg_nc_u16(bp1 + gb) : 0u;
+                const uint32_t a0 = __byte_perm(b0a, 0u, 0x1010u), a1 = __byte_perm(b1a, 0u, 0x1010u);
+                const uint32_t a2 = __byte_perm(b0b, 0u, 0x1010u), a3 = __byte_perm(b1b, 0u, 0x1010u);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const uint32_t rowx = xg + uint32_t((g + 8 * mt) * p.gpad) * 4u;
+                    uint32_t xb0, xb1;
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(xb0) : "r"(rowx + uint32_t(ga) * 4u));
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(xb1) : "r"(rowx + uint32_t(gb) * 4u));
+                    mma_16816(t[mt], a0, a1, a2, a3, xb0, xb1);
+                }
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[mt][i] = fmaf(128.f, t[mt][i], acc[mt][i]);
         }
         step_base += csteps;
     }
@@ -317,7 +458,7 @@ __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(cons
         for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int m = 8 * mt + 2 * t + (i & 1);
+                const int m = 8 * mt + 2 * c + (i & 1);
                 const int n = (i < 2) ? r0 : r1;
                 if (m < p.M && n < p.N) {
                     const float v = acc[mt][i] * yscale;
@@ -338,7 +479,7 @@ __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(cons
     for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int col = 8 * mt + 2 * t + (i & 1);
+            const int col = 8 * mt + 2 * c + (i & 1);
             red[col * R + rl + (i < 2 ? 0 : 8)] = acc[mt][i] * yscale;
         }
     }
@@ -400,8 +541,11 @@ int log2_exact(int v) {
 
 }  // namespace
 
+int mma_gpad(const MmaConfig& c) { return (c.xchunk / c.group + 7) / 8 * 8; }
+
 size_t mma_smem_bytes(const MmaConfig& c) {
-    const size_t xbytes = size_t(8 * c.mt) * size_t(c.xchunk) * 2;
+    // staged x rows (with padding) + group sums, or the split-K partials
+    const size_t xbytes = size_t(8 * c.mt) * (size_t(c.xchunk) * 2 + XPAD * 16 + size_t(mma_gpad(c)) * 4);
     const size_t rbytes = c.split > 1 ? size_t(16 * c.warps) * size_t(8 * c.mt) * 4 : 0;
     return xbytes > rbytes ? xbytes : rbytes;
 }
@@ -420,10 +564,12 @@ cudaError_t launch_mma(const QmmArgs& a, const MmaConfig& c, cudaStream_t stream
     p.K = int(a.K);
     p.G = int(a.K / a.group);
     p.KW = int(a.K * a.bits / 32);
+    p.group = a.group;
     p.gshift = log2_exact(a.group);
     p.is_bf16 = a.is_bf16;
     p.kslice = c.kslice;
     p.xchunk = c.xchunk;
+    p.gpad = mma_gpad(c);
     p.split = c.split;
     p.static_w = c.static_weights ? 1 : 0;
 

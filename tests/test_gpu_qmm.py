@@ -84,11 +84,22 @@ def test_empty_m_and_n():
     assert y.shape == (4, 0)
 
 
+def _ulp(v, dtype):
+    """Spacing of the output type at |v| (fp16: 11-bit significand, bf16: 8-bit)."""
+    mant = 10 if dtype == torch.float16 else 7
+    emin = -14 if dtype == torch.float16 else -126
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** emin)))
+    return 2.0 ** (e - mant)
+
+
 @pytest.mark.parametrize("bits,group", [(4, 64), (6, 32), (8, 128)])
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
-def test_one_hot_within_one_ulp(oracle_mod, bits, group, dtype):
-    """x = e_k rows give y[:, n] = dequantized column k; the GPU may differ from
-    RNE_out(d) by at most one unit in the last place of the output dtype."""
+@pytest.mark.parametrize("kernel", ["auto", "mma", "tc"])
+def test_one_hot_reproduces_dequantized_columns(oracle_mod, bits, group, dtype, kernel):
+    """x = e_k rows give y[:, n] = d[n, k] = s*q + b (the oracle's dequantized column).  The
+    kernels round s*q (or s*q + b) to fp16 once, add b exactly in fp32 and round once more
+    to the output type, so |y - d| <= 2^-11 |d - b| + one unit in the last place of the
+    output type at |d| (plus the subnormal and fp32 terms below)."""
     N, K = 256, 512
     w = w_input(N, K, dtype, 3, 1.0 if dtype == torch.float16 else 0.02)
     op, os_, ob = oracle_quantize(oracle_mod, w, bits, group)
@@ -97,17 +108,19 @@ def test_one_hot_within_one_ulp(oracle_mod, bits, group, dtype):
     x = torch.zeros((len(ks), K), dtype=dtype)
     for i, k in enumerate(ks):
         x[i, k] = 1.0
-    y = q.qmm(x.cuda(), P, S, B, bits, group)
+    plan = None if kernel == "auto" else q.make_plan(kernel=q.KERNEL_MMA if kernel == "mma" else q.KERNEL_TC)
+    y = q.qmm(x.cuda(), P, S, B, bits, group, plan=plan)
     torch.cuda.synchronize()
-    ref_bits = oracle_mod.dequantize(op, os_, ob, K, bits, group, dtype == torch.bfloat16)
-    got = u16(y.cpu()).astype(np.int32)
+    d = oracle_mod.dequantize_f32(op, os_, ob, K, bits, group).astype(np.float64)
+    bias = ob.view(np.float16).astype(np.float64)
+    got = y.float().cpu().numpy().astype(np.float64)
     for i, k in enumerate(ks):
-        r = ref_bits[:, k].astype(np.int32)
-        # ordered comparison of same-sign patterns: |bits difference| <= 1 ulp
-        same_sign = (got[i] & 0x8000) == (r & 0x8000)
-        zero = ((got[i] & 0x7FFF) == 0) & ((r & 0x7FFF) == 0)
-        assert np.all(same_sign | zero)
-        assert np.max(np.abs((got[i] & 0x7FFF) - (r & 0x7FFF))) <= 1
+        ref = d[:, k]
+        b = bias[:, k // group]
+        # (2^-25: the fp16 rounding step of a subnormal s*q; 2^-20 |d|: d's own fp32 rounding)
+        bound = 2.0 ** -11 * np.abs(ref - b) + _ulp(ref, dtype) + 2.0 ** -25 + 2.0 ** -20 * np.abs(ref)
+        err = np.abs(got[i] - ref)
+        assert np.all(err <= bound), f"k={k}: max excess {np.max(err - bound)}"
 
 
 def test_bf16_large_activations_do_not_overflow(oracle_mod):
