@@ -25,7 +25,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "qmm.h")
 
 QMM_OK, QMM_ERR_INVALID_ARG, QMM_ERR_UNSUPPORTED, QMM_ERR_CUDA = 0, 1, 2, 3
 QMM_F16, QMM_BF16 = 0, 1
-KERNEL_AUTO, KERNEL_MMA, KERNEL_TC = 0, 1, 2
+KERNEL_AUTO, KERNEL_MMA, KERNEL_TC, KERNEL_STREAM = 0, 1, 2, 3
 PLAN_PDL, PLAN_STATIC_WEIGHTS = 1, 2
 
 

@@ -116,6 +116,7 @@ struct Resolved {
     int kernel;
     MmaConfig mma;
     TcConfig tc;
+    StreamConfig st;
 };
 
 TcConfig tc_config(int64_t M, int64_t N, int64_t K, int bits, int split_req) {
@@ -152,13 +153,23 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
     qmm_plan p;
     memset(&p, 0, sizeof(p));
     if (in) p = *in;
-    if (p.kernel != QMM_KERNEL_AUTO && p.kernel != QMM_KERNEL_MMA && p.kernel != QMM_KERNEL_TC)
+    if (p.kernel != QMM_KERNEL_AUTO && p.kernel != QMM_KERNEL_MMA && p.kernel != QMM_KERNEL_TC &&
+        p.kernel != QMM_KERNEL_STREAM)
         return fail(QMM_ERR_INVALID_ARG, "kernel=%d", p.kernel);
     if (p.split < 0 || p.split > 16) return fail(QMM_ERR_INVALID_ARG, "split=%d (1..16)", p.split);
     if (p.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS))
         return fail(QMM_ERR_INVALID_ARG, "unknown plan flags 0x%x", p.flags);
     const bool tc_ok = tc_supported(M, N, K, bits, group) && aligned(scales, 4) && aligned(biases, 4);
-    if (p.kernel == QMM_KERNEL_AUTO) p.kernel = (tc_ok && prefer_tc(M, N, K)) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
+    const bool st_ok = stream_supported(M, N, K, bits, group) && aligned(scales, 16) && aligned(biases, 16) &&
+                       stream_config(M, N, K, bits, group, p.split).ring >= 2;
+    if (p.kernel == QMM_KERNEL_AUTO) {
+        if (st_ok && M <= 16) p.kernel = QMM_KERNEL_STREAM;
+        else p.kernel = (tc_ok && prefer_tc(M, N, K)) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
+    }
+    if (p.kernel == QMM_KERNEL_STREAM && !st_ok)
+        return fail(QMM_ERR_UNSUPPORTED,
+                    "streaming kernel needs 1 <= M <= 16, K a multiple of 8 groups, a 16-byte "
+                    "multiple of packed bytes per row and 16-byte aligned scales/biases");
     if (p.kernel == QMM_KERNEL_TC && !tc_ok)
         return fail(QMM_ERR_UNSUPPORTED,
                     "tensor-core kernel needs K >= 128, an even number of groups per row, a 16-byte "
@@ -182,6 +193,13 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
         p.warps = c.warps;
         p.split = c.split;
         res.mma = c;
+    } else if (p.kernel == QMM_KERNEL_STREAM) {
+        StreamConfig c = stream_config(M, N, K, bits, group, p.split);
+        c.pdl = pdl;
+        c.static_weights = stat;
+        p.warps = 9;
+        p.split = c.split;
+        res.st = c;
     } else {
         TcConfig c = tc_config(M, N, K, bits, p.split);
         c.pdl = pdl;
@@ -284,7 +302,9 @@ qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
     a.bits = bits;
     a.group = group;
     a.is_bf16 = dtype == QMM_BF16;
-    cudaError_t e = r.kernel == QMM_KERNEL_TC ? launch_tc(a, r.tc, st) : launch_mma(a, r.mma, st);
+    cudaError_t e = r.kernel == QMM_KERNEL_TC       ? launch_tc(a, r.tc, st)
+                    : r.kernel == QMM_KERNEL_STREAM ? launch_stream(a, r.st, st)
+                                                    : launch_mma(a, r.mma, st);
     return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm launch");
 }
 
@@ -346,7 +366,10 @@ qmm_status qmm_device_errors(uint32_t* bits) {
     unsigned v = 0;
     cudaError_t e = tc_read_and_clear_errors(&v);
     if (e != cudaSuccess) return cuda_fail(e, "qmm_device_errors");
-    *bits = v;
+    unsigned w = 0;
+    e = stream_read_and_clear_errors(&w);
+    if (e != cudaSuccess) return cuda_fail(e, "qmm_device_errors");
+    *bits = v | w;
     return QMM_OK;
 }
 

@@ -1,6 +1,7 @@
 // qmm_internal.h -- host-side declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -60,6 +61,26 @@ int tc_ring_for(int bits, int mp);
 int tc_kc(int bits);  // K elements per pipeline stage
 size_t tc_smem_bytes(int bits, int mp, int ring);
 cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream);
+
+// Fully resolved launch configuration of the TMA-fed streaming kernel (qmm_stream.cu).
+struct StreamConfig {
+    int mt;        // 8-token column tiles (1 or 2)
+    int split;     // K slices = cluster size along grid.y
+    int kslice;    // K codes per slice
+    int ring;      // shared-memory stages (0: the shape does not fit this kernel)
+    int grid_x;    // blocks along N (persistent when split == 1)
+    size_t smem;   // dynamic shared memory per block
+    bool pdl;
+    bool static_weights;
+};
+bool stream_supported(int64_t M, int64_t N, int64_t K, int bits, int group);
+StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group, int split_req);
+cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream);
+cudaError_t stream_read_and_clear_errors(unsigned* out);
+
+// 2-D tiled TMA descriptor over a row-major [outer, inner] array (row pitch inner*esize bytes).
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
+                 uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 cudaError_t tc_read_and_clear_errors(unsigned* out);
 int tc_max_active_clusters(int bits, int mp, int ring, int split);
 // Tensor-core path with scratch in a fixed device array (qmm_noalloc).

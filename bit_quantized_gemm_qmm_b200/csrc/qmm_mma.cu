@@ -30,6 +30,7 @@
 #include <cooperative_groups.h>
 
 #include "qmm_common.cuh"
+#include "qmm_dq.cuh"
 #include "qmm_internal.h"
 
 namespace cg = cooperative_groups;
@@ -37,16 +38,8 @@ namespace cg = cooperative_groups;
 namespace qmm_impl {
 namespace {
 
-// Per format: U codes per lane per row per step (one K-span of a lane), NREG 32-bit words
-// holding them, UN codes per staging unit (the block the K permutation acts on).  A step
-// covers KS = 4*U codes of K (the four lanes of a row side by side).
-template <int BITS> struct Fmt;
-template <> struct Fmt<4> { static constexpr int U = 32, NREG = 4, UN = 8; };   // 16 bytes
-template <> struct Fmt<6> { static constexpr int U = 32, NREG = 6, UN = 16; };  // 24 bytes
-template <> struct Fmt<8> { static constexpr int U = 16, NREG = 4, UN = 8; };   // 16 bytes
-
 constexpr int PF = 4;    // steps of codes in flight per lane
-constexpr int XPAD = 4;  // 16-byte chunks of padding after each staged x row
+constexpr int XPAD = kXPad;
 
 struct Params {
     const uint16_t* x;
@@ -67,59 +60,9 @@ struct Params {
     int static_w;
 };
 
-// fp16x2 constants of the code -> value conversion.  A code q placed in mantissa bits
-// [o, o+n) of an fp16 whose exponent makes bit o worth 1 reads as M + q exactly, where
-// M = 2^(10-o): 1024 for o = 0, 256 for o = 2, 64 for o = 4.
-constexpr uint32_t kM1024x2 = 0x64006400u;   // (1024, 1024)
-constexpr uint32_t kM64x2 = 0x54005400u;     // (64, 64)
-constexpr uint32_t kM1024_256 = 0x5C006400u; // (lo 1024, hi 256)
-constexpr uint32_t kM64_1024 = 0x64005400u;  // (lo 64, hi 1024)
-constexpr uint32_t kN1024x2 = 0xE400E400u;   // (-1024, -1024)
-constexpr uint32_t kN64x2 = 0xD400D400u;     // (-64, -64)
-constexpr uint32_t kN1024_256 = 0xDC00E400u; // (lo -1024, hi -256)
-constexpr uint32_t kN64_1024 = 0xE400D400u;  // (lo -64, hi -1024)
-
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-// Per-row constants of one step: S = (s, s) and the offsets -M*s for the two magic layouts
-// the format uses.  All are exact while |s| < 64 (then 1024*s is a finite fp16).
-struct RowConst {
-    uint32_t S, NA, NB;
-};
-
-template <int BITS>
-__device__ __forceinline__ RowConst row_const(uint32_t sbits) {
-    RowConst r;
-    r.S = __byte_perm(sbits, 0u, 0x1010u);
-    if constexpr (BITS == 6) {
-        r.NA = hmul2(r.S, kN1024_256);
-        r.NB = hmul2(r.S, kN64_1024);
-    } else {
-        r.NA = hmul2(r.S, kN1024x2);
-        r.NB = hmul2(r.S, kN64x2);
-    }
-    return r;
-}
-
-// s*q for the two codes held in v = M + q (per half): one rounding of the exact product.
-template <bool SAFE>
-__device__ __forceinline__ uint32_t scaled(uint32_t v, uint32_t magic, uint32_t S, uint32_t N) {
-    if constexpr (SAFE) return hmul2(hsub2(v, magic), S);  // |s| >= 64: -M*s would overflow
-    else return hfma2(v, S, N);                            // s*(M+q) - M*s
-}
-
 // ---------------------------------------------------------------- loads of one step
 template <int BITS>
-__device__ __forceinline__ void load_codes(const uint32_t* wp, uint32_t (&w)[Fmt<BITS>::NREG]) {
+__device__ __forceinline__ void load_codes(const uint32_t* wp, uint32_t (&w)[StepFmt<BITS>::NREG]) {
     if constexpr (BITS == 6) {
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
@@ -130,179 +73,6 @@ __device__ __forceinline__ void load_codes(const uint32_t* wp, uint32_t (&w)[Fmt
     } else {
         const uint4 v = ldg_stream_v4(wp);
         w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    }
-}
-
-// ---------------------------------------------------------------- one step of MMAs
-// w[r]: the lane's U codes of rows g (r=0) and g+8 (r=1); C[r]: their step constants.
-// xa: shared address of the lane's first staged x chunk of this step for token row g;
-// xmt: byte distance between 8-token tiles.  Each MMA takes two code pairs per row; the
-// staged x of the lane's K-span is stored in exactly that pair order.
-template <int BITS, int MT, bool SAFE>
-__device__ __forceinline__ void compute_step(const uint32_t (&w)[2][Fmt<BITS>::NREG],
-                                             const RowConst (&C)[2], uint32_t xa, uint32_t xmt,
-                                             float (&acc)[MT][4]) {
-    if constexpr (BITS == 4) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {  // word j: codes 8j..8j+7, pairs (0,4) (1,5) (2,6) (3,7)
-            uint32_t a[2][4];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const uint32_t v = w[r][j], v8 = v >> 8;
-                a[r][0] = scaled<SAFE>((v & 0x000F000Fu) | kM1024x2, kM1024x2, C[r].S, C[r].NA);
-                a[r][1] = scaled<SAFE>((v & 0x00F000F0u) | kM64x2, kM64x2, C[r].S, C[r].NB);
-                a[r][2] = scaled<SAFE>((v8 & 0x000F000Fu) | kM1024x2, kM1024x2, C[r].S, C[r].NA);
-                a[r][3] = scaled<SAFE>((v8 & 0x00F000F0u) | kM64x2, kM64x2, C[r].S, C[r].NB);
-            }
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const uint4 xb = lds_v4(xa + j * 64 + mt * xmt);
-                mma_16816(acc[mt], a[0][0], a[1][0], a[0][1], a[1][1], xb.x, xb.y);
-                mma_16816(acc[mt], a[0][2], a[1][2], a[0][3], a[1][3], xb.z, xb.w);
-            }
-        }
-    } else if constexpr (BITS == 8) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {  // words 2j, 2j+1: codes 8j..8j+7 in natural pairs
-            uint32_t a[2][4];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t v = w[r][2 * j + h];
-                    a[r][2 * h] = scaled<SAFE>(__byte_perm(v, 0x64646464u, 0x4140u), kM1024x2, C[r].S, C[r].NA);
-                    a[r][2 * h + 1] = scaled<SAFE>(__byte_perm(v, 0x64646464u, 0x4342u), kM1024x2, C[r].S, C[r].NA);
-                }
-            }
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const uint4 xb = lds_v4(xa + j * 64 + mt * xmt);
-                mma_16816(acc[mt], a[0][0], a[1][0], a[0][1], a[1][1], xb.x, xb.y);
-                mma_16816(acc[mt], a[0][2], a[1][2], a[0][3], a[1][3], xb.z, xb.w);
-            }
-        }
-    } else {  // BITS == 6: two triplets of words, 16 codes each
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            uint32_t a[2][8];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const uint32_t A = w[r][3 * t], B = w[r][3 * t + 1], Cw = w[r][3 * t + 2];
-                // code i sits at bits 6i..6i+5 of the 96-bit triplet.  Each shifted word holds
-                // a pair at (bits 0-5, bits 18-23) -> magic (1024, 256), or at (bits 4-9,
-                // bits 16-21) -> magic (64, 1024).
-                const uint32_t fa[6] = {A, A >> 6, __funnelshift_r(A, B, 12), B >> 4,
-                                        __funnelshift_r(B, Cw, 10), __funnelshift_r(B, Cw, 16)};
-                const uint32_t fb[2] = {Cw >> 4, Cw >> 10};
-#pragma unroll
-                for (int i = 0; i < 6; ++i)
-                    a[r][i] = scaled<SAFE>((fa[i] & 0x00FC003Fu) | kM1024_256, kM1024_256, C[r].S, C[r].NA);
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-                    a[r][6 + i] = scaled<SAFE>((fb[i] & 0x003F03F0u) | kM64_1024, kM64_1024, C[r].S, C[r].NB);
-            }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const uint4 xb = lds_v4(xa + (2 * t + h) * 64 + mt * xmt);
-                    mma_16816(acc[mt], a[0][4 * h], a[1][4 * h], a[0][4 * h + 1], a[1][4 * h + 1], xb.x, xb.y);
-                    mma_16816(acc[mt], a[0][4 * h + 2], a[1][4 * h + 2], a[0][4 * h + 3], a[1][4 * h + 3], xb.z, xb.w);
-                }
-            }
-        }
-    }
-}
-
-// ---------------------------------------------------------------- x staging
-// Position, within the lane's staged K-span, of each code of a staging unit: the MMA pair
-// order of compute_step.  4-bit: word pairs (i, i+4); 6-bit: the triplet pairs
-// (0,3) (1,4) (2,5) (6,9) (7,10) (8,11) (12,14) (13,15); 8-bit: natural order.
-template <int BITS>
-__host__ __device__ constexpr int perm_src(int i) {
-    if (BITS == 4) return (i & 1) ? 4 + (i >> 1) : (i >> 1);  // 0 4 1 5 2 6 3 7
-    if (BITS == 6) {
-        constexpr int t[16] = {0, 3, 1, 4, 2, 5, 6, 9, 7, 10, 8, 11, 12, 14, 13, 15};
-        return t[i];
-    }
-    return i;
-}
-
-// Stage x[0:8*MT, kc : kc + xchunk) as fp16 (zero outside [0,M) x [kc, kend)) in the lane
-// layout: row m, step s, lane span c, chunk j at 16-byte chunk m*RS + s*(KS/8) + 4j + c
-// (RS = xchunk/8 + XPAD), codes in pair order.  Also the per-group sums X of the same
-// (scaled) values, times 2^-7 so any group of fp16 values stays finite, as fp16 (hi, lo)
-// with X*2^-7 = hi + lo to about 2^-22 relative: xg[m*gpad + group] = (hi, lo).
-template <int BITS, int MT, int NTHREADS>
-__device__ __forceinline__ void stage_x(const Params& p, uint32_t xs, uint32_t xg, int kc, int kend,
-                                        float xscale) {
-    using F = Fmt<BITS>;
-    constexpr int UN = F::UN, KS = 4 * F::U, UPS = KS / UN;  // units per step
-    constexpr int UPL = F::U / UN;                            // units per lane span
-    const int upr = p.xchunk / UN;                            // units per row
-    const int total = 8 * MT * upr;                           // a multiple of 32
-    const int RS = p.xchunk / 8 + XPAD;
-    const int upg = p.group / UN;                             // units per group
-    for (int u0 = 0; u0 < total; u0 += NTHREADS) {
-        const int u = u0 + int(threadIdx.x);
-        if (u0 + int(threadIdx.x & ~31u) >= total) break;     // whole warps only
-        const int m = u / upr, kk = u - m * upr;
-        const int k = kc + kk * UN;
-        float f[UN];
-        if (m < p.M && k < kend) {
-            const uint16_t* src = p.x + int64_t(m) * p.K + k;
-#pragma unroll
-            for (int h = 0; h < UN / 8; ++h) {
-                const uint4 v = ldg_nc_v4(src + 8 * h);
-                const uint32_t r[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if (p.is_bf16) {
-                        f[8 * h + 2 * i] = bf16lo_to_f32(r[i]) * xscale;
-                        f[8 * h + 2 * i + 1] = bf16hi_to_f32(r[i]) * xscale;
-                    } else {
-                        const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
-                        f[8 * h + 2 * i] = t.x;
-                        f[8 * h + 2 * i + 1] = t.y;
-                    }
-                }
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < UN; ++i) f[i] = 0.f;
-        }
-        // group sum over the upg consecutive lanes holding one group
-        float sum = 0.f;
-#pragma unroll
-        for (int i = 0; i < UN; ++i) sum += f[i];
-        for (int o = 1; o < upg; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if ((kk & (upg - 1)) == 0) {
-            const float X = sum * 0.0078125f;
-            const __half hi = __float2half_rn(X);
-            const __half lo = __float2half_rn(X - __half2float(hi));
-            const uint32_t pk = uint32_t(__half_as_ushort(hi)) | (uint32_t(__half_as_ushort(lo)) << 16);
-            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(m * p.gpad + kk / upg) * 4u), "r"(pk));
-        }
-        // permuted fp16 chunks
-        const int s = kk / UPS, wu = kk - s * UPS;
-        const int c = wu / UPL, t = wu - c * UPL;
-#pragma unroll
-        for (int h = 0; h < UN / 8; ++h) {
-            const int j = t * (UN / 8) + h;
-            uint4 o;
-            uint32_t* ov = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                ov[i] = f32x2_to_f16x2(f[perm_src<BITS>(8 * h + 2 * i)], f[perm_src<BITS>(8 * h + 2 * i + 1)]);
-            sts_v4(xs + uint32_t(m * RS + s * (KS / 8) + 4 * j + c) * 16u, o);
-        }
-    }
-    // group slots past this pass's groups read as zero
-    const int npg = p.xchunk / p.group;
-    const int extra = p.gpad - npg;
-    for (int e = threadIdx.x; e < 8 * MT * extra; e += NTHREADS) {
-        const int m = e / extra, gi = npg + (e - m * extra);
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(m * p.gpad + gi) * 4u), "r"(0u));
     }
 }
 
@@ -339,8 +109,8 @@ __device__ __forceinline__ int bf16_block_exponent(const Params& p, int kb, int 
 template <int BITS, int MT, int NWARP>
 __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(const Params p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    using F = Fmt<BITS>;
-    constexpr int U = F::U, NREG = F::NREG, KS = 4 * U;
+    using F = StepFmt<BITS>;
+    constexpr int U = F::U, NREG = F::NREG, KS = F::KS;
     constexpr int WPS = KS * BITS / 32;  // words per row per step
     constexpr int NTHREADS = NWARP * 32;
     constexpr int R = 16 * NWARP;
@@ -399,7 +169,8 @@ __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(cons
     for (int kc = k_begin; kc < k_end; kc += p.xchunk) {
         const int csteps = (min(p.xchunk, k_end - kc) + KS - 1) / KS;
         __syncthreads();
-        stage_x<BITS, MT, NTHREADS>(p, xs, xg, kc, k_end, xscale);
+        stage_x_tile<BITS, MT>(p.x, p.M, p.K, p.is_bf16, p.group, p.xchunk, p.gpad, NTHREADS, xs, xg, kc, k_end,
+                               xscale);
         __syncthreads();
         for (int s0 = 0; s0 < csteps; s0 += PF) {
 #pragma unroll
@@ -410,9 +181,9 @@ __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(cons
                     const bool big = ((sb[slot][0] & 0x7FFFu) >= 0x5400u) | ((sb[slot][1] & 0x7FFFu) >= 0x5400u);
                     const uint32_t xa = xlane + uint32_t(cs * KS * 2);
                     if (__any_sync(0xffffffffu, big))
-                        compute_step<BITS, MT, true>(wb[slot], C, xa, xmt, acc);
+                        step_mma<BITS, MT, true>(wb[slot], C, xa, xmt, acc);
                     else
-                        compute_step<BITS, MT, false>(wb[slot], C, xa, xmt, acc);
+                        step_mma<BITS, MT, false>(wb[slot], C, xa, xmt, acc);
                     load(wb[slot], sb[slot], step_base + cs + PF);
                 }
             }
@@ -432,16 +203,7 @@ __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(cons
                 const uint32_t b1a = ga < npg ? ldg_nc_u16(bp1 + ga) : 0u;
                 const uint32_t b0b = gb < npg ? ldg_nc_u16(bp0 + gb) : 0u;
                 const uint32_t b1b = gb < npg ? ldg_nc_u16(bp1 + gb) : 0u;
-                const uint32_t a0 = __byte_perm(b0a, 0u, 0x1010u), a1 = __byte_perm(b1a, 0u, 0x1010u);
-                const uint32_t a2 = __byte_perm(b0b, 0u, 0x1010u), a3 = __byte_perm(b1b, 0u, 0x1010u);
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const uint32_t rowx = xg + uint32_t((g + 8 * mt) * p.gpad) * 4u;
-                    uint32_t xb0, xb1;
-                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(xb0) : "r"(rowx + uint32_t(ga) * 4u));
-                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(xb1) : "r"(rowx + uint32_t(gb) * 4u));
-                    mma_16816(t[mt], a0, a1, a2, a3, xb0, xb1);
-                }
+                bias_mma<MT>(b0a, b1a, b0b, b1b, xg + uint32_t(g * p.gpad + gi) * 4u, uint32_t(8 * p.gpad * 4), c, t);
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)

@@ -1,0 +1,544 @@
+// qmm_stream.cu -- small-M quantized matmul with TMA-staged weights (sm_100a).
+//
+// y[m,n] = sum_k x[m,k] * (s[n,k/g] * q[n,k] + b[n,k/g])      (MLX issue #4720, "To Reproduce":
+// quantized_matmul(x, *w, transpose=True); formats from "What Are NAX Verify Kernels ...",
+// "Supported Data Formats and Quantization Schemes").
+//
+// At M <= 16 the matmul streams the packed weights once and does little arithmetic per byte,
+// so the kernel is built around keeping HBM busy.  The warp-tile kernel (qmm_mma.cu) holds
+// its codes in flight in registers, which caps the warps per SM and with them the bytes in
+// flight; here the tensor memory accelerator (TMA) moves the codes into a shared-memory ring
+// and the warps only compute:
+//   * one producer thread issues, per 128-row tile, one TMA box of scales and one of biases
+//     (double-buffered per tile) and, per K stage, one box of packed codes (128 rows x 128 B,
+//     192 B for 6-bit), each completing on an mbarrier; the ring runs across tiles, so a
+//     persistent block streams without gaps;
+//   * eight consumer warps own 16 rows each.  Per stage a lane reads its 64 codes (32 for
+//     8-bit) of two rows from shared memory, dequantizes them in registers to A = RN_fp16(s q)
+//     (qmm_dq.cuh) and runs mma.sync m16n8k16 against x held in shared memory for the whole
+//     K range of the block, staged once in the matching pair order.  The bias enters as b
+//     times the group sum of x, one more MMA per eight groups at the end of the tile;
+//   * K is split across the blocks of a cluster when there are too few tiles to fill the
+//     GPU; partial sums are added over distributed shared memory in rank order, so results
+//     are deterministic.
+// Every wait is bounded; a wait that runs out sets an error bit (qmm_device_errors), makes the
+// block stop issuing and leave once its copies in flight have landed.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "qmm_common.cuh"
+#include "qmm_dq.cuh"
+#include "qmm_internal.h"
+#include "sm100.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace qmm_impl {
+
+__device__ unsigned int g_stream_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int ST_ROWS = 128;                  // weight rows per tile
+constexpr int ST_CW = 16;                     // consumer warps: 8 row groups x 2 K halves
+constexpr int ST_THREADS = (ST_CW + 1) * 32;  // + the producer warp
+constexpr int ST_SS = 4;                      // scale / bias boxes in flight
+constexpr long long ST_TIMEOUT = 4000000000LL;  // cycles (about 2 s)
+
+// A stage is 128 rows x KS codes (two steps of StepFmt, one per K half): 128 bytes a row
+// (192 for 6-bit).  Scales and biases arrive per block of 8 groups (8 x 2 bytes a row).
+template <int BITS>
+__host__ __device__ constexpr int stage_codes() { return 2 * StepFmt<BITS>::KS; }
+
+struct StParams {
+    const uint16_t* x;
+    uint16_t* y;
+    int M, N, K;
+    int group, gshift;
+    int is_bf16;
+    int T;        // 128-row tiles
+    int kslice;   // K codes per split (a multiple of the stage and of 8 groups)
+    int split;
+    int ring;     // stages in the shared-memory ring
+    int static_w;
+};
+
+struct StLayout {
+    uint32_t w_stage, sb_off, x_off, xrs, xg_off, gpad, xf_off, red_off, bar_off, total;
+};
+
+constexpr uint32_t kSbSlot = 2 * ST_ROWS * 8 * 2;  // one scale box + one bias box (4 KB)
+
+__host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split) {
+    StLayout L;
+    L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 128));  // 16 or 24 KB
+    L.sb_off = uint32_t(ring) * L.w_stage;
+    uint32_t off = L.sb_off + ST_SS * kSbSlot;
+    L.x_off = off;
+    L.xrs = uint32_t(kslice / 8 + kXPad);                     // 16-byte chunks per staged x row
+    off += uint32_t(8 * mt) * L.xrs * 16;
+    L.xg_off = off;
+    L.gpad = uint32_t((kslice / group + 7) / 8 * 8);
+    off += uint32_t(8 * mt) * L.gpad * 4;
+    L.xf_off = off;                                           // K-half partials: [8 warps][32][4*MT]
+    off += uint32_t(8 * 32 * 4 * mt * 4);
+    L.red_off = off;
+    if (split > 1) off += uint32_t(ST_ROWS * 8 * mt * 4);
+    off = (off + 15) & ~15u;
+    L.bar_off = off;
+    off += 8 * uint32_t(2 * ring + 2 * ST_SS + 16) + 16;
+    L.total = off;
+    return L;
+}
+
+__device__ __forceinline__ void set_error(unsigned bit) { atomicOr(&g_stream_error, bit); }
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+
+// Bounded mbarrier wait that gives up at once when the block is aborting, so that after a
+// timeout every warp runs through the rest of its loop without waiting (no warp is left
+// behind at a barrier).  A timeout sets the error bit and the block's abort flag.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, long long dl, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    while (true) {
+        if (*abort_flag) return false;
+        if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+        if (clock64() > dl) {
+            set_error(1u);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+
+// Exponent E >= 0 such that max|x| * 2^-E < 2^15 over x[:, kb:ke] (bf16 activations only).
+__device__ __forceinline__ int bf16_exponent(const StParams& p, int kb, int ke, float* red) {
+    const int cpr = (ke - kb) >> 3;
+    float amax = 0.f;
+    for (int u = threadIdx.x; u < p.M * cpr; u += ST_CW * 32) {
+        const int m = u / cpr, c = u - m * cpr;
+        const uint4 v = ldg_nc_v4(p.x + int64_t(m) * p.K + kb + 8 * c);
+        const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            amax = fmaxf(amax, fmaxf(fabsf(bf16lo_to_f32(r[i])), fabsf(bf16hi_to_f32(r[i]))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    consumer_sync();
+    float a = red[0];
+#pragma unroll
+    for (int i = 1; i < ST_CW; ++i) a = fmaxf(a, red[i]);
+    const int eb = int(__float_as_uint(a) >> 23) & 0xFF;  // a < 2^(eb-126)
+    return eb > 141 ? eb - 141 : 0;
+}
+
+template <int BITS, int MT>
+__global__ void __launch_bounds__(ST_THREADS, 1)
+    qmm_stream_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
+                      const __grid_constant__ CUtensorMap bmap, const StParams p) {
+    using F = StepFmt<BITS>;
+    constexpr int KSS = F::KS;                 // codes per step (one K half of a stage)
+    constexpr int KS = stage_codes<BITS>();    // codes per stage
+    constexpr int NREG = F::NREG, U = F::U;
+    constexpr int WPS = KS * BITS / 32;        // 32-bit words per row per stage
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ float s_red[ST_CW];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const StLayout L = st_layout(BITS, MT, p.ring, p.kslice, p.group, p.split);
+    const int S = p.ring;
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t bar_full = sbase + L.bar_off;
+    const uint32_t bar_empty = bar_full + 8 * S;
+    const uint32_t bar_sfull = bar_empty + 8 * S;       // [ST_SS]
+    const uint32_t bar_sempty = bar_sfull + 8 * ST_SS;  // [ST_SS]
+    const uint32_t bar_xfull = bar_sempty + 8 * ST_SS;  // [8]: K-half partials written
+    const uint32_t bar_xempty = bar_xfull + 8 * 8;      // [8]: ... and read
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bar_off + 8 * (2 * S + 2 * ST_SS + 16));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kb = blockIdx.y * p.kslice;
+    const int ke = min(p.K, kb + p.kslice);
+    const int nst = (ke - kb + KS - 1) / KS;
+    const int spb = (8 * p.group) / KS;         // stages per block of 8 groups (1..8)
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(bar_full + 8 * i, 1);
+            mbar_init(bar_empty + 8 * i, ST_CW);
+        }
+        for (int i = 0; i < ST_SS; ++i) {
+            mbar_init(bar_sfull + 8 * i, 1);
+            mbar_init(bar_sempty + 8 * i, ST_CW);
+        }
+        for (int i = 0; i < 8; ++i) {
+            mbar_init(bar_xfull + 8 * i, 1);
+            mbar_init(bar_xempty + 8 * i, 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x == 32 * ST_CW) {
+        prefetch_tensormap(&wmap);
+        prefetch_tensormap(&smap);
+        prefetch_tensormap(&bmap);
+    }
+    __syncthreads();
+
+    if (warp == ST_CW) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            if (!p.static_w) grid_dependency_wait();
+            const int wcol0 = kb / 32 * BITS;  // kb * BITS / 32 (kb is a multiple of 256)
+            const int gcol0 = kb >> p.gshift;  // a multiple of 8
+            int it = 0, blk = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.T && ok; t += gridDim.x) {
+                const long long dl = clock64() + ST_TIMEOUT;
+                for (int st = 0; st < nst; ++st, ++it) {
+                    if (st % spb == 0) {  // scales and biases of the next 8 groups
+                        const int ss = blk % ST_SS;
+                        if (blk >= ST_SS && !wait_or_abort(bar_sempty + 8 * ss, ((blk / ST_SS) & 1) ^ 1, dl, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t dst = sbase + L.sb_off + ss * kSbSlot;
+                        mbar_arrive_expect_tx(bar_sfull + 8 * ss, kSbSlot);
+                        tma_load_2d(dst, &smap, bar_sfull + 8 * ss, gcol0 + 8 * (st / spb), t * ST_ROWS);
+                        tma_load_2d(dst + kSbSlot / 2, &bmap, bar_sfull + 8 * ss, gcol0 + 8 * (st / spb), t * ST_ROWS);
+                        ++blk;
+                    }
+                    const int s = it % S;
+                    if ((it >= S && !wait_or_abort(bar_empty + 8 * s, ((it / S) & 1) ^ 1, dl, abort_flag)) || *abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar_full + 8 * s, L.w_stage);
+                    tma_load_2d(sbase + s * L.w_stage, &wmap, bar_full + 8 * s, wcol0 + st * WPS, t * ST_ROWS);
+                }
+            }
+            // nothing may still be landing in shared memory when the block exits
+            const long long dl = clock64() + ST_TIMEOUT;
+            for (int i = max(0, it - S); i < it; ++i)
+                if (!mbar_wait(bar_full + 8 * (i % S), (i / S) & 1, dl)) set_error(2u);
+            for (int i = max(0, blk - ST_SS); i < blk; ++i)
+                if (!mbar_wait(bar_sfull + 8 * (i % ST_SS), (i / ST_SS) & 1, dl)) set_error(2u);
+        }
+    } else {
+        // ------------------------------------------------------------ consumers
+        const int g = lane >> 2, c = lane & 3;
+        const int half = warp >> 3;                        // K half of each stage
+        const int rg = warp & 7;                           // 16-row group of the tile
+        const int rA = rg * 16 + ((g >> 1) | ((g & 1) << 2));  // rows of "g" and "g + 8": the
+        const int rB = rA + 8;                             // permutation keeps the code reads conflict-free
+        grid_dependency_wait();
+        const int E = p.is_bf16 ? bf16_exponent(p, kb, ke, s_red) : 0;
+        const uint32_t xs = sbase + L.x_off, xg = sbase + L.xg_off;
+        stage_x_tile<BITS, MT>(p.x, p.M, p.K, p.is_bf16, p.group, p.kslice, int(L.gpad), ST_CW * 32, xs, xg, kb, ke,
+                               exp2i(-E));
+        consumer_sync();
+        grid_dependents_launch();
+
+        const uint32_t xmt = 8 * L.xrs * 16;
+        const uint32_t xlane = xs + uint32_t(g * int(L.xrs) + c) * 16u + uint32_t(half * KSS * 2);
+        const uint32_t xgrow = xg + uint32_t(g * int(L.gpad)) * 4u;
+        const uint32_t xg_mt = 8 * L.gpad * 4;
+        float* xf = reinterpret_cast<float*>(smem + L.xf_off) + (rg * 32 + lane) * 4 * MT;
+        const float yscale = exp2i(E);
+        int it = 0, blk = 0, tc = 0;
+        for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++tc) {
+            // After a timeout (abort flag set) every wait below returns at once and the work
+            // is skipped, so all warps leave the loop together.
+            const long long dl = clock64() + ST_TIMEOUT;
+            float acc[MT][4], tb[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[mt][i] = tb[mt][i] = 0.f;
+            uint32_t sbuf = 0;
+            bool sok = true;
+            for (int st = 0; st < nst; ++st, ++it) {
+                const int ss = blk % ST_SS;
+                if (st % spb == 0) {
+                    sok = wait_or_abort(bar_sfull + 8 * ss, (blk / ST_SS) & 1, dl, abort_flag);
+                    sbuf = sbase + L.sb_off + ss * kSbSlot;
+                }
+                const int s = it % S;
+                const bool ok = sok && wait_or_abort(bar_full + 8 * s, (it / S) & 1, dl, abort_flag);
+                if (ok) {
+                    uint32_t w[2][NREG];
+                    const uint32_t stage = sbase + s * L.w_stage;
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int row = r == 0 ? rA : rB;
+                        if constexpr (BITS == 6) {
+#pragma unroll
+                            for (int i = 0; i < 3; ++i) {
+                                const uint2 v = lds_v2(stage + row * 192 + half * 96 + 24 * c + 8 * i);
+                                w[r][2 * i] = v.x;
+                                w[r][2 * i + 1] = v.y;
+                            }
+                        } else {  // 128-byte swizzle: 16-byte chunk ^= row & 7
+                            const uint4 v = lds_v4(stage + row * 128 + ((((4 * half + c) ^ row) & 7) << 4));
+                            w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
+                        }
+                    }
+                    // the group of the lane's span within the current block of 8 groups
+                    const int gl = ((st * KS + half * KSS + c * U) >> p.gshift) & 7;
+                    const uint32_t s0 = lds_u16(sbuf + uint32_t(rA * 8 + gl) * 2u);
+                    const uint32_t s1 = lds_u16(sbuf + uint32_t(rB * 8 + gl) * 2u);
+                    const RowConst C[2] = {row_const<BITS>(s0), row_const<BITS>(s1)};
+                    const bool big = ((s0 & 0x7FFFu) >= 0x5400u) | ((s1 & 0x7FFFu) >= 0x5400u);
+                    const uint32_t xa = xlane + uint32_t(st * KS * 2);
+                    if (__any_sync(0xffffffffu, big))
+                        step_mma<BITS, MT, true>(w, C, xa, xmt, acc);
+                    else
+                        step_mma<BITS, MT, false>(w, C, xa, xmt, acc);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+                }
+                if (st % spb == spb - 1) {
+                    if (sok && half == 0) {  // bias term of the block's 8 groups: y += b * X
+                        const uint32_t bb = sbuf + kSbSlot / 2;
+                        bias_mma<MT>(lds_u16(bb + uint32_t(rA * 8 + c) * 2u), lds_u16(bb + uint32_t(rB * 8 + c) * 2u),
+                                     lds_u16(bb + uint32_t(rA * 8 + c + 4) * 2u),
+                                     lds_u16(bb + uint32_t(rB * 8 + c + 4) * 2u), xgrow + uint32_t(st / spb) * 32u,
+                                     xg_mt, c, tb);
+                    }
+                    __syncwarp();
+                    if (sok && lane == 0) mbar_arrive(bar_sempty + 8 * ss);
+                    ++blk;
+                }
+            }
+            // the two K halves meet: half 1 hands its partial sums to half 0 (mbarrier handshake)
+            if (half == 1) {
+                if (tc == 0 || wait_or_abort(bar_xempty + 8 * rg, ((tc - 1) & 1), dl, abort_flag)) {
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) xf[4 * mt + i] = acc[mt][i];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_xfull + 8 * rg);
+                }
+            } else if (wait_or_abort(bar_xfull + 8 * rg, tc & 1, dl, abort_flag)) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        acc[mt][i] = (acc[mt][i] + xf[4 * mt + i] + 128.f * tb[mt][i]) * yscale;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_xempty + 8 * rg);
+                if (p.split == 1) {
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int m = 8 * mt + 2 * c + (i & 1);
+                            const int n = t * ST_ROWS + (i < 2 ? rA : rB);
+                            if (m < p.M && n < p.N)
+                                p.y[int64_t(m) * p.N + n] = p.is_bf16
+                                                                ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][i]))
+                                                                : __half_as_ushort(__float2half_rn(acc[mt][i]));
+                        }
+                } else {
+                    // one tile per block when K is split: partials [8*MT cols][128 rows]
+                    float* red = reinterpret_cast<float*>(smem + L.red_off);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            red[(8 * mt + 2 * c + (i & 1)) * ST_ROWS + (i < 2 ? rA : rB)] = acc[mt][i];
+                }
+            }
+        }
+    }
+
+    if (p.split > 1) {
+        // K split over the cluster (grid.x == T: one tile per block): block `rank` sums a slice
+        // of the tile's rows over ranks 0..split-1 in order.
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        const int t = blockIdx.x;
+        const int rank = int(cluster.block_rank());
+        const int rows_per = (ST_ROWS + p.split - 1) / p.split;
+        const int rlo = rank * rows_per, rhi = min(ST_ROWS, rlo + rows_per);
+        const int nrows = max(0, rhi - rlo);
+        const int ncols = min(8 * MT, p.M);
+        float* red = reinterpret_cast<float*>(smem + L.red_off);
+        const bool ok = *abort_flag == 0;
+        for (int e = threadIdx.x; e < nrows * ncols; e += ST_THREADS) {
+            const int col = e / nrows, row = rlo + (e - col * nrows);
+            const int n = t * ST_ROWS + row;
+            float sum = 0.f;
+            for (int q = 0; q < p.split; ++q) sum += cluster.map_shared_rank(red, q)[col * ST_ROWS + row];
+            if (n < p.N && ok)
+                p.y[int64_t(col) * p.N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sum))
+                                                        : __half_as_ushort(__float2half_rn(sum));
+        }
+        cluster.sync();
+    }
+}
+
+using StKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const StParams);
+
+StKernelFn pick_stream(int bits, int mt) {
+    if (bits == 4) return mt == 1 ? qmm_stream_kernel<4, 1> : mt == 2 ? qmm_stream_kernel<4, 2> : nullptr;
+    if (bits == 6) return mt == 1 ? qmm_stream_kernel<6, 1> : mt == 2 ? qmm_stream_kernel<6, 2> : nullptr;
+    if (bits == 8) return mt == 1 ? qmm_stream_kernel<8, 1> : mt == 2 ? qmm_stream_kernel<8, 2> : nullptr;
+    return nullptr;
+}
+
+int ks_for(int bits) { return bits == 8 ? 128 : 256; }
+int ilog2(int v) {
+    int s = 0;
+    while ((1 << s) < v) ++s;
+    return s;
+}
+int cdiv(int64_t a, int64_t b) { return int((a + b - 1) / b); }
+int rup(int64_t a, int64_t b) { return int((a + b - 1) / b * b); }
+
+constexpr int kNumSM = 148;
+constexpr size_t kMaxSmem = 226 * 1024;  // dynamic, per block (static shared memory is tiny)
+constexpr size_t kSmSmem = 228 * 1024;   // per SM (including 1 KB reserved per block)
+
+size_t st_smem(int bits, int mt, int ring, int kslice, int group, int split) {
+    return size_t(st_layout(bits, mt, ring, kslice, group, split).total) + 1024;  // + alignment slack
+}
+
+}  // namespace
+
+bool stream_supported(int64_t M, int64_t N, int64_t K, int bits, int group) {
+    if (M < 1 || M > 16 || N < 1) return false;
+    if (bits != 4 && bits != 6 && bits != 8) return false;
+    if ((K * bits / 8) % 16) return false;       // code rows must be 16-byte pitched for TMA
+    if (K % (8 * int64_t(group))) return false;  // scale / bias rows too (groups per row % 8)
+    return K >= 8 * int64_t(group);
+}
+
+StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group, int split_req) {
+    StreamConfig c = {};
+    c.mt = M > 8 ? 2 : 1;
+    const int KS = ks_for(bits);
+    const int T = cdiv(N, ST_ROWS);
+    const int unit = std::max(KS, 8 * group);  // kslice granularity: whole stages and 8-group blocks
+    const int units = cdiv(K, unit);
+    int split = split_req;
+    if (split <= 0) {
+        // Fewer tiles than SMs: split K over up to 8 blocks (a portable cluster), keeping the
+        // grid within one wave of resident blocks and at least two stages per block.
+        split = 1;
+        if (T < kNumSM) {
+            for (int s = std::min(8, units); s >= 2; --s) {
+                const int ks = rup(cdiv(K, s), unit);
+                if (cdiv(K, ks) != s || ks / KS < 2) continue;
+                if (T * s <= kNumSM) {
+                    split = s;
+                    break;
+                }
+            }
+        }
+    }
+    split = std::max(1, std::min(8, split));
+    for (;; ++split) {
+        const int kslice = rup(cdiv(K, split), unit);
+        const int sp = cdiv(K, kslice);
+        const int nst = kslice / KS;
+        int ring = sp > 1 ? std::min(nst, 8) : 8;
+        ring = std::max(ring, 2);
+        while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp) > kMaxSmem) --ring;
+        if (st_smem(bits, c.mt, ring, kslice, group, sp) > kMaxSmem) {
+            if (split < 8) continue;
+            c.ring = 0;  // does not fit: the caller uses another kernel
+            return c;
+        }
+        c.split = sp;
+        c.kslice = kslice;
+        c.ring = ring;
+        c.smem = st_smem(bits, c.mt, ring, kslice, group, sp);
+        const int per_sm = std::max(1, int(kSmSmem / (c.smem + 1024)));
+        c.grid_x = sp > 1 ? T : std::min(T, kNumSM * per_sm);
+        return c;
+    }
+}
+
+cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream) {
+    const int mt = int(a.M) > 8 ? 2 : 1;
+    StKernelFn fn = pick_stream(a.bits, mt);
+    if (!fn || c.ring < 2) return cudaErrorInvalidValue;
+    const int KS = ks_for(a.bits);  // codes per stage
+    const uint64_t KW = uint64_t(a.K) * a.bits / 32;
+    const uint64_t G = uint64_t(a.K / a.group);
+    CUtensorMap wmap, smap, bmap;
+    const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
+                     uint32_t(KS * a.bits / 32), ST_ROWS, wsw) ||
+        !make_map_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, G, uint64_t(a.N), 8, ST_ROWS,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_2d(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.biases, G, uint64_t(a.N), 8, ST_ROWS,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+
+    StParams p;
+    p.x = a.x;
+    p.y = a.y;
+    p.M = int(a.M);
+    p.N = int(a.N);
+    p.K = int(a.K);
+    p.group = a.group;
+    p.gshift = ilog2(a.group);
+    p.is_bf16 = a.is_bf16;
+    p.T = cdiv(a.N, ST_ROWS);
+    p.kslice = c.kslice;
+    p.split = c.split;
+    p.ring = c.ring;
+    p.static_w = c.static_weights ? 1 : 0;
+
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(c.grid_x), unsigned(c.split), 1);
+    cfg.blockDim = dim3(ST_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = c.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    if (c.split > 1) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = unsigned(c.split);
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (c.pdl) {
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = unsigned(na);
+    return cudaLaunchKernelEx(&cfg, fn, wmap, smap, bmap, p);
+}
+
+cudaError_t stream_read_and_clear_errors(unsigned* out) {
+    unsigned v = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_stream_error, sizeof(v));
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyToSymbol(g_stream_error, &zero, sizeof(zero));
+    *out = v;
+    return e;
+}
+
+}  // namespace qmm_impl

@@ -110,6 +110,8 @@ enum {
     QMM_KERNEL_AUTO = 0,   /* let the dispatch table decide                                 */
     QMM_KERNEL_MMA = 1,    /* warp-per-16-row tile, register-streamed codes, mma.sync       */
     QMM_KERNEL_TC = 2,     /* swap-AB tcgen05 tile: 128 weight rows x M tokens, TMEM accum   */
+    QMM_KERNEL_STREAM = 3, /* M <= 16: TMA-staged codes, mma.sync consumer warps; K split over
+                              a cluster only when the 128-row tiles cannot fill the GPU      */
 };
 
 enum {
@@ -122,7 +124,8 @@ typedef struct {
     int32_t kernel;   /* QMM_KERNEL_*                                                       */
     int32_t split;    /* number of K slices (thread-block cluster size along K), 1..16      */
     int32_t warps;    /* warps per block: 4 or 8 for QMM_KERNEL_MMA (0 = default); the      
-                         tensor-core kernel always uses 18 and ignores this field           */
+                         tensor-core kernel always uses 18 and the streaming kernel 9, and
+                         both ignore this field                                             */
     uint32_t flags;   /* QMM_PLAN_* bits                                                     */
     int32_t reserved[4];
 } qmm_plan;

@@ -1,0 +1,109 @@
+"""GPU parity of the TMA-fed streaming kernel (QMM_KERNEL_STREAM, M <= 16) against the fp64 CPU
+oracle, through the C ABI with the kernel forced.
+
+Operation: MLX issue #4720, "To Reproduce" (quantized_matmul(x, *w, transpose=True)); formats:
+"What Are NAX Verify Kernels ...", "Supported Data Formats and Quantization Schemes".  Covers
+every format, each M up to 16, K split over clusters and the persistent (unsplit) grid with
+more tiles than blocks, ragged N, bf16 activations beyond the fp16 range and bitwise
+determinism.  Tolerances: tests/helpers.py.
+"""
+import pytest
+import torch
+
+import bit_quantized_gemm_qmm_b200 as q
+from bit_quantized_gemm_qmm_b200.inputs import randn, w_input, x_input
+from helpers import check_close, oracle_qmm, oracle_quantize, to_device_weights
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(oracle_mod, M, N, K, bits, group, dtype, sigma=1.0, split=0, flags=q.PLAN_PDL, wseed=0, x=None):
+    w = w_input(N, K, dtype, wseed, sigma)
+    if x is None:
+        x = x_input(M, K, dtype)
+    op, os_, ob = oracle_quantize(oracle_mod, w, bits, group)
+    P, S, B = to_device_weights(op, os_, ob)
+    plan = q.make_plan(kernel=q.KERNEL_STREAM, split=split, flags=flags)
+    y = q.qmm(x.cuda(), P, S, B, bits, group, plan=plan)
+    torch.cuda.synchronize()
+    assert q.device_errors() == 0
+    ref = oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group)
+    return check_close(y, ref, dtype, f"stream M={M} N={N} K={K} b{bits} g{group} {dtype} split={split}")
+
+
+@pytest.mark.parametrize("M", list(range(1, 17)))
+def test_every_m(oracle_mod, M):
+    _run(oracle_mod, M, 384, 2048, 4, 64, torch.float16)
+
+
+@pytest.mark.parametrize("bits", [4, 6, 8])
+@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("M", [1, 7, 16])
+def test_formats(oracle_mod, bits, group, dtype, M):
+    sigma = 1.0 if dtype == torch.float16 else 0.02
+    _run(oracle_mod, M, 272, 2048, bits, group, dtype, sigma)
+
+
+@pytest.mark.parametrize("split", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("bits,group", [(4, 64), (6, 32), (8, 128)])
+def test_forced_splits(oracle_mod, split, bits, group):
+    for flags in (0, q.PLAN_PDL | q.PLAN_STATIC_WEIGHTS):
+        _run(oracle_mod, 5, 256, 8192, bits, group, torch.float16, split=split, flags=flags)
+
+
+@pytest.mark.parametrize("N", [1, 17, 129, 1000])
+def test_ragged_n(oracle_mod, N):
+    _run(oracle_mod, 6, N, 1024, 4, 64, torch.float16)
+    _run(oracle_mod, 13, N, 1024, 6, 32, torch.bfloat16, 0.02)
+
+
+def test_persistent_more_tiles_than_blocks(oracle_mod):
+    """N = 40000 rows = 313 tiles with an unsplit K: each block streams several tiles with
+    the shared-memory ring running across tile boundaries."""
+    pd = q.plan_default(3, 40000, 1024, 4, 64, torch.float16)
+    assert pd.kernel == q.KERNEL_STREAM and pd.split == 1
+    _run(oracle_mod, 3, 40000, 1024, 4, 64, torch.float16)
+    _run(oracle_mod, 11, 40000, 1024, 8, 32, torch.bfloat16, 0.02)
+
+
+def test_bf16_large_activations(oracle_mod):
+    M, K = 4, 1024
+    x = randn((M, K), 1.0, torch.bfloat16, 5)
+    x[0] *= 1e6
+    x[1, :7] = 3.0e5
+    w = w_input(128, K, torch.bfloat16, 1, 0.02)
+    op, os_, ob = oracle_quantize(oracle_mod, w, 4, 64)
+    P, S, B = to_device_weights(op, os_, ob)
+    y = q.qmm(x.cuda(), P, S, B, 4, 64, plan=q.make_plan(kernel=q.KERNEL_STREAM))
+    torch.cuda.synchronize()
+    ref = oracle_qmm(oracle_mod, x, op, os_, ob, K, 4, 64)
+    for m in range(M):
+        check_close(y[m:m + 1], ref[m:m + 1], torch.bfloat16, f"row {m}")
+
+
+def test_large_scales_take_the_exact_path(oracle_mod):
+    """Scales of 64 and above (weights spanning more than 960) cannot use the fused offset
+    -M*s in fp16; those steps switch to the subtract-then-multiply form."""
+    M, N, K = 4, 256, 1024
+    w = w_input(N, K, torch.float16, 4, 1.0) * 300.0
+    op, os_, ob = oracle_quantize(oracle_mod, w, 4, 64)
+    P, S, B = to_device_weights(op, os_, ob)
+    assert float(S.float().abs().max()) >= 64.0
+    x = x_input(M, K, torch.float16)
+    y = q.qmm(x.cuda(), P, S, B, 4, 64, plan=q.make_plan(kernel=q.KERNEL_STREAM))
+    torch.cuda.synchronize()
+    ref = oracle_qmm(oracle_mod, x, op, os_, ob, K, 4, 64)
+    check_close(y, ref, torch.float16, "large scales")
+
+
+def test_deterministic_bitwise():
+    M, N, K = 9, 4096, 8192
+    w = w_input(N, K, torch.float16, 2).cuda()
+    x = x_input(M, K, torch.float16).cuda()
+    P, S, B = q.quantize(w, 4, 64)
+    plan = q.make_plan(kernel=q.KERNEL_STREAM)
+    y1 = q.qmm(x, P, S, B, 4, 64, plan=plan)
+    y2 = q.qmm(x, P, S, B, 4, 64, plan=plan)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
