@@ -102,10 +102,11 @@ qmm_status validate_qmm(const void* x, const uint32_t* packed, const uint16_t* s
     return QMM_OK;
 }
 
-// Dispatch between the two kernels, from the measured per-shape sweeps (bench.py --sweep; the
-// crossovers are recorded in the profiles): the tensor-core kernel wins for wide N at every M
-// and for large weight matrices from M = 9 up; on the 4096-wide and narrower projections the
-// warp-tile kernel keeps the lead to M = 32.
+// Dispatch, from the measured per-shape sweeps (bench.py --sweep; the crossovers are recorded
+// in the profiles): up to M = 8 the TMA-fed streaming kernel, where the shape suits it (K a
+// whole number of its stages and scale blocks); above that the tensor-core kernel for wide N
+// and for large weight matrices, and the warp-tile kernel on the 4096-wide and narrower
+// projections up to M = 32.
 bool prefer_tc(int64_t M, int64_t N, int64_t K) {
     if (N >= 8192 && N * K <= (int64_t(1) << 27)) return true;  // gate/up-like: wide N, moderate size
     if (N * K >= (int64_t(1) << 25)) return M >= 9;             // >= 32M codes (down, LM head)
@@ -163,7 +164,7 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
     const bool st_ok = stream_supported(M, N, K, bits, group) && aligned(scales, 16) && aligned(biases, 16) &&
                        stream_config(M, N, K, bits, group, p.split).ring >= 2;
     if (p.kernel == QMM_KERNEL_AUTO) {
-        if (st_ok && M <= 16) p.kernel = QMM_KERNEL_STREAM;
+        if (st_ok && M <= 8) p.kernel = QMM_KERNEL_STREAM;
         else p.kernel = (tc_ok && prefer_tc(M, N, K)) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
     }
     if (p.kernel == QMM_KERNEL_STREAM && !st_ok)

@@ -177,12 +177,14 @@ __device__ __forceinline__ void step_mma(const uint32_t (&w)[2][StepFmt<BITS>::N
 // ---------------------------------------------------------------- x staging
 constexpr int kXPad = 4;  // 16-byte chunks of padding after each staged x row
 
-// Stage x[0:8*MT, kc : kc + xchunk) as fp16 (zero outside [0,M) x [kc, kend)) in the lane
+// Stage x[0:M, kc : kc + xchunk) as fp16 (zero past kend) in the lane
 // layout: row m, step s, lane span c, chunk j at 16-byte chunk m*RS + s*(KS/8) + 4j + c
 // (RS = xchunk/8 + kXPad, which keeps the B-fragment reads free of bank conflicts), codes in
 // pair order.  Also the per-group sums X of the same (scaled) values, times 2^-7 so any group
 // of fp16 values stays finite, as fp16 (hi, lo) with X*2^-7 = hi + lo to about 2^-22
-// relative: xg[m*gpad + group] = (hi, lo); slots gpad > xchunk/group read as zero.
+// relative: xg[m*gpad + group] = (hi, lo); slots gpad > xchunk/group read as zero.  Token rows
+// M..8*MT-1 are left as they are: an MMA column depends only on its own B column, so those
+// rows only reach accumulator columns that are never stored.
 // Run by `nthreads` threads (whole warps, threadIdx.x < nthreads); xchunk is a multiple of
 // the step and of the group.
 template <int BITS, int MT>
@@ -193,16 +195,19 @@ __device__ __forceinline__ void stage_x_tile(const uint16_t* __restrict__ x, int
     constexpr int UN = F::UN, KS = F::KS, UPS = KS / UN;  // units per step
     constexpr int UPL = F::U / UN;                         // units per lane span
     const int upr = xchunk / UN;                           // units per row
-    const int total = 8 * MT * upr;                        // a multiple of 32
+    const int rows = M < 8 * MT ? M : 8 * MT;              // token rows >= M are never read back
+    const int total = rows * upr;
+    const int totp = (total + 31) & ~31;                   // whole warps take part in the shuffles
     const int RS = xchunk / 8 + kXPad;
     const int upg = group / UN;                            // units per group
-    for (int u0 = 0; u0 < total; u0 += nthreads) {
-        if (u0 + int(threadIdx.x & ~31u) >= total) break;  // whole warps only
+    for (int u0 = 0; u0 < totp; u0 += nthreads) {
+        if (u0 + int(threadIdx.x & ~31u) >= totp) break;   // whole warps only
         const int u = u0 + int(threadIdx.x);
+        const bool valid = u < total;
         const int m = u / upr, kk = u - m * upr;
         const int k = kc + kk * UN;
         float f[UN];
-        if (m < M && k < kend) {
+        if (valid && k < kend) {
             const uint16_t* src = x + int64_t(m) * K + k;
 #pragma unroll
             for (int h = 0; h < UN / 8; ++h) {
@@ -229,6 +234,7 @@ __device__ __forceinline__ void stage_x_tile(const uint16_t* __restrict__ x, int
 #pragma unroll
         for (int i = 0; i < UN; ++i) sum += f[i];
         for (int o = 1; o < upg; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (!valid) continue;  // (after the shuffles: padding units end whole groups)
         if ((kk & (upg - 1)) == 0) {
             const float X = sum * 0.0078125f;
             const __half hi = __float2half_rn(X);
@@ -252,7 +258,7 @@ __device__ __forceinline__ void stage_x_tile(const uint16_t* __restrict__ x, int
     }
     const int npg = xchunk / group;
     const int extra = gpad - npg;
-    for (int e = threadIdx.x; e < 8 * MT * extra; e += nthreads) {
+    for (int e = threadIdx.x; e < rows * extra; e += nthreads) {
         const int m = e / extra, gi = npg + (e - m * extra);
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(m * gpad + gi) * 4u), "r"(0u));
     }

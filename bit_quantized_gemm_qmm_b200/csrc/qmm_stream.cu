@@ -45,13 +45,23 @@ using namespace sm100;
 constexpr int ST_ROWS = 128;                  // weight rows per tile
 constexpr int ST_CW = 16;                     // consumer warps: 8 row groups x 2 K halves
 constexpr int ST_THREADS = (ST_CW + 1) * 32;  // + the producer warp
-constexpr int ST_SS = 4;                      // scale / bias boxes in flight
+constexpr int ST_SS = 3;                      // scale / bias boxes in flight
 constexpr long long ST_TIMEOUT = 4000000000LL;  // cycles (about 2 s)
 
-// A stage is 128 rows x KS codes (two steps of StepFmt, one per K half): 128 bytes a row
-// (192 for 6-bit).  Scales and biases arrive per block of 8 groups (8 x 2 bytes a row).
-template <int BITS>
-__host__ __device__ constexpr int stage_codes() { return 2 * StepFmt<BITS>::KS; }
+// A stage is 128 rows x stage_codes() codes: two TMA boxes of 128 bytes a row for 4/8-bit
+// (one per K half, SPH = 2 steps of StepFmt each), one box of 192 bytes a row for 6-bit (one
+// step per K half).  Scales and biases arrive per block of block_codes() codes (a whole
+// number of stages and of 8 groups).
+template <int BITS> struct SFmt {
+    static constexpr int SPH = BITS == 6 ? 1 : 2;              // steps per K half
+    static constexpr int KSTG = 2 * SPH * StepFmt<BITS>::KS;   // codes per stage
+};
+
+__host__ __device__ inline int st_stage_codes(int bits) { return bits == 6 ? 256 : (bits == 4 ? 512 : 256); }
+__host__ __device__ inline int st_block_codes(int bits, int group) {
+    const int a = 8 * group, b = st_stage_codes(bits);
+    return a > b ? a : b;
+}
 
 struct StParams {
     const uint16_t* x;
@@ -60,23 +70,22 @@ struct StParams {
     int group, gshift;
     int is_bf16;
     int T;        // 128-row tiles
-    int kslice;   // K codes per split (a multiple of the stage and of 8 groups)
+    int kslice;   // K codes per split (a multiple of the scale block)
     int split;
     int ring;     // stages in the shared-memory ring
     int static_w;
 };
 
 struct StLayout {
-    uint32_t w_stage, sb_off, x_off, xrs, xg_off, gpad, xf_off, red_off, bar_off, total;
+    uint32_t w_stage, sb_off, sb_slot, x_off, xrs, xg_off, gpad, xf_off, red_off, bar_off, total;
 };
-
-constexpr uint32_t kSbSlot = 2 * ST_ROWS * 8 * 2;  // one scale box + one bias box (4 KB)
 
 __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split) {
     StLayout L;
-    L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 128));  // 16 or 24 KB
+    L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 256));  // 24 or 32 KB
     L.sb_off = uint32_t(ring) * L.w_stage;
-    uint32_t off = L.sb_off + ST_SS * kSbSlot;
+    L.sb_slot = uint32_t(2 * ST_ROWS * (st_block_codes(bits, group) / group) * 2);  // scales + biases
+    uint32_t off = L.sb_off + ST_SS * L.sb_slot;
     L.x_off = off;
     L.xrs = uint32_t(kslice / 8 + kXPad);                     // 16-byte chunks per staged x row
     off += uint32_t(8 * mt) * L.xrs * 16;
@@ -151,10 +160,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     qmm_stream_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                       const __grid_constant__ CUtensorMap bmap, const StParams p) {
     using F = StepFmt<BITS>;
-    constexpr int KSS = F::KS;                 // codes per step (one K half of a stage)
-    constexpr int KS = stage_codes<BITS>();    // codes per stage
+    using SF = SFmt<BITS>;
+    constexpr int KSS = F::KS;                 // codes per step
+    constexpr int SPH = SF::SPH;               // steps per K half of a stage
+    constexpr int KS = SF::KSTG;               // codes per stage
     constexpr int NREG = F::NREG, U = F::U;
-    constexpr int WPS = KS * BITS / 32;        // 32-bit words per row per stage
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ float s_red[ST_CW];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -173,7 +183,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     const int kb = blockIdx.y * p.kslice;
     const int ke = min(p.K, kb + p.kslice);
     const int nst = (ke - kb + KS - 1) / KS;
-    const int spb = (8 * p.group) / KS;         // stages per block of 8 groups (1..8)
+    const int blkc = st_block_codes(BITS, p.group);
+    const int gbb = blkc >> p.gshift;            // groups per scale block (8 or 16)
+    const int spb = blkc / KS;                   // stages per scale block (1..4)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
@@ -202,6 +214,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             if (!p.static_w) grid_dependency_wait();
+            constexpr int BOXW = BITS == 6 ? 48 : 32;          // words per box row
+            constexpr int NBOX = BITS == 6 ? 1 : 2;            // boxes per stage
             const int wcol0 = kb / 32 * BITS;  // kb * BITS / 32 (kb is a multiple of 256)
             const int gcol0 = kb >> p.gshift;  // a multiple of 8
             int it = 0, blk = 0;
@@ -209,16 +223,17 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             for (int t = blockIdx.x; t < p.T && ok; t += gridDim.x) {
                 const long long dl = clock64() + ST_TIMEOUT;
                 for (int st = 0; st < nst; ++st, ++it) {
-                    if (st % spb == 0) {  // scales and biases of the next 8 groups
+                    if (st % spb == 0) {  // scales and biases of the next block of groups
                         const int ss = blk % ST_SS;
                         if (blk >= ST_SS && !wait_or_abort(bar_sempty + 8 * ss, ((blk / ST_SS) & 1) ^ 1, dl, abort_flag)) {
                             ok = false;
                             break;
                         }
-                        const uint32_t dst = sbase + L.sb_off + ss * kSbSlot;
-                        mbar_arrive_expect_tx(bar_sfull + 8 * ss, kSbSlot);
-                        tma_load_2d(dst, &smap, bar_sfull + 8 * ss, gcol0 + 8 * (st / spb), t * ST_ROWS);
-                        tma_load_2d(dst + kSbSlot / 2, &bmap, bar_sfull + 8 * ss, gcol0 + 8 * (st / spb), t * ST_ROWS);
+                        const uint32_t dst = sbase + L.sb_off + ss * L.sb_slot;
+                        mbar_arrive_expect_tx(bar_sfull + 8 * ss, L.sb_slot);
+                        tma_load_2d(dst, &smap, bar_sfull + 8 * ss, gcol0 + gbb * (st / spb), t * ST_ROWS);
+                        tma_load_2d(dst + L.sb_slot / 2, &bmap, bar_sfull + 8 * ss, gcol0 + gbb * (st / spb),
+                                    t * ST_ROWS);
                         ++blk;
                     }
                     const int s = it % S;
@@ -227,7 +242,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(bar_full + 8 * s, L.w_stage);
-                    tma_load_2d(sbase + s * L.w_stage, &wmap, bar_full + 8 * s, wcol0 + st * WPS, t * ST_ROWS);
+#pragma unroll
+                    for (int b = 0; b < NBOX; ++b)
+                        tma_load_2d(sbase + s * L.w_stage + b * (ST_ROWS * 128), &wmap, bar_full + 8 * s,
+                                    wcol0 + (st * NBOX + b) * BOXW, t * ST_ROWS);
                 }
             }
             // nothing may still be landing in shared memory when the block exits
@@ -240,10 +258,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     } else {
         // ------------------------------------------------------------ consumers
         const int g = lane >> 2, c = lane & 3;
-        const int half = warp >> 3;                        // K half of each stage
-        const int rg = warp & 7;                           // 16-row group of the tile
+        const int half = warp >> 3;                             // K half of each stage
+        const int rg = warp & 7;                                // 16-row group of the tile
         const int rA = rg * 16 + ((g >> 1) | ((g & 1) << 2));  // rows of "g" and "g + 8": the
-        const int rB = rA + 8;                             // permutation keeps the code reads conflict-free
+        const int rB = rA + 8;                                  // permutation keeps the code reads conflict-free
         grid_dependency_wait();
         const int E = p.is_bf16 ? bf16_exponent(p, kb, ke, s_red) : 0;
         const uint32_t xs = sbase + L.x_off, xg = sbase + L.xg_off;
@@ -253,7 +271,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         grid_dependents_launch();
 
         const uint32_t xmt = 8 * L.xrs * 16;
-        const uint32_t xlane = xs + uint32_t(g * int(L.xrs) + c) * 16u + uint32_t(half * KSS * 2);
+        const uint32_t xlane = xs + uint32_t(g * int(L.xrs) + c) * 16u + uint32_t(half * SPH * KSS * 2);
         const uint32_t xgrow = xg + uint32_t(g * int(L.gpad)) * 4u;
         const uint32_t xg_mt = 8 * L.gpad * 4;
         float* xf = reinterpret_cast<float*>(smem + L.xf_off) + (rg * 32 + lane) * 4 * MT;
@@ -274,12 +292,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 const int ss = blk % ST_SS;
                 if (st % spb == 0) {
                     sok = wait_or_abort(bar_sfull + 8 * ss, (blk / ST_SS) & 1, dl, abort_flag);
-                    sbuf = sbase + L.sb_off + ss * kSbSlot;
+                    sbuf = sbase + L.sb_off + ss * L.sb_slot;
                 }
                 const int s = it % S;
                 const bool ok = sok && wait_or_abort(bar_full + 8 * s, (it / S) & 1, dl, abort_flag);
                 if (ok) {
-                    uint32_t w[2][NREG];
+                    // the lane's codes of rows rA and rB for the SPH steps of its K half; the
+                    // ring slot is released as soon as they are in registers
+                    uint32_t w[SPH][2][NREG];
                     const uint32_t stage = sbase + s * L.w_stage;
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
@@ -288,35 +308,45 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
                             for (int i = 0; i < 3; ++i) {
                                 const uint2 v = lds_v2(stage + row * 192 + half * 96 + 24 * c + 8 * i);
-                                w[r][2 * i] = v.x;
-                                w[r][2 * i + 1] = v.y;
+                                w[0][r][2 * i] = v.x;
+                                w[0][r][2 * i + 1] = v.y;
                             }
-                        } else {  // 128-byte swizzle: 16-byte chunk ^= row & 7
-                            const uint4 v = lds_v4(stage + row * 128 + ((((4 * half + c) ^ row) & 7) << 4));
-                            w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
+                        } else {  // box `half`, 128-byte swizzle: 16-byte chunk ^= row & 7
+#pragma unroll
+                            for (int j = 0; j < SPH; ++j) {
+                                const uint4 v = lds_v4(stage + half * (ST_ROWS * 128) + row * 128 +
+                                                       ((((4 * j + c) ^ row) & 7) << 4));
+                                w[j][r][0] = v.x; w[j][r][1] = v.y; w[j][r][2] = v.z; w[j][r][3] = v.w;
+                            }
                         }
                     }
-                    // the group of the lane's span within the current block of 8 groups
-                    const int gl = ((st * KS + half * KSS + c * U) >> p.gshift) & 7;
-                    const uint32_t s0 = lds_u16(sbuf + uint32_t(rA * 8 + gl) * 2u);
-                    const uint32_t s1 = lds_u16(sbuf + uint32_t(rB * 8 + gl) * 2u);
-                    const RowConst C[2] = {row_const<BITS>(s0), row_const<BITS>(s1)};
-                    const bool big = ((s0 & 0x7FFFu) >= 0x5400u) | ((s1 & 0x7FFFu) >= 0x5400u);
-                    const uint32_t xa = xlane + uint32_t(st * KS * 2);
-                    if (__any_sync(0xffffffffu, big))
-                        step_mma<BITS, MT, true>(w, C, xa, xmt, acc);
-                    else
-                        step_mma<BITS, MT, false>(w, C, xa, xmt, acc);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+#pragma unroll
+                    for (int j = 0; j < SPH; ++j) {
+                        // the lane's group within the current scale block
+                        const int kr = st * KS + (half * SPH + j) * KSS + c * U;
+                        const int gl = (kr >> p.gshift) - (st / spb) * gbb;
+                        const uint32_t s0 = lds_u16(sbuf + uint32_t(rA * gbb + gl) * 2u);
+                        const uint32_t s1 = lds_u16(sbuf + uint32_t(rB * gbb + gl) * 2u);
+                        const RowConst C[2] = {row_const<BITS>(s0), row_const<BITS>(s1)};
+                        const bool big = ((s0 & 0x7FFFu) >= 0x5400u) | ((s1 & 0x7FFFu) >= 0x5400u);
+                        const uint32_t xa = xlane + uint32_t(st * KS * 2 + j * KSS * 2);
+                        if (__any_sync(0xffffffffu, big))
+                            step_mma<BITS, MT, true>(w[j], C, xa, xmt, acc);
+                        else
+                            step_mma<BITS, MT, false>(w[j], C, xa, xmt, acc);
+                    }
                 }
                 if (st % spb == spb - 1) {
-                    if (sok && half == 0) {  // bias term of the block's 8 groups: y += b * X
-                        const uint32_t bb = sbuf + kSbSlot / 2;
-                        bias_mma<MT>(lds_u16(bb + uint32_t(rA * 8 + c) * 2u), lds_u16(bb + uint32_t(rB * 8 + c) * 2u),
-                                     lds_u16(bb + uint32_t(rA * 8 + c + 4) * 2u),
-                                     lds_u16(bb + uint32_t(rB * 8 + c + 4) * 2u), xgrow + uint32_t(st / spb) * 32u,
-                                     xg_mt, c, tb);
+                    if (sok && half == 0) {  // bias term of the block's groups: y += b * X
+                        const uint32_t bb = sbuf + L.sb_slot / 2;
+                        for (int q = 0; q < gbb; q += 8)
+                            bias_mma<MT>(lds_u16(bb + uint32_t(rA * gbb + q + c) * 2u),
+                                         lds_u16(bb + uint32_t(rB * gbb + q + c) * 2u),
+                                         lds_u16(bb + uint32_t(rA * gbb + q + c + 4) * 2u),
+                                         lds_u16(bb + uint32_t(rB * gbb + q + c + 4) * 2u),
+                                         xgrow + uint32_t((st / spb) * gbb + q) * 4u, xg_mt, c, tb);
                     }
                     __syncwarp();
                     if (sok && lane == 0) mbar_arrive(bar_sempty + 8 * ss);
@@ -401,7 +431,7 @@ StKernelFn pick_stream(int bits, int mt) {
     return nullptr;
 }
 
-int ks_for(int bits) { return bits == 8 ? 128 : 256; }
+int ks_for(int bits) { return st_stage_codes(bits); }
 int ilog2(int v) {
     int s = 0;
     while ((1 << s) < v) ++s;
@@ -425,7 +455,7 @@ bool stream_supported(int64_t M, int64_t N, int64_t K, int bits, int group) {
     if (bits != 4 && bits != 6 && bits != 8) return false;
     if ((K * bits / 8) % 16) return false;       // code rows must be 16-byte pitched for TMA
     if (K % (8 * int64_t(group))) return false;  // scale / bias rows too (groups per row % 8)
-    return K >= 8 * int64_t(group);
+    return K % st_block_codes(bits, group) == 0;  // whole stages and scale blocks
 }
 
 StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group, int split_req) {
@@ -433,7 +463,7 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
     c.mt = M > 8 ? 2 : 1;
     const int KS = ks_for(bits);
     const int T = cdiv(N, ST_ROWS);
-    const int unit = std::max(KS, 8 * group);  // kslice granularity: whole stages and 8-group blocks
+    const int unit = st_block_codes(bits, group);  // kslice granularity: whole stages and scale blocks
     const int units = cdiv(K, unit);
     int split = split_req;
     if (split <= 0) {
@@ -456,10 +486,13 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         const int kslice = rup(cdiv(K, split), unit);
         const int sp = cdiv(K, kslice);
         const int nst = kslice / KS;
-        int ring = sp > 1 ? std::min(nst, 8) : 8;
-        ring = std::max(ring, 2);
+        // ring: up to 6 stages (at most the stages a block streams when K is split); at least
+        // 3 when the whole K range has more, else K is split further to make room
+        const int want = std::min(sp > 1 ? nst : 6, 6);
+        int ring = std::max(want, 2);
         while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp) > kMaxSmem) --ring;
-        if (st_smem(bits, c.mt, ring, kslice, group, sp) > kMaxSmem) {
+        const bool fits = st_smem(bits, c.mt, ring, kslice, group, sp) <= kMaxSmem;
+        if (!fits || (ring < std::min(want, 3) && split < 8)) {
             if (split < 8) continue;
             c.ring = 0;  // does not fit: the caller uses another kernel
             return c;
@@ -483,11 +516,12 @@ cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t 
     const uint64_t G = uint64_t(a.K / a.group);
     CUtensorMap wmap, smap, bmap;
     const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+    const uint32_t gbb = uint32_t(st_block_codes(a.bits, a.group) / a.group);  // groups per scale box
     if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
-                     uint32_t(KS * a.bits / 32), ST_ROWS, wsw) ||
-        !make_map_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, G, uint64_t(a.N), 8, ST_ROWS,
+                     a.bits == 6 ? 48u : 32u, ST_ROWS, wsw) ||
+        !make_map_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, G, uint64_t(a.N), gbb, ST_ROWS,
                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_2d(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.biases, G, uint64_t(a.N), 8, ST_ROWS,
+        !make_map_2d(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.biases, G, uint64_t(a.N), gbb, ST_ROWS,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
 

@@ -84,11 +84,11 @@ def test_plans(L):
     assert p.kernel in (q.KERNEL_MMA, q.KERNEL_TC, q.KERNEL_STREAM) and 1 <= p.split <= 16
     # the streaming kernel takes M <= 16 when K is a multiple of eight groups; its K split
     # stays within a portable cluster
-    for M in (1, 6, 16):
+    for M in (1, 6, 8):
         p = q.plan_default(M, 4096, 14336, 4, 64, f16)
         assert p.kernel == q.KERNEL_STREAM and 1 <= p.split <= 8
     assert q.plan_default(4, 151936, 4096, 4, 64, f16).split == 1  # enough tiles: no split
-    assert q.plan_default(17, 4096, 4096, 4, 64, f16).kernel != q.KERNEL_STREAM
+    assert q.plan_default(9, 4096, 4096, 4, 64, f16).kernel != q.KERNEL_STREAM
     assert q.plan_default(4, 4096, 4096 + 64, 4, 64, f16).kernel != q.KERNEL_STREAM
     st = q.make_plan(kernel=q.KERNEL_STREAM)
     assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(st), None) == q.QMM_ERR_UNSUPPORTED
