@@ -218,26 +218,32 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
             constexpr int NBOX = BITS == 6 ? 1 : 2;            // boxes per stage
             const int wcol0 = kb / 32 * BITS;  // kb * BITS / 32 (kb is a multiple of 256)
             const int gcol0 = kb >> p.gshift;  // a multiple of 8
-            int it = 0, blk = 0;
+            int it = 0, blk = 0;               // stages and scale blocks issued
+            int s = 0, ss = 0;                 // their ring slots
+            uint32_t ph = 0, sph = 0;          // ... and phases
             bool ok = true;
             for (int t = blockIdx.x; t < p.T && ok; t += gridDim.x) {
                 const long long dl = clock64() + ST_TIMEOUT;
+                int sib = 0, gcol = gcol0, wcol = wcol0;
                 for (int st = 0; st < nst; ++st, ++it) {
-                    if (st % spb == 0) {  // scales and biases of the next block of groups
-                        const int ss = blk % ST_SS;
-                        if (blk >= ST_SS && !wait_or_abort(bar_sempty + 8 * ss, ((blk / ST_SS) & 1) ^ 1, dl, abort_flag)) {
+                    if (sib == 0) {  // scales and biases of the next block of groups
+                        if (blk >= ST_SS && !wait_or_abort(bar_sempty + 8 * ss, sph ^ 1u, dl, abort_flag)) {
                             ok = false;
                             break;
                         }
                         const uint32_t dst = sbase + L.sb_off + ss * L.sb_slot;
                         mbar_arrive_expect_tx(bar_sfull + 8 * ss, L.sb_slot);
-                        tma_load_2d(dst, &smap, bar_sfull + 8 * ss, gcol0 + gbb * (st / spb), t * ST_ROWS);
-                        tma_load_2d(dst + L.sb_slot / 2, &bmap, bar_sfull + 8 * ss, gcol0 + gbb * (st / spb),
-                                    t * ST_ROWS);
+                        tma_load_2d(dst, &smap, bar_sfull + 8 * ss, gcol, t * ST_ROWS);
+                        tma_load_2d(dst + L.sb_slot / 2, &bmap, bar_sfull + 8 * ss, gcol, t * ST_ROWS);
+                        gcol += gbb;
                         ++blk;
+                        if (++ss == ST_SS) {
+                            ss = 0;
+                            sph ^= 1u;
+                        }
                     }
-                    const int s = it % S;
-                    if ((it >= S && !wait_or_abort(bar_empty + 8 * s, ((it / S) & 1) ^ 1, dl, abort_flag)) || *abort_flag) {
+                    if (++sib == spb) sib = 0;
+                    if ((it >= S && !wait_or_abort(bar_empty + 8 * s, ph ^ 1u, dl, abort_flag)) || *abort_flag) {
                         ok = false;
                         break;
                     }
@@ -245,7 +251,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
                     for (int b = 0; b < NBOX; ++b)
                         tma_load_2d(sbase + s * L.w_stage + b * (ST_ROWS * 128), &wmap, bar_full + 8 * s,
-                                    wcol0 + (st * NBOX + b) * BOXW, t * ST_ROWS);
+                                    wcol + b * BOXW, t * ST_ROWS);
+                    wcol += NBOX * BOXW;
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             // nothing may still be landing in shared memory when the block exits
@@ -276,7 +287,14 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         const uint32_t xg_mt = 8 * L.gpad * 4;
         float* xf = reinterpret_cast<float*>(smem + L.xf_off) + (rg * 32 + lane) * 4 * MT;
         const float yscale = exp2i(E);
-        int it = 0, blk = 0, tc = 0;
+        // ring position (slot s, phase ph) and scale-block position (slot ss, phase sph) advance
+        // incrementally; no division in the loop
+        int s = 0, ss = 0, tc = 0;
+        uint32_t ph = 0, sph = 0;
+        int lane_off[SPH];  // code offset of the lane span of each step within a stage
+#pragma unroll
+        for (int j = 0; j < SPH; ++j) lane_off[j] = (half * SPH + j) * KSS + c * U;
+        const uint32_t rAg = uint32_t(rA * gbb) * 2u, rBg = uint32_t(rB * gbb) * 2u;
         for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++tc) {
             // After a timeout (abort flag set) every wait below returns at once and the work
             // is skipped, so all warps leave the loop together.
@@ -288,14 +306,15 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
                 for (int i = 0; i < 4; ++i) acc[mt][i] = tb[mt][i] = 0.f;
             uint32_t sbuf = 0;
             bool sok = true;
-            for (int st = 0; st < nst; ++st, ++it) {
-                const int ss = blk % ST_SS;
-                if (st % spb == 0) {
-                    sok = wait_or_abort(bar_sfull + 8 * ss, (blk / ST_SS) & 1, dl, abort_flag);
+            int sib = 0;             // stage within the scale block
+            uint32_t xblk = xgrow;   // group sums of the current block
+            uint32_t xst = xlane;    // staged x of the current stage
+            for (int st = 0; st < nst; ++st) {
+                if (sib == 0) {
+                    sok = wait_or_abort(bar_sfull + 8 * ss, sph, dl, abort_flag);
                     sbuf = sbase + L.sb_off + ss * L.sb_slot;
                 }
-                const int s = it % S;
-                const bool ok = sok && wait_or_abort(bar_full + 8 * s, (it / S) & 1, dl, abort_flag);
+                const bool ok = sok && wait_or_abort(bar_full + 8 * s, ph, dl, abort_flag);
                 if (ok) {
                     // the lane's codes of rows rA and rB for the SPH steps of its K half; the
                     // ring slot is released as soon as they are in registers
@@ -325,32 +344,40 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < SPH; ++j) {
                         // the lane's group within the current scale block
-                        const int kr = st * KS + (half * SPH + j) * KSS + c * U;
-                        const int gl = (kr >> p.gshift) - (st / spb) * gbb;
-                        const uint32_t s0 = lds_u16(sbuf + uint32_t(rA * gbb + gl) * 2u);
-                        const uint32_t s1 = lds_u16(sbuf + uint32_t(rB * gbb + gl) * 2u);
+                        const uint32_t gl2 = uint32_t((sib * KS + lane_off[j]) >> p.gshift) * 2u;
+                        const uint32_t s0 = lds_u16(sbuf + rAg + gl2);
+                        const uint32_t s1 = lds_u16(sbuf + rBg + gl2);
                         const RowConst C[2] = {row_const<BITS>(s0), row_const<BITS>(s1)};
                         const bool big = ((s0 & 0x7FFFu) >= 0x5400u) | ((s1 & 0x7FFFu) >= 0x5400u);
-                        const uint32_t xa = xlane + uint32_t(st * KS * 2 + j * KSS * 2);
+                        const uint32_t xa = xst + uint32_t(j * KSS * 2);
                         if (__any_sync(0xffffffffu, big))
                             step_mma<BITS, MT, true>(w[j], C, xa, xmt, acc);
                         else
                             step_mma<BITS, MT, false>(w[j], C, xa, xmt, acc);
                     }
                 }
-                if (st % spb == spb - 1) {
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                xst += uint32_t(KS * 2);
+                if (++sib == spb) {
                     if (sok && half == 0) {  // bias term of the block's groups: y += b * X
                         const uint32_t bb = sbuf + L.sb_slot / 2;
                         for (int q = 0; q < gbb; q += 8)
-                            bias_mma<MT>(lds_u16(bb + uint32_t(rA * gbb + q + c) * 2u),
-                                         lds_u16(bb + uint32_t(rB * gbb + q + c) * 2u),
-                                         lds_u16(bb + uint32_t(rA * gbb + q + c + 4) * 2u),
-                                         lds_u16(bb + uint32_t(rB * gbb + q + c + 4) * 2u),
-                                         xgrow + uint32_t((st / spb) * gbb + q) * 4u, xg_mt, c, tb);
+                            bias_mma<MT>(lds_u16(bb + rAg + uint32_t(q + c) * 2u), lds_u16(bb + rBg + uint32_t(q + c) * 2u),
+                                         lds_u16(bb + rAg + uint32_t(q + c + 4) * 2u),
+                                         lds_u16(bb + rBg + uint32_t(q + c + 4) * 2u), xblk + uint32_t(q) * 4u, xg_mt, c,
+                                         tb);
                     }
                     __syncwarp();
                     if (sok && lane == 0) mbar_arrive(bar_sempty + 8 * ss);
-                    ++blk;
+                    sib = 0;
+                    xblk += uint32_t(gbb) * 4u;
+                    if (++ss == ST_SS) {
+                        ss = 0;
+                        sph ^= 1u;
+                    }
                 }
             }
             // the two K halves meet: half 1 hands its partial sums to half 0 (mbarrier handshake)
