@@ -69,6 +69,7 @@ struct StreamConfig {
     int kslice;    // K codes per slice
     int ring;      // shared-memory stages (0: the shape does not fit this kernel)
     int grid_x;    // blocks along N (persistent when split == 1)
+    int ncw;       // consumer warps per block (8 or 16)
     size_t smem;   // dynamic shared memory per block
     bool pdl;
     bool static_weights;
