@@ -36,6 +36,7 @@ METRIC = "effective weight GB/s (and % of HBM roofline) per shape vs M=1..64, 1Ã
 WORKLOAD = "qo"
 BENCH_MS = (1, 4, 5, 6)
 NOMINAL_HBM_GBS = 8000.0
+KERNEL_NAMES = {1: "qmm_mma_kernel", 2: "qmm_tc_kernel", 3: "qmm_stream_kernel"}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -52,7 +53,7 @@ def parse():
                     "JSON file instead of running the headline benchmark")
     ap.add_argument("--sweep-configs", default="qo,down,gateup_6b,gateup_8b,kv_6b,kv_8b,lmhead")
     ap.add_argument("--sweep-ms", default="1-64", help="e.g. 1-64 or 1,4,16")
-    ap.add_argument("--sweep-plan", default="", help="kernel:split:warps override, e.g. 1:4:8")
+    ap.add_argument("--sweep-plan", default="", help="kernel:split:warps[:flags] override, e.g. 1:4:8")
     return ap.parse_args()
 
 
@@ -79,12 +80,20 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of the ranks' values (every rank gets it); identity on one process."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_gbs(bytes_per_rank_step: float, ms_per_step: float, world: int) -> float:
+    """Whole-job rate for weak scaling: every rank streams the same bytes per step, and the
+    step time is the slowest rank's."""
+    return bytes_per_rank_step * world / (ms_per_step * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -230,7 +239,7 @@ def run_ours(args, rank, world):
     clk = clocks.stop()
     t_ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_per_step = t_ms / args.steps
-    value = step_wbytes * world / (ms_per_step * 1e-3) / 1e9
+    value = job_gbs(step_wbytes, ms_per_step, world)
     achieved = step_algo_bytes / (ms_per_step * 1e-3) / 1e9  # per GPU: the only kernel in the step
 
     # ---- eager figure (same calls, launched one by one)
@@ -284,7 +293,7 @@ def run_ours(args, rank, world):
                    "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(),
-                     "peak_kind": peak_kind, "kernel": "qmm_mma_kernel",
+                     "peak_kind": peak_kind, "kernel": KERNEL_NAMES.get(plans[BENCH_MS[0]].kernel, "?"),
                      "algorithmic_bytes_per_launch": "weight bytes + 2*M*K (x) + 2*M*N (y)"},
         "breakdown": breakdown,
         "e2e": e2e,
@@ -450,9 +459,10 @@ def run_sweep(args):
             x = x_input(M, wl.K, wl.dtype).to(dev)
             y = torch.empty((M, wl.N), dtype=wl.dtype, device=dev)
             if args.sweep_plan:
-                kern, split, warps = (int(v) for v in args.sweep_plan.split(":"))
-                plan = q.make_plan(kernel=kern, split=split, warps=warps,
-                                   flags=q.PLAN_PDL | q.PLAN_STATIC_WEIGHTS)
+                f = [int(v) for v in args.sweep_plan.split(":")]
+                kern, split, warps = f[:3]
+                flags = f[3] if len(f) > 3 else q.PLAN_PDL | q.PLAN_STATIC_WEIGHTS
+                plan = q.make_plan(kernel=kern, split=split, warps=warps, flags=flags)
             else:
                 plan = q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype)
                 plan.flags |= q.PLAN_STATIC_WEIGHTS
