@@ -26,6 +26,8 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <cstring>
+#include <unordered_map>
 
 #include "qmm_common.cuh"
 #include "qmm_dq.cuh"
@@ -567,23 +569,87 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
     }
 }
 
+namespace {
+
+// Per-thread cache of encoded weight descriptors, keyed by the arrays and the format.
+struct StMaps {
+    CUtensorMap w, s, b;
+};
+struct MapKey {
+    const void *packed, *scales, *biases;
+    int64_t N, K;
+    int bits, group;
+    bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey& k) const {
+        size_t h = 1469598103934665603ull;
+        const unsigned char* p = reinterpret_cast<const unsigned char*>(&k);
+        for (size_t i = 0; i < sizeof(MapKey); ++i) h = (h ^ p[i]) * 1099511628211ull;
+        return h;
+    }
+};
+
+const StMaps* weight_maps(const QmmArgs& a) {
+    thread_local std::unordered_map<MapKey, StMaps, MapKeyHash> cache;
+    MapKey k;
+    std::memset(&k, 0, sizeof(k));  // padding bytes take part in the key
+    k.packed = a.packed;
+    k.scales = a.scales;
+    k.biases = a.biases;
+    k.N = a.N;
+    k.K = a.K;
+    k.bits = a.bits;
+    k.group = a.group;
+    auto it = cache.find(k);
+    if (it != cache.end()) return &it->second;
+    const uint64_t KW = uint64_t(a.K) * a.bits / 32;
+    const uint64_t G = uint64_t(a.K / a.group);
+    const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+    const uint32_t gbb = uint32_t(st_block_codes(a.bits, a.group) / a.group);  // groups per scale box
+    StMaps m;
+    if (!make_map_2d(&m.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N), a.bits == 6 ? 48u : 32u,
+                     ST_ROWS, wsw) ||
+        !make_map_2d(&m.s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, G, uint64_t(a.N), gbb, ST_ROWS,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_2d(&m.b, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.biases, G, uint64_t(a.N), gbb, ST_ROWS,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return nullptr;
+    if (cache.size() >= 1024) cache.clear();  // bounded: many distinct weight sets just re-encode
+    return &cache.emplace(k, m).first->second;
+}
+
+// The dynamic shared memory limit of a kernel is raised once per device and size.
+cudaError_t ensure_smem_attr(StKernelFn fn, size_t smem) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    struct FnDev {
+        StKernelFn fn;
+        int dev;
+        bool operator==(const FnDev& o) const { return fn == o.fn && dev == o.dev; }
+    };
+    struct FnDevHash {
+        size_t operator()(const FnDev& k) const { return std::hash<const void*>()((const void*)k.fn) ^ size_t(k.dev); }
+    };
+    thread_local std::unordered_map<FnDev, size_t, FnDevHash> done;
+    size_t& have = done[FnDev{fn, dev}];
+    if (have >= smem) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e == cudaSuccess) have = smem;
+    return e;
+}
+
+}  // namespace
+
 cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream) {
     const int mt = int(a.M) > 8 ? 2 : 1;
     StKernelFn fn = pick_stream(a.bits, mt, c.ncw);
     if (!fn || c.ring < 2) return cudaErrorInvalidValue;
-    const int KS = ks_for(a.bits);  // codes per stage
-    const uint64_t KW = uint64_t(a.K) * a.bits / 32;
-    const uint64_t G = uint64_t(a.K / a.group);
-    CUtensorMap wmap, smap, bmap;
-    const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
-    const uint32_t gbb = uint32_t(st_block_codes(a.bits, a.group) / a.group);  // groups per scale box
-    if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
-                     a.bits == 6 ? 48u : 32u, ST_ROWS, wsw) ||
-        !make_map_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, G, uint64_t(a.N), gbb, ST_ROWS,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_2d(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.biases, G, uint64_t(a.N), gbb, ST_ROWS,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
+    // The three descriptors depend only on the weight arrays and the format; a call that
+    // repeats them (the usual case: the same weights every step) reuses the encoded copies.
+    const StMaps* maps = weight_maps(a);
+    if (!maps) return cudaErrorInvalidValue;
 
     StParams p;
     p.x = a.x;
@@ -600,7 +666,7 @@ cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t 
     p.ring = c.ring;
     p.static_w = c.static_weights ? 1 : 0;
 
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem));
+    cudaError_t e = ensure_smem_attr(fn, c.smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(c.grid_x), unsigned(c.split), 1);
@@ -623,7 +689,7 @@ cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t 
     }
     cfg.attrs = attrs;
     cfg.numAttrs = unsigned(na);
-    return cudaLaunchKernelEx(&cfg, fn, wmap, smap, bmap, p);
+    return cudaLaunchKernelEx(&cfg, fn, maps->w, maps->s, maps->b, p);
 }
 
 cudaError_t stream_read_and_clear_errors(unsigned* out) {
