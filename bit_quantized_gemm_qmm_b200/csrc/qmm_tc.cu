@@ -30,6 +30,7 @@
 #include <unordered_map>
 
 #include "qmm_common.cuh"
+#include "qmm_dq.cuh"
 #include "qmm_internal.h"
 #include "sm100.cuh"
 
@@ -134,18 +135,45 @@ __host__ __device__ inline TcSmemLayout tc_layout(int x_stage, int w_bytes, int 
     L.w_off = L.x_off + ring * L.x_stage;
     L.sc_off = L.w_off + ring * L.w_stage;
     L.bar_off = L.sc_off + TC_SPF * TC_NDQ * 32 * 8;
-    L.total = L.bar_off + 8 * (2 * ring + 2 * na + 1) + 16;
+    L.total = L.bar_off + 8 * (4 * ring + 2 * na + 1) + 16;
     return L;
 }
 
 __device__ __forceinline__ void set_error(unsigned bit) { atomicOr(&g_tc_error, bit); }
 
 // ---------------------------------------------------------------- dequantization into A
-// One thread: U codes of one row (a quarter stage) -> U/2 fp16x2 columns of the A buffer, in
-// natural K order (column j = codes 2j, 2j+1).  s_pair/b_pair: fp16 pair holding the scale
-// (bias) of the thread's groups; two_groups: the U codes span two groups (lo half, hi half).
+// One thread: U codes of one row (a quarter stage), already in registers (wd), -> U/2 fp16x2
+// columns of the A buffer.  Column j holds K slots (2j, 2j+1), which hold the codes the x
+// tiles put there (xprep_kernel): for 4-bit the pairs (i, i+4) of each word, for 6-bit the
+// triplet pairs of qmm_dq.cuh, for 8-bit natural pairs.  Each column is RN_fp16(s*q + b):
+// q = (M + q) - M exactly, then one fused multiply-add.  s_pair/b_pair: fp16 pair holding the
+// scale (bias) of the thread's groups; two_groups: the U codes span two groups (lo, hi half).
+__device__ __forceinline__ uint32_t fold(uint32_t v, uint32_t magic, uint32_t s2, uint32_t b2) {
+    return hfma2(hsub2(v, magic), s2, b2);
+}
+
+template <int BITS> struct TcWords { static constexpr int N = BITS == 6 ? 12 : 8; };
+
 template <int BITS>
-__device__ __forceinline__ void dequant_quarter(uint32_t w_row, int row, int quarter, uint32_t s_pair,
+__device__ __forceinline__ void load_quarter(uint32_t w_row, int row, int quarter, uint32_t (&wd)[TcWords<BITS>::N]) {
+    if constexpr (BITS == 6) {  // 192-byte rows, no swizzle: 48 bytes
+#pragma unroll
+        for (int cc = 0; cc < 3; ++cc) {
+            const uint4 v = lds_v4(w_row + uint32_t(quarter * 48 + cc * 16));
+            wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
+        }
+    } else {  // 128-byte rows, 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r & 7)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * quarter + cc;
+            const uint4 v = lds_v4(w_row + uint32_t((c ^ (row & 7)) << 4));
+            wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
+        }
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ void dequant_quarter(const uint32_t (&wd)[TcWords<BITS>::N], uint32_t s_pair,
                                                 uint32_t b_pair, int two_groups, int sel,
                                                 uint32_t (&out)[TcFmt<BITS, 16>::COLS]) {
     uint32_t s_lo, b_lo, s_hi, b_hi;
@@ -158,60 +186,32 @@ __device__ __forceinline__ void dequant_quarter(uint32_t w_row, int row, int qua
         b_lo = b_hi = __byte_perm(b_pair, 0u, ps);
     }
     if constexpr (BITS == 4) {
-        // 128-byte rows, 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r & 7).
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * quarter + cc;
-            const uint4 v = lds_v4(w_row + uint32_t((c ^ (row & 7)) << 4));
-            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-            const uint32_t s2 = cc ? s_hi : s_lo, b2 = cc ? b_hi : b_lo;
-#pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t t = __byte_perm(wd[wi], 0u, 0x4040u | uint32_t(j) | (uint32_t(j) << 8));
-                    const uint32_t h = (t & 0x00F0000Fu) | kMagic1024x2;
-                    const uint32_t q = hfma2(h, kOneSixteenth, kMinus1024_64);
-                    out[cc * 16 + wi * 4 + j] = hfma2(q, s2, b2);
-                }
-            }
+        for (int wi = 0; wi < 8; ++wi) {
+            const uint32_t s2 = wi < 4 ? s_lo : s_hi, b2 = wi < 4 ? b_lo : b_hi;
+            const uint32_t v = wd[wi], v8 = v >> 8;
+            out[wi * 4 + 0] = fold((v & 0x000F000Fu) | kM1024x2, kM1024x2, s2, b2);
+            out[wi * 4 + 1] = fold((v & 0x00F000F0u) | kM64x2, kM64x2, s2, b2);
+            out[wi * 4 + 2] = fold((v8 & 0x000F000Fu) | kM1024x2, kM1024x2, s2, b2);
+            out[wi * 4 + 3] = fold((v8 & 0x00F000F0u) | kM64x2, kM64x2, s2, b2);
         }
     } else if constexpr (BITS == 8) {
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * quarter + cc;
-            const uint4 v = lds_v4(w_row + uint32_t((c ^ (row & 7)) << 4));
-            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const uint32_t h = __byte_perm(wd[wi], 0x64646464u, j ? 0x4342u : 0x4140u);
-                    const uint32_t q = hfma2(h, kOnes, kMinus1024x2);
-                    out[cc * 8 + wi * 2 + j] = hfma2(q, s_lo, b_lo);
-                }
-            }
+        for (int wi = 0; wi < 8; ++wi) {
+            out[wi * 2 + 0] = fold(__byte_perm(wd[wi], 0x64646464u, 0x4140u), kM1024x2, s_lo, b_lo);
+            out[wi * 2 + 1] = fold(__byte_perm(wd[wi], 0x64646464u, 0x4342u), kM1024x2, s_lo, b_lo);
         }
     } else {
-        // 192-byte rows, no swizzle; the thread's 48 bytes are 4 triplets of 16 codes.
-        uint32_t wd[12];
-#pragma unroll
-        for (int cc = 0; cc < 3; ++cc) {
-            const uint4 v = lds_v4(w_row + uint32_t(quarter * 48 + cc * 16));
-            wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
-        }
 #pragma unroll
         for (int tr = 0; tr < 4; ++tr) {
             const uint32_t A = wd[3 * tr], B = wd[3 * tr + 1], C = wd[3 * tr + 2];
-            const uint32_t f[8] = {A, A >> 12, __funnelshift_r(A, B, 24), B >> 4,
-                                   B >> 16, __funnelshift_r(B, C, 28), C >> 8, C >> 20};
             const uint32_t s2 = tr < 2 ? s_lo : s_hi, b2 = tr < 2 ? b_lo : b_hi;
+            const uint32_t fa[6] = {A, A >> 6, __funnelshift_r(A, B, 12), B >> 4, __funnelshift_r(B, C, 10),
+                                    __funnelshift_r(B, C, 16)};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t h = (f[j] & 0x3Fu) | ((f[j] << 10) & 0x3F0000u) | kMagic1024x2;
-                const uint32_t q = hfma2(h, kOnes, kMinus1024x2);
-                out[tr * 8 + j] = hfma2(q, s2, b2);
-            }
+            for (int i = 0; i < 6; ++i) out[tr * 8 + i] = fold((fa[i] & 0x00FC003Fu) | kM1024_256, kM1024_256, s2, b2);
+            out[tr * 8 + 6] = fold(((C >> 4) & 0x003F03F0u) | kM64_1024, kM64_1024, s2, b2);
+            out[tr * 8 + 7] = fold(((C >> 10) & 0x003F03F0u) | kM64_1024, kM64_1024, s2, b2);
         }
     }
 }
@@ -227,12 +227,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const TcSmemLayout L = tc_layout(XS, F::W_BYTES, p.ring, F::NA);
     const int S = L.ring;
     const uint32_t sbase = smem_addr(smem);
-    const uint32_t bar_full = sbase + L.bar_off;              // [S]
-    const uint32_t bar_empty = bar_full + 8 * S;               // [S]
-    const uint32_t bar_afull = bar_empty + 8 * S;              // [NA]
+    // Codes and x tiles have rings of their own: a code slot is free as soon as the
+    // dequantizers have read it, an x slot only when the MMAs that read it have completed.
+    const uint32_t bar_full = sbase + L.bar_off;              // [S] codes landed
+    const uint32_t bar_empty = bar_full + 8 * S;               // [S] codes read
+    const uint32_t bar_xfull = bar_empty + 8 * S;              // [S] x tile landed
+    const uint32_t bar_xempty = bar_xfull + 8 * S;             // [S] x tile consumed by the MMAs
+    const uint32_t bar_afull = bar_xempty + 8 * S;             // [NA]
     const uint32_t bar_aempty = bar_afull + 8 * F::NA;         // [NA]
     const uint32_t bar_acc = bar_aempty + 8 * F::NA;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.bar_off + 8 * (2 * S + 2 * F::NA + 1));
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.bar_off + 8 * (4 * S + 2 * F::NA + 1));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -253,7 +257,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(bar_full + 8 * i, 1);
-            mbar_init(bar_empty + 8 * i, TC_NDQ + TC_NMMA);
+            mbar_init(bar_empty + 8 * i, TC_NDQ);
+            mbar_init(bar_xfull + 8 * i, 1);
+            mbar_init(bar_xempty + 8 * i, TC_NMMA);
         }
         for (int i = 0; i < F::NA; ++i) {
             mbar_init(bar_afull + 8 * i, TC_NDQ);
@@ -280,40 +286,57 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        // lane 0 streams the code tiles (TMA), lane 1 the x tiles (bulk copies); each runs
+        // ahead as far as its own ring allows.
         if (lane == 0) {
             constexpr int WCOLS = F::ROW_BYTES / 4;
-            const uint32_t stage_tx = uint32_t(F::W_BYTES + XS);
-            const uint8_t* xt = reinterpret_cast<const uint8_t*>(p.xt);
-            const int pre = p.static_w ? min(S, nst) : 0;
-            // codes of the first stages do not depend on earlier kernels when weights are static
-            for (int i = 0; i < pre; ++i) {
-                TC_TRACE(0, i);
-                mbar_arrive_expect_tx(bar_full + 8 * i, stage_tx);
-                tma_load_2d(sbase + L.w_off + i * L.w_stage, &wmap, bar_full + 8 * i, (st0 + i) * WCOLS, n0);
-            }
-            grid_dependency_wait();
+            // codes never depend on earlier kernels when the weights are static
+            if (!p.static_w) grid_dependency_wait();
             deadline = clock64() + TC_TIMEOUT_CYCLES;
-            for (int i = 0; i < pre; ++i)
-                bulk_load(sbase + L.x_off + i * L.x_stage, xt + size_t(st0 + i) * XS, XS, bar_full + 8 * i);
-            int issued = pre;
-            for (int i = pre; i < nst; ++i) {
-                const int s = i % S;
-                if (i >= S && !mbar_wait(bar_empty + 8 * s, ((i / S) & 1) ^ 1, deadline)) {
+            int issued = 0, s = 0;
+            uint32_t ph = 0;
+            for (int i = 0; i < nst; ++i) {
+                if (i >= S && !mbar_wait(bar_empty + 8 * s, ph ^ 1u, deadline)) {
                     set_error(1u);
                     *abort_flag = 1;
                     break;
                 }
                 if (*abort_flag) break;
                 TC_TRACE(0, i);
-                mbar_arrive_expect_tx(bar_full + 8 * s, stage_tx);
+                mbar_arrive_expect_tx(bar_full + 8 * s, uint32_t(F::W_BYTES));
                 tma_load_2d(sbase + L.w_off + s * L.w_stage, &wmap, bar_full + 8 * s, (st0 + i) * WCOLS, n0);
-                bulk_load(sbase + L.x_off + s * L.x_stage, xt + size_t(st0 + i) * XS, XS, bar_full + 8 * s);
                 issued = i + 1;
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
-            // drain: every issued stage's copy must land before the block may exit
+            // drain: every issued copy must land before the block may exit
             const long long drain_deadline = clock64() + TC_TIMEOUT_CYCLES;
             for (int i = max(0, issued - S); i < issued; ++i)
                 if (!mbar_wait(bar_full + 8 * (i % S), (i / S) & 1, drain_deadline)) set_error(1u);
+        } else if (lane == 1) {
+            const uint8_t* xt = reinterpret_cast<const uint8_t*>(p.xt);
+            int issued = 0, s = 0;
+            uint32_t ph = 0;
+            for (int i = 0; i < nst; ++i) {
+                if (i >= S && !mbar_wait(bar_xempty + 8 * s, ph ^ 1u, deadline)) {
+                    set_error(1u);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                mbar_arrive_expect_tx(bar_xfull + 8 * s, uint32_t(XS));
+                bulk_load(sbase + L.x_off + s * L.x_stage, xt + size_t(st0 + i) * XS, XS, bar_xfull + 8 * s);
+                issued = i + 1;
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            const long long drain_deadline = clock64() + TC_TIMEOUT_CYCLES;
+            for (int i = max(0, issued - S); i < issued; ++i)
+                if (!mbar_wait(bar_xfull + 8 * (i % S), (i / S) & 1, drain_deadline)) set_error(1u);
         }
     } else if (warp < TC_DQ0) {
         // ------------------------------------------------------------ MMA issuers
@@ -324,11 +347,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int j = warp - 1;
         constexpr uint32_t idesc = idesc_f16_f32(TC_ROWS, MP);
         const uint32_t dcol = tmem + uint32_t(j * MP);
+        int s = 0, a = 0;
+        uint32_t ph = 0, pa = 0;
         for (int i = 0; i < nst; ++i) {
-            const int s = i % S, a = i % F::NA;
-            const bool got_full = mbar_wait(bar_full + 8 * s, (i / S) & 1, deadline);
+            const bool got_full = mbar_wait(bar_xfull + 8 * s, ph, deadline);
             if (j == 0 && lane == 0) TC_TRACE(10, i);
-            if (!got_full || !mbar_wait(bar_afull + 8 * a, (i / F::NA) & 1, deadline)) {
+            if (!got_full || !mbar_wait(bar_afull + 8 * a, pa, deadline)) {
                 if (lane == 0) {
                     set_error(1u);
                     *abort_flag = 1;
@@ -345,11 +369,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     const uint64_t bdesc = smem_desc_sw128(xs + (kk >> 2) * (MP * 128) + (kk & 3) * 32, 1024);
                     umma_f16_ts(dcol, acol + kk * 8, bdesc, idesc, (i > 0 || kk > j) ? 1u : 0u);
                 }
-                umma_commit(bar_empty + 8 * s);
+                umma_commit(bar_xempty + 8 * s);
                 umma_commit(bar_aempty + 8 * a);
             }
             __syncwarp();
             if (j == 0 && lane == 0) TC_TRACE(2, i);
+            if (++s == S) {
+                s = 0;
+                ph ^= 1u;
+            }
+            if (++a == F::NA) {
+                a = 0;
+                pa ^= 1u;
+            }
         }
         if (elect_one()) umma_commit(bar_acc);  // fires once every MMA issued above has completed
         __syncwarp();
@@ -379,27 +411,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < TC_SPF; ++i) issue_scales(i);
 
+        int s = 0, a = 0;
+        uint32_t ph = 0, pa = 0;
         for (int i = 0; i < nst; ++i) {
-            const int s = i % S, a = i % F::NA;
-            if (!mbar_wait(bar_full + 8 * s, (i / S) & 1, deadline)) {
+            if (!mbar_wait(bar_full + 8 * s, ph, deadline)) {
                 set_error(1u);
                 *abort_flag = 1;
                 break;
             }
             if (warp == TC_DQ0 && lane == 0) TC_TRACE(3, i);
+            // the thread's codes into registers; the code slot is free again at once
+            uint32_t wd[TcWords<BITS>::N];
+            load_quarter<BITS>(sbase + L.w_off + s * L.w_stage + row * F::ROW_BYTES, row, quarter, wd);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_empty + 8 * s);
             cp_async_wait<TC_SPF - 1>();
             const uint32_t sp = sc_base + uint32_t(i % TC_SPF) * (TC_NDQ * 32 * 8);
             uint32_t s_pair, b_pair;
             asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(s_pair), "=r"(b_pair) : "r"(sp));
             const int k = (st0 + i) * F::KC + quarter * F::U;
             uint32_t vals[F::COLS];
-            dequant_quarter<BITS>(sbase + L.w_off + s * L.w_stage + row * F::ROW_BYTES, row, quarter, s_pair,
-                                  b_pair, two_groups, (k >> p.gshift) & 1, vals);
-            __syncwarp();
+            dequant_quarter<BITS>(wd, s_pair, b_pair, two_groups, (k >> p.gshift) & 1, vals);
             if (warp == TC_DQ0 && lane == 0) TC_TRACE(4, i);
-            if (lane == 0) mbar_arrive(bar_empty + 8 * s);   // codes of stage s consumed
             issue_scales(i + TC_SPF);
-            if (i >= F::NA && !mbar_wait(bar_aempty + 8 * a, ((i / F::NA) & 1) ^ 1, deadline)) {
+            if (i >= F::NA && !mbar_wait(bar_aempty + 8 * a, pa ^ 1u, deadline)) {
                 set_error(1u);
                 *abort_flag = 1;
                 break;
@@ -416,6 +451,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             __syncwarp();
             if (warp == TC_DQ0 && lane == 0) TC_TRACE(6, i);
             if (lane == 0) mbar_arrive(bar_afull + 8 * a);
+            if (++s == S) {
+                s = 0;
+                ph ^= 1u;
+            }
+            if (++a == F::NA) {
+                a = 0;
+                pa ^= 1u;
+            }
         }
         cp_async_wait<0>();
     }
@@ -533,12 +576,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 // ---------------------------------------------------------------- activations -> stage tiles
 // One block per padded token row m (MP blocks).  Writes x'[stage][m][k] (fp16) in the layout
 // the MMA reads: per stage, KC/64 swizzle atoms of [MP rows x 128 B], 16-byte chunk c of row m
-// at chunk c ^ (m & 7).  Rows m >= M and columns k >= K are zero.  bf16 rows are scaled by
-// 2^-E_m, E_m = max(0, e - 141) where max|x[m,:]| < 2^(e-126), so every value fits fp16.
-template <int KC>
+// at chunk c ^ (m & 7); within each block of 8 (4/8-bit) or 16 (6-bit) K positions the values
+// are permuted into the code-pair order of the dequantizers (perm_src).  Rows m >= M and
+// columns k >= K are zero.  bf16 rows are scaled by 2^-E_m, E_m = max(0, e - 141) where
+// max|x[m,:]| < 2^(e-126), so every value fits fp16.
+template <int KC, int BITS>
 __global__ void __launch_bounds__(256) xprep_kernel(const uint16_t* __restrict__ x, int M, int K, int is_bf16,
                                                     int MP, int nst, uint16_t* __restrict__ xt,
                                                     int* __restrict__ xexp) {
+    constexpr int UN = BITS == 6 ? 16 : 8;  // K positions per permutation block
     __shared__ float red[8];
     grid_dependents_launch();
     grid_dependency_wait();
@@ -566,22 +612,43 @@ __global__ void __launch_bounds__(256) xprep_kernel(const uint16_t* __restrict__
     }
     if (threadIdx.x == 0 && m < M && xexp) xexp[m] = E;
     const float sc = exp2i(-E);
-    const int nchunks = nst * (KC / 8);
-    for (int u = threadIdx.x; u < nchunks; u += 256) {
-        const int k = u * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (m < M && k < K) {
-            v = ldg_nc_v4(xr + k);
-            if (is_bf16) {
-                v.x = f32x2_to_f16x2(bf16lo_to_f32(v.x) * sc, bf16hi_to_f32(v.x) * sc);
-                v.y = f32x2_to_f16x2(bf16lo_to_f32(v.y) * sc, bf16hi_to_f32(v.y) * sc);
-                v.z = f32x2_to_f16x2(bf16lo_to_f32(v.z) * sc, bf16hi_to_f32(v.z) * sc);
-                v.w = f32x2_to_f16x2(bf16lo_to_f32(v.w) * sc, bf16hi_to_f32(v.w) * sc);
+    const int nunits = nst * (KC / UN);
+    for (int u = threadIdx.x; u < nunits; u += 256) {
+        const int k = u * UN;
+        float f[UN];
+#pragma unroll
+        for (int i = 0; i < UN; ++i) f[i] = 0.f;
+        if (m < M && k < K) {  // K is a multiple of 32, so a unit is all in or all out
+#pragma unroll
+            for (int h = 0; h < UN / 8; ++h) {
+                const uint4 v = ldg_nc_v4(xr + k + 8 * h);
+                const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (is_bf16) {
+                        f[8 * h + 2 * i] = bf16lo_to_f32(r[i]) * sc;
+                        f[8 * h + 2 * i + 1] = bf16hi_to_f32(r[i]) * sc;
+                    } else {
+                        const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
+                        f[8 * h + 2 * i] = t.x;
+                        f[8 * h + 2 * i + 1] = t.y;
+                    }
+                }
             }
         }
-        const int st = k / KC, kk = k % KC, atom = kk / 64, c = (kk % 64) / 8;
-        const int64_t off = int64_t(st) * MP * KC + int64_t(atom) * MP * 64 + int64_t(m) * 64 + ((c ^ (m & 7)) * 8);
-        *reinterpret_cast<uint4*>(xt + off) = v;
+#pragma unroll
+        for (int h = 0; h < UN / 8; ++h) {
+            uint4 o;
+            uint32_t* ov = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                ov[i] = f32x2_to_f16x2(f[perm_src<BITS>(8 * h + 2 * i)], f[perm_src<BITS>(8 * h + 2 * i + 1)]);
+            const int kh = k + 8 * h;
+            const int st = kh / KC, kk = kh % KC, atom = kk / 64, c = (kk % 64) / 8;
+            const int64_t off =
+                int64_t(st) * MP * KC + int64_t(atom) * MP * 64 + int64_t(m) * 64 + ((c ^ (m & 7)) * 8);
+            *reinterpret_cast<uint4*>(xt + off) = o;
+        }
     }
 }
 
@@ -730,8 +797,9 @@ cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) 
     pc.stream = stream;
     pc.attrs = &pdl_attr;
     pc.numAttrs = c.pdl ? 1 : 0;
-    e = KC == 256 ? cudaLaunchKernelEx(&pc, xprep_kernel<256>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
-                  : cudaLaunchKernelEx(&pc, xprep_kernel<128>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp);
+    e = a.bits == 4   ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 4>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
+        : a.bits == 6 ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 6>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
+                      : cudaLaunchKernelEx(&pc, xprep_kernel<128, 8>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp);
     if (e != cudaSuccess) return finish(e);
 
     CUtensorMap wmap;
@@ -918,8 +986,9 @@ cudaError_t launch_tc_noalloc(const QmmArgs& a, const TcConfig& c, cudaStream_t 
     pc.stream = stream;
     pc.attrs = &pdl_attr;
     pc.numAttrs = c.pdl ? 1 : 0;
-    e = KC == 256 ? cudaLaunchKernelEx(&pc, xprep_kernel<256>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
-                  : cudaLaunchKernelEx(&pc, xprep_kernel<128>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp);
+    e = a.bits == 4   ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 4>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
+        : a.bits == 6 ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 6>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
+                      : cudaLaunchKernelEx(&pc, xprep_kernel<128, 8>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp);
     if (e != cudaSuccess) return e;
 
     CUtensorMap wmap;
