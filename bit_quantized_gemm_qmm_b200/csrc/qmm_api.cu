@@ -110,6 +110,7 @@ qmm_status validate_qmm(const void* x, const uint32_t* packed, const uint16_t* s
 bool prefer_tc(int64_t M, int64_t N, int64_t K) {
     if (N >= 8192 && N * K <= (int64_t(1) << 27)) return true;  // gate/up-like: wide N, moderate size
     if (N * K >= (int64_t(1) << 25)) return M >= 9;             // >= 32M codes (down, LM head)
+    if (N * K < (int64_t(1) << 23)) return M >= 24;             // k/v-like: < 8M codes
     return M >= 33;
 }
 
