@@ -3,6 +3,7 @@
 // Entry points and their contracts are documented in include/qmm.h.  Every check happens
 // on the host before anything is launched; there is no fallback path: a shape or format the
 // kernels do not handle returns QMM_ERR_UNSUPPORTED.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -162,10 +163,16 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
     if (p.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS))
         return fail(QMM_ERR_INVALID_ARG, "unknown plan flags 0x%x", p.flags);
     const bool tc_ok = tc_supported(M, N, K, bits, group) && aligned(scales, 4) && aligned(biases, 4);
-    const bool st_ok = stream_supported(M, N, K, bits, group) && aligned(scales, 16) && aligned(biases, 16) &&
-                       stream_config(M, N, K, bits, group, p.split).ring >= 2;
+    const bool st_shape = stream_supported(M, N, K, bits, group) && aligned(scales, 16) && aligned(biases, 16);
+    StreamConfig stc = {};
+    if (st_shape) stc = stream_config(M, N, K, bits, group, p.split);
+    const bool st_ok = stc.ring >= 2;
     if (p.kernel == QMM_KERNEL_AUTO) {
-        if (st_ok && M <= 8) p.kernel = QMM_KERNEL_STREAM;
+        // the streaming kernel up to M = 8, and up to 16 while staging x still leaves room
+        // for a 4-stage ring (or for all the stages a block streams) without splitting K
+        // further than the tile count asks for
+        if (st_ok && (M <= 8 || (!stc.split_raised && stc.ring >= std::min(4, stc.stages))))
+            p.kernel = QMM_KERNEL_STREAM;
         else p.kernel = (tc_ok && prefer_tc(M, N, K)) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
     }
     if (p.kernel == QMM_KERNEL_STREAM && !st_ok)

@@ -68,6 +68,8 @@ struct StreamConfig {
     int split;     // K slices = cluster size along grid.y
     int kslice;    // K codes per slice
     int ring;      // shared-memory stages (0: the shape does not fit this kernel)
+    int stages;    // K stages each block streams per tile
+    bool split_raised;  // K split beyond the tile-count choice only to make x fit
     int grid_x;    // blocks along N (persistent when split == 1)
     int ncw;       // consumer warps per block (8 or 16)
     size_t smem;   // dynamic shared memory per block

@@ -86,7 +86,10 @@ struct StLayout {
     uint32_t w_stage, sb_off, sb_slot, x_off, xrs, xg_off, gpad, xf_off, red_off, bar_off, total;
 };
 
-__host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split, int ncw) {
+// x and its group sums are staged for the M real token rows only (reads for token rows >= M
+// are redirected to row M-1: they feed accumulator columns that are never stored).
+__host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split, int ncw,
+                                              int mrows) {
     StLayout L;
     L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 256));  // 24 or 32 KB
     L.sb_off = uint32_t(ring) * L.w_stage;
@@ -94,10 +97,10 @@ __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int ks
     uint32_t off = L.sb_off + ST_SS * L.sb_slot;
     L.x_off = off;
     L.xrs = uint32_t(kslice / 8 + kXPad);                     // 16-byte chunks per staged x row
-    off += uint32_t(8 * mt) * L.xrs * 16;
+    off += uint32_t(mrows) * L.xrs * 16;
     L.xg_off = off;
     L.gpad = uint32_t((kslice / group + 7) / 8 * 8);
-    off += uint32_t(8 * mt) * L.gpad * 4;
+    off += uint32_t(mrows) * L.gpad * 4;
     L.xf_off = off;                                           // K-half partials: [8 warps][32][4*MT]
     if (ncw == 16) off += uint32_t(8 * 32 * 4 * mt * 4);
     L.red_off = off;
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ float s_red[NCW];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const StLayout L = st_layout(BITS, MT, p.ring, p.kslice, p.group, p.split, NCW);
+    const StLayout L = st_layout(BITS, MT, p.ring, p.kslice, p.group, p.split, NCW, p.M);
     const int S = p.ring;
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar_full = sbase + L.bar_off;
@@ -292,10 +295,11 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         consumer_sync<NCW>();
         grid_dependents_launch();
 
-        const uint32_t xmt = 8 * L.xrs * 16;
-        const uint32_t xlane = xs + uint32_t(g * int(L.xrs) + c) * 16u + uint32_t(hbase * SPH * KSS * 2);
-        const uint32_t xgrow = xg + uint32_t(g * int(L.gpad)) * 4u;
-        const uint32_t xg_mt = 8 * L.gpad * 4;
+        const int tr0 = min(g, p.M - 1), tr1 = min(g + 8, p.M - 1);  // token rows of the two x tiles
+        const uint32_t xmt = uint32_t(tr1 - tr0) * L.xrs * 16;
+        const uint32_t xlane = xs + uint32_t(tr0 * int(L.xrs) + c) * 16u + uint32_t(hbase * SPH * KSS * 2);
+        const uint32_t xgrow = xg + uint32_t(tr0 * int(L.gpad)) * 4u;
+        const uint32_t xg_mt = uint32_t(tr1 - tr0) * L.gpad * 4;
         float* xf = reinterpret_cast<float*>(smem + L.xf_off) + (rg * 32 + lane) * 4 * MT;
         const float yscale = exp2i(E);
         // ring position (slot s, phase ph) and scale-block position (slot ss, phase sph) advance
@@ -502,8 +506,8 @@ constexpr int kNumSM = 148;
 constexpr size_t kMaxSmem = 226 * 1024;  // dynamic, per block (static shared memory is tiny)
 constexpr size_t kSmSmem = 228 * 1024;   // per SM (including 1 KB reserved per block)
 
-size_t st_smem(int bits, int mt, int ring, int kslice, int group, int split, int ncw) {
-    return size_t(st_layout(bits, mt, ring, kslice, group, split, ncw).total) + 1024;  // + alignment slack
+size_t st_smem(int bits, int mt, int ring, int kslice, int group, int split, int ncw, int mrows) {
+    return size_t(st_layout(bits, mt, ring, kslice, group, split, ncw, mrows).total) + 1024;  // + alignment slack
 }
 
 }  // namespace
@@ -540,6 +544,7 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         }
     }
     split = std::max(1, std::min(8, split));
+    const int split0 = split;
     for (;; ++split) {
         const int kslice = rup(cdiv(K, split), unit);
         const int sp = cdiv(K, kslice);
@@ -551,8 +556,8 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         // 16 consumer warps measured faster than 8 on every configuration of the sweep (the
         // 8-warp blocks fit two to an SM, but that bought no overlap between calls)
         const int ncw = 16;
-        while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp, ncw) > kMaxSmem) --ring;
-        const bool fits = st_smem(bits, c.mt, ring, kslice, group, sp, ncw) <= kMaxSmem;
+        while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M)) > kMaxSmem) --ring;
+        const bool fits = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M)) <= kMaxSmem;
         if (!fits || (ring < std::min(want, 3) && split < 8)) {
             if (split < 8) continue;
             c.ring = 0;  // does not fit: the caller uses another kernel
@@ -561,8 +566,10 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         c.split = sp;
         c.kslice = kslice;
         c.ring = ring;
+        c.stages = nst;
+        c.split_raised = split > split0;
         c.ncw = ncw;
-        c.smem = st_smem(bits, c.mt, ring, kslice, group, sp, ncw);
+        c.smem = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M));
         const int per_sm = std::max(1, int(kSmSmem / (c.smem + 1024)));
         c.grid_x = sp > 1 ? T : std::min(T, kNumSM * per_sm);
         return c;

@@ -88,7 +88,7 @@ def test_plans(L):
         p = q.plan_default(M, 4096, 14336, 4, 64, f16)
         assert p.kernel == q.KERNEL_STREAM and 1 <= p.split <= 8
     assert q.plan_default(4, 151936, 4096, 4, 64, f16).split == 1  # enough tiles: no split
-    assert q.plan_default(9, 4096, 4096, 4, 64, f16).kernel != q.KERNEL_STREAM
+    assert q.plan_default(17, 4096, 4096, 4, 64, f16).kernel != q.KERNEL_STREAM
     assert q.plan_default(4, 4096, 4096 + 64, 4, 64, f16).kernel != q.KERNEL_STREAM
     st = q.make_plan(kernel=q.KERNEL_STREAM)
     assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(st), None) == q.QMM_ERR_UNSUPPORTED
