@@ -104,4 +104,25 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
 // 2^e as float for -126 <= e <= 127.
 __device__ __forceinline__ float exp2i(int e) { return __uint_as_float(uint32_t(e + 127) << 23); }
 
+// Sum of one float from each block of a cluster (ranks 0..n-1, n <= 16), added in rank order so
+// the result does not depend on timing.  The remote loads are all issued before the first add.
+__device__ __forceinline__ float cluster_sum_in_order(const float* local, int n) {
+    float v[16];
+    const uint32_t la = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        v[q] = 0.f;
+        if (q < n) {
+            uint32_t ra;
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(la), "r"(uint32_t(q)));
+            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v[q]) : "r"(ra));
+        }
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+        if (q < n) sum += v[q];
+    return sum;
+}
+
 }  // namespace qmm_impl

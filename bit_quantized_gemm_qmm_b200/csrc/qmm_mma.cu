@@ -255,8 +255,7 @@ __global__ void __launch_bounds__(NWARP * 32, 8 / NWARP * 2) qmm_mma_kernel(cons
     for (int e = threadIdx.x; e < nrows * ncols; e += NTHREADS) {
         const int col = e / nrows, row = rlo + (e - col * nrows);
         const int n = blockIdx.x * R + row;
-        float sum = 0.f;
-        for (int q = 0; q < p.split; ++q) sum += cluster.map_shared_rank(red, q)[col * R + row];
+        const float sum = cluster_sum_in_order(red + col * R + row, p.split);
         if (n < p.N)
             p.y[int64_t(col) * p.N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sum))
                                                     : __half_as_ushort(__float2half_rn(sum));

@@ -470,8 +470,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         for (int e = threadIdx.x; e < nrows * ncols; e += StWarps<NCW>::THREADS) {
             const int col = e / nrows, row = rlo + (e - col * nrows);
             const int n = t * ST_ROWS + row;
-            float sum = 0.f;
-            for (int q = 0; q < p.split; ++q) sum += cluster.map_shared_rank(red, q)[col * ST_ROWS + row];
+            const float sum = cluster_sum_in_order(red + col * ST_ROWS + row, p.split);
             if (n < p.N && ok)
                 p.y[int64_t(col) * p.N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sum))
                                                         : __half_as_ushort(__float2half_rn(sum));

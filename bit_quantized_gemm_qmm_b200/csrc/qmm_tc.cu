@@ -549,8 +549,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int nrows = rhi - rlo, ncols = min(MP, p.M);
         for (int e = threadIdx.x; e < nrows * ncols; e += TC_THREADS) {
             const int col = e / nrows, r = rlo + (e - col * nrows);
-            float sum = 0.f;
-            for (int z = 0; z < p.split; ++z) sum += cluster.map_shared_rank(red, z)[col * TC_ROWS + r];
+            const float sum = cluster_sum_in_order(red + col * TC_ROWS + r, p.split);
             const int nn = n0 + r;
             if (nn < p.N)
                 p.y[int64_t(col) * p.N + nn] = p.out_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sum))
