@@ -321,14 +321,15 @@ def run_e2e(wl, weights, plans, dev, steps):
     hy = {M: torch.empty((S, M, wl.N), dtype=wl.dtype).pin_memory() for M in BENCH_MS}
     dx = {M: torch.empty((M, wl.K), dtype=wl.dtype, device=dev) for M in BENCH_MS}
     dy = {M: torch.empty((S, M, wl.N), dtype=wl.dtype, device=dev) for M in BENCH_MS}
+    outs = {M: list(dy[M].unbind(0)) for M in BENCH_MS}  # each call's own output slice
     stream = torch.cuda.current_stream(dev)
 
     def one_step():
         for M in BENCH_MS:
             dx[M].copy_(hx[M], non_blocking=True)
         for M in BENCH_MS:
-            for i, (P, S_, B) in enumerate(weights):
-                q.qmm(dx[M], P, S_, B, wl.bits, wl.group, out=dy[M][i], plan=plans[M])
+            for (P, S_, B), y in zip(weights, outs[M]):
+                q.qmm(dx[M], P, S_, B, wl.bits, wl.group, out=y, plan=plans[M])
         for M in BENCH_MS:
             hy[M].copy_(dy[M], non_blocking=True)
         stream.synchronize()

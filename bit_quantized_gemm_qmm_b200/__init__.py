@@ -169,28 +169,73 @@ def make_plan(kernel: int = KERNEL_AUTO, split: int = 0, warps: int = 0, flags: 
     return p
 
 
+_call = None
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _caller():
+    """The C hand-off of qmm() (module _qmm_call), bound to the loaded library's qmm_ex."""
+    global _call
+    if _call is None:
+        L = lib()
+        try:
+            from . import _qmm_call
+        except ImportError as e:
+            raise QmmUnavailable(f"the _qmm_call module is missing ({e}); run __graft_entry__.build()") from e
+        _qmm_call.bind(ctypes.cast(L.qmm_ex, ctypes.c_void_p).value)
+        _call = _qmm_call.qmm_ex
+    return _call
+
+
+def _current_stream(dev_index: int) -> int:
+    if _raw_stream is not None:
+        return _raw_stream(dev_index)
+    return torch.cuda.current_stream(dev_index).cuda_stream
+
+
 def qmm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
         bits: int, group: int, out: torch.Tensor | None = None, plan: Plan | None = None):
-    """y[M,N] = x[M,K] . dequant(packed, scales, biases)^T on the current CUDA stream."""
+    """y[M,N] = x[M,K] . dequant(packed, scales, biases)^T on the current CUDA stream.
+
+    The checks here guard what the C ABI cannot see (devices, contiguity, the arrays' sizes
+    and element types); the format, M and the pointers' alignment are checked by the library.
+    """
+    if not (x.is_cuda and packed.is_cuda and scales.is_cuda and biases.is_cuda):
+        raise ValueError("x, packed, scales and biases must be CUDA tensors")
+    dev = x.get_device()
+    if packed.get_device() != dev or scales.get_device() != dev or biases.get_device() != dev:
+        raise ValueError("all tensors must be on the same CUDA device")
+    if not (x.is_contiguous() and packed.is_contiguous() and scales.is_contiguous() and biases.is_contiguous()):
+        raise ValueError("tensors must be contiguous")
     if x.dim() != 2 or packed.dim() != 2:
         raise ValueError("x must be [M, K] and packed [N, K*bits/32]")
-    dev = _need_cuda(x, packed, scales, biases)
     M, K = x.shape
-    N = packed.shape[0]
-    if packed.shape[1] * 32 != K * bits:
-        raise ValueError(f"packed has {packed.shape[1]} words per row; K={K} at {bits} bits needs {K * bits // 32}")
-    if out is None:
-        out = torch.empty((M, N), dtype=x.dtype, device=dev)
-    elif out.shape != (M, N) or out.dtype != x.dtype:
-        raise ValueError("out must be [M, N] with x's dtype")
-    L = lib()
-    if plan is None:
-        st = L.qmm(_ptr(x), _ptr(packed), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, bits, group,
-                   _dtype_code(x.dtype), _stream(dev))
+    N, KW = packed.shape
+    if KW * 32 != K * bits:
+        raise ValueError(f"packed has {KW} words per row; K={K} at {bits} bits needs {K * bits // 32}")
+    if packed.element_size() != 4:
+        raise ValueError("packed must hold 32-bit words")
+    if scales.dtype is not torch.float16 or biases.dtype is not torch.float16:
+        raise ValueError("scales and biases must be fp16")
+    if group > 0 and K % group == 0 and (scales.numel() != N * (K // group) or biases.numel() != N * (K // group)):
+        raise ValueError(f"scales and biases must hold [N, K/group] = [{N}, {K // group}] values")
+    dt = x.dtype
+    if dt is torch.float16:
+        code = QMM_F16
+    elif dt is torch.bfloat16:
+        code = QMM_BF16
     else:
-        st = L.qmm_ex(_ptr(x), _ptr(packed), _ptr(scales), _ptr(biases), _ptr(out), M, N, K, bits, group,
-                      _dtype_code(x.dtype), ctypes.byref(plan), _stream(dev))
-    _check(st)
+        raise ValueError(f"unsupported activation dtype {dt} (fp16 or bf16)")
+    if out is None:
+        out = torch.empty((M, N), dtype=dt, device=x.device)
+    elif not (out.is_cuda and out.get_device() == dev and out.is_contiguous() and out.dtype is dt
+              and out.dim() == 2 and out.shape[0] == M and out.shape[1] == N):
+        raise ValueError("out must be a contiguous [M, N] CUDA tensor with x's dtype on x's device")
+    st = _caller()(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
+                   M, N, K, bits, group, code, 0 if plan is None else ctypes.addressof(plan),
+                   _current_stream(dev))
+    if st:
+        _check(st)
     return out
 
 

@@ -1,4 +1,5 @@
-"""Build the CUDA library in-tree: csrc/*.cu -> libqmm_b200.so (sm_100a only).
+"""Build the CUDA library in-tree: csrc/*.cu -> libqmm_b200.so (sm_100a only), and the small
+CPython module _qmm_call that hands each qmm() call to the library's C ABI.
 
 Each translation unit is compiled on its own (in parallel) and linked into one shared
 library with the CUDA runtime linked statically, so the .so loads on a host without a GPU
@@ -12,11 +13,14 @@ import os
 import shutil
 import subprocess
 import sys
+import sysconfig
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqmm_b200.so")
+CALL_SRC = os.path.join(HERE, "_qmm_call.c")
+CALL_LIB = os.path.join(HERE, "_qmm_call" + (sysconfig.get_config_var("EXT_SUFFIX") or ".so"))
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]
 
@@ -37,7 +41,23 @@ def _stale(srcs, target) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+def build_call_module(force: bool = False) -> str:
+    """gcc the CPython hand-off module (plain C against the interpreter's headers)."""
+    if not force and os.path.exists(CALL_LIB) and os.path.getmtime(CALL_LIB) >= max(
+            os.path.getmtime(CALL_SRC), os.path.getmtime(__file__)):
+        return CALL_LIB
+    cc = os.environ.get("CC") or shutil.which("gcc") or shutil.which("cc")
+    if not cc:
+        raise RuntimeError("no C compiler for the _qmm_call module")
+    tmp = CALL_LIB + ".tmp"
+    subprocess.check_call([cc, "-O2", "-shared", "-fPIC", "-Wall", "-Werror",
+                           "-I" + sysconfig.get_paths()["include"], CALL_SRC, "-o", tmp])
+    os.replace(tmp, CALL_LIB)
+    return CALL_LIB
+
+
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
+    build_call_module(force)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     if not force and not _stale(srcs, LIB):
         return LIB

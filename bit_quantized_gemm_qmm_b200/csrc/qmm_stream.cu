@@ -361,19 +361,30 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+                    // the scales of all steps of the stage first, then one vote for the stage:
+                    // a single branch keeps the steps' dequant and MMAs in one straight run
+                    uint32_t sv[HPW * SPH][2];
+                    bool big = false;
 #pragma unroll
                     for (int j = 0; j < HPW * SPH; ++j) {
                         // the lane's group within the current scale block
                         const uint32_t gl2 = uint32_t((sib * KS + lane_off[j]) >> p.gshift) * 2u;
-                        const uint32_t s0 = lds_u16(sbuf + rAg + gl2);
-                        const uint32_t s1 = lds_u16(sbuf + rBg + gl2);
-                        const RowConst C[2] = {row_const<BITS>(s0), row_const<BITS>(s1)};
-                        const bool big = ((s0 & 0x7FFFu) >= 0x5400u) | ((s1 & 0x7FFFu) >= 0x5400u);
-                        const uint32_t xa = xst + uint32_t(j * KSS * 2);
-                        if (__any_sync(0xffffffffu, big))
-                            step_mma<BITS, MT, true>(w[j], C, xa, xmt, acc);
-                        else
-                            step_mma<BITS, MT, false>(w[j], C, xa, xmt, acc);
+                        sv[j][0] = lds_u16(sbuf + rAg + gl2);
+                        sv[j][1] = lds_u16(sbuf + rBg + gl2);
+                        big |= ((sv[j][0] & 0x7FFFu) >= 0x5400u) | ((sv[j][1] & 0x7FFFu) >= 0x5400u);
+                    }
+                    if (__any_sync(0xffffffffu, big)) {
+#pragma unroll
+                        for (int j = 0; j < HPW * SPH; ++j) {
+                            const RowConst C[2] = {row_const<BITS>(sv[j][0]), row_const<BITS>(sv[j][1])};
+                            step_mma<BITS, MT, true>(w[j], C, xst + uint32_t(j * KSS * 2), xmt, acc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < HPW * SPH; ++j) {
+                            const RowConst C[2] = {row_const<BITS>(sv[j][0]), row_const<BITS>(sv[j][1])};
+                            step_mma<BITS, MT, false>(w[j], C, xst + uint32_t(j * KSS * 2), xmt, acc);
+                        }
                     }
                 }
                 if (++s == S) {

@@ -62,6 +62,41 @@ def test_qmm_rejects_before_launch(L, kw, status):
     assert L.qmm_last_error()
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=5), q.QMM_ERR_UNSUPPORTED),
+    (dict(M=65), q.QMM_ERR_UNSUPPORTED),
+    (dict(K=96), q.QMM_ERR_INVALID_ARG),
+    (dict(dtype=7), q.QMM_ERR_INVALID_ARG),
+    (dict(ptr=0), q.QMM_ERR_INVALID_ARG),
+    (dict(y=24), q.QMM_ERR_INVALID_ARG),
+    (dict(M=0, ptr=0, y=0, scales=0), q.QMM_OK),
+])
+def test_call_module_forwards_to_qmm_ex(L, kw, status):
+    """The C hand-off qmm() uses passes every argument through unchanged: the library gives
+    the same verdicts as through ctypes, with the default plan (address 0) and with a plan."""
+    call = q._caller()
+    a = dict(M=4, N=64, K=128, bits=4, group=64, dtype=0, ptr=16, y=16, scales=16)
+    a.update(kw)
+    args = (a["ptr"], a["ptr"], a["scales"], a["scales"], a["y"], a["M"], a["N"], a["K"], a["bits"], a["group"],
+            a["dtype"])
+    assert call(*args, 0, 0) == status
+    plan = q.make_plan(kernel=q.KERNEL_MMA)
+    assert call(*args, ctypes.addressof(plan), 0) == status
+    with pytest.raises(TypeError):
+        call(*args, 0)
+
+
+def test_python_qmm_checks_tensors(L):
+    """What the C ABI cannot see is checked in Python before any call: devices, sizes and
+    element types (CPU tensors here, so nothing reaches the library)."""
+    import torch
+    x = torch.zeros((4, 128), dtype=torch.float16)
+    P = torch.zeros((16, 16), dtype=torch.int32)
+    S = torch.zeros((16, 2), dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA"):
+        q.qmm(x, P, S, S, 4, 64)
+
+
 def test_empty_shapes_are_noops(L):
     # M == 0 or N == 0 returns before touching any pointer or the device
     assert _qmm(L, M=0, ptr=0, y=0, scales=0) == q.QMM_OK
