@@ -313,7 +313,8 @@ def run_ours(args, rank, world):
 def run_e2e(wl, weights, plans, dev, steps):
     """Each step through the Python API: the step's inputs (x for each M) go from pinned host
     memory to the device, every call of the step runs with its own output, and all outputs
-    come back to pinned host memory; the weights stay resident, as a model's do."""
+    come back to pinned host memory; the weights stay resident, as a model's do.  The outputs
+    of one M go back on a copy stream while the calls of the next M run."""
     import bit_quantized_gemm_qmm_b200 as q
     from bit_quantized_gemm_qmm_b200.inputs import x_input
     S = len(weights)
@@ -323,6 +324,8 @@ def run_e2e(wl, weights, plans, dev, steps):
     dy = {M: torch.empty((S, M, wl.N), dtype=wl.dtype, device=dev) for M in BENCH_MS}
     outs = {M: list(dy[M].unbind(0)) for M in BENCH_MS}  # each call's own output slice
     stream = torch.cuda.current_stream(dev)
+    copy_stream = torch.cuda.Stream(dev)
+    done = {M: torch.cuda.Event() for M in BENCH_MS}
 
     def one_step():
         for M in BENCH_MS:
@@ -330,8 +333,11 @@ def run_e2e(wl, weights, plans, dev, steps):
         for M in BENCH_MS:
             for (P, S_, B), y in zip(weights, outs[M]):
                 q.qmm(dx[M], P, S_, B, wl.bits, wl.group, out=y, plan=plans[M])
-        for M in BENCH_MS:
-            hy[M].copy_(dy[M], non_blocking=True)
+            done[M].record(stream)
+            copy_stream.wait_event(done[M])
+            with torch.cuda.stream(copy_stream):
+                hy[M].copy_(dy[M], non_blocking=True)
+        copy_stream.synchronize()
         stream.synchronize()
 
     one_step()
