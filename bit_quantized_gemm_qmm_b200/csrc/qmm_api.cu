@@ -112,7 +112,8 @@ bool prefer_tc(int64_t M, int64_t N, int64_t K) {
     if (N >= 8192 && N * K <= (int64_t(1) << 27)) return true;  // gate/up-like: wide N, moderate size
     if (N * K >= (int64_t(1) << 25)) return M >= 9;             // >= 32M codes (down, LM head)
     if (N * K < (int64_t(1) << 23)) return M >= 24;             // k/v-like: < 8M codes
-    return M >= 33;
+    return M >= 28;  // q/o-like: the tensor-core kernel's time is flat over M = 17..32 (one
+                     // 32-column tile) while the warp-tile kernel's grows; they cross near 28
 }
 
 struct Resolved {
@@ -170,8 +171,11 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
     if (p.kernel == QMM_KERNEL_AUTO) {
         // the streaming kernel up to M = 8, and up to 16 while staging x still leaves room
         // for a 4-stage ring (or for all the stages a block streams) without splitting K
-        // further than the tile count asks for
-        if (st_ok && (M <= 8 || (!stc.split_raised && stc.ring >= std::min(4, stc.stages))))
+        // further than the tile count asks for; on an unsplit grid, whose blocks stream back
+        // to back, 96 KB in flight suffice (3 stages of 4- or 8-bit codes, 4 of 6-bit)
+        const int ring_need =
+            (st_ok && stc.split == 1) ? (96 * 1024 + stc.stage_bytes - 1) / std::max(1, stc.stage_bytes) : 4;
+        if (st_ok && (M <= 8 || (!stc.split_raised && stc.ring >= std::min(ring_need, stc.stages))))
             p.kernel = QMM_KERNEL_STREAM;
         else p.kernel = (tc_ok && prefer_tc(M, N, K)) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
     }

@@ -69,6 +69,7 @@ struct StreamConfig {
     int kslice;    // K codes per slice
     int ring;      // shared-memory stages (0: the shape does not fit this kernel)
     int stages;    // K stages each block streams per tile
+    int stage_bytes;  // shared memory of one ring stage
     bool split_raised;  // K split beyond the tile-count choice only to make x fit
     int grid_x;    // blocks along N (persistent when split == 1)
     int ncw;       // consumer warps per block (8 or 16)

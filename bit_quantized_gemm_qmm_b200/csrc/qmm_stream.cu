@@ -577,6 +577,7 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         c.kslice = kslice;
         c.ring = ring;
         c.stages = nst;
+        c.stage_bytes = ST_ROWS * KS * bits / 8;
         c.split_raised = split > split0;
         c.ncw = ncw;
         c.smem = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M));

@@ -124,6 +124,10 @@ def test_plans(L):
         assert p.kernel == q.KERNEL_STREAM and 1 <= p.split <= 8
     assert q.plan_default(4, 151936, 4096, 4, 64, f16).split == 1  # enough tiles: no split
     assert q.plan_default(17, 4096, 4096, 4, 64, f16).kernel != q.KERNEL_STREAM
+    # LM head (unsplit grid): x of up to 13 rows leaves a 3-stage ring, 14 does not
+    bf16 = __import__("torch").bfloat16
+    assert q.plan_default(13, 151936, 4096, 4, 64, bf16).kernel == q.KERNEL_STREAM
+    assert q.plan_default(14, 151936, 4096, 4, 64, bf16).kernel != q.KERNEL_STREAM
     assert q.plan_default(4, 4096, 4096 + 64, 4, 64, f16).kernel != q.KERNEL_STREAM
     st = q.make_plan(kernel=q.KERNEL_STREAM)
     assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(st), None) == q.QMM_ERR_UNSUPPORTED

@@ -67,6 +67,16 @@ def test_persistent_more_tiles_than_blocks(oracle_mod):
     _run(oracle_mod, 11, 40000, 1024, 8, 32, torch.bfloat16, 0.02)
 
 
+@pytest.mark.parametrize("M,bits,group", [(10, 4, 64), (12, 4, 64), (13, 8, 128)])
+def test_unsplit_grid_with_three_stage_ring(oracle_mod, M, bits, group):
+    """K = 4096 with 10-13 token rows on an unsplit grid with more tiles than blocks: staged x
+    leaves room for a 3-stage ring only, and the default plan takes this kernel."""
+    N, K = 20000, 4096
+    pd = q.plan_default(M, N, K, bits, group, torch.bfloat16)
+    assert pd.kernel == q.KERNEL_STREAM and pd.split == 1
+    _run(oracle_mod, M, N, K, bits, group, torch.bfloat16, 0.02)
+
+
 def test_bf16_large_activations(oracle_mod):
     M, K = 4, 1024
     x = randn((M, K), 1.0, torch.bfloat16, 5)
