@@ -106,6 +106,19 @@ __device__ __forceinline__ float exp2i(int e) { return __uint_as_float(uint32_t(
 
 // Sum of one float from each block of a cluster (ranks 0..n-1, n <= 16), added in rank order so
 // the result does not depend on timing.  The remote loads are all issued before the first add.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Store v at shared address `local` (this block's layout) of block `rank` of the cluster.
+__device__ __forceinline__ void st_cluster_f32(uint32_t local, uint32_t rank, float v) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ float cluster_sum_in_order(const float* local, int n) {
     float v[16];
     const uint32_t la = static_cast<uint32_t>(__cvta_generic_to_shared(local));

@@ -104,7 +104,7 @@ __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int ks
     L.xf_off = off;                                           // K-half partials: [8 warps][32][4*MT]
     if (ncw == 16) off += uint32_t(8 * 32 * 4 * mt * 4);
     L.red_off = off;
-    if (split > 1) off += uint32_t(ST_ROWS * 8 * mt * 4);
+    if (split > 1) off += uint32_t(split * ((ST_ROWS + split - 1) / split) * 8 * mt * 4);
     off = (off + 15) & ~15u;
     L.bar_off = off;
     off += 8 * uint32_t(2 * ring + 2 * ST_SS + 16) + 16;
@@ -217,6 +217,11 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // K split: every block of the cluster must be running before another one writes into its
+    // shared memory (the partial sums are pushed there); this arrival is waited for just
+    // before the first such write
+    if (p.split > 1) asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+    bool cl_waited = false;
     if (threadIdx.x == 32 * NCW) {
         prefetch_tensormap(&wmap);
         prefetch_tensormap(&smap);
@@ -453,40 +458,58 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                                                                 : __half_as_ushort(__float2half_rn(acc[mt][i]));
                         }
                 } else {
-                    // one tile per block when K is split: partials [8*MT cols][128 rows]
-                    float* red = reinterpret_cast<float*>(smem + L.red_off);
+                    // one tile per block when K is split: each partial goes straight into the
+                    // shared memory of the block that sums its row (rows dealt out evenly over
+                    // the ranks), at [this rank][column][row within the owner's slice]
+                    if (!cl_waited) {
+                        asm volatile("barrier.cluster.wait;" ::: "memory");
+                        cl_waited = true;
+                    }
+                    const int rows_per = (ST_ROWS + p.split - 1) / p.split;
+                    const uint32_t me = cluster_ctarank();
+                    const uint32_t red_la = sbase + L.red_off;
+                    const int oA = rA / rows_per, oB = rB / rows_per;
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            red[(8 * mt + 2 * c + (i & 1)) * ST_ROWS + (i < 2 ? rA : rB)] = acc[mt][i];
+                        for (int i = 0; i < 4; ++i) {
+                            const int col = 8 * mt + 2 * c + (i & 1);
+                            const int owner = i < 2 ? oA : oB;
+                            const int rl = (i < 2 ? rA : rB) - owner * rows_per;
+                            if (col < p.M)
+                                st_cluster_f32(red_la + uint32_t(((int(me) * 8 * MT + col) * rows_per + rl) * 4),
+                                               uint32_t(owner), acc[mt][i]);
+                        }
                 }
             }
         }
     }
 
     if (p.split > 1) {
-        // K split over the cluster (grid.x == T: one tile per block): block `rank` sums a slice
-        // of the tile's rows over ranks 0..split-1 in order.
-        cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();
+        // K split over the cluster (grid.x == T: one tile per block): once every block has
+        // pushed its partials (cluster barrier, release/acquire), block `rank` sums the rows
+        // it owns over ranks 0..split-1 in order, from its own shared memory; no block reads
+        // another's shared memory after this barrier, so none waits for the others to finish
+        if (!cl_waited) asm volatile("barrier.cluster.wait;" ::: "memory");
+        asm volatile("barrier.cluster.arrive;" ::: "memory");
+        asm volatile("barrier.cluster.wait;" ::: "memory");
         const int t = blockIdx.x;
-        const int rank = int(cluster.block_rank());
+        const int rank = int(cluster_ctarank());
         const int rows_per = (ST_ROWS + p.split - 1) / p.split;
         const int rlo = rank * rows_per, rhi = min(ST_ROWS, rlo + rows_per);
         const int nrows = max(0, rhi - rlo);
         const int ncols = min(8 * MT, p.M);
-        float* red = reinterpret_cast<float*>(smem + L.red_off);
+        const float* red = reinterpret_cast<const float*>(smem + L.red_off);
         const bool ok = *abort_flag == 0;
         for (int e = threadIdx.x; e < nrows * ncols; e += StWarps<NCW>::THREADS) {
-            const int col = e / nrows, row = rlo + (e - col * nrows);
-            const int n = t * ST_ROWS + row;
-            const float sum = cluster_sum_in_order(red + col * ST_ROWS + row, p.split);
+            const int col = e / nrows, rl = e - col * nrows;
+            const int n = t * ST_ROWS + rlo + rl;
+            float sum = 0.f;
+            for (int q = 0; q < p.split; ++q) sum += red[(q * 8 * MT + col) * rows_per + rl];
             if (n < p.N && ok)
                 p.y[int64_t(col) * p.N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sum))
                                                         : __half_as_ushort(__float2half_rn(sum));
         }
-        cluster.sync();
     }
 }
 
