@@ -141,19 +141,33 @@ def quantize(w: torch.Tensor, bits: int, group: int):
     packed = torch.empty((N, K * bits // 32), dtype=torch.int32, device=dev)
     scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
     biases = torch.empty((N, K // group), dtype=torch.float16, device=dev)
-    _check(L.qmm_quantize(_ptr(w), _dtype_code(w.dtype), N, K, bits, group, _ptr(packed),
-                          _ptr(scales), _ptr(biases), _stream(dev)))
+    with torch.cuda.device(dev):
+        _check(L.qmm_quantize(_ptr(w), _dtype_code(w.dtype), N, K, bits, group, _ptr(packed),
+                              _ptr(scales), _ptr(biases), _stream(dev)))
     return packed, scales, biases
 
 
 def dequantize(packed: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor, K: int, bits: int,
                group: int, dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None):
     dev = _need_cuda(packed, scales, biases)
+    if packed.dim() != 2:
+        raise ValueError("packed must be [N, K*bits/32]")
     N = packed.shape[0]
+    if packed.shape[1] * 32 != K * bits or packed.element_size() != 4:
+        raise ValueError(f"packed must hold K*bits/32 = {K * bits // 32} 32-bit words per row")
+    if group > 0 and K % group == 0 and (scales.numel() != N * (K // group) or biases.numel() != N * (K // group)):
+        raise ValueError(f"scales and biases must hold [N, K/group] = [{N}, {K // group}] values")
+    if scales.dtype != torch.float16 or biases.dtype != torch.float16:
+        raise ValueError("scales and biases must be fp16")
     if out is None:
         out = torch.empty((N, K), dtype=dtype, device=dev)
-    _check(lib().qmm_dequantize(_ptr(packed), _ptr(scales), _ptr(biases), N, K, bits, group,
-                                _dtype_code(out.dtype), _ptr(out), _stream(dev)))
+    else:
+        _need_cuda(packed, out)
+        if out.shape != (N, K):
+            raise ValueError(f"out must be [N, K] = [{N}, {K}]")
+    with torch.cuda.device(dev):
+        _check(lib().qmm_dequantize(_ptr(packed), _ptr(scales), _ptr(biases), N, K, bits, group,
+                                    _dtype_code(out.dtype), _ptr(out), _stream(dev)))
     return out
 
 
@@ -231,9 +245,13 @@ def qmm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, biases: tor
     elif not (out.is_cuda and out.get_device() == dev and out.is_contiguous() and out.dtype is dt
               and out.dim() == 2 and out.shape[0] == M and out.shape[1] == N):
         raise ValueError("out must be a contiguous [M, N] CUDA tensor with x's dtype on x's device")
-    st = _caller()(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
-                   M, N, K, bits, group, code, 0 if plan is None else ctypes.addressof(plan),
-                   _current_stream(dev))
+    args = (x.data_ptr(), packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
+            M, N, K, bits, group, code, 0 if plan is None else ctypes.addressof(plan), _current_stream(dev))
+    if dev == torch.cuda.current_device():
+        st = _caller()(*args)
+    else:  # the library launches on the calling thread's current device
+        with torch.cuda.device(dev):
+            st = _caller()(*args)
     if st:
         _check(st)
     return out

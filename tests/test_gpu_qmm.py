@@ -84,6 +84,37 @@ def test_empty_m_and_n():
     assert y.shape == (4, 0)
 
 
+def test_binding_rejects_mismatched_tensors():
+    """The binding checks what the C ABI cannot see before any launch: array sizes and element
+    types, and the output's shape, dtype and contiguity."""
+    dev = "cuda"
+    x = torch.zeros((4, 128), dtype=torch.float16, device=dev)
+    P = torch.zeros((16, 16), dtype=torch.int32, device=dev)   # N=16, K=128 at 4 bits
+    S = torch.zeros((16, 2), dtype=torch.float16, device=dev)  # group 64
+    q.qmm(x, P, S, S, 4, 64)                                   # consistent: accepted
+    torch.cuda.synchronize()
+    bad = [
+        dict(S=torch.zeros((16, 1), dtype=torch.float16, device=dev)),      # too few groups
+        dict(S=torch.zeros((16, 2), dtype=torch.float32, device=dev)),      # not fp16
+        dict(P=torch.zeros((16, 15), dtype=torch.int32, device=dev)),       # K mismatch
+        dict(P=torch.zeros((16, 16), dtype=torch.int16, device=dev)),       # not 32-bit words
+        dict(out=torch.zeros((4, 17), dtype=torch.float16, device=dev)),    # wrong shape
+        dict(out=torch.zeros((4, 16), dtype=torch.bfloat16, device=dev)),   # wrong dtype
+        dict(out=torch.zeros((16, 4), dtype=torch.float16, device=dev).t()),  # not contiguous
+        dict(out=torch.zeros((4, 16), dtype=torch.float16)),                # on the host
+    ]
+    for kw in bad:
+        a = dict(P=P, S=S, out=None)
+        a.update(kw)
+        with pytest.raises(ValueError):
+            q.qmm(x, a["P"], a["S"], a["S"], 4, 64, out=a["out"])
+    with pytest.raises(ValueError):
+        q.dequantize(P, torch.zeros((16, 1), dtype=torch.float16, device=dev), S, 128, 4, 64)
+    with pytest.raises(ValueError):
+        q.dequantize(P, S, S, 128, 4, 64, out=torch.zeros((16, 64), dtype=torch.float16, device=dev))
+    assert q.device_errors() == 0
+
+
 def _ulp(v, dtype):
     """Spacing of the output type at |v| (fp16: 11-bit significand, bf16: 8-bit)."""
     mant = 10 if dtype == torch.float16 else 7
