@@ -15,6 +15,19 @@ def pytest_configure(config):
 
 @pytest.fixture(scope="session")
 def oracle_mod():
+    mutant = os.environ.get("QMM_ORACLE_MUTANT_SRC")
+    if mutant:
+        # tests/test_oracle_mutations.py: the pins run against a copy of the oracle's C source
+        # with one planted mistake, built beside that copy (a separate module instance)
+        import importlib.util
+        spec = importlib.util.spec_from_file_location("oracle_mutant", os.path.join(ROOT, "oracle", "__init__.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod._SRC = mutant
+        mod._LIB_PATH = os.path.splitext(mutant)[0] + ".so"
+        mod._lib = None
+        mod.build(force=True)
+        return mod
     import oracle
     oracle.build()
     return oracle
