@@ -143,3 +143,17 @@ def test_status_strings(L):
     for s in range(4):
         assert L.qmm_status_string(s)
     assert L.qmm_version() >= 100
+
+
+def test_default_plan_for_every_workload_and_m(L):
+    """The dispatch table gives a valid plan for every benchmark shape at every M = 1..64: a
+    known kernel, a K split within a cluster, the streaming kernel only up to M = 16, and the
+    same answer on a second query."""
+    from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS
+    for name, wl in WORKLOADS.items():
+        for M in range(1, 65):
+            p = q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype)
+            assert p.kernel in (q.KERNEL_MMA, q.KERNEL_TC, q.KERNEL_STREAM), (name, M, p.as_dict())
+            assert 1 <= p.split <= 16, (name, M, p.as_dict())
+            assert p.kernel != q.KERNEL_STREAM or M <= 16, (name, M)
+            assert q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype).as_dict() == p.as_dict()
