@@ -73,7 +73,7 @@ def test_qmm_rejects_before_launch(L, kw, status):
 ])
 def test_call_module_forwards_to_qmm_ex(L, kw, status):
     """The C hand-off qmm() uses passes every argument through unchanged: the library gives
-    the same verdicts as through ctypes, with the default plan (address 0) and with a plan."""
+    the same statuses as through ctypes, with the default plan (address 0) and with a plan."""
     call = q._caller()
     a = dict(M=4, N=64, K=128, bits=4, group=64, dtype=0, ptr=16, y=16, scales=16)
     a.update(kw)
