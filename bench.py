@@ -353,9 +353,14 @@ def run_e2e(wl, weights, plans, dev, steps):
             "calls_per_step": len(BENCH_MS) * S}
 
 
+# The sources that decide the benchmark's launches: the streaming kernel, the headers it is
+# compiled from, and the dispatch that picks it and its plan.
+TRAFFIC_SOURCES = ("qmm_api.cu", "qmm_common.cuh", "qmm_dq.cuh", "qmm_internal.h", "qmm_stream.cu", "sm100.cuh")
+
+
 def traffic_per_launch():
-    """DRAM bytes per launch from the committed ncu capture, if the kernel source still
-    matches the one that was profiled (else null)."""
+    """DRAM bytes per launch from the committed ncu capture, if the sources of the profiled
+    kernel and its dispatch still match the ones that were profiled (else null)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
@@ -363,7 +368,7 @@ def traffic_per_launch():
     except Exception:
         return None
     h = hashlib.sha256()
-    for name in sorted(os.listdir(os.path.join(ROOT, "bit_quantized_gemm_qmm_b200", "csrc"))):
+    for name in TRAFFIC_SOURCES:
         h.update(open(os.path.join(ROOT, "bit_quantized_gemm_qmm_b200", "csrc", name), "rb").read())
     if d.get("csrc_sha256") != h.hexdigest():
         return None

@@ -76,6 +76,12 @@ constexpr int TC_NDQ = 16;                       // dequantizer warps (four per 
 constexpr int TC_DQ0 = 1 + TC_NMMA;              // first dequantizer warp
 constexpr int TC_THREADS = (TC_DQ0 + TC_NDQ) * 32;  // 672
 constexpr int TC_SPF = 4;                        // stages of scales in flight per thread
+// Scales and biases by TMA (shapes with a multiple of 8 groups per row): per block of 8
+// groups, one [128 rows x 8] box of scales and one of biases into a TC_SS-slot ring that
+// reuses the per-thread scale area.
+constexpr int TC_SS = 3;
+constexpr int TC_SB_SLOT = 2 * TC_ROWS * 8 * 2;  // 4 KB: scales, then biases
+static_assert(TC_SS * TC_SB_SLOT <= TC_SPF * TC_NDQ * 32 * 8, "scale ring must fit the scale area");
 constexpr int TC_TMEM_COLS = 512;
 constexpr long long TC_TIMEOUT_CYCLES = 4000000000LL;  // ~2 s at 2 GHz
 
@@ -135,7 +141,7 @@ __host__ __device__ inline TcSmemLayout tc_layout(int x_stage, int w_bytes, int 
     L.w_off = L.x_off + ring * L.x_stage;
     L.sc_off = L.w_off + ring * L.w_stage;
     L.bar_off = L.sc_off + TC_SPF * TC_NDQ * 32 * 8;
-    L.total = L.bar_off + 8 * (4 * ring + 2 * na + 1) + 16;
+    L.total = L.bar_off + 8 * (4 * ring + 2 * na + 1 + 2 * TC_SS) + 16;
     return L;
 }
 
@@ -217,9 +223,10 @@ __device__ __forceinline__ void dequant_quarter(const uint32_t (&wd)[TcWords<BIT
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int BITS, int MP>
+template <int BITS, int MP, bool STMA>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    qmm_tc_kernel(const __grid_constant__ CUtensorMap wmap, const TcParams p) {
+    qmm_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
+                  const __grid_constant__ CUtensorMap bmap, const TcParams p) {
     using F = TcFmt<BITS, MP>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -236,7 +243,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t bar_afull = bar_xempty + 8 * S;             // [NA]
     const uint32_t bar_aempty = bar_afull + 8 * F::NA;         // [NA]
     const uint32_t bar_acc = bar_aempty + 8 * F::NA;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.bar_off + 8 * (4 * S + 2 * F::NA + 1));
+    const uint32_t bar_sfull = bar_acc + 8;                    // [TC_SS] scale block landed (STMA)
+    const uint32_t bar_sempty = bar_sfull + 8 * TC_SS;         // [TC_SS] scale block read (STMA)
+    uint32_t* tmem_holder =
+        reinterpret_cast<uint32_t*>(smem + L.bar_off + 8 * (4 * S + 2 * F::NA + 1 + 2 * TC_SS));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -266,9 +276,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             mbar_init(bar_aempty + 8 * i, TC_NMMA);
         }
         mbar_init(bar_acc, TC_NMMA);
+        for (int i = 0; i < TC_SS; ++i) {
+            mbar_init(bar_sfull + 8 * i, 1);
+            mbar_init(bar_sempty + 8 * i, TC_NDQ);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&wmap);
+        if (STMA) {
+            prefetch_tensormap(&smap);
+            prefetch_tensormap(&bmap);
+        }
     }
     if (warp == 0) {
         tmem_alloc(smem_addr(tmem_holder), TC_TMEM_COLS);
@@ -281,7 +299,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // Everything except the producer's first code tiles depends on earlier kernels; the
     // producer waits after issuing those tiles, everyone else waits here.  Deadlines start
     // after the wait so a slow predecessor never looks like a stalled pipeline.
-    if (!(warp == 0 && lane == 0)) grid_dependency_wait();
+    if (!(warp == 0 && (lane == 0 || (STMA && lane == 2)))) grid_dependency_wait();
     long long deadline = clock64() + TC_TIMEOUT_CYCLES;
 
     if (warp == 0) {
@@ -337,6 +355,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const long long drain_deadline = clock64() + TC_TIMEOUT_CYCLES;
             for (int i = max(0, issued - S); i < issued; ++i)
                 if (!mbar_wait(bar_xfull + 8 * (i % S), (i / S) & 1, drain_deadline)) set_error(1u);
+        } else if (STMA && lane == 2) {
+            // scales and biases never depend on earlier kernels when the weights are static
+            if (!p.static_w) grid_dependency_wait();
+            deadline = clock64() + TC_TIMEOUT_CYCLES;
+            const int spb = (8 << p.gshift) / F::KC;  // stages per block of 8 groups (1..8)
+            int gcol = (st0 * F::KC) >> p.gshift;     // a multiple of 8 (the host checks)
+            int blk = 0, ss = 0;
+            uint32_t sph = 0;
+            for (int i = 0; i < nst; i += spb) {
+                if (blk >= TC_SS && !mbar_wait(bar_sempty + 8 * ss, sph ^ 1u, deadline)) {
+                    set_error(1u);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                const uint32_t dst = sbase + L.sc_off + uint32_t(ss * TC_SB_SLOT);
+                mbar_arrive_expect_tx(bar_sfull + 8 * ss, uint32_t(TC_SB_SLOT));
+                tma_load_2d(dst, &smap, bar_sfull + 8 * ss, gcol, n0);
+                tma_load_2d(dst + TC_SB_SLOT / 2, &bmap, bar_sfull + 8 * ss, gcol, n0);
+                gcol += 8;
+                if (++ss == TC_SS) {
+                    ss = 0;
+                    sph ^= 1u;
+                }
+                ++blk;
+            }
+            const long long drain_deadline = clock64() + TC_TIMEOUT_CYCLES;
+            for (int b = max(0, blk - TC_SS); b < blk; ++b)
+                if (!mbar_wait(bar_sfull + 8 * (b % TC_SS), (b / TC_SS) & 1, drain_deadline)) set_error(1u);
         }
     } else if (warp < TC_DQ0) {
         // ------------------------------------------------------------ MMA issuers
@@ -408,12 +455,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             cp_async_4(dst + 4, p.biases + off, ok ? 4u : 0u);
             cp_async_commit();
         };
+        if (!STMA) {
 #pragma unroll
-        for (int i = 0; i < TC_SPF; ++i) issue_scales(i);
+            for (int i = 0; i < TC_SPF; ++i) issue_scales(i);
+        }
+        const int spb = (8 << p.gshift) / F::KC;  // (STMA) stages per scale block
+        int ss = 0, sib = 0;
+        uint32_t sph = 0, sbuf = 0;
 
         int s = 0, a = 0;
         uint32_t ph = 0, pa = 0;
         for (int i = 0; i < nst; ++i) {
+            if (STMA && sib == 0) {
+                if (!mbar_wait(bar_sfull + 8 * ss, sph, deadline)) {
+                    set_error(1u);
+                    *abort_flag = 1;
+                    break;
+                }
+                sbuf = sbase + L.sc_off + uint32_t(ss * TC_SB_SLOT);
+            }
             if (!mbar_wait(bar_full + 8 * s, ph, deadline)) {
                 set_error(1u);
                 *abort_flag = 1;
@@ -425,15 +485,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             load_quarter<BITS>(sbase + L.w_off + s * L.w_stage + row * F::ROW_BYTES, row, quarter, wd);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_empty + 8 * s);
-            cp_async_wait<TC_SPF - 1>();
-            const uint32_t sp = sc_base + uint32_t(i % TC_SPF) * (TC_NDQ * 32 * 8);
             uint32_t s_pair, b_pair;
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(s_pair), "=r"(b_pair) : "r"(sp));
+            if (STMA) {
+                // the pair of groups (scale block positions gl & ~1, gl | 1) of this row; the
+                // block starts at a multiple of 8 groups, so gl & 1 is the global parity too
+                const int gl = (sib * F::KC + quarter * F::U) >> p.gshift;
+                const uint32_t off = uint32_t(row * 8 + (gl & ~1)) * 2u;
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(s_pair) : "r"(sbuf + off));
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b_pair) : "r"(sbuf + uint32_t(TC_SB_SLOT / 2) + off));
+            } else {
+                cp_async_wait<TC_SPF - 1>();
+                const uint32_t sp = sc_base + uint32_t(i % TC_SPF) * (TC_NDQ * 32 * 8);
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(s_pair), "=r"(b_pair) : "r"(sp));
+            }
             const int k = (st0 + i) * F::KC + quarter * F::U;
             uint32_t vals[F::COLS];
             dequant_quarter<BITS>(wd, s_pair, b_pair, two_groups, (k >> p.gshift) & 1, vals);
+            if (STMA && ++sib == spb) {  // the block's scales are in registers: free the slot
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_sempty + 8 * ss);
+                sib = 0;
+                if (++ss == TC_SS) {
+                    ss = 0;
+                    sph ^= 1u;
+                }
+            }
             if (warp == TC_DQ0 && lane == 0) TC_TRACE(4, i);
-            issue_scales(i + TC_SPF);
+            if (!STMA) issue_scales(i + TC_SPF);
             if (i >= F::NA && !mbar_wait(bar_aempty + 8 * a, pa ^ 1u, deadline)) {
                 set_error(1u);
                 *abort_flag = 1;
@@ -685,24 +763,29 @@ cudaError_t device_pool(cudaMemPool_t* out) {
     return cudaSuccess;
 }
 
-using TcKernelFn = void (*)(const CUtensorMap, const TcParams);
+using TcKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const TcParams);
 
-template <int BITS>
+template <int BITS, bool STMA>
 TcKernelFn pick_tc_mp(int mp) {
     switch (mp) {
-        case 16: return qmm_tc_kernel<BITS, 16>;
-        case 32: return qmm_tc_kernel<BITS, 32>;
-        case 48: return qmm_tc_kernel<BITS, 48>;
-        case 64: return qmm_tc_kernel<BITS, 64>;
+        case 16: return qmm_tc_kernel<BITS, 16, STMA>;
+        case 32: return qmm_tc_kernel<BITS, 32, STMA>;
+        case 48: return qmm_tc_kernel<BITS, 48, STMA>;
+        case 64: return qmm_tc_kernel<BITS, 64, STMA>;
         default: return nullptr;
     }
 }
 
-TcKernelFn pick_tc(int bits, int mp) {
-    if (bits == 4) return pick_tc_mp<4>(mp);
-    if (bits == 6) return pick_tc_mp<6>(mp);
-    if (bits == 8) return pick_tc_mp<8>(mp);
+template <bool STMA>
+TcKernelFn pick_tc_s(int bits, int mp) {
+    if (bits == 4) return pick_tc_mp<4, STMA>(mp);
+    if (bits == 6) return pick_tc_mp<6, STMA>(mp);
+    if (bits == 8) return pick_tc_mp<8, STMA>(mp);
     return nullptr;
+}
+
+TcKernelFn pick_tc(int bits, int mp, bool stma = false) {
+    return stma ? pick_tc_s<true>(bits, mp) : pick_tc_s<false>(bits, mp);
 }
 
 int kc_for(int bits) { return bits == 8 ? 128 : 256; }
@@ -742,6 +825,24 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Scales and biases by TMA (8 groups = 16 bytes per box row, boxes starting at multiples of
+// 8 groups): every row holds a multiple of 8 groups, each block's K range starts at one, and
+// both arrays are 16-byte aligned.  Otherwise each thread fetches its scale pairs itself.
+static bool tc_scale_tma_ok(const QmmArgs& a, int stages_per_split, int split) {
+    if ((a.K / a.group) % 8) return false;
+    if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) return false;
+    const int spb = 8 * a.group / kc_for(a.bits);
+    return split == 1 || stages_per_split % spb == 0;
+}
+
+static bool make_scale_maps(const QmmArgs& a, CUtensorMap* smap, CUtensorMap* bmap) {
+    const uint64_t G = uint64_t(a.K / a.group);
+    return make_map_2d(smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, G, uint64_t(a.N), 8, TC_ROWS,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           make_map_2d(bmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.biases, G, uint64_t(a.N), 8, TC_ROWS,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 bool tc_supported(int64_t M, int64_t N, int64_t K, int bits, int group) {
     if (M < 1 || M > 64 || N < 1 || K < 128) return false;
     if ((K / group) % 2) return false;              // scale pairs are fetched 4 bytes at a time
@@ -767,10 +868,11 @@ size_t tc_smem_bytes(int bits, int mp, int ring) {
 }
 
 cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) {
-    TcKernelFn fn = pick_tc(a.bits, c.mp);
-    if (!fn) return cudaErrorInvalidValue;
     const int KC = kc_for(a.bits);
     const int nst_k = int((a.K + KC - 1) / KC);
+    const bool stma = tc_scale_tma_ok(a, c.stages_per_split, (nst_k + c.stages_per_split - 1) / c.stages_per_split);
+    TcKernelFn fn = pick_tc(a.bits, c.mp, stma);
+    if (!fn) return cudaErrorInvalidValue;
 
     // stage tiles of x (fp16) and the per-token exponents, in stream-ordered scratch memory
     cudaMemPool_t pool;
@@ -807,6 +909,8 @@ cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) 
     if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
                      uint32_t(KC * a.bits / 32), TC_ROWS, wsw))
         return finish(cudaErrorInvalidValue);
+    CUtensorMap smap = wmap, bmap = wmap;  // unused unless stma
+    if (stma && !make_scale_maps(a, &smap, &bmap)) return finish(cudaErrorInvalidValue);
 
     TcParams p;
     p.scales = a.scales;
@@ -850,7 +954,7 @@ cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) 
     if (c.pdl) attrs[na++] = pdl_attr;
     cfg.attrs = attrs;
     cfg.numAttrs = unsigned(na);
-    return finish(cudaLaunchKernelEx(&cfg, fn, wmap, p));
+    return finish(cudaLaunchKernelEx(&cfg, fn, wmap, smap, bmap, p));
 }
 
 // How many clusters of `split` blocks of this kernel can be resident at once (0 if the query
@@ -964,10 +1068,11 @@ size_t tc_noalloc_need(int64_t M, int64_t K, int bits) {
 size_t tc_noalloc_capacity() { return kNoAllocXBytes; }
 
 cudaError_t launch_tc_noalloc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) {
-    TcKernelFn fn = pick_tc(a.bits, c.mp);
-    if (!fn) return cudaErrorInvalidValue;
     const int KC = kc_for(a.bits);
     const int nst_k = int((a.K + KC - 1) / KC);
+    const bool stma = tc_scale_tma_ok(a, c.stages_per_split, (nst_k + c.stages_per_split - 1) / c.stages_per_split);
+    TcKernelFn fn = pick_tc(a.bits, c.mp, stma);
+    if (!fn) return cudaErrorInvalidValue;
     const size_t xt_bytes = size_t(nst_k) * size_t(c.mp) * size_t(KC) * 2;
     if (xt_bytes > kNoAllocXBytes) return cudaErrorInvalidValue;
     void* ws = nullptr;
@@ -996,6 +1101,8 @@ cudaError_t launch_tc_noalloc(const QmmArgs& a, const TcConfig& c, cudaStream_t 
     if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
                      uint32_t(KC * a.bits / 32), TC_ROWS, wsw))
         return cudaErrorInvalidValue;
+    CUtensorMap smap = wmap, bmap = wmap;  // unused unless stma
+    if (stma && !make_scale_maps(a, &smap, &bmap)) return cudaErrorInvalidValue;
 
     TcParams p;
     p.scales = a.scales;
@@ -1039,7 +1146,7 @@ cudaError_t launch_tc_noalloc(const QmmArgs& a, const TcConfig& c, cudaStream_t 
     if (c.pdl) attrs[na++] = pdl_attr;
     cfg.attrs = attrs;
     cfg.numAttrs = unsigned(na);
-    return cudaLaunchKernelEx(&cfg, fn, wmap, p);
+    return cudaLaunchKernelEx(&cfg, fn, wmap, smap, bmap, p);
 }
 
 }  // namespace qmm_impl
