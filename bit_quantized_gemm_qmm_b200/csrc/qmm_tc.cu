@@ -12,15 +12,18 @@
 //           two so none overflows fp16), written straight into the 128-byte-swizzled tile
 //           layout the MMA reads, one contiguous [MP x KC] tile per K stage;
 //   qmm_tc  warp 0      producer: per stage one TMA box of packed codes [128 rows x 128 B] and
-//                       one bulk copy of the stage's x tile into an S-stage ring;
+//                       one bulk copy of the stage's x tile into an S-stage ring; per block of
+//                       8 groups one TMA box of scales and one of biases [128 rows x 8];
 //           warp 1      MMA issuer: tcgen05.mma kind::f16, A from tensor memory, B = x from
 //                       shared memory, D (fp32, 128 lanes x MP columns) in tensor memory;
 //           warps 2-17  dequantizers, four per tensor-memory lane quadrant: one thread per
 //                       weight row and quarter stage; codes -> fp16 (s*q + b, one rounding)
 //                       -> tcgen05.st into an A buffer; afterwards they read D and write y.
 // Few, large copies keep the copy engine's per-request cost off the critical path (a 2D box
-// costs about the same whether it moves 2 KB or 16 KB).  Scales and biases are fetched per
-// thread with cp.async a few stages ahead.  K may be split across a thread-block cluster;
+// costs about the same whether it moves 2 KB or 16 KB).  Scales and biases come by TMA where
+// every row holds a multiple of 8 groups and each block's K range starts at one; otherwise
+// each thread fetches its pair with cp.async a few stages ahead.  K may be split across a
+// thread-block cluster;
 // partial tiles are summed over DSMEM in rank order.  Every mbarrier wait is bounded: on
 // timeout the block records an error, drains its own copies and frees its tensor memory.
 #include <cooperative_groups.h>
