@@ -89,7 +89,9 @@ qmm_status qmm_dequantize(const uint32_t* packed, const uint16_t* scales,
  * output dtype.  Split-K partial sums are combined in a fixed order, so the result is
  * bitwise reproducible run to run.  M == 0 or N == 0 is a no-op; K == 0 writes zeros.
  * Alignment: x, packed and y 16-byte aligned; scales and biases 2-byte (4-byte alignment is
- * needed for the tensor-core kernel, which the dispatcher otherwise avoids).
+ * needed for the tensor-core kernel, which the dispatcher otherwise avoids; with 16-byte
+ * alignment the streaming and tensor-core kernels fetch them as TMA tiles, which is faster,
+ * and the streaming kernel requires it).
  * Scratch memory: the tensor-core kernel stages x in a small buffer (about 2*64*K bytes) taken
  * on `stream` from a memory pool the library owns (cudaMallocFromPoolAsync) and released on
  * the same stream after the call; this is also valid while the stream is being captured into
