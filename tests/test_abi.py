@@ -128,6 +128,12 @@ def test_plans(L):
     bf16 = __import__("torch").bfloat16
     assert q.plan_default(13, 151936, 4096, 4, 64, bf16).kernel == q.KERNEL_STREAM
     assert q.plan_default(14, 151936, 4096, 4, 64, bf16).kernel != q.KERNEL_STREAM
+    # 6-bit stages are smaller (24 KB): 4 of them are needed, so 6-bit gate/up leaves at M = 13
+    assert q.plan_default(12, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_STREAM
+    assert q.plan_default(13, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_TC
+    # q/o size: the warp-tile kernel up to M = 27, the tensor-core kernel from 28
+    assert q.plan_default(27, 4096, 4096, 4, 64, f16).kernel == q.KERNEL_MMA
+    assert q.plan_default(28, 4096, 4096, 4, 64, f16).kernel == q.KERNEL_TC
     assert q.plan_default(4, 4096, 4096 + 64, 4, 64, f16).kernel != q.KERNEL_STREAM
     st = q.make_plan(kernel=q.KERNEL_STREAM)
     assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(st), None) == q.QMM_ERR_UNSUPPORTED
