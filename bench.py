@@ -5,11 +5,16 @@ Metric (MLX issue #4720, "To Reproduce"): weight bytes per call = N*K*bits/8 + N
 (packed codes + one fp16 scale and bias per group), divided by the time per call, with the
 weight copies rotated so that they do not sit in L2.
 
-Workload: the q/o projection verify shapes, K = N = 4096, 4-bit, group 64, fp16 x and W
-~ N(0,1), M in {1, 4, 5, 6}.  27 weight sets (255 MB, twice the 126 MB L2) are rotated, so
-every call streams its weights from HBM.  One step = one call per weight set for each M
-(108 calls).  Weights and x are resident in HBM before the timed region; the step is
-captured once in a CUDA graph and replayed (an eager-launch figure is reported beside it).
+Headline workload: the 151936-wide LM head (K = 4096, 4-bit, group 64, bf16 x and W ~
+N(0, 0.02^2)) at M in {1, 4, 6, 16}, the largest configuration.  Its single 350 MB matrix
+is larger than the 126 MB L2, so every call streams its weights from HBM.  One step = one
+call per M (4 calls); weights and x are resident in HBM before the timed region; the step
+is captured once in a CUDA graph and replayed.
+
+`breakdown` covers the metric as stated, per shape and per M: every M = 1..64 on the three
+4-bit shapes (q/o 4096 -> 4096, down 14336 -> 4096, LM head 4096 -> 151936) and M in
+{4, 16, 64} on the mixed-precision gate/up and k/v shapes, each cell one CUDA graph of one
+call per rotated weight set (>= 2x L2 in total), timed with CUDA events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -32,28 +37,33 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-METRIC = "effective weight GB/s (and % of HBM roofline) per shape vs M=1..64, 1×B200"
-WORKLOAD = "qo"
-BENCH_MS = (1, 4, 5, 6)
+METRIC = "effective weight GB/s (and % of HBM roofline) per shape vs M=1..64, 1\u00d7B200"
+WORKLOAD = "lmhead"
+BENCH_MS = (1, 4, 6, 16)
+GATED = ("qo", "down", "lmhead")          # every M = 1..64
+MIXED = ("gateup_6b", "gateup_8b", "kv_6b", "kv_8b")
+MIXED_MS = (4, 16, 64)
 NOMINAL_HBM_GBS = 8000.0
-KERNEL_NAMES = {1: "qmm_mma_kernel", 2: "qmm_tc_kernel", 3: "qmm_stream_kernel"}
+KERNEL_NAMES = {1: "qmm_mma_kernel", 2: "qmm_tc_kernel", 3: "qmm_stream_kernel", 4: "qmm_sk_kernel"}
 FALLBACK_HBM_GBS = 6650.0
+CLOCK_SOAK_S = 2.5  # the step replayed (untimed) while the clocks are sampled, right before timing
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--breakdown-out", default="", help="also write the per-M breakdown JSON here")
+    ap.add_argument("--no-breakdown", action="store_true", help="skip the per-shape, per-M table")
+    ap.add_argument("--breakdown-out", default="", help="also write the whole JSON line, indented, here")
     ap.add_argument("--sweep", default="", help="write a per-configuration, per-M GB/s sweep to this "
                     "JSON file instead of running the headline benchmark")
     ap.add_argument("--sweep-configs", default="qo,down,gateup_6b,gateup_8b,kv_6b,kv_8b,lmhead")
     ap.add_argument("--sweep-ms", default="1-64", help="e.g. 1-64 or 1,4,16")
-    ap.add_argument("--sweep-plan", default="", help="kernel:split:warps[:flags] override, e.g. 1:4:8")
+    ap.add_argument("--sweep-plan", default="", help="kernel:split:warps[:flags] override, e.g. 4:1:0:3")
     return ap.parse_args()
 
 
@@ -173,24 +183,184 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- our arm
-def setup_workload(dev):
-    import bit_quantized_gemm_qmm_b200 as q
-    from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS, w_input, x_input
-    wl = WORKLOADS[WORKLOAD]
+def launches_per_call(plan) -> int:
+    """Kernels one call launches: the tensor-core kernels with x staged in the workspace run a
+    small x kernel first."""
+    if plan.kernel == 2 or (plan.kernel == 4 and plan.split == 2):
+        return 2
+    return 1
+
+
+def make_weights(q, wl, dev):
+    from bit_quantized_gemm_qmm_b200.inputs import w_input
     weights = []
     for i in range(wl.sets):
         w = w_input(wl.N, wl.K, wl.dtype, i, wl.w_sigma).to(dev)
         weights.append(q.quantize(w, wl.bits, wl.group))
         del w
+    return weights
+
+
+def default_plan(q, wl, M):
+    p = q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype)
+    p.flags |= q.PLAN_STATIC_WEIGHTS  # weights are written once, before any timed call
+    return p
+
+
+def setup_workload(dev):
+    import bit_quantized_gemm_qmm_b200 as q
+    from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS, x_input
+    wl = WORKLOADS[WORKLOAD]
+    weights = make_weights(q, wl, dev)
     xs = {M: x_input(M, wl.K, wl.dtype).to(dev) for M in BENCH_MS}
     ys = {M: torch.empty((M, wl.N), dtype=wl.dtype, device=dev) for M in BENCH_MS}
-    plans = {}
-    for M in BENCH_MS:
-        p = q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype)
-        p.flags |= q.PLAN_STATIC_WEIGHTS  # weights are written once, before any timed call
-        plans[M] = p
+    plans = {M: default_plan(q, wl, M) for M in BENCH_MS}
     torch.cuda.synchronize()
     return wl, weights, xs, ys, plans
+
+
+def time_cell(q, wl, weights, M, dev, plan, target_s=0.12):
+    """Seconds per call of one (shape, M) cell: a CUDA graph of one call per rotated weight set,
+    replayed; the best of three timed batches of replays."""
+    from bit_quantized_gemm_qmm_b200.inputs import x_input
+    x = x_input(M, wl.K, wl.dtype).to(dev)
+    y = torch.empty((M, wl.N), dtype=wl.dtype, device=dev)
+    for (P, S, B) in weights:
+        q.qmm(x, P, S, B, wl.bits, wl.group, out=y, plan=plan)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for (P, S, B) in weights:
+            q.qmm(x, P, S, B, wl.bits, wl.group, out=y, plan=plan)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    e1.synchronize()
+    one = max(e0.elapsed_time(e1) * 1e-3, 1e-6)
+    reps = max(2, min(200, int(target_s / 3 / one)))
+    best = float("inf")
+    for _ in range(3):
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1) * 1e-3 / reps / len(weights))
+    del g
+    return best
+
+
+def run_breakdown(q, dev, peak):
+    """GB/s per shape and M (default dispatch, static-weight plans): every M = 1..64 on the
+    three 4-bit shapes, M in {4, 16, 64} on the mixed-precision ones."""
+    from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS
+    out = {}
+    for name in GATED + MIXED:
+        wl = WORKLOADS[name]
+        weights = make_weights(q, wl, dev)
+        torch.cuda.synchronize()
+        wbytes = wl.weight_bytes()
+        Ms = range(1, 65) if name in GATED else MIXED_MS
+        cells = {}
+        for M in Ms:
+            plan = default_plan(q, wl, M)
+            t = time_cell(q, wl, weights, M, dev, plan)
+            gbs = wbytes / t / 1e9
+            cells[str(M)] = {"gbs": round(gbs, 1), "us": round(t * 1e6, 3), "frac_of_measured": round(gbs / peak, 4),
+                             "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                             "kernel": KERNEL_NAMES.get(plan.kernel, "?"), "plan": plan.as_dict()}
+        g = [c["gbs"] for c in cells.values()]
+        drops = [(int(a), round(1 - cells[b]["gbs"] / cells[a]["gbs"], 4)) for a, b in zip(list(cells)[:-1], list(cells)[1:])]
+        worst = max(drops, key=lambda d: d[1]) if drops else (None, 0.0)
+        out[name] = {"shape": f"K={wl.K} N={wl.N} {wl.bits}-bit g{wl.group} {str(wl.dtype).replace('torch.', '')}",
+                     "weight_sets": len(weights), "weight_bytes_per_call": wbytes,
+                     "min_frac_of_measured": round(min(g) / peak, 4), "mean_frac_of_measured": round(sum(g) / len(g) / peak, 4),
+                     "largest_adjacent_drop": {"from_M": worst[0], "drop": worst[1]}, "M": cells}
+        del weights
+        torch.cuda.empty_cache()
+        print(f"[breakdown] {name}: " + " ".join(f"{m}:{c['gbs']:.0f}" for m, c in cells.items()),
+              file=sys.stderr, flush=True)
+    return out
+
+
+GROUPS = {  # one decoder layer's projections that share x (Qwen3-8B-like widths), 4-bit g64 fp16
+    "qkv": {"K": 4096, "Ns": (4096, 1024, 1024), "sets": 18},
+    "gate_up": {"K": 4096, "Ns": (14336, 14336), "sets": 4},
+}
+GROUP_MS = (1, 4, 16, 64)
+
+
+def run_grouped(q, dev, peak):
+    """One launch over a layer's matrices (qmm_grouped) against the same matrices as separate
+    calls: GB/s of the group's weight bytes per M, weight sets rotated (>= 2x L2)."""
+    from bit_quantized_gemm_qmm_b200.inputs import w_input, x_input
+    out = {}
+    stream = torch.cuda.current_stream(dev)
+    for name, cfg in GROUPS.items():
+        K, Ns = cfg["K"], cfg["Ns"]
+        sets = []
+        for i in range(cfg["sets"]):
+            mats = []
+            for j, N in enumerate(Ns):
+                w = w_input(N, K, torch.float16, 500 + 10 * i + j, 1.0).to(dev)
+                mats.append(q.quantize(w, 4, 64))
+                del w
+            sets.append(mats)
+        torch.cuda.synchronize()
+        gbytes = sum(N * K // 2 + N * (K // 64) * 4 for N in Ns)
+        cells = {}
+        for M in GROUP_MS:
+            x = x_input(M, K, torch.float16).to(dev)
+            outs = [torch.empty((M, N), dtype=torch.float16, device=dev) for N in Ns]
+            plans = [q.plan_default(M, N, K, 4, 64, torch.float16) for N in Ns]
+            for p_ in plans:
+                p_.flags |= q.PLAN_STATIC_WEIGHTS
+            gplan = q.make_plan(kernel=q.KERNEL_SK, flags=q.PLAN_PDL | q.PLAN_STATIC_WEIGHTS)
+
+            def grouped():
+                for mats in sets:
+                    q.qmm_grouped(x, mats, 4, 64, outs=outs, plan=gplan)
+
+            def separate():
+                for mats in sets:
+                    for (P, S, B), y, p_ in zip(mats, outs, plans):
+                        q.qmm(x, P, S, B, 4, 64, out=y, plan=p_)
+
+            res = {}
+            for label, fn in (("grouped", grouped), ("separate", separate)):
+                fn()
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    fn()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                best = float("inf")
+                for _ in range(3):
+                    g.replay()
+                    torch.cuda.synchronize()
+                    e0.record(stream)
+                    for _ in range(10):
+                        g.replay()
+                    e1.record(stream)
+                    e1.synchronize()
+                    best = min(best, e0.elapsed_time(e1) * 1e-3 / 10 / len(sets))
+                del g
+                gbs = gbytes / best / 1e9
+                res[label] = {"gbs": round(gbs, 1), "us": round(best * 1e6, 3), "frac_of_measured": round(gbs / peak, 4)}
+            res["speedup"] = round(res["separate"]["us"] / res["grouped"]["us"], 3)
+            cells[str(M)] = res
+        out[name] = {"K": K, "Ns": list(Ns), "format": "4-bit g64 fp16", "weight_sets": len(sets),
+                     "weight_bytes_per_group": gbytes, "M": cells}
+        del sets
+        torch.cuda.empty_cache()
+        print(f"[grouped] {name}: " + " ".join(f"{m}:{c['grouped']['gbs']:.0f}/{c['separate']['gbs']:.0f}"
+                                               for m, c in cells.items()), file=sys.stderr, flush=True)
+    return out
 
 
 def run_ours(args, rank, world):
@@ -199,9 +369,11 @@ def run_ours(args, rank, world):
     q.lib()  # loud failure if the CUDA library is missing
     wl, weights, xs, ys, plans = setup_workload(dev)
     wbytes = wl.weight_bytes()
-    calls_per_step = len(BENCH_MS) * len(weights)
+    nsets = len(weights)
+    calls_per_step = len(BENCH_MS) * nsets
     step_wbytes = wbytes * calls_per_step
     step_algo_bytes = sum((wbytes + 2 * M * wl.K + 2 * M * wl.N) * len(weights) for M in BENCH_MS)
+    launches_per_step = sum(launches_per_call(plans[M]) * len(weights) for M in BENCH_MS)
 
     def step(Ms=BENCH_MS):
         for M in Ms:
@@ -210,28 +382,33 @@ def run_ours(args, rank, world):
                 q.qmm(x, P, S, B, wl.bits, wl.group, out=y, plan=p)
 
     stream = torch.cuda.current_stream(dev)
-    # eager warm-up, then one CUDA graph per step (and one per M for the breakdown)
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
-    graphs = {}
-    for key, Ms in [("all", BENCH_MS)] + [(M, (M,)) for M in BENCH_MS]:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(Ms)
-        graphs[key] = g
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
     for _ in range(max(3, args.warmup)):
-        graphs["all"].replay()
+        g.replay()
     torch.cuda.synchronize()
 
-    # ---- timed region: exactly K graph replays of the step
+    # ---- clocks: sampled from a soak of the same replays right before the timed region
+    # through to its end (the timed region alone is too short for a 200 ms sampler)
     clocks = ClockSampler(dev.index, not args.no_clocks)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if clocks.proc is not None:
+        t_end = time.perf_counter() + CLOCK_SOAK_S
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                g.replay()
+            torch.cuda.synchronize()
+
+    # ---- timed region: exactly K graph replays of the step
     barrier(world)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        graphs["all"].replay()
+        g.replay()
     e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize()
@@ -240,10 +417,10 @@ def run_ours(args, rank, world):
     t_ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_per_step = t_ms / args.steps
     value = job_gbs(step_wbytes, ms_per_step, world)
-    achieved = step_algo_bytes / (ms_per_step * 1e-3) / 1e9  # per GPU: the only kernel in the step
+    achieved = step_algo_bytes / (ms_per_step * 1e-3) / 1e9  # per GPU: the only kernels in the step
 
     # ---- eager figure (same calls, launched one by one)
-    reps = max(10, args.steps // 20)
+    reps = max(5, args.steps // 4)
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(reps):
@@ -253,53 +430,52 @@ def run_ours(args, rank, world):
     eager_ms = e0.elapsed_time(e1) / reps
     eager_value = step_wbytes / (eager_ms * 1e-3) / 1e9
 
-    # ---- per-M breakdown (graph replays)
     peak, peak_kind = measured_peaks()
-    breakdown = {}
-    reps_m = max(20, args.steps // 4)
+    per_m = {}
     for M in BENCH_MS:
-        for _ in range(3):
-            graphs[M].replay()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(reps_m):
-            graphs[M].replay()
-        e1.record(stream)
-        e1.synchronize()
-        per_call_ms = e0.elapsed_time(e1) / reps_m / len(weights)
-        gbs = wbytes / (per_call_ms * 1e-3) / 1e9
-        breakdown[f"M={M}"] = {"gbs": round(gbs, 1), "us_per_call": round(per_call_ms * 1e3, 3),
-                               "frac_of_measured": round(gbs / peak, 4),
-                               "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
-                               "plan": plans[M].as_dict()}
+        t = time_cell(q, wl, weights, M, dev, plans[M])
+        gbs = wbytes / t / 1e9
+        per_m[f"M={M}"] = {"gbs": round(gbs, 1), "us_per_call": round(t * 1e6, 3),
+                           "frac_of_measured": round(gbs / peak, 4), "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                           "plan": plans[M].as_dict()}
 
     # ---- end-to-end through the public API with host buffers
-    e2e = run_e2e(wl, weights, plans, dev, max(5, args.steps // 100))
-
-    del graphs
+    e2e = run_e2e(wl, weights, plans, dev, max(5, args.steps // 10))
+    del g
     torch.cuda.synchronize()
+    breakdown = grouped = None
+    if not args.no_breakdown:
+        del weights
+        torch.cuda.empty_cache()
+        breakdown = run_breakdown(q, dev, peak)
+        grouped = run_grouped(q, dev, peak)
 
+    kernel = KERNEL_NAMES.get(plans[BENCH_MS[0]].kernel, "?")
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16 (fp16 dequantized weights x fp16 activations, fp32 accumulation)",
-        "data": "synthetic (seeded N(0,1) fp16 x and W, quantized by the library)",
-        "config": {"workload": "qo: K=4096 N=4096 4-bit g64 fp16, M in {1,4,5,6}",
-                   "weight_sets": len(weights), "calls_per_step": calls_per_step,
+        "dtype": "f16 (fp16 dequantized weights x fp16-converted bf16 activations, fp32 accumulation)",
+        "data": "synthetic (seeded N(0,1) bf16 x, N(0,0.02^2) bf16 W, quantized by the library)",
+        "config": {"workload": "lmhead: K=4096 N=151936 4-bit g64 bf16, M in {1,4,6,16}",
+                   "weight_sets": nsets, "calls_per_step": calls_per_step,
                    "weight_bytes_per_call": wbytes,
-                   "l2": f"rotated weight sets totalling {len(weights) * wbytes / 1e6:.0f} MB > 126 MB L2",
+                   "l2": f"one {wbytes / 1e6:.0f} MB weight matrix > 126 MB L2 (inputs larger than L2)",
                    "launch": "CUDA graph replay of the step", "eager_value_gbs": round(eager_value, 2),
-                   "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4)},
+                   "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4), "per_M": per_m},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(),
-                     "peak_kind": peak_kind, "kernel": KERNEL_NAMES.get(plans[BENCH_MS[0]].kernel, "?"),
-                     "algorithmic_bytes_per_launch": "weight bytes + 2*M*K (x) + 2*M*N (y)"},
-        "breakdown": breakdown,
+                     "peak_kind": peak_kind, "kernel": kernel,
+                     "algorithmic_bytes_per_launch": "weight bytes + 2*M*K (x) + 2*M*N (y), averaged over the "
+                                                     "step's calls; time = step time / calls (launch gaps included)"},
         "e2e": e2e,
-        "gpu_launches": calls_per_step * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
     }
+    if breakdown is not None:
+        out["breakdown"] = breakdown
+        out["grouped"] = grouped
     if clk:
+        clk["window"] = f"{CLOCK_SOAK_S:.1f} s of the same replays immediately before the timed region, and the timed region"
         out["clocks"] = clk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=12.0)
@@ -312,9 +488,9 @@ def run_ours(args, rank, world):
 
 def run_e2e(wl, weights, plans, dev, steps):
     """Each step through the Python API: the step's inputs (x for each M) go from pinned host
-    memory to the device, every call of the step runs with its own output, and all outputs
-    come back to pinned host memory; the weights stay resident, as a model's do.  The outputs
-    of one M go back on a copy stream while the calls of the next M run."""
+    memory to the device, every call of the step runs, and every output comes back to pinned
+    host memory; the weights stay resident, as a model's do.  The output of one M goes back on
+    a copy stream while the calls of the next M run."""
     import bit_quantized_gemm_qmm_b200 as q
     from bit_quantized_gemm_qmm_b200.inputs import x_input
     S = len(weights)
@@ -353,9 +529,10 @@ def run_e2e(wl, weights, plans, dev, steps):
             "calls_per_step": len(BENCH_MS) * S}
 
 
-# The sources that decide the benchmark's launches: the streaming kernel, the headers it is
-# compiled from, and the dispatch that picks it and its plan.
-TRAFFIC_SOURCES = ("qmm_api.cu", "qmm_common.cuh", "qmm_dq.cuh", "qmm_internal.h", "qmm_stream.cu", "sm100.cuh")
+# The sources that decide the benchmark's launches: the kernels, the headers they are
+# compiled from, and the dispatch that picks them and their plans.
+TRAFFIC_SOURCES = ("qmm_api.cu", "qmm_common.cuh", "qmm_dq.cuh", "qmm_internal.h", "qmm_sk.cu", "qmm_stream.cu",
+                   "sm100.cuh")
 
 
 def traffic_per_launch():
@@ -398,19 +575,21 @@ def _oracle_pass(wl, pq, xs, rows: int) -> float:
     return time.perf_counter() - t0
 
 
-def cpu_baseline(wl, budget_s: float = 12.0):
-    """The CPU oracle as it stands, on the host cores: whole calls (all N rows of one weight
-    set) for every M, repeated for about `budget_s` seconds."""
+def cpu_baseline(wl, budget_s: float = 12.0, rows: int = 8192):
+    """The CPU oracle as it stands, on the host cores: one call per M on the first `rows` rows
+    of the weight matrix, repeated for about `budget_s` seconds; GB/s counts the weight bytes
+    of those rows."""
     cores = int(os.environ.get("OMP_NUM_THREADS", host_cores()))
-    pq, xs = _oracle_inputs(wl, wl.N)
+    rows = min(rows, wl.N)
+    pq, xs = _oracle_inputs(wl, rows)
     t_total, passes = 0.0, 0
     while passes == 0 or t_total < budget_s:
-        t_total += _oracle_pass(wl, pq, xs, wl.N)
+        t_total += _oracle_pass(wl, pq, xs, rows)
         passes += 1
-    nbytes = passes * len(BENCH_MS) * wl.weight_bytes()
+    nbytes = passes * len(BENCH_MS) * wl.weight_bytes() * rows / wl.N
     return {"value": round(nbytes / t_total / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{passes} pass(es) of one full call per M in {list(BENCH_MS)} on weight set 0 "
-                      f"({t_total:.1f} s)"}
+            "sample": f"{passes} pass(es) of one call per M in {list(BENCH_MS)} on rows 0..{rows - 1} of the "
+                      f"{wl.N}-row weight matrix ({t_total:.1f} s)"}
 
 
 def run_reference(args, rank, world):
@@ -422,9 +601,10 @@ def run_reference(args, rank, world):
     from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS
     wl = WORKLOADS[WORKLOAD]
     cores = int(os.environ.get("OMP_NUM_THREADS", host_cores()))
-    pq, xs = _oracle_inputs(wl, wl.N)
-    t_full = _oracle_pass(wl, pq, xs, wl.N)
-    rows = int(min(wl.N, max(64, wl.N * (120.0 / max(1, args.steps + args.warmup)) / max(t_full, 1e-6))))
+    probe = min(wl.N, 4096)
+    pq, xs = _oracle_inputs(wl, probe)
+    t_probe = _oracle_pass(wl, pq, xs, probe)
+    rows = int(min(probe, max(64, probe * (120.0 / max(1, args.steps + args.warmup)) / max(t_probe, 1e-6))))
     for _ in range(args.warmup):
         _oracle_pass(wl, pq, xs, rows)
     t_total = 0.0
@@ -436,8 +616,8 @@ def run_reference(args, rank, world):
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_total * 1e3 / max(1, args.steps), 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
-           "data": "synthetic (seeded N(0,1) fp16 x and W)",
-           "config": {"workload": "qo: K=4096 N=4096 4-bit g64 fp16, M in {1,4,5,6}"},
+           "data": "synthetic (seeded N(0,1) bf16 x, N(0,0.02^2) bf16 W)",
+           "config": {"workload": "lmhead: K=4096 N=151936 4-bit g64 bf16, M in {1,4,6,16}"},
            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)

@@ -25,8 +25,8 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "qmm.h")
 
 QMM_OK, QMM_ERR_INVALID_ARG, QMM_ERR_UNSUPPORTED, QMM_ERR_CUDA = 0, 1, 2, 3
 QMM_F16, QMM_BF16 = 0, 1
-KERNEL_AUTO, KERNEL_MMA, KERNEL_TC, KERNEL_STREAM = 0, 1, 2, 3
-PLAN_PDL, PLAN_STATIC_WEIGHTS = 1, 2
+KERNEL_AUTO, KERNEL_MMA, KERNEL_TC, KERNEL_STREAM, KERNEL_SK = 0, 1, 2, 3, 4
+PLAN_PDL, PLAN_STATIC_WEIGHTS, PLAN_TEST_TIMEOUT = 1, 2, 1 << 30
 
 
 class QmmUnavailable(RuntimeError):
@@ -46,6 +46,11 @@ class Plan(ctypes.Structure):
 
     def as_dict(self):
         return {"kernel": self.kernel, "split": self.split, "warps": self.warps, "flags": self.flags}
+
+
+class Item(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("biases", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("N", ctypes.c_int64)]
 
 
 _lib = None
@@ -84,6 +89,8 @@ def lib() -> ctypes.CDLL:
     L.qmm_device_errors.restype = I
     L.qmm_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, I, I, U, P]
     L.qmm_noalloc.restype = I
+    L.qmm_grouped.argtypes = [P, ctypes.POINTER(Item), I, I64, I64, I, I, U, ctypes.POINTER(Plan), P]
+    L.qmm_grouped.restype = I
     _lib = L
     return L
 
@@ -255,6 +262,38 @@ def qmm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, biases: tor
     if st:
         _check(st)
     return out
+
+
+def qmm_grouped(x: torch.Tensor, weights, bits: int, group: int, outs=None, plan: Plan | None = None):
+    """[x . dequant(W_i)^T for each (packed, scales, biases) W_i in `weights`] in one launch:
+    up to four matrices that share x (a layer's q/k/v or gate/up projections).  Returns the
+    list of outputs [M, N_i] (or fills `outs`)."""
+    if not x.is_cuda or not x.is_contiguous() or x.dim() != 2:
+        raise ValueError("x must be a contiguous [M, K] CUDA tensor")
+    dev = x.get_device()
+    M, K = x.shape
+    if not 1 <= len(weights) <= 4:
+        raise ValueError("between one and four weight matrices")
+    if outs is None:
+        outs = [torch.empty((M, P.shape[0]), dtype=x.dtype, device=x.device) for (P, _, _) in weights]
+    items = (Item * len(weights))()
+    for i, ((P, S, B), y) in enumerate(zip(weights, outs)):
+        for t in (P, S, B, y):
+            if not (t.is_cuda and t.get_device() == dev and t.is_contiguous()):
+                raise ValueError("all tensors must be contiguous and on x's device")
+        N, KW = P.shape
+        if KW * 32 != K * bits or P.element_size() != 4:
+            raise ValueError(f"matrix {i}: packed has {KW} words per row; K={K} at {bits} bits needs {K * bits // 32}")
+        if S.dtype is not torch.float16 or B.dtype is not torch.float16 or S.numel() != N * (K // group) \
+                or B.numel() != N * (K // group):
+            raise ValueError(f"matrix {i}: scales and biases must be fp16 [N, K/group]")
+        if y.dtype is not x.dtype or tuple(y.shape) != (M, N):
+            raise ValueError(f"matrix {i}: output must be [M, N] = [{M}, {N}] in x's dtype")
+        items[i] = Item(P.data_ptr(), S.data_ptr(), B.data_ptr(), y.data_ptr(), N)
+    with torch.cuda.device(dev):
+        _check(lib().qmm_grouped(x.data_ptr(), items, len(weights), M, K, bits, group, _dtype_code(x.dtype),
+                                 None if plan is None else ctypes.byref(plan), _current_stream(dev)))
+    return outs
 
 
 def device_errors() -> int:

@@ -28,6 +28,16 @@ qmm_status cuda_fail(cudaError_t e, const char* what) {
     return fail(QMM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
+// A launch helper's result: cudaErrorNotSupported means the kernel turned the shape or the
+// arrays down before launching anything (for example a tensor map that cannot be encoded).
+qmm_status launch_result(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return QMM_OK;
+    if (e == cudaErrorNotSupported)
+        return fail(QMM_ERR_UNSUPPORTED, "%s: the kernel cannot describe these arrays (tensor map or "
+                    "scratch size); nothing was launched", what);
+    return cuda_fail(e, what);
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 bool bits_ok(int bits) { return bits == 4 || bits == 6 || bits == 8; }
@@ -46,7 +56,8 @@ qmm_status check_format(int64_t N, int64_t K, int bits, int group) {
 }
 
 constexpr int kNumSM = 148;
-constexpr int kMaxM = 64;
+constexpr int kMaxM = 64;                        // the small-M kernels' range
+constexpr int64_t kMaxTotalM = int64_t(1) << 20;  // larger M runs as chunks of up to 128 tokens
 
 int ceil_div(int64_t a, int64_t b) { return int((a + b - 1) / b); }
 int round_up(int64_t a, int64_t b) { return int((a + b - 1) / b * b); }
@@ -90,7 +101,7 @@ qmm_status validate_qmm(const void* x, const uint32_t* packed, const uint16_t* s
     if (s != QMM_OK) return s;
     if (dtype != QMM_F16 && dtype != QMM_BF16) return fail(QMM_ERR_INVALID_ARG, "dtype=%d", int(dtype));
     if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M=%lld", (long long)M);
-    if (M > kMaxM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %d", (long long)M, kMaxM);
+    if (M > kMaxTotalM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %lld", (long long)M, (long long)kMaxTotalM);
     if (M == 0 || N == 0) return QMM_OK;
     if (!y) return fail(QMM_ERR_INVALID_ARG, "y is null");
     if (!aligned(y, 16)) return fail(QMM_ERR_INVALID_ARG, "y must be 16-byte aligned");
@@ -116,11 +127,14 @@ bool prefer_tc(int64_t M, int64_t N, int64_t K) {
                      // 32-column tile) while the warp-tile kernel's grows; they cross near 28
 }
 
+constexpr bool kSkByDefault = false;
+
 struct Resolved {
     int kernel;
     MmaConfig mma;
     TcConfig tc;
     StreamConfig st;
+    SkConfig sk;
 };
 
 TcConfig tc_config(int64_t M, int64_t N, int64_t K, int bits, int split_req) {
@@ -158,16 +172,31 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
     memset(&p, 0, sizeof(p));
     if (in) p = *in;
     if (p.kernel != QMM_KERNEL_AUTO && p.kernel != QMM_KERNEL_MMA && p.kernel != QMM_KERNEL_TC &&
-        p.kernel != QMM_KERNEL_STREAM)
+        p.kernel != QMM_KERNEL_STREAM && p.kernel != QMM_KERNEL_SK)
         return fail(QMM_ERR_INVALID_ARG, "kernel=%d", p.kernel);
+    if (p.kernel == QMM_KERNEL_SK && (p.split < 0 || p.split > 2))
+        return fail(QMM_ERR_INVALID_ARG, "split=%d (the even-split kernel takes 0, 1 or 2: the x mode)", p.split);
     if (p.split < 0 || p.split > 16) return fail(QMM_ERR_INVALID_ARG, "split=%d (1..16)", p.split);
-    if (p.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS))
+    if (p.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS | QMM_PLAN_TEST_TIMEOUT))
         return fail(QMM_ERR_INVALID_ARG, "unknown plan flags 0x%x", p.flags);
+    if ((p.flags & QMM_PLAN_TEST_TIMEOUT) && p.kernel != QMM_KERNEL_SK)
+        return fail(QMM_ERR_INVALID_ARG, "QMM_PLAN_TEST_TIMEOUT applies to the even-split kernel only");
+    if (M > kMaxM) {
+        // prefill-sized M: only the even-split kernel covers it (up to 128 tokens a launch)
+        if (p.kernel != QMM_KERNEL_AUTO && p.kernel != QMM_KERNEL_SK)
+            return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %d runs on the even-split kernel only", (long long)M, kMaxM);
+        p.kernel = QMM_KERNEL_SK;
+    }
     const bool tc_ok = tc_supported(M, N, K, bits, group) && aligned(scales, 4) && aligned(biases, 4);
     const bool st_shape = stream_supported(M, N, K, bits, group) && aligned(scales, 16) && aligned(biases, 16);
     StreamConfig stc = {};
-    if (st_shape) stc = stream_config(M, N, K, bits, group, p.split);
+    if (st_shape && p.kernel != QMM_KERNEL_SK) stc = stream_config(M, N, K, bits, group, p.split);
     const bool st_ok = stc.ring >= 2;
+    const bool sk_shape = sk_supported(M, N, K, bits, group) && aligned(scales, 16) && aligned(biases, 16);
+    SkConfig skc = {};
+    if (sk_shape) skc = sk_config(M, N, K, bits, group, p.kernel == QMM_KERNEL_SK ? p.split : 0);
+    const bool sk_ok = sk_shape && skc.ok;
+    if (p.kernel == QMM_KERNEL_AUTO && sk_ok && kSkByDefault) p.kernel = QMM_KERNEL_SK;
     if (p.kernel == QMM_KERNEL_AUTO) {
         // the streaming kernel up to M = 8, and up to 16 while staging x still leaves room
         // for a 4-stage ring (or for all the stages a block streams) without splitting K
@@ -183,6 +212,10 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
         return fail(QMM_ERR_UNSUPPORTED,
                     "streaming kernel needs 1 <= M <= 16, K a multiple of 8 groups, a 16-byte "
                     "multiple of packed bytes per row and 16-byte aligned scales/biases");
+    if (p.kernel == QMM_KERNEL_SK && !sk_ok)
+        return fail(QMM_ERR_UNSUPPORTED,
+                    "even-split kernel needs a multiple of 8 groups per row, a 16-byte multiple of packed "
+                    "bytes per row and 16-byte aligned scales/biases (and so does any M > %d)", kMaxM);
     if (p.kernel == QMM_KERNEL_TC && !tc_ok)
         return fail(QMM_ERR_UNSUPPORTED,
                     "tensor-core kernel needs K >= 128, an even number of groups per row, a 16-byte "
@@ -213,6 +246,14 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
         p.warps = 9;
         p.split = c.split;
         res.st = c;
+    } else if (p.kernel == QMM_KERNEL_SK) {
+        SkConfig c = skc;
+        c.pdl = pdl;
+        c.static_weights = stat;
+        c.test_timeout = (p.flags & QMM_PLAN_TEST_TIMEOUT) != 0;
+        p.warps = 20;
+        p.split = c.x_staged ? 1 : 2;
+        res.sk = c;
     } else {
         TcConfig c = tc_config(M, N, K, bits, p.split);
         c.pdl = pdl;
@@ -222,7 +263,8 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
         p.split = ceil_div(ceil_div(K, tc_kc(bits)), c.stages_per_split);
         res.tc = c;
     }
-    p.flags = (pdl ? QMM_PLAN_PDL : 0u) | (stat ? QMM_PLAN_STATIC_WEIGHTS : 0u);
+    p.flags = (pdl ? QMM_PLAN_PDL : 0u) | (stat ? QMM_PLAN_STATIC_WEIGHTS : 0u) |
+              (p.flags & QMM_PLAN_TEST_TIMEOUT);
     if (out) *out = p;
     if (r) *r = res;
     return QMM_OK;
@@ -282,8 +324,9 @@ qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group
     if (s != QMM_OK) return s;
     if (dtype != QMM_F16 && dtype != QMM_BF16) return fail(QMM_ERR_INVALID_ARG, "dtype=%d", int(dtype));
     if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M");
-    if (M > kMaxM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %d", (long long)M, kMaxM);
+    if (M > kMaxTotalM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %lld", (long long)M, (long long)kMaxTotalM);
     if (!plan) return fail(QMM_ERR_INVALID_ARG, "plan is null");
+    if (M > kSkMaxTokens) M = kSkMaxTokens;  // the plan of each chunk
     // the default plan assumes 4-byte aligned scales and biases (any allocation is)
     return resolve_plan(M, N, K, bits, group, nullptr, reinterpret_cast<const void*>(16),
                         reinterpret_cast<const void*>(16), plan, nullptr);
@@ -300,6 +343,20 @@ qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
         cudaError_t e = cudaMemsetAsync(y, 0, size_t(M) * size_t(N) * 2, st);
         return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm zero fill");
     }
+    if (M > kSkMaxTokens) {
+        // chunks of at most 128 tokens, as even as possible; each streams the weights once
+        const int64_t nch = (M + kSkMaxTokens - 1) / kSkMaxTokens;
+        const size_t esz = 2;
+        int64_t m0 = 0;
+        for (int64_t i = 0; i < nch; ++i) {
+            const int64_t mc = (M - m0) / (nch - i);
+            s = qmm_ex(static_cast<const char*>(x) + size_t(m0) * size_t(K) * esz, packed, scales, biases,
+                       static_cast<char*>(y) + size_t(m0) * size_t(N) * esz, mc, N, K, bits, group, dtype, plan, stream);
+            if (s != QMM_OK) return s;
+            m0 += mc;
+        }
+        return QMM_OK;
+    }
     Resolved r;
     s = resolve_plan(M, N, K, bits, group, plan, scales, biases, nullptr, &r);
     if (s != QMM_OK) return s;
@@ -315,10 +372,11 @@ qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
     a.bits = bits;
     a.group = group;
     a.is_bf16 = dtype == QMM_BF16;
-    cudaError_t e = r.kernel == QMM_KERNEL_TC       ? launch_tc(a, r.tc, st)
+    cudaError_t e = r.kernel == QMM_KERNEL_SK       ? launch_sk(a, r.sk, st)
+                    : r.kernel == QMM_KERNEL_TC     ? launch_tc(a, r.tc, st)
                     : r.kernel == QMM_KERNEL_STREAM ? launch_stream(a, r.st, st)
                                                     : launch_mma(a, r.mma, st);
-    return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm launch");
+    return launch_result(e, "qmm launch");
 }
 
 qmm_status qmm(const void* x, const uint32_t* packed, const uint16_t* scales,
@@ -327,11 +385,78 @@ qmm_status qmm(const void* x, const uint32_t* packed, const uint16_t* scales,
     return qmm_ex(x, packed, scales, biases, y, M, N, K, bits, group, dtype, nullptr, stream);
 }
 
+qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t M, int64_t K,
+                       int bits, int group, qmm_dtype dtype, const qmm_plan* plan, void* stream) {
+    if (count < 1 || count > kSkMaxItems) return fail(QMM_ERR_INVALID_ARG, "count=%d (1..%d)", count, kSkMaxItems);
+    if (!items) return fail(QMM_ERR_INVALID_ARG, "items is null");
+    if (dtype != QMM_F16 && dtype != QMM_BF16) return fail(QMM_ERR_INVALID_ARG, "dtype=%d", int(dtype));
+    if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M=%lld", (long long)M);
+    if (M > kSkMaxTokens) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %d", (long long)M, kSkMaxTokens);
+    SkItem live[kSkMaxItems];
+    int n = 0;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        qmm_status st = check_format(items[i].N, K, bits, group);
+        if (st != QMM_OK) return st;
+        if (items[i].N == 0) continue;
+        if (M > 0 && (!items[i].y || !aligned(items[i].y, 16)))
+            return fail(QMM_ERR_INVALID_ARG, "item %d: y must be a 16-byte aligned pointer", i);
+        live[n++] = SkItem{items[i].packed, items[i].scales, items[i].biases, static_cast<uint16_t*>(items[i].y),
+                           items[i].N};
+        tiles += (items[i].N + 127) / 128;
+    }
+    if (M == 0 || n == 0) return QMM_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) {
+        for (int i = 0; i < n; ++i) {
+            cudaError_t e = cudaMemsetAsync(live[i].y, 0, size_t(M) * size_t(live[i].N) * 2, st);
+            if (e != cudaSuccess) return cuda_fail(e, "qmm_grouped zero fill");
+        }
+        return QMM_OK;
+    }
+    if (!x || !aligned(x, 16)) return fail(QMM_ERR_INVALID_ARG, "x must be a 16-byte aligned pointer");
+    for (int i = 0; i < n; ++i) {
+        if (!live[i].packed || !live[i].scales || !live[i].biases)
+            return fail(QMM_ERR_INVALID_ARG, "item %d: null weight pointer", i);
+        if (!aligned(live[i].packed, 16) || !aligned(live[i].scales, 16) || !aligned(live[i].biases, 16))
+            return fail(QMM_ERR_UNSUPPORTED, "item %d: grouped calls need 16-byte aligned packed/scales/biases", i);
+        if (!sk_supported(M, live[i].N, K, bits, group))
+            return fail(QMM_ERR_UNSUPPORTED,
+                        "item %d: grouped calls run on the even-split kernel, which needs a multiple of 8 groups "
+                        "per row and a 16-byte multiple of packed bytes per row", i);
+    }
+    qmm_plan pl;
+    memset(&pl, 0, sizeof(pl));
+    if (plan) pl = *plan;
+    if (pl.kernel != QMM_KERNEL_AUTO && pl.kernel != QMM_KERNEL_SK)
+        return fail(QMM_ERR_INVALID_ARG, "grouped calls run on the even-split kernel (kernel=%d)", pl.kernel);
+    if (pl.split < 0 || pl.split > 2) return fail(QMM_ERR_INVALID_ARG, "split=%d (x mode 0, 1 or 2)", pl.split);
+    if (pl.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS))
+        return fail(QMM_ERR_INVALID_ARG, "unknown or unsupported plan flags 0x%x", pl.flags);
+    if (tiles * 128 > (int64_t(1) << 30)) return fail(QMM_ERR_UNSUPPORTED, "too many rows in one grouped call");
+    SkConfig c = sk_config(M, tiles * 128, K, bits, group, pl.split);
+    if (!c.ok) return fail(QMM_ERR_UNSUPPORTED, "even-split plan does not fit shared memory");
+    c.pdl = plan ? (pl.flags & QMM_PLAN_PDL) != 0 : true;
+    c.static_weights = plan ? (pl.flags & QMM_PLAN_STATIC_WEIGHTS) != 0 : false;
+    c.test_timeout = false;
+    QmmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = static_cast<const uint16_t*>(x);
+    a.M = M;
+    a.N = tiles * 128;
+    a.K = K;
+    a.bits = bits;
+    a.group = group;
+    a.is_bf16 = dtype == QMM_BF16;
+    return launch_result(launch_sk_items(a, live, n, c, st), "qmm_grouped launch");
+}
+
 qmm_status qmm_noalloc(const void* x, const uint32_t* packed, const uint16_t* scales,
                        const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                        int group, qmm_dtype dtype, void* stream) {
     qmm_status s = validate_qmm(x, packed, scales, biases, y, M, N, K, bits, group, dtype);
     if (s != QMM_OK) return s;
+    if (M > kMaxM) return fail(QMM_ERR_UNSUPPORTED, "qmm_noalloc takes M <= %d", kMaxM);
     if (M == 0 || N == 0 || K == 0)
         return fail(QMM_ERR_UNSUPPORTED, "qmm_noalloc needs M, N, K > 0 (use qmm for empty shapes)");
     if (!tc_supported(M, N, K, bits, group) || !aligned(scales, 4) || !aligned(biases, 4))
@@ -359,7 +484,7 @@ qmm_status qmm_noalloc(const void* x, const uint32_t* packed, const uint16_t* sc
     a.group = group;
     a.is_bf16 = dtype == QMM_BF16;
     cudaError_t e = launch_tc_noalloc(a, c, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm_noalloc launch");
+    return launch_result(e, "qmm_noalloc launch");
 }
 
 const char* qmm_status_string(qmm_status status) {
@@ -382,7 +507,10 @@ qmm_status qmm_device_errors(uint32_t* bits) {
     unsigned w = 0;
     e = stream_read_and_clear_errors(&w);
     if (e != cudaSuccess) return cuda_fail(e, "qmm_device_errors");
-    *bits = v | w;
+    unsigned z = 0;
+    e = sk_read_and_clear_errors(&z);
+    if (e != cudaSuccess) return cuda_fail(e, "qmm_device_errors");
+    *bits = v | w | z;
     return QMM_OK;
 }
 

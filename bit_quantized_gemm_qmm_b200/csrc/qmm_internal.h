@@ -78,6 +78,40 @@ struct StreamConfig {
     bool static_weights;
 };
 bool stream_supported(int64_t M, int64_t N, int64_t K, int bits, int group);
+
+// Fully resolved launch configuration of the evenly split tensor-core kernel (qmm_sk.cu).
+struct SkConfig {
+    int mp;          // MMA N: M rounded up to a multiple of 16 (16..128)
+    int T, S, U;     // 128-row tiles, 256-code stages per tile, units (T * S)
+    int per, grid;   // units per block, blocks
+    bool x_staged;   // x staged in shared memory by the kernel (else by a small kernel, per call)
+    int nslots;      // x stages in shared memory (staged mode)
+    int sc, sx;      // code ring and x ring depths
+    size_t smem;     // dynamic shared memory per block
+    bool ok;         // the configuration fits
+    bool pdl;
+    bool static_weights;
+    bool test_timeout;  // testing aid (QMM_PLAN_TEST_TIMEOUT)
+};
+constexpr int kSkMaxTokens = 128;  // tokens one launch of the even-split kernel covers
+bool sk_supported(int64_t M, int64_t N, int64_t K, int bits, int group);
+// xmode: 0 = choose, 1 = x staged in shared memory, 2 = x staged in the workspace
+SkConfig sk_config(int64_t M, int64_t N, int64_t K, int bits, int group, int xmode);
+cudaError_t launch_sk(const QmmArgs& a, const SkConfig& c, cudaStream_t stream);
+// One launch over several weight matrices that share x (a's packed/scales/biases/y/N are
+// ignored; the matrices come from `items`).  c must come from sk_config with N = 128 * the
+// total of the matrices' 128-row tiles.
+struct SkItem {
+    const uint32_t* packed;
+    const uint16_t* scales;
+    const uint16_t* biases;
+    uint16_t* y;
+    int64_t N;
+};
+constexpr int kSkMaxItems = 4;
+cudaError_t launch_sk_items(const QmmArgs& a, const SkItem* items, int nitems, const SkConfig& c,
+                            cudaStream_t stream);
+cudaError_t sk_read_and_clear_errors(unsigned* out);
 StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group, int split_req);
 cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream);
 cudaError_t stream_read_and_clear_errors(unsigned* out);

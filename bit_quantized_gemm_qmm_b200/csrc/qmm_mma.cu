@@ -313,7 +313,7 @@ size_t mma_smem_bytes(const MmaConfig& c) {
 
 cudaError_t launch_mma(const QmmArgs& a, const MmaConfig& c, cudaStream_t stream) {
     KernelFn fn = pick_kernel(a.bits, c.mt, c.warps);
-    if (!fn) return cudaErrorInvalidValue;
+    if (!fn) return cudaErrorNotSupported;
     Params p;
     p.x = a.x;
     p.packed = a.packed;

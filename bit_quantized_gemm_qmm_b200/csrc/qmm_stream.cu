@@ -686,11 +686,11 @@ cudaError_t ensure_smem_attr(StKernelFn fn, size_t smem) {
 cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream) {
     const int mt = int(a.M) > 8 ? 2 : 1;
     StKernelFn fn = pick_stream(a.bits, mt, c.ncw);
-    if (!fn || c.ring < 2) return cudaErrorInvalidValue;
+    if (!fn || c.ring < 2) return cudaErrorNotSupported;
     // The three descriptors depend only on the weight arrays and the format; a call that
     // repeats them (the usual case: the same weights every step) reuses the encoded copies.
     const StMaps* maps = weight_maps(a);
-    if (!maps) return cudaErrorInvalidValue;
+    if (!maps) return cudaErrorNotSupported;
 
     StParams p;
     p.x = a.x;

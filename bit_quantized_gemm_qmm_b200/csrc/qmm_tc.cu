@@ -45,29 +45,6 @@ namespace qmm_impl {
 // qmm_device_errors().
 __device__ unsigned int g_tc_error = 0;
 
-#ifdef QMM_TC_TRACE
-// Pipeline trace of block (0,0) for performance analysis (built only with -DQMM_TC_TRACE):
-// g_tc_trace[event * 256 + stage] = %globaltimer at that event.
-__device__ unsigned long long g_tc_trace[16 * 256];
-__device__ unsigned long long g_tc_blocks[4096 * 8];  // per block: start, end, smid, nstages, clk0, clk1
-__device__ __forceinline__ unsigned long long gtimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void tc_trace(int ev, int i) {
-    if (blockIdx.x == 0 && blockIdx.y == 0 && i < 256) g_tc_trace[ev * 256 + i] = gtimer();
-}
-__device__ __forceinline__ void tc_trace_block(int which, unsigned long long v) {
-    const int b = blockIdx.y * gridDim.x + blockIdx.x;
-    if (b < 4096) g_tc_blocks[b * 8 + which] = v;
-}
-#define TC_TRACE(ev, i) tc_trace(ev, i)
-#define TC_TRACE_BLOCK(which, v) tc_trace_block(which, v)
-#else
-#define TC_TRACE(ev, i) ((void)0)
-#define TC_TRACE_BLOCK(which, v) ((void)0)
-#endif
 
 namespace {
 
@@ -253,16 +230,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) TC_TRACE(9, 0);
-#ifdef QMM_TC_TRACE
-    if (threadIdx.x == 0) {
-        unsigned smid;
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        TC_TRACE_BLOCK(0, gtimer());
-        TC_TRACE_BLOCK(2, smid);
-        TC_TRACE_BLOCK(4, clock64());
-    }
-#endif
     const int n0 = blockIdx.x * TC_ROWS;
     const int st0 = blockIdx.y * p.stages_per_split;
     const int nst = min(p.stages_per_split, p.nstages_k - st0);
@@ -323,7 +290,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     break;
                 }
                 if (*abort_flag) break;
-                TC_TRACE(0, i);
                 mbar_arrive_expect_tx(bar_full + 8 * s, uint32_t(F::W_BYTES));
                 tma_load_2d(sbase + L.w_off + s * L.w_stage, &wmap, bar_full + 8 * s, (st0 + i) * WCOLS, n0);
                 issued = i + 1;
@@ -401,7 +367,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         uint32_t ph = 0, pa = 0;
         for (int i = 0; i < nst; ++i) {
             const bool got_full = mbar_wait(bar_xfull + 8 * s, ph, deadline);
-            if (j == 0 && lane == 0) TC_TRACE(10, i);
             if (!got_full || !mbar_wait(bar_afull + 8 * a, pa, deadline)) {
                 if (lane == 0) {
                     set_error(1u);
@@ -410,7 +375,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 break;
             }
             tc_fence_after();
-            if (j == 0 && lane == 0) TC_TRACE(1, i);
             const uint32_t xs = sbase + L.x_off + s * L.x_stage;
             const uint32_t acol = tmem + F::ACC_COLS + F::A_COLS * a;
             if (elect_one()) {
@@ -423,7 +387,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 umma_commit(bar_aempty + 8 * a);
             }
             __syncwarp();
-            if (j == 0 && lane == 0) TC_TRACE(2, i);
             if (++s == S) {
                 s = 0;
                 ph ^= 1u;
@@ -482,7 +445,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 *abort_flag = 1;
                 break;
             }
-            if (warp == TC_DQ0 && lane == 0) TC_TRACE(3, i);
             // the thread's codes into registers; the code slot is free again at once
             uint32_t wd[TcWords<BITS>::N];
             load_quarter<BITS>(sbase + L.w_off + s * L.w_stage + row * F::ROW_BYTES, row, quarter, wd);
@@ -513,7 +475,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     sph ^= 1u;
                 }
             }
-            if (warp == TC_DQ0 && lane == 0) TC_TRACE(4, i);
             if (!STMA) issue_scales(i + TC_SPF);
             if (i >= F::NA && !mbar_wait(bar_aempty + 8 * a, pa ^ 1u, deadline)) {
                 set_error(1u);
@@ -530,7 +491,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (warp == TC_DQ0 && lane == 0) TC_TRACE(6, i);
             if (lane == 0) mbar_arrive(bar_afull + 8 * a);
             if (++s == S) {
                 s = 0;
@@ -558,7 +518,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (dq_warp) {
         const long long d2 = clock64() + TC_TIMEOUT_CYCLES;
         const bool have_acc = mbar_wait(bar_acc, 0, d2);
-        if (warp == TC_DQ0 && lane == 0) TC_TRACE(8, 0);
         if (!have_acc) set_error(1u);
         tc_fence_after();
         const bool ok = have_acc && *abort_flag == 0;
@@ -640,13 +599,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
 
     // ---------------------------------------------------------------- teardown
-#ifdef QMM_TC_TRACE
-    if (threadIdx.x == 0) {
-        TC_TRACE_BLOCK(1, gtimer());
-        TC_TRACE_BLOCK(3, nst);
-        TC_TRACE_BLOCK(5, clock64());
-    }
-#endif
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, TC_TMEM_COLS);
@@ -870,28 +822,70 @@ size_t tc_smem_bytes(int bits, int mp, int ring) {
     return body + 1024;  // alignment slack
 }
 
-cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) {
-    const int KC = kc_for(a.bits);
-    const int nst_k = int((a.K + KC - 1) / KC);
-    const bool stma = tc_scale_tma_ok(a, c.stages_per_split, (nst_k + c.stages_per_split - 1) / c.stages_per_split);
-    TcKernelFn fn = pick_tc(a.bits, c.mp, stma);
-    if (!fn) return cudaErrorInvalidValue;
+// Everything a tensor-core call needs before its first launch: the kernel, its three tensor
+// maps, its parameters (all but the scratch pointers) and its launch shape.  Computed in
+// full before anything is enqueued, so a call that cannot run launches nothing.
+struct TcLaunch {
+    TcKernelFn fn;
+    CUtensorMap wmap, smap, bmap;
+    TcParams p;
+    int nst_k, KC;
+    size_t xt_bytes, smem;
+};
 
-    // stage tiles of x (fp16) and the per-token exponents, in stream-ordered scratch memory
-    cudaMemPool_t pool;
-    cudaError_t e = device_pool(&pool);
+// cudaErrorNotSupported: the shape or the arrays do not suit the kernel (nothing launched;
+// the API reports QMM_ERR_UNSUPPORTED).
+static cudaError_t tc_prepare(const QmmArgs& a, const TcConfig& c, TcLaunch* L) {
+    L->KC = kc_for(a.bits);
+    L->nst_k = int((a.K + L->KC - 1) / L->KC);
+    const int split = (L->nst_k + c.stages_per_split - 1) / c.stages_per_split;
+    const bool stma = tc_scale_tma_ok(a, c.stages_per_split, split);
+    L->fn = pick_tc(a.bits, c.mp, stma);
+    if (!L->fn || c.ring < 2) return cudaErrorNotSupported;
+    L->xt_bytes = size_t(L->nst_k) * size_t(c.mp) * size_t(L->KC) * 2;
+    const uint64_t KW = uint64_t(a.K) * a.bits / 32;
+    const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_map_2d(&L->wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
+                     uint32_t(L->KC * a.bits / 32), TC_ROWS, wsw))
+        return cudaErrorNotSupported;
+    L->smap = L->wmap;  // unused unless stma
+    L->bmap = L->wmap;
+    if (stma && !make_scale_maps(a, &L->smap, &L->bmap)) return cudaErrorNotSupported;
+    TcParams& p = L->p;
+    p.scales = a.scales;
+    p.biases = a.biases;
+    p.y = a.y;
+    p.xt = nullptr;
+    p.xexp = nullptr;
+    p.M = int(a.M);
+    p.N = int(a.N);
+    p.K = int(a.K);
+    p.G = int(a.K / a.group);
+    p.gshift = a.group == 32 ? 5 : a.group == 64 ? 6 : 7;
+    p.nstages_k = L->nst_k;
+    p.stages_per_split = c.stages_per_split;
+    p.split = split;
+    p.out_bf16 = a.is_bf16;
+    p.static_w = c.static_weights ? 1 : 0;
+    p.ring = c.ring;
+    L->smem = tc_smem_bytes(a.bits, c.mp, c.ring);
+    cudaError_t e = cudaFuncSetAttribute(L->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L->smem));
     if (e != cudaSuccess) return e;
-    const size_t xt_bytes = size_t(nst_k) * size_t(c.mp) * size_t(KC) * 2;
-    void* ws = nullptr;
-    e = cudaMallocFromPoolAsync(&ws, xt_bytes + 64 * sizeof(int), pool, stream);
-    if (e != cudaSuccess) return e;
-    auto finish = [&](cudaError_t err) {
-        cudaError_t f = cudaFreeAsync(ws, stream);  // after everything enqueued above
-        return err == cudaSuccess ? f : err;
-    };
-    uint16_t* xt = static_cast<uint16_t*>(ws);
-    int* xexp = a.is_bf16 ? reinterpret_cast<int*>(static_cast<char*>(ws) + xt_bytes) : nullptr;
+    if (p.split > 8) {
+        e = cudaFuncSetAttribute(L->fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
 
+// Enqueue the x kernel and the tensor-core kernel of a prepared call, with the fp16 x tiles
+// at `xt` (xt_bytes) and, for bf16 activations, the per-token exponents at `xexp` (64 ints).
+// The x kernel waits for the previous grid in the stream before it writes `xt`, so calls
+// that share the scratch on one stream never overlap on it.
+static cudaError_t tc_enqueue(const QmmArgs& a, const TcConfig& c, TcLaunch* L, uint16_t* xt, int* xexp,
+                              cudaStream_t stream) {
+    L->p.xt = xt;
+    L->p.xexp = a.is_bf16 ? xexp : nullptr;
     cudaLaunchAttribute pdl_attr;
     pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl_attr.val.programmaticStreamSerializationAllowed = 1;
@@ -901,63 +895,47 @@ cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) 
     pc.stream = stream;
     pc.attrs = &pdl_attr;
     pc.numAttrs = c.pdl ? 1 : 0;
-    e = a.bits == 4   ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 4>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
-        : a.bits == 6 ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 6>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
-                      : cudaLaunchKernelEx(&pc, xprep_kernel<128, 8>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp);
-    if (e != cudaSuccess) return finish(e);
-
-    CUtensorMap wmap;
-    const uint64_t KW = uint64_t(a.K) * a.bits / 32;
-    const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
-    if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
-                     uint32_t(KC * a.bits / 32), TC_ROWS, wsw))
-        return finish(cudaErrorInvalidValue);
-    CUtensorMap smap = wmap, bmap = wmap;  // unused unless stma
-    if (stma && !make_scale_maps(a, &smap, &bmap)) return finish(cudaErrorInvalidValue);
-
-    TcParams p;
-    p.scales = a.scales;
-    p.biases = a.biases;
-    p.y = a.y;
-    p.xt = xt;
-    p.xexp = xexp;
-    p.M = int(a.M);
-    p.N = int(a.N);
-    p.K = int(a.K);
-    p.G = int(a.K / a.group);
-    p.gshift = a.group == 32 ? 5 : a.group == 64 ? 6 : 7;
-    p.nstages_k = nst_k;
-    p.stages_per_split = c.stages_per_split;
-    p.split = (nst_k + c.stages_per_split - 1) / c.stages_per_split;
-    p.out_bf16 = a.is_bf16;
-    p.static_w = c.static_weights ? 1 : 0;
-    p.ring = c.ring;
-
-    const size_t smem = tc_smem_bytes(a.bits, c.mp, c.ring);
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return finish(e);
-    if (p.split > 8) {
-        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return finish(e);
-    }
+    int* xe = L->p.xexp ? xexp : nullptr;
+    cudaError_t e =
+        a.bits == 4   ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 4>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, L->nst_k, xt, xe)
+        : a.bits == 6 ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 6>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, L->nst_k, xt, xe)
+                      : cudaLaunchKernelEx(&pc, xprep_kernel<128, 8>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, L->nst_k, xt, xe);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned((a.N + TC_ROWS - 1) / TC_ROWS), unsigned(p.split), 1);
+    cfg.gridDim = dim3(unsigned((a.N + TC_ROWS - 1) / TC_ROWS), unsigned(L->p.split), 1);
     cfg.blockDim = dim3(TC_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = L->smem;
     cfg.stream = stream;
     cudaLaunchAttribute attrs[2];
     int na = 0;
-    if (p.split > 1) {
+    if (L->p.split > 1) {
         attrs[na].id = cudaLaunchAttributeClusterDimension;
         attrs[na].val.clusterDim.x = 1;
-        attrs[na].val.clusterDim.y = unsigned(p.split);
+        attrs[na].val.clusterDim.y = unsigned(L->p.split);
         attrs[na].val.clusterDim.z = 1;
         ++na;
     }
     if (c.pdl) attrs[na++] = pdl_attr;
     cfg.attrs = attrs;
     cfg.numAttrs = unsigned(na);
-    return finish(cudaLaunchKernelEx(&cfg, fn, wmap, smap, bmap, p));
+    return cudaLaunchKernelEx(&cfg, L->fn, L->wmap, L->smap, L->bmap, L->p);
+}
+
+cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) {
+    TcLaunch L;
+    cudaError_t e = tc_prepare(a, c, &L);
+    if (e != cudaSuccess) return e;
+    // stage tiles of x (fp16) and the per-token exponents, in stream-ordered scratch memory
+    cudaMemPool_t pool;
+    e = device_pool(&pool);
+    if (e != cudaSuccess) return e;
+    void* ws = nullptr;
+    e = cudaMallocFromPoolAsync(&ws, L.xt_bytes + 64 * sizeof(int), pool, stream);
+    if (e != cudaSuccess) return e;
+    e = tc_enqueue(a, c, &L, static_cast<uint16_t*>(ws),
+                   reinterpret_cast<int*>(static_cast<char*>(ws) + L.xt_bytes), stream);
+    const cudaError_t f = cudaFreeAsync(ws, stream);  // after everything enqueued above
+    return e == cudaSuccess ? f : e;
 }
 
 // How many clusters of `split` blocks of this kernel can be resident at once (0 if the query
@@ -1000,14 +978,6 @@ int tc_max_active_clusters(int bits, int mp, int ring, int split) {
     return n;
 }
 
-#ifdef QMM_TC_TRACE
-extern "C" cudaError_t qmm_tc_trace_read(unsigned long long* host16x256) {
-    return cudaMemcpyFromSymbol(host16x256, g_tc_trace, sizeof(g_tc_trace));
-}
-extern "C" cudaError_t qmm_tc_trace_blocks(unsigned long long* host4096x8) {
-    return cudaMemcpyFromSymbol(host4096x8, g_tc_blocks, sizeof(g_tc_blocks));
-}
-#endif
 
 cudaError_t tc_read_and_clear_errors(unsigned* out) {
     unsigned v = 0, zero = 0;
@@ -1071,85 +1041,18 @@ size_t tc_noalloc_need(int64_t M, int64_t K, int bits) {
 size_t tc_noalloc_capacity() { return kNoAllocXBytes; }
 
 cudaError_t launch_tc_noalloc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream) {
-    const int KC = kc_for(a.bits);
-    const int nst_k = int((a.K + KC - 1) / KC);
-    const bool stma = tc_scale_tma_ok(a, c.stages_per_split, (nst_k + c.stages_per_split - 1) / c.stages_per_split);
-    TcKernelFn fn = pick_tc(a.bits, c.mp, stma);
-    if (!fn) return cudaErrorInvalidValue;
-    const size_t xt_bytes = size_t(nst_k) * size_t(c.mp) * size_t(KC) * 2;
-    if (xt_bytes > kNoAllocXBytes) return cudaErrorInvalidValue;
+    TcLaunch L;
+    cudaError_t e = tc_prepare(a, c, &L);
+    if (e != cudaSuccess) return e;
+    if (L.xt_bytes > kNoAllocXBytes) return cudaErrorNotSupported;
     void* ws = nullptr;
-    cudaError_t e = noalloc_scratch(&ws);
+    e = noalloc_scratch(&ws);
     if (e != cudaSuccess) return e;
-    uint16_t* xt = static_cast<uint16_t*>(ws);
-    int* xexp = a.is_bf16 ? reinterpret_cast<int*>(static_cast<char*>(ws) + kNoAllocXBytes) : nullptr;
-
-    cudaLaunchAttribute pdl_attr;
-    pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl_attr.val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t pc = {};
-    pc.gridDim = dim3(unsigned(c.mp), 1, 1);
-    pc.blockDim = dim3(256, 1, 1);
-    pc.stream = stream;
-    pc.attrs = &pdl_attr;
-    pc.numAttrs = c.pdl ? 1 : 0;
-    e = a.bits == 4   ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 4>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
-        : a.bits == 6 ? cudaLaunchKernelEx(&pc, xprep_kernel<256, 6>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp)
-                      : cudaLaunchKernelEx(&pc, xprep_kernel<128, 8>, a.x, int(a.M), int(a.K), a.is_bf16, c.mp, nst_k, xt, xexp);
-    if (e != cudaSuccess) return e;
-
-    CUtensorMap wmap;
-    const uint64_t KW = uint64_t(a.K) * a.bits / 32;
-    const CUtensorMapSwizzle wsw = a.bits == 6 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
-    if (!make_map_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, KW, uint64_t(a.N),
-                     uint32_t(KC * a.bits / 32), TC_ROWS, wsw))
-        return cudaErrorInvalidValue;
-    CUtensorMap smap = wmap, bmap = wmap;  // unused unless stma
-    if (stma && !make_scale_maps(a, &smap, &bmap)) return cudaErrorInvalidValue;
-
-    TcParams p;
-    p.scales = a.scales;
-    p.biases = a.biases;
-    p.y = a.y;
-    p.xt = xt;
-    p.xexp = xexp;
-    p.M = int(a.M);
-    p.N = int(a.N);
-    p.K = int(a.K);
-    p.G = int(a.K / a.group);
-    p.gshift = a.group == 32 ? 5 : a.group == 64 ? 6 : 7;
-    p.nstages_k = nst_k;
-    p.stages_per_split = c.stages_per_split;
-    p.split = (nst_k + c.stages_per_split - 1) / c.stages_per_split;
-    p.out_bf16 = a.is_bf16;
-    p.static_w = c.static_weights ? 1 : 0;
-    p.ring = c.ring;
-
-    const size_t smem = tc_smem_bytes(a.bits, c.mp, c.ring);
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    if (p.split > 8) {
-        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned((a.N + TC_ROWS - 1) / TC_ROWS), unsigned(p.split), 1);
-    cfg.blockDim = dim3(TC_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attrs[2];
-    int na = 0;
-    if (p.split > 1) {
-        attrs[na].id = cudaLaunchAttributeClusterDimension;
-        attrs[na].val.clusterDim.x = 1;
-        attrs[na].val.clusterDim.y = unsigned(p.split);
-        attrs[na].val.clusterDim.z = 1;
-        ++na;
-    }
-    if (c.pdl) attrs[na++] = pdl_attr;
-    cfg.attrs = attrs;
-    cfg.numAttrs = unsigned(na);
-    return cudaLaunchKernelEx(&cfg, fn, wmap, smap, bmap, p);
+    // the x kernel waits for the previous grid on the stream before it rewrites the shared
+    // array (griddepcontrol.wait ahead of its first store), so back-to-back calls on one
+    // stream never overwrite x tiles that an earlier call is still reading
+    return tc_enqueue(a, c, &L, static_cast<uint16_t*>(ws),
+                      reinterpret_cast<int*>(static_cast<char*>(ws) + kNoAllocXBytes), stream);
 }
 
 }  // namespace qmm_impl

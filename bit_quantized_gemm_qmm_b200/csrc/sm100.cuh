@@ -55,11 +55,7 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long deadline) {
     if (mbar_try_wait(bar, parity)) return true;
     while (true) {
-#ifdef QMM_NO_SUSPEND
-        if (mbar_try_wait(bar, parity)) return true;
-#else
         if (mbar_try_wait_suspend(bar, parity, 1000000u)) return true;
-#endif
         if (clock64() > deadline) return false;
     }
 }
@@ -158,6 +154,12 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
         : "memory");
 }
 
+// 32 lanes x 2 columns of 32-bit.
+__device__ __forceinline__ void tmem_st_32x32b_x2(uint32_t taddr, uint32_t v0, uint32_t v1) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(v0), "r"(v1)
+                 : "memory");
+}
+
 // 32 lanes x 8 columns of 32-bit -> 8 registers per thread.
 __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&v)[8]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
@@ -178,6 +180,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t sbo)
     d |= uint64_t((sbo >> 4) & 0x3FFF) << 32;      // stride byte offset
     d |= uint64_t(1) << 46;                        // descriptor version (sm_100)
     d |= uint64_t(2) << 61;                        // layout: 128-byte swizzle
+    return d;
+}
+
+// Shared-memory matrix descriptor, K-major operand without swizzle: 8-row x 16-byte core
+// matrices stored as 128 contiguous bytes, `lbo` bytes between the core matrices adjacent in
+// K and `sbo` bytes between those adjacent in M/N.
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFF);
+    d |= uint64_t((lbo >> 4) & 0x3FFF) << 16;
+    d |= uint64_t((sbo >> 4) & 0x3FFF) << 32;
+    d |= uint64_t(1) << 46;  // descriptor version (sm_100); layout type 0 = no swizzle
     return d;
 }
 

@@ -114,12 +114,23 @@ enum {
     QMM_KERNEL_TC = 2,     /* swap-AB tcgen05 tile: 128 weight rows x M tokens, TMEM accum   */
     QMM_KERNEL_STREAM = 3, /* M <= 16: TMA-staged codes, mma.sync consumer warps; K split over
                               a cluster only when the 128-row tiles cannot fill the GPU      */
+    QMM_KERNEL_SK = 4,     /* 1 <= M <= 64: tcgen05 tile of 128 weight rows x M tokens with the
+                              weight stream split evenly over at most one block per SM; the
+                              partial sums of a tile split between blocks are added by the last
+                              of them in a fixed order.  Its `split` plan field selects where x
+                              is staged: 0 = choose, 1 = in shared memory by the kernel itself
+                              (one launch), 2 = once per call in the workspace (two launches) */
 };
 
 enum {
     QMM_PLAN_PDL = 1u << 0,            /* launch with programmatic dependent launch          */
     QMM_PLAN_STATIC_WEIGHTS = 1u << 1, /* weights are not written by earlier stream work:
                                           prefetch them before waiting on the previous kernel */
+    QMM_PLAN_TEST_TIMEOUT = 1u << 30,  /* testing aid for QMM_KERNEL_SK only, never set by qmm():
+                                          block 0 withholds its first stage of codes and every
+                                          pipeline wait gives up after about a millisecond, so
+                                          the call takes the timeout path and reports bit 0 in
+                                          qmm_device_errors(); y is not valid after such a call */
 };
 
 typedef struct {
@@ -143,6 +154,35 @@ qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group
 qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
                   const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                   int group, qmm_dtype dtype, const qmm_plan* plan, void* stream);
+
+/* One weight matrix of a grouped call: its arrays as for qmm(), its N, and its output. */
+typedef struct {
+    const uint32_t* packed;  /* [N, K*bits/32] codes                                           */
+    const uint16_t* scales;  /* [N, K/group] fp16                                              */
+    const uint16_t* biases;  /* [N, K/group] fp16                                              */
+    void* y;                 /* [M, N] output, dtype of x                                      */
+    int64_t N;               /* rows of this matrix (0: the item is skipped)                    */
+} qmm_item;
+
+/*
+ * qmm_grouped -- y_i = x . dequant(items[i])^T for 1 <= count <= 4 weight matrices that share
+ * x, K and the format (bits, group, dtype): a decoder layer's q, k and v projections, or its
+ * gate and up projections, in ONE launch of the even-split kernel (two when x is staged in
+ * the workspace).  "How the NAX Verify Kernel Path Improves Decode Performance in MTPLX",
+ * section "Architectural Differences: Stock MLX vs. NAX Verify", puts the small verify
+ * calls' cost in per-call dispatch overhead; one launch over the layer's matrices pays it
+ * once and splits all their weight bytes evenly over the SMs.
+ * Each item must meet the even-split kernel's shape rules (1 <= M <= 64, a multiple of 8
+ * groups per row, a 16-byte multiple of packed bytes per row; packed, scales, biases, x and
+ * y 16-byte aligned), else QMM_ERR_UNSUPPORTED and nothing is launched.  `plan` may be NULL
+ * or name QMM_KERNEL_AUTO / QMM_KERNEL_SK with its x mode in `split` and the QMM_PLAN_PDL /
+ * QMM_PLAN_STATIC_WEIGHTS flags (NULL = PDL, weights not static).  Each y_i meets the same
+ * tolerance as a qmm() call and is bitwise reproducible run to run (the split points, and so
+ * the order partial sums meet in, depend on the whole group).  M == 0 is a no-op; K == 0
+ * writes zeros to every y.  Stream, scratch memory and errors as for qmm().
+ */
+qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t M, int64_t K,
+                       int bits, int group, qmm_dtype dtype, const qmm_plan* plan, void* stream);
 
 /*
  * qmm_noalloc -- qmm() on the tensor-core kernel without allocating anything.  The pages have

@@ -145,6 +145,18 @@ def test_plans(L):
     assert L.qmm_ex(16, 16, 16, 16, 16, 4, 64, 128, 4, 64, 0, ctypes.byref(bad), None) == q.QMM_ERR_INVALID_ARG
 
 
+def test_prefill_m_routes_to_the_even_split_kernel(L):
+    """Above 64 tokens only the even-split kernel runs (up to 128 tokens a launch, larger M as
+    even chunks); shapes it cannot take are refused before anything is launched."""
+    f16 = __import__("torch").float16
+    for M in (65, 80, 128, 129, 1000):
+        assert q.plan_default(M, 4096, 4096, 4, 64, f16).kernel == q.KERNEL_SK
+    assert _qmm(L, M=65) == q.QMM_ERR_UNSUPPORTED  # K = 128, g64: 2 groups per row, not a multiple of 8
+    assert _qmm(L, M=(1 << 20) + 1) == q.QMM_ERR_UNSUPPORTED
+    mma = q.make_plan(kernel=q.KERNEL_MMA)
+    assert L.qmm_ex(16, 16, 16, 16, 16, 65, 64, 512, 4, 64, 0, ctypes.byref(mma), None) == q.QMM_ERR_UNSUPPORTED
+
+
 def test_status_strings(L):
     for s in range(4):
         assert L.qmm_status_string(s)

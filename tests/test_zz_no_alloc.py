@@ -63,6 +63,27 @@ def test_noalloc_matches_qmm_on_consecutive_calls():
     assert q.device_errors() == 0
 
 
+def test_noalloc_back_to_back_without_host_sync():
+    """Six calls issued back to back on one stream, each into its own output, with one
+    synchronization at the end: every call's x kernel must wait for the call before it
+    before it rewrites the shared array."""
+    tc_plan = q.make_plan(kernel=q.KERNEL_TC)
+    prepared = [_inputs(*c, seed=20 + i) for i, c in enumerate(CASES)]
+    refs = [q.qmm(x, P, S, B, c[3], c[4], plan=tc_plan).double().cpu().numpy()
+            for (x, P, S, B), c in zip(prepared, CASES)]
+    torch.cuda.synchronize()
+    order = [0, 1, 2, 0, 2, 1]
+    outs = []
+    for i in order:
+        (x, P, S, B), (M, N, K, bits, group, dtype, _) = prepared[i], CASES[i]
+        y = torch.full((M, N), float("nan"), dtype=dtype, device="cuda")
+        outs.append(_noalloc(x, P, S, B, bits, group, y))
+    torch.cuda.synchronize()
+    for i, y in zip(order, outs):
+        check_close(y, refs[i], CASES[i][5], f"qmm_noalloc back to back, case {i}")
+    assert q.device_errors() == 0
+
+
 def test_noalloc_rejects_oversize_without_launching():
     # staged activations: roundup(K, 256) * 64 * 2 bytes > 2 MiB
     M, N, K, bits, group = 64, 128, 16384 + 256, 4, 64
