@@ -327,7 +327,8 @@ qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group
     if (M > kMaxTotalM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %lld", (long long)M, (long long)kMaxTotalM);
     if (!plan) return fail(QMM_ERR_INVALID_ARG, "plan is null");
     if (M > kSkMaxTokens) M = kSkMaxTokens;  // the plan of each chunk
-    // the default plan assumes 4-byte aligned scales and biases (any allocation is)
+    // the plan qmm() picks for 16-byte aligned scales and biases (any allocation is), as the
+    // header states
     return resolve_plan(M, N, K, bits, group, nullptr, reinterpret_cast<const void*>(16),
                         reinterpret_cast<const void*>(16), plan, nullptr);
 }

@@ -198,37 +198,30 @@ __device__ __forceinline__ uint32_t lds_u16v(uint32_t a) {
 }
 
 // ---------------------------------------------------------------- x -> staged tiles
-// One 8- (4/8-bit) or 16-value (6-bit) block of x row m at K offset k (relative to the
-// stage start kk within the stage): converted to fp16 (bf16 values times 2^-E first), put
-// in the dequantizers' pair order and stored in the 128-byte-swizzled tile of the stage
-// ([4 atoms][MP rows][128 B], 16-byte chunk c of row m at c ^ (m & 7)).  Returns the block's
-// sum (of the converted values) for the x sums.  Nothing is stored unless `store`; values
-// are read only when `valid` (zeros otherwise).
+// One 8- (4/8-bit) or 16-value (6-bit) block of x row m at K offset kk within its stage,
+// already loaded (`raw`, zeros when out of range): converted to fp16 (bf16 values times 2^-E
+// first), put in the dequantizers' pair order and stored in the 128-byte-swizzled tile of the
+// stage ([4 atoms][MP rows][128 B], 16-byte chunk c of row m at c ^ (m & 7)).  Returns the
+// block's sum (of the converted values) for the x sums.  Nothing is stored unless `store`.
 template <int BITS>
-__device__ __forceinline__ float stage_x_block(const uint16_t* src, bool valid, bool store, int is_bf16,
+__device__ __forceinline__ float stage_x_block(const uint4 (&raw)[SkFmt<BITS>::UN / 8], bool store, int is_bf16,
                                                float xscale, int mp, int m, int kk, uint8_t* gdst, uint32_t sdst) {
     constexpr int UN = SkFmt<BITS>::UN;
     float f[UN];
-    if (valid) {
 #pragma unroll
-        for (int h = 0; h < UN / 8; ++h) {
-            const uint4 v = ldg_x16(src + 8 * h);
-            const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+    for (int h = 0; h < UN / 8; ++h) {
+        const uint32_t r[4] = {raw[h].x, raw[h].y, raw[h].z, raw[h].w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                if (is_bf16) {
-                    f[8 * h + 2 * i] = bf16lo_to_f32(r[i]) * xscale;
-                    f[8 * h + 2 * i + 1] = bf16hi_to_f32(r[i]) * xscale;
-                } else {
-                    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
-                    f[8 * h + 2 * i] = t.x;
-                    f[8 * h + 2 * i + 1] = t.y;
-                }
+        for (int i = 0; i < 4; ++i) {
+            if (is_bf16) {
+                f[8 * h + 2 * i] = bf16lo_to_f32(r[i]) * xscale;
+                f[8 * h + 2 * i + 1] = bf16hi_to_f32(r[i]) * xscale;
+            } else {
+                const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
+                f[8 * h + 2 * i] = t.x;
+                f[8 * h + 2 * i + 1] = t.y;
             }
         }
-    } else {
-#pragma unroll
-        for (int i = 0; i < UN; ++i) f[i] = 0.f;
     }
     float sum = 0.f;
 #pragma unroll
@@ -249,6 +242,50 @@ __device__ __forceinline__ float stage_x_block(const uint16_t* src, bool valid, 
         }
     }
     return sum;
+}
+
+template <int BITS>
+__device__ __forceinline__ void load_x_block(const uint16_t* src, bool valid, uint4 (&raw)[SkFmt<BITS>::UN / 8]) {
+#pragma unroll
+    for (int h = 0; h < SkFmt<BITS>::UN / 8; ++h) raw[h] = valid ? ldg_x16(src + 8 * h) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Stage blocks i = i0, i0 + stride, ... (< totp) of a [rows x (KC or K)] range of x: `XB`
+// blocks per thread are loaded before any is converted, so their loads overlap.  `at(i)`
+// gives (row, K offset, stage-relative offset, destination) of block i; blocks past `total`
+// or past K contribute zeros and store nothing.  The x sums of each 32-value stretch are
+// reduced over the lanes that hold it (consecutive lanes hold consecutive blocks of a row).
+template <int BITS, int XB, class At, class Sum>
+__device__ __forceinline__ void stage_x_range(const uint16_t* x, int K, int is_bf16, const float* xscale, int mp,
+                                              int i0, int stride, int total, At at, Sum put_sum) {
+    constexpr int UN = SkFmt<BITS>::UN, UPS = 32 / UN;
+    const int totp = (total + 31) & ~31;
+    for (int ib = i0; ib < totp; ib += XB * stride) {
+        uint4 raw[XB][UN / 8];
+#pragma unroll
+        for (int b = 0; b < XB; ++b) {
+            const int i = ib + b * stride;
+            int m, k, kk;
+            uint8_t* gd;
+            uint32_t sd;
+            at(i < total ? i : 0, m, k, kk, gd, sd);
+            load_x_block<BITS>(x + int64_t(m) * K + k, i < total && k < K, raw[b]);
+        }
+#pragma unroll
+        for (int b = 0; b < XB; ++b) {
+            const int i = ib + b * stride;
+            if (i >= totp) break;  // warp-uniform: totp and stride are multiples of 32
+            const bool valid = i < total;
+            int m, k, kk;
+            uint8_t* gd;
+            uint32_t sd;
+            at(valid ? i : 0, m, k, kk, gd, sd);
+            float sum = stage_x_block<BITS>(raw[b], valid, is_bf16, xscale ? xscale[m] : 1.f, mp, m, kk, gd, sd);
+            if (UPS >= 2) sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            if (UPS >= 4) sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            if (valid && ((kk / UN) % UPS) == 0) put_sum(i, m, kk, sum);
+        }
+    }
 }
 
 // Byte offset of the x sum of 32-code stretch j (0..7) of token m in a stage's x-sum tile:
@@ -556,28 +593,38 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         // per-token exponents of bf16 activations: E_m with max|x_m| * 2^-E_m < 2^15 over the
         // K range this block reads (its own choice; the tile's partial sums are rescaled by
         // 2^E_m before they meet)
-        if (XS) {
-            if (p.is_bf16) {
-                const int nst = min(p.per, p.S);
-                for (int m = 0; m < p.M; ++m) {
-                    float amax_v = 0.f;
-                    for (int e = tid; e < nst * (SK_KC / 8); e += SK_NISS * 32) {
-                        const int sl = e / (SK_KC / 8), v = e - sl * (SK_KC / 8);
+        if (XS && p.is_bf16) {
+            // every (token, 8-value block) of the block's K range; eight loads in flight per
+            // thread, each block's maximum folded into amax[m] with a shared-memory atomicMax
+            // on the float bits (all values >= 0)
+            const int nst = min(p.per, p.S);
+            const int per_row = nst * (SK_KC / 8);
+            const int total = p.M * per_row;
+            for (int e0 = tid; e0 < total; e0 += SK_NISS * 32 * 8) {
+                uint4 v[8];
+#pragma unroll
+                for (int bb = 0; bb < 8; ++bb) {
+                    const int e = e0 + bb * SK_NISS * 32;
+                    v[bb] = make_uint4(0u, 0u, 0u, 0u);
+                    if (e < total) {
+                        const int m = e / per_row, cc = e - m * per_row, sl = cc / (SK_KC / 8);
                         int s = s_a + sl;
                         if (s >= p.S) s -= p.S;
-                        const int k = s * SK_KC + v * 8;
-                        if (k < p.K) {
-                            const uint4 xv = ldg_x16(p.x + int64_t(m) * p.K + k);
-                            const uint32_t r[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                amax_v = fmaxf(amax_v, fmaxf(fabsf(bf16lo_to_f32(r[i])), fabsf(bf16hi_to_f32(r[i]))));
-                        }
+                        const int k = s * SK_KC + (cc - sl * (SK_KC / 8)) * 8;
+                        if (k < p.K) v[bb] = ldg_x16(p.x + int64_t(m) * p.K + k);
                     }
+                }
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) amax_v = fmaxf(amax_v, __shfl_xor_sync(0xffffffffu, amax_v, o));
-                    // warp maxima meet in amax[m] through atomicMax on the float bits (>= 0)
-                    if (lane == 0) atomicMax(amax + m, __float_as_int(amax_v));
+                for (int bb = 0; bb < 8; ++bb) {
+                    const int e = e0 + bb * SK_NISS * 32;
+                    if (e < total) {
+                        const uint32_t r[4] = {v[bb].x, v[bb].y, v[bb].z, v[bb].w};
+                        float mx = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            mx = fmaxf(mx, fmaxf(fabsf(bf16lo_to_f32(r[i])), fabsf(bf16hi_to_f32(r[i]))));
+                        atomicMax(amax + e / per_row, __float_as_int(mx));
+                    }
                 }
             }
         }
@@ -623,22 +670,22 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                 xbase = sbase + L.x_off + uint32_t(slot * MP * 512);
                 xsbase = sbase + L.xs_off + uint32_t(slot * MP * 32);
                 if (slot >= nstaged) {
-                    // stage this stage's x: M rows x 256 values, 8 (16) per thread step
-                    constexpr int UN = F::UN, UPR = SK_KC / UN, UPS = 32 / UN;
-                    const int total = p.M * UPR;
-                    const int totp = (total + 31) & ~31;
-                    for (int i = tid; i < totp; i += SK_NISS * 32) {
-                        const bool valid = i < total;
-                        const int m = valid ? i / UPR : 0, v = i - m * UPR;
-                        const int k = s * SK_KC + v * UN;
-                        float sum = stage_x_block<BITS>(p.x + int64_t(m) * p.K + k, valid && k < p.K, valid,
-                                                        p.is_bf16, escale[m], MP, m, v * UN, nullptr, xbase);
-                        if (UPS >= 2) sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                        if (UPS >= 4) sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-                        if (valid && (v % UPS) == 0)
-                            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xsbase + xsum_off(m, v / UPS)),
+                    // stage this stage's x: M rows x 256 values
+                    constexpr int UN = F::UN, UPR = SK_KC / UN;
+                    const int k0 = s * SK_KC;
+                    stage_x_range<BITS, 64 / UN>(
+                        p.x, p.K, p.is_bf16, escale, MP, tid, SK_NISS * 32, p.M * UPR,
+                        [&](int i, int& m, int& k, int& kk, uint8_t*& gd, uint32_t& sd) {
+                            m = i / UPR;
+                            kk = (i - m * UPR) * UN;
+                            k = k0 + kk;
+                            gd = nullptr;
+                            sd = xbase;
+                        },
+                        [&](int, int m, int kk, float sum) {
+                            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xsbase + xsum_off(m, kk / 32)),
                                          "r"(xsum_pack(sum)));
-                    }
+                        });
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_xstage);
@@ -895,8 +942,9 @@ template <int BITS>
 __global__ void __launch_bounds__(256) sk_xprep_kernel(const uint16_t* __restrict__ x, int M, int K, int is_bf16,
                                                        int MP, int S, uint8_t* __restrict__ xt,
                                                        uint8_t* __restrict__ xsum, int* __restrict__ xexp) {
-    constexpr int UN = SkFmt<BITS>::UN, UPR = SK_KC / UN, UPS = 32 / UN;
+    constexpr int UN = SkFmt<BITS>::UN, UPR = SK_KC / UN;
     __shared__ float red[8];
+    __shared__ float scl[64];
     grid_dependents_launch();
     grid_dependency_wait();
     const int m = blockIdx.x;
@@ -921,21 +969,24 @@ __global__ void __launch_bounds__(256) sk_xprep_kernel(const uint16_t* __restric
         const int eb = int(__float_as_uint(a) >> 23) & 0xFF;
         E = eb > 141 ? eb - 141 : 0;
     }
-    if (threadIdx.x == 0) xexp[m] = E;
-    const float sc = exp2i(-E);
-    const int total = S * UPR;
-    const int totp = (total + 31) & ~31;
-    for (int i = threadIdx.x; i < totp; i += 256) {
-        const bool valid = i < total;
-        const int s = valid ? i / UPR : 0, v = i - s * UPR;
-        const int k = s * SK_KC + v * UN;
-        float sum = stage_x_block<BITS>(xr + k, valid && k < K, valid, is_bf16, sc, MP, m, v * UN,
-                                        xt + size_t(s) * MP * 512, 0u);
-        if (UPS >= 2) sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        if (UPS >= 4) sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (valid && (v % UPS) == 0)
-            *reinterpret_cast<uint32_t*>(xsum + size_t(s) * MP * 32 + xsum_off(m, v / UPS)) = xsum_pack(sum);
+    if (threadIdx.x == 0) {
+        xexp[m] = E;
+        scl[m] = exp2i(-E);
     }
+    __syncthreads();
+    stage_x_range<BITS, 64 / UN>(
+        x, K, is_bf16, scl, MP, threadIdx.x, 256, S * UPR,
+        [&](int i, int& mm, int& k, int& kk, uint8_t*& gd, uint32_t& sd) {
+            const int s = i / UPR;
+            mm = m;
+            kk = (i - s * UPR) * UN;
+            k = s * SK_KC + kk;
+            gd = xt + size_t(s) * MP * 512;
+            sd = 0u;
+        },
+        [&](int i, int mm, int kk, float sum) {
+            *reinterpret_cast<uint32_t*>(xsum + size_t(i / UPR) * MP * 32 + xsum_off(mm, kk / 32)) = xsum_pack(sum);
+        });
 }
 
 using SkKernelFn = void (*)(const SkMapSet, const SkParams);

@@ -144,7 +144,10 @@ typedef struct {
 } qmm_plan;
 
 /* Fill *plan with the dispatch table's choice for this shape (QMM_OK), or report why the
- * shape is unsupported.  Sizes as for qmm(). */
+ * shape is unsupported.  Sizes as for qmm().  The choice is the one qmm() makes when
+ * `scales` and `biases` are 16-byte aligned (every allocation from cudaMalloc or torch is);
+ * with less aligned arrays qmm() falls back to kernels that need less, so the plan may
+ * differ.  For M > 128 it is the plan of each 128-token chunk. */
 qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group,
                             qmm_dtype dtype, qmm_plan* plan);
 
