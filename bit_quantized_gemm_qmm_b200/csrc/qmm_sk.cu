@@ -744,33 +744,31 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         int aused = 0;
         bool have_sb = false, ok = true, e_waited = false;
         uint32_t sbuf = 0;
-        int t = u0 / p.S, s = s_a, prev_b = -1;
-        for (int u = u0; u < u1 && ok; ++u) {
-            const bool seg_first = (u == u0) || s == 0;
-            const bool seg_last = (u == u1 - 1) || s == p.S - 1;
-            const int b = (s * SK_KC) >> (p.gshift + 3);
-            if (seg_first || b != prev_b) {
+        int prev_b = -1;
+        // The loop is software-pipelined: the codes, scales and biases of the next stage are
+        // read while this one converts, and the tensor-memory stores of a stage are waited
+        // for only after the next stage has been converted (or at the end of a tile).
+        uint32_t wd[F::NW];
+        uint32_t s0 = 0, s1 = 0, b0 = 0, b1 = 0;
+        // fetch stage (tt, ss_) into wd / s0.. (returns false on timeout)
+        auto fetch = [&](int uu, int ss_) -> bool {
+            const bool first = (uu == u0) || ss_ == 0;
+            const int bb = (ss_ * SK_KC) >> (p.gshift + 3);
+            if (first || bb != prev_b) {
                 if (have_sb) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_sempty + 8 * ss);
                     if (++ss == SK_SS) { ss = 0; sph ^= 1u; }
                 }
-                ok = sk_wait(bar_sfull + 8 * ss, sph, abort_flag, p.timeout);
+                if (!sk_wait(bar_sfull + 8 * ss, sph, abort_flag, p.timeout)) return false;
                 have_sb = true;
                 sbuf = sbase + L.sb_off + uint32_t(ss * SK_SB);
-                prev_b = b;
+                prev_b = bb;
             }
-            ok = ok && sk_wait(bar_full + 8 * sc, ph, abort_flag, p.timeout);
-            if (!ok) break;
-            uint32_t wd[F::NW];
+            if (!sk_wait(bar_full + 8 * sc, ph, abort_flag, p.timeout)) return false;
             sk_load_codes<BITS>(sbase + L.code_off + uint32_t(sc * F::CST), row, uq, wd);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_empty + 8 * sc);
-            if (++sc == p.sc) { sc = 0; ph ^= 1u; }
             // scale and bias of the quarter's group(s) within the block's 8
-            const int k0 = s * SK_KC + uq * 64;
-            const int gi = (k0 >> p.gshift) & 7;
-            uint32_t s0, s1, b0, b1;
+            const int gi = ((ss_ * SK_KC + uq * 64) >> p.gshift) & 7;
             if (g == 32) {
                 const uint32_t sv = lds_u32(sbuf + uint32_t(row * 16 + gi * 2));
                 const uint32_t bv = lds_u32(sbuf + uint32_t(SK_SB / 2 + row * 16 + gi * 2));
@@ -780,6 +778,26 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                 s0 = s1 = lds_u16v(sbuf + uint32_t(row * 16 + gi * 2));
                 b0 = b1 = lds_u16v(sbuf + uint32_t(SK_SB / 2 + row * 16 + gi * 2));
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_empty + 8 * sc);
+            if (++sc == p.sc) { sc = 0; ph ^= 1u; }
+            return true;
+        };
+        bool pending = false;  // a stage's tensor-memory stores not yet waited for and signalled
+        int pend_a = 0;
+        auto signal_pending = [&]() {
+            if (pending) {
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_afull + 8 * pend_a);
+                pending = false;
+            }
+        };
+        int t = u0 / p.S, s = s_a;
+        ok = fetch(u0, s_a);
+        for (int u = u0; u < u1 && ok; ++u) {
+            const bool seg_last = (u == u1 - 1) || s == p.S - 1;
             uint32_t vals[32];
             if constexpr (TM::FOLD) {
                 sk_dequant_fold<BITS>(wd, s0, b0, s1, b1, vals);
@@ -789,6 +807,15 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                 if (__any_sync(0xffffffffu, big)) sk_dequant<BITS, true>(wd, C0, C1, vals);
                 else sk_dequant<BITS, false>(wd, C0, C1, vals);
             }
+            const uint32_t bp0 = __byte_perm(b0, 0u, 0x1010u), bp1 = __byte_perm(b1, 0u, 0x1010u);
+            signal_pending();
+            if (u + 1 < u1) {
+                const int sn = s + 1 == p.S ? 0 : s + 1;
+                if (!fetch(u + 1, sn)) {
+                    ok = false;
+                    break;
+                }
+            }
             if (aused >= NA) {
                 if (!sk_wait(bar_aempty + 8 * a, pa ^ 1u, abort_flag, p.timeout)) break;
             }
@@ -796,14 +823,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             tc_fence_after();
             const uint32_t acol = tmem + lane_base + uint32_t(TM::ABASE + a * TM::ACOLS);
             tmem_st_32x32b_x32(acol + uint32_t(uq * 32), vals);
-            if constexpr (!TM::FOLD)
-                tmem_st_32x32b_x2(acol + uint32_t(SK_KC / 2 + 2 * uq), __byte_perm(b0, 0u, 0x1010u),
-                                  __byte_perm(b1, 0u, 0x1010u));
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_afull + 8 * a);
+            if constexpr (!TM::FOLD) tmem_st_32x32b_x2(acol + uint32_t(SK_KC / 2 + 2 * uq), bp0, bp1);
+            pending = true;
+            pend_a = a;
             if (++a == NA) { a = 0; pa ^= 1u; }
+            if (seg_last) signal_pending();
 
             if (seg_last) {
                 // ---------------------------------------------------- epilogue of tile t
@@ -823,7 +847,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                 const int N = p.Ns[it];
                 uint16_t* const y = p.y[it];
                 float* part = P > 1 ? p.partials + size_t(sk_slot(c, t, p.per, p.S)) * MP * SK_ROWS : nullptr;
-#pragma unroll
+#pragma unroll 1
                 for (int cw = 0; cw < (MP / 8 + 3) / 4; ++cw) {
                     const int ch = uq + 4 * cw;
                     if (ch < MP / 8) {
@@ -898,7 +922,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                     if (!ok) break;
                     if (*verdict) {
                         __threadfence();
-#pragma unroll
+#pragma unroll 1
                         for (int cw = 0; cw < (MP / 8 + 3) / 4; ++cw) {
                             const int ch = uq + 4 * cw;
                             if (ch < MP / 8 && n < N) {

@@ -77,7 +77,12 @@ def test_sk_grid_shapes(oracle_mod, N, K, M):
     op, os_, ob = oracle_quantize(oracle_mod, w, 4, 64)
     P, S, B = to_device_weights(op, os_, ob)
     for xmode in XMODES:
-        y = q.qmm(x.cuda(), P, S, B, 4, 64, plan=_plan(xmode)).cpu()
+        try:
+            y = q.qmm(x.cuda(), P, S, B, 4, 64, plan=_plan(xmode)).cpu()
+        except q.QmmError as e:
+            # x staged in shared memory is refused when the block's stages of it do not fit
+            assert xmode == 1 and e.status == q.QMM_ERR_UNSUPPORTED, e
+            continue
         assert q.device_errors() == 0
         rows = np.unique(np.concatenate([np.arange(0, N, max(1, N // 700)), np.arange(max(0, N - 300), N)]))
         ref = oracle_qmm(oracle_mod, x, op[rows], os_[rows], ob[rows], K, 4, 64)
