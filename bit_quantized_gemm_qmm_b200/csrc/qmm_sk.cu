@@ -302,39 +302,6 @@ __device__ __forceinline__ uint32_t xsum_pack(float s) {
 }
 
 // ---------------------------------------------------------------- dequantization
-// One thread's quarter stage (64 codes of one row, in registers) -> 32 fp16x2 A columns of
-// s*q in pair order.  C0 covers the first 32 codes, C1 the other 32 (the same constants when
-// a group spans the quarter).
-template <int BITS, bool SAFE>
-__device__ __forceinline__ void sk_dequant(const uint32_t (&wd)[SkFmt<BITS>::NW], const RowConst& C0,
-                                           const RowConst& C1, uint32_t (&out)[32]) {
-    if constexpr (BITS == 4) {
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            uint32_t a[4];
-            dq4_word<SAFE>(wd[w], w < 4 ? C0 : C1, a);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) out[4 * w + i] = a[i];
-        }
-    } else if constexpr (BITS == 8) {
-#pragma unroll
-        for (int w = 0; w < 16; ++w) {
-            uint32_t a[2];
-            dq8_word<SAFE>(wd[w], w < 8 ? C0 : C1, a);
-            out[2 * w] = a[0];
-            out[2 * w + 1] = a[1];
-        }
-    } else {
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            uint32_t a[8];
-            dq6_triplet<SAFE>(wd[3 * t], wd[3 * t + 1], wd[3 * t + 2], t < 2 ? C0 : C1, a);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) out[8 * t + i] = a[i];
-        }
-    }
-}
-
 // The same quarter stage with the bias folded in: each pair is RN_fp16(s*q + b), with q taken
 // exactly out of its magic-number form first ((M + q) - M) and then one fused multiply-add.
 // Never overflows for weights that fit fp16.
@@ -376,31 +343,43 @@ __device__ __forceinline__ void sk_dequant_fold(const uint32_t (&wd)[SkFmt<BITS>
     }
 }
 
-// The thread's codes of one stage: row `row`, quarter `uq` of the stage's K range.
-template <int BITS>
-__device__ __forceinline__ void sk_load_codes(uint32_t stage, int row, int uq, uint32_t (&wd)[SkFmt<BITS>::NW]) {
-    if constexpr (BITS == 4) {  // 128-byte rows, 128-byte swizzle; 32 bytes per quarter
+// Convert a quarter stage and store it to its 32 A columns as it goes (a few columns per
+// tcgen05.st, straight from the registers the conversion wrote).
+template <int BITS, bool SAFE>
+__device__ __forceinline__ void sk_dequant_store(const uint32_t (&wd)[SkFmt<BITS>::NW], const RowConst& C0,
+                                                 const RowConst& C1, uint32_t acol) {
+    if constexpr (BITS == 4) {
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * uq + cc;
-            const uint4 v = lds_v4(stage + uint32_t(row * 128 + ((c ^ (row & 7)) << 4)));
-            wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
+        for (int w = 0; w < 8; ++w) {
+            uint32_t a[4];
+            dq4_word<SAFE>(wd[w], w < 4 ? C0 : C1, a);
+            tmem_st_32x32b_x4(acol + uint32_t(4 * w), a[0], a[1], a[2], a[3]);
         }
-    } else if constexpr (BITS == 8) {  // two 128-byte boxes per row; 64 bytes per quarter
-        const uint32_t box = stage + uint32_t((uq >> 1) * SK_ROWS * 128 + row * 128);
+    } else if constexpr (BITS == 8) {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            const int c = (uq & 1) * 4 + cc;
-            const uint4 v = lds_v4(box + uint32_t((c ^ (row & 7)) << 4));
-            wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
+        for (int w = 0; w < 16; w += 2) {
+            uint32_t a[2], b2[2];
+            dq8_word<SAFE>(wd[w], w < 8 ? C0 : C1, a);
+            dq8_word<SAFE>(wd[w + 1], w < 8 ? C0 : C1, b2);
+            tmem_st_32x32b_x4(acol + uint32_t(2 * w), a[0], a[1], b2[0], b2[1]);
         }
-    } else {  // 192-byte rows, no swizzle; 48 bytes per quarter
+    } else {
 #pragma unroll
-        for (int cc = 0; cc < 3; ++cc) {
-            const uint4 v = lds_v4(stage + uint32_t(row * 192 + uq * 48 + cc * 16));
-            wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
+        for (int t = 0; t < 4; ++t) {
+            uint32_t a[8];
+            dq6_triplet<SAFE>(wd[3 * t], wd[3 * t + 1], wd[3 * t + 2], t < 2 ? C0 : C1, a);
+            tmem_st_32x32b_x8(acol + uint32_t(8 * t), a);
         }
     }
+}
+
+template <int BITS>
+__device__ __forceinline__ void sk_dequant_fold_store(const uint32_t (&wd)[SkFmt<BITS>::NW], uint32_t s0, uint32_t b0,
+                                                      uint32_t s1, uint32_t b1, uint32_t acol) {
+    uint32_t v[32];
+    sk_dequant_fold<BITS>(wd, s0, b0, s1, b1, v);
+#pragma unroll
+    for (int c = 0; c < 32; c += 8) tmem_st_32x32b_x8(acol + uint32_t(c), v + c);
 }
 
 // Which matrix tile t belongs to.
@@ -705,9 +684,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             if (issuer && sk_elect_one()) {
                 const uint32_t acol = tmem + uint32_t(TM::ABASE + a * TM::ACOLS);
                 const uint32_t dcol = tmem + uint32_t(j * MP);
+                // descriptors of the K16 steps differ only in their start address field, which
+                // never carries (shared addresses are below 2^18): add the offsets to one
+                const uint64_t xd0 = smem_desc_sw128(xbase, 1024);
 #pragma unroll
                 for (int kk = j; kk < SK_KC / 16; kk += NACC) {
-                    const uint64_t bdesc = smem_desc_sw128(xbase + uint32_t((kk >> 2) * (MP * 128) + (kk & 3) * 32), 1024);
+                    const uint64_t bdesc = xd0 + uint64_t(((kk >> 2) * (MP * 128) + (kk & 3) * 32) >> 4);
                     umma_f16_ts(dcol, acol + uint32_t(kk * 8), bdesc, idesc, (seg_first && kk == j) ? 0u : 1u);
                 }
                 if (!TM::FOLD && j == 0) {
@@ -739,95 +721,92 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         const int row = q * 32 + lane;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         const int g = 1 << p.gshift;
-        int sc = 0, ss = 0, a = 0, nseg = 0, nsplit = 0;
+        // per-thread constants: where its codes sit in a stage, its scale row, its A columns
+        uint32_t coff[F::NW / 4];  // byte offsets of the thread's 16-byte code chunks
+#pragma unroll
+        for (int cc = 0; cc < F::NW / 4; ++cc) {
+            if constexpr (BITS == 4) {
+                coff[cc] = uint32_t(row * 128 + (((2 * uq + cc) ^ (row & 7)) << 4));
+            } else if constexpr (BITS == 8) {
+                coff[cc] = uint32_t((uq >> 1) * SK_ROWS * 128 + row * 128 + ((((uq & 1) * 4 + cc) ^ (row & 7)) << 4));
+            } else {
+                coff[cc] = uint32_t(row * 192 + uq * 48 + cc * 16);
+            }
+        }
+        const uint32_t soff = uint32_t(row * 16);
+        const int spb = (8 << p.gshift) / SK_KC;         // stages per scale block (1, 2, 4)
+        const int gps = SK_KC >> p.gshift;               // groups per stage (8, 4, 2)
+        const int qg = (uq * 64) >> p.gshift;            // the quarter's first group in its stage
+        const uint32_t a_base = tmem + lane_base + uint32_t(TM::ABASE + uq * 32);
+        const uint32_t ab_base = tmem + lane_base + uint32_t(TM::ABASE + SK_KC / 2 + 2 * uq);
+        int sc = 0, ss = 0, a = 0, nseg = 0, nsplit = 0, aused = 0;
         uint32_t ph = 0, sph = 0, pa = 0;
-        int aused = 0;
         bool have_sb = false, ok = true, e_waited = false;
         uint32_t sbuf = 0;
-        int prev_b = -1;
-        // The loop is software-pipelined: the codes, scales and biases of the next stage are
-        // read while this one converts, and the tensor-memory stores of a stage are waited
-        // for only after the next stage has been converted (or at the end of a tile).
-        uint32_t wd[F::NW];
-        uint32_t s0 = 0, s1 = 0, b0 = 0, b1 = 0;
-        // fetch stage (tt, ss_) into wd / s0.. (returns false on timeout)
-        auto fetch = [&](int uu, int ss_) -> bool {
-            const bool first = (uu == u0) || ss_ == 0;
-            const int bb = (ss_ * SK_KC) >> (p.gshift + 3);
-            if (first || bb != prev_b) {
+        uint32_t cstage = sbase + L.code_off;  // code ring slot sc
+        int t = u0 / p.S, s = s_a, sib = s_a % spb;
+        for (int u = u0; u < u1 && ok; ++u) {
+            const bool seg_first = (u == u0) || s == 0;
+            const bool seg_last = (u == u1 - 1) || s == p.S - 1;
+            if (seg_first || sib == 0) {  // the next block of 8 groups' scales and biases
                 if (have_sb) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_sempty + 8 * ss);
                     if (++ss == SK_SS) { ss = 0; sph ^= 1u; }
                 }
-                if (!sk_wait(bar_sfull + 8 * ss, sph, abort_flag, p.timeout)) return false;
+                ok = sk_wait(bar_sfull + 8 * ss, sph, abort_flag, p.timeout);
                 have_sb = true;
-                sbuf = sbase + L.sb_off + uint32_t(ss * SK_SB);
-                prev_b = bb;
+                sbuf = sbase + L.sb_off + uint32_t(ss * SK_SB) + soff;
             }
-            if (!sk_wait(bar_full + 8 * sc, ph, abort_flag, p.timeout)) return false;
-            sk_load_codes<BITS>(sbase + L.code_off + uint32_t(sc * F::CST), row, uq, wd);
-            // scale and bias of the quarter's group(s) within the block's 8
-            const int gi = ((ss_ * SK_KC + uq * 64) >> p.gshift) & 7;
-            if (g == 32) {
-                const uint32_t sv = lds_u32(sbuf + uint32_t(row * 16 + gi * 2));
-                const uint32_t bv = lds_u32(sbuf + uint32_t(SK_SB / 2 + row * 16 + gi * 2));
-                s0 = sv & 0xFFFFu; s1 = sv >> 16;
-                b0 = bv & 0xFFFFu; b1 = bv >> 16;
-            } else {
-                s0 = s1 = lds_u16v(sbuf + uint32_t(row * 16 + gi * 2));
-                b0 = b1 = lds_u16v(sbuf + uint32_t(SK_SB / 2 + row * 16 + gi * 2));
+            ok = ok && sk_wait(bar_full + 8 * sc, ph, abort_flag, p.timeout);
+            if (!ok) break;
+            uint32_t wd[F::NW];
+#pragma unroll
+            for (int cc = 0; cc < F::NW / 4; ++cc) {
+                const uint4 v = lds_v4(cstage + coff[cc]);
+                wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_empty + 8 * sc);
-            if (++sc == p.sc) { sc = 0; ph ^= 1u; }
-            return true;
-        };
-        bool pending = false;  // a stage's tensor-memory stores not yet waited for and signalled
-        int pend_a = 0;
-        auto signal_pending = [&]() {
-            if (pending) {
-                tc_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_afull + 8 * pend_a);
-                pending = false;
-            }
-        };
-        int t = u0 / p.S, s = s_a;
-        ok = fetch(u0, s_a);
-        for (int u = u0; u < u1 && ok; ++u) {
-            const bool seg_last = (u == u1 - 1) || s == p.S - 1;
-            uint32_t vals[32];
-            if constexpr (TM::FOLD) {
-                sk_dequant_fold<BITS>(wd, s0, b0, s1, b1, vals);
+            if (++sc == p.sc) {
+                sc = 0;
+                ph ^= 1u;
+                cstage = sbase + L.code_off;
             } else {
-                const RowConst C0 = row_const<BITS>(s0), C1 = row_const<BITS>(s1);
-                const bool big = ((s0 & 0x7FFFu) >= 0x5400u) | ((s1 & 0x7FFFu) >= 0x5400u);
-                if (__any_sync(0xffffffffu, big)) sk_dequant<BITS, true>(wd, C0, C1, vals);
-                else sk_dequant<BITS, false>(wd, C0, C1, vals);
+                cstage += uint32_t(F::CST);
             }
-            const uint32_t bp0 = __byte_perm(b0, 0u, 0x1010u), bp1 = __byte_perm(b1, 0u, 0x1010u);
-            signal_pending();
-            if (u + 1 < u1) {
-                const int sn = s + 1 == p.S ? 0 : s + 1;
-                if (!fetch(u + 1, sn)) {
-                    ok = false;
-                    break;
-                }
+            // scale and bias of the quarter's group(s) within the block's 8
+            const uint32_t gaddr = sbuf + uint32_t((sib * gps + qg) * 2);
+            uint32_t s0, s1, b0, b1;
+            if (g == 32) {
+                const uint32_t sv = lds_u32(gaddr), bv = lds_u32(gaddr + SK_SB / 2);
+                s0 = sv & 0xFFFFu; s1 = sv >> 16;
+                b0 = bv & 0xFFFFu; b1 = bv >> 16;
+            } else {
+                s0 = s1 = lds_u16v(gaddr);
+                b0 = b1 = lds_u16v(gaddr + SK_SB / 2);
             }
             if (aused >= NA) {
                 if (!sk_wait(bar_aempty + 8 * a, pa ^ 1u, abort_flag, p.timeout)) break;
             }
             ++aused;
             tc_fence_after();
-            const uint32_t acol = tmem + lane_base + uint32_t(TM::ABASE + a * TM::ACOLS);
-            tmem_st_32x32b_x32(acol + uint32_t(uq * 32), vals);
-            if constexpr (!TM::FOLD) tmem_st_32x32b_x2(acol + uint32_t(SK_KC / 2 + 2 * uq), bp0, bp1);
-            pending = true;
-            pend_a = a;
+            const uint32_t acol = a_base + uint32_t(a * TM::ACOLS);
+            if constexpr (TM::FOLD) {
+                sk_dequant_fold_store<BITS>(wd, s0, b0, s1, b1, acol);
+            } else {
+                const RowConst C0 = row_const<BITS>(s0), C1 = row_const<BITS>(s1);
+                const bool big = ((s0 & 0x7FFFu) >= 0x5400u) | ((s1 & 0x7FFFu) >= 0x5400u);
+                if (__any_sync(0xffffffffu, big)) sk_dequant_store<BITS, true>(wd, C0, C1, acol);
+                else sk_dequant_store<BITS, false>(wd, C0, C1, acol);
+                tmem_st_32x32b_x2(ab_base + uint32_t(a * TM::ACOLS), __byte_perm(b0, 0u, 0x1010u),
+                                  __byte_perm(b1, 0u, 0x1010u));
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_afull + 8 * a);
             if (++a == NA) { a = 0; pa ^= 1u; }
-            if (seg_last) signal_pending();
 
             if (seg_last) {
                 // ---------------------------------------------------- epilogue of tile t
@@ -946,7 +925,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                     // dequantizer warp has read it: the next gather barrier orders that
                 }
             }
-            if (++s == p.S) { s = 0; ++t; }
+            if (++s == p.S) {
+                s = 0;
+                sib = 0;
+                ++t;
+            } else if (++sib == spb) {
+                sib = 0;
+            }
         }
     }
 
