@@ -21,10 +21,11 @@
 //
 // Warps: 0 = producer (lane 0: TMA boxes of codes, scales and biases; lane 1: the staged x
 // tiles when they come from the workspace), 1-3 = MMA issuers (one accumulator each; they
-// also stage x in shared memory when it fits there), 4-19 = dequantizers, four per tensor-
-// memory lane quadrant, one thread per weight row and quarter stage; at the end of each
-// tile they read the accumulators and write y or the tile's partial sums.  Twenty warps are
-// five per SM sub-partition, which leaves 96 registers a thread.
+// also stage x in shared memory when it fits there), 4-11 = dequantizers, two per tensor-
+// memory lane quadrant, one thread per weight row and half stage (128 codes between two
+// barrier round trips: the fixed cost of a round trip is spread over as many codes as the
+// registers allow); at the end of each tile they read the accumulators and write y or the
+// tile's partial sums.
 // Every mbarrier wait is bounded; a wait that runs out sets an error bit (qmm_device_errors)
 // and the block drops its work, drains its copies in flight and frees its tensor memory.
 #include <cuda.h>
@@ -52,8 +53,8 @@ constexpr int SK_ROWS = 128;                        // weight rows per tile (MMA
 constexpr int SK_KC = 256;                          // codes per stage and row
 constexpr int SK_NISS = 3;                          // MMA issuer warps (1..3)
 constexpr int SK_DQ0 = 1 + SK_NISS;                 // first dequantizer warp
-constexpr int SK_NDQ = 16;                          // dequantizer warps
-constexpr int SK_THREADS = (SK_DQ0 + SK_NDQ) * 32;  // 640: five warps per SM sub-partition
+constexpr int SK_NDQ = 8;                           // dequantizer warps (two per TMEM lane quadrant)
+constexpr int SK_THREADS = (SK_DQ0 + SK_NDQ) * 32;  // 384: three warps per SM sub-partition
 constexpr int SK_SS = 3;                            // scale/bias blocks in flight
 constexpr int SK_SB = 2 * SK_ROWS * 16;             // one block: [128 x 8] scales + biases
 constexpr long long SK_TIMEOUT = 2000000000LL;      // cycles (about 1 s) a pipeline wait may take
@@ -79,7 +80,8 @@ template <int MP> struct SkTm {
 template <int BITS> struct SkFmt {
     static constexpr int CST = SK_ROWS * SK_KC * BITS / 8;  // code bytes per stage (16/24/32 KB)
     static constexpr int WPS = SK_KC * BITS / 32;            // code words per stage and row
-    static constexpr int NW = WPS / 4;                       // words per dequant thread (quarter)
+    static constexpr int NW = WPS / 4;                       // words per 64-code sub-block
+    static constexpr int NWH = WPS / 2;                      // words per dequant thread (half stage)
     static constexpr int UN = BITS == 6 ? 16 : 8;            // x values per permutation block
 };
 
@@ -183,6 +185,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ uint4 ldg_x16(const void* p) {
     uint4 v;
     asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
 
@@ -371,6 +379,17 @@ __device__ __forceinline__ void sk_dequant_store(const uint32_t (&wd)[SkFmt<BITS
             tmem_st_32x32b_x8(acol + uint32_t(8 * t), a);
         }
     }
+}
+
+// Scales of 64 or more (rare: weight ranges above ~1000 at 4 bits): the sub-block is converted
+// again with the subtract-then-multiply form, over the columns the fused form just wrote.
+// Kept out of line so the hot loop holds one conversion path.
+template <int BITS>
+__device__ __noinline__ void sk_dequant_store_safe(const uint32_t* wd, uint32_t s0, uint32_t s1, uint32_t acol) {
+    uint32_t w[SkFmt<BITS>::NW];
+#pragma unroll
+    for (int i = 0; i < SkFmt<BITS>::NW; ++i) w[i] = wd[i];
+    sk_dequant_store<BITS, true>(w, row_const<BITS>(s0), row_const<BITS>(s1), acol);
 }
 
 template <int BITS>
@@ -717,28 +736,28 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         // ------------------------------------------------------------ dequantizers + epilogue
         const int dw = warp - SK_DQ0;
         const int q = warp & 3;       // tensor-memory lane quadrant this warp may access
-        const int uq = dw >> 2;       // quarter of the stage's K range
+        const int uh = dw >> 2;       // half of the stage's K range
         const int row = q * 32 + lane;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         const int g = 1 << p.gshift;
         // per-thread constants: where its codes sit in a stage, its scale row, its A columns
-        uint32_t coff[F::NW / 4];  // byte offsets of the thread's 16-byte code chunks
+        uint32_t coff[F::NWH / 4];  // byte offsets of the thread's 16-byte code chunks
 #pragma unroll
-        for (int cc = 0; cc < F::NW / 4; ++cc) {
+        for (int cc = 0; cc < F::NWH / 4; ++cc) {
             if constexpr (BITS == 4) {
-                coff[cc] = uint32_t(row * 128 + (((2 * uq + cc) ^ (row & 7)) << 4));
+                coff[cc] = uint32_t(row * 128 + (((4 * uh + cc) ^ (row & 7)) << 4));
             } else if constexpr (BITS == 8) {
-                coff[cc] = uint32_t((uq >> 1) * SK_ROWS * 128 + row * 128 + ((((uq & 1) * 4 + cc) ^ (row & 7)) << 4));
+                coff[cc] = uint32_t(uh * SK_ROWS * 128 + row * 128 + ((cc ^ (row & 7)) << 4));
             } else {
-                coff[cc] = uint32_t(row * 192 + uq * 48 + cc * 16);
+                coff[cc] = uint32_t(row * 192 + uh * 96 + cc * 16);
             }
         }
         const uint32_t soff = uint32_t(row * 16);
         const int spb = (8 << p.gshift) / SK_KC;         // stages per scale block (1, 2, 4)
         const int gps = SK_KC >> p.gshift;               // groups per stage (8, 4, 2)
-        const int qg = (uq * 64) >> p.gshift;            // the quarter's first group in its stage
-        const uint32_t a_base = tmem + lane_base + uint32_t(TM::ABASE + uq * 32);
-        const uint32_t ab_base = tmem + lane_base + uint32_t(TM::ABASE + SK_KC / 2 + 2 * uq);
+        const int hg = (uh * 128) >> p.gshift;           // the half's first group in its stage
+        const uint32_t a_base = tmem + lane_base + uint32_t(TM::ABASE + uh * 64);
+        const uint32_t ab_base = tmem + lane_base + uint32_t(TM::ABASE + SK_KC / 2 + 4 * uh);
         int sc = 0, ss = 0, a = 0, nseg = 0, nsplit = 0, aused = 0;
         uint32_t ph = 0, sph = 0, pa = 0;
         bool have_sb = false, ok = true, e_waited = false;
@@ -760,9 +779,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             }
             ok = ok && sk_wait(bar_full + 8 * sc, ph, abort_flag, p.timeout);
             if (!ok) break;
-            uint32_t wd[F::NW];
+            uint32_t wd[F::NWH];
 #pragma unroll
-            for (int cc = 0; cc < F::NW / 4; ++cc) {
+            for (int cc = 0; cc < F::NWH / 4; ++cc) {
                 const uint4 v = lds_v4(cstage + coff[cc]);
                 wd[4 * cc] = v.x; wd[4 * cc + 1] = v.y; wd[4 * cc + 2] = v.z; wd[4 * cc + 3] = v.w;
             }
@@ -775,16 +794,20 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             } else {
                 cstage += uint32_t(F::CST);
             }
-            // scale and bias of the quarter's group(s) within the block's 8
-            const uint32_t gaddr = sbuf + uint32_t((sib * gps + qg) * 2);
-            uint32_t s0, s1, b0, b1;
-            if (g == 32) {
-                const uint32_t sv = lds_u32(gaddr), bv = lds_u32(gaddr + SK_SB / 2);
-                s0 = sv & 0xFFFFu; s1 = sv >> 16;
-                b0 = bv & 0xFFFFu; b1 = bv >> 16;
-            } else {
-                s0 = s1 = lds_u16v(gaddr);
-                b0 = b1 = lds_u16v(gaddr + SK_SB / 2);
+            // scales and biases of the half's groups: sv[i] covers its i-th 32-code stretch
+            const uint32_t gaddr = sbuf + uint32_t((sib * gps + hg) * 2);
+            uint32_t sv[4], bv[4];
+            if (g == 32) {  // four groups: one per stretch
+                const uint2 sp = lds_v2(gaddr), bp = lds_v2(gaddr + SK_SB / 2);
+                sv[0] = sp.x & 0xFFFFu; sv[1] = sp.x >> 16; sv[2] = sp.y & 0xFFFFu; sv[3] = sp.y >> 16;
+                bv[0] = bp.x & 0xFFFFu; bv[1] = bp.x >> 16; bv[2] = bp.y & 0xFFFFu; bv[3] = bp.y >> 16;
+            } else if (g == 64) {  // two groups: stretches (0,1) and (2,3)
+                const uint32_t sp = lds_u32(gaddr), bp = lds_u32(gaddr + SK_SB / 2);
+                sv[0] = sv[1] = sp & 0xFFFFu; sv[2] = sv[3] = sp >> 16;
+                bv[0] = bv[1] = bp & 0xFFFFu; bv[2] = bv[3] = bp >> 16;
+            } else {  // one group for the whole half
+                sv[0] = sv[1] = sv[2] = sv[3] = lds_u16v(gaddr);
+                bv[0] = bv[1] = bv[2] = bv[3] = lds_u16v(gaddr + SK_SB / 2);
             }
             if (aused >= NA) {
                 if (!sk_wait(bar_aempty + 8 * a, pa ^ 1u, abort_flag, p.timeout)) break;
@@ -793,14 +816,33 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             tc_fence_after();
             const uint32_t acol = a_base + uint32_t(a * TM::ACOLS);
             if constexpr (TM::FOLD) {
-                sk_dequant_fold_store<BITS>(wd, s0, b0, s1, b1, acol);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    uint32_t w[F::NW];
+#pragma unroll
+                    for (int i = 0; i < F::NW; ++i) w[i] = wd[j * F::NW + i];
+                    sk_dequant_fold_store<BITS>(w, sv[2 * j], bv[2 * j], sv[2 * j + 1], bv[2 * j + 1], acol + 32 * j);
+                }
             } else {
-                const RowConst C0 = row_const<BITS>(s0), C1 = row_const<BITS>(s1);
-                const bool big = ((s0 & 0x7FFFu) >= 0x5400u) | ((s1 & 0x7FFFu) >= 0x5400u);
-                if (__any_sync(0xffffffffu, big)) sk_dequant_store<BITS, true>(wd, C0, C1, acol);
-                else sk_dequant_store<BITS, false>(wd, C0, C1, acol);
-                tmem_st_32x32b_x2(ab_base + uint32_t(a * TM::ACOLS), __byte_perm(b0, 0u, 0x1010u),
-                                  __byte_perm(b1, 0u, 0x1010u));
+                bool big = false;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) big |= (sv[i] & 0x7FFFu) >= 0x5400u;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    uint32_t w[F::NW];
+#pragma unroll
+                    for (int i = 0; i < F::NW; ++i) w[i] = wd[j * F::NW + i];
+                    sk_dequant_store<BITS, false>(w, row_const<BITS>(sv[2 * j]), row_const<BITS>(sv[2 * j + 1]),
+                                                  acol + 32 * j);
+                }
+                if (__any_sync(0xffffffffu, big)) {
+#pragma unroll 1
+                    for (int j = 0; j < 2; ++j)
+                        sk_dequant_store_safe<BITS>(wd + j * F::NW, sv[2 * j], sv[2 * j + 1], acol + 32 * j);
+                }
+                tmem_st_32x32b_x4(ab_base + uint32_t(a * TM::ACOLS), __byte_perm(bv[0], 0u, 0x1010u),
+                                  __byte_perm(bv[1], 0u, 0x1010u), __byte_perm(bv[2], 0u, 0x1010u),
+                                  __byte_perm(bv[3], 0u, 0x1010u));
             }
             tc_wait_st();
             tc_fence_before();
@@ -827,8 +869,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                 uint16_t* const y = p.y[it];
                 float* part = P > 1 ? p.partials + size_t(sk_slot(c, t, p.per, p.S)) * MP * SK_ROWS : nullptr;
 #pragma unroll 1
-                for (int cw = 0; cw < (MP / 8 + 3) / 4; ++cw) {
-                    const int ch = uq + 4 * cw;
+                for (int cw = 0; cw < (MP / 8 + 1) / 2; ++cw) {
+                    const int ch = uh + 2 * cw;
                     if (ch < MP / 8) {
                         // accumulators 0..NACC-1 added in order, then 64 x the bias accumulator
                         float acc[8];
@@ -902,8 +944,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                     if (*verdict) {
                         __threadfence();
 #pragma unroll 1
-                        for (int cw = 0; cw < (MP / 8 + 3) / 4; ++cw) {
-                            const int ch = uq + 4 * cw;
+                        for (int cw = 0; cw < (MP / 8 + 1) / 2; ++cw) {
+                            const int ch = uh + 2 * cw;
                             if (ch < MP / 8 && n < N) {
 #pragma unroll
                                 for (int i = 0; i < 8; ++i) {
