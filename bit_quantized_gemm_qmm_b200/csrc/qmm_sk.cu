@@ -62,13 +62,16 @@ constexpr float SK_XS_SCALE = 0.015625f;            // the x sums are staged tim
 constexpr float SK_XS_UNSCALE = 64.f;
 constexpr int SK_MAX_ITEMS = 4;                     // weight matrices one launch may cover
 
-// Tensor memory (512 columns): NACC accumulators and the bias accumulator, MP columns each,
-// then NA buffers of A (128 columns of codes + 8 of biases).  Above 64 tokens there is no
-// room for a second accumulator: the bias is folded into A (FOLD: A = RN_fp16(s*q + b), two
-// fp16 operations per code pair instead of one), one accumulator, no bias MMA.
+// Tensor memory (512 columns): the accumulator and the bias accumulator, MP columns each,
+// then NA buffers of A (128 columns of codes + 8 of biases).  One thread issues every MMA:
+// measured on B200, back-to-back tcgen05.mma (M = 128, K = 16, N <= 64) issue every ~46
+// cycles from one thread, with A in tensor or shared memory alike, while three issuing
+// warps together managed only one per ~125 cycles.  Above 64 tokens there is no room for a
+// second accumulator: the bias is folded into A (FOLD: A = RN_fp16(s*q + b), two fp16
+// operations per code pair instead of one), no bias MMA.
 template <int MP> struct SkTm {
     static constexpr bool FOLD = MP > 64;
-    static constexpr int NACC = FOLD ? 1 : (MP == 64 ? 2 : 3);
+    static constexpr int NACC = 1;
     static constexpr int NBIAS = FOLD ? 0 : 1;
     static constexpr int ABASE = (NACC + NBIAS) * MP;
     static constexpr int ACOLS = SK_KC / 2 + (FOLD ? 0 : 8);
@@ -653,7 +656,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         sk_wait(bar_eready, 0, abort_flag, p.timeout);
 
         constexpr uint32_t idesc = idesc_f16_f32(SK_ROWS, MP);
-        const bool issuer = j < NACC;
+        const bool issuer = j == 0;
         int a = 0, sx = 0, nseg = 0, nstaged = 0;
         uint32_t pa = 0, px = 0;
         int t = u0 / p.S, s = s_a;
@@ -693,6 +696,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             } else {
                 xbase = sbase + L.x_off + uint32_t(sx * MP * 512);
                 xsbase = sbase + L.xs_off + uint32_t(sx * MP * 32);
+            }
+            if (!issuer) {  // the other warps only help stage x
+                if (++s == p.S) { s = 0; ++t; }
+                continue;
             }
             bool ok = true;
             if (!XS) ok = sk_wait(bar_xfull + 8 * sx, px, abort_flag, p.timeout);
