@@ -657,7 +657,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
 
         constexpr uint32_t idesc = idesc_f16_f32(SK_ROWS, MP);
         const bool issuer = j == 0;
-        int a = 0, sx = 0, nseg = 0, nstaged = 0;
+        int a = 0, sx = 0, nseg = 0;
         uint32_t pa = 0, px = 0;
         int t = u0 / p.S, s = s_a;
         (void)t;
@@ -670,28 +670,33 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                 if (slot < 0) slot += p.S;
                 xbase = sbase + L.x_off + uint32_t(slot * MP * 512);
                 xsbase = sbase + L.xs_off + uint32_t(slot * MP * 32);
-                if (slot >= nstaged) {
-                    // stage this stage's x: M rows x 256 values
+                if (u == u0) {
+                    // every stage of x this block reads, in one batch: the loads of all of
+                    // them are in flight together (the call is waiting for x at this point)
                     constexpr int UN = F::UN, UPR = SK_KC / UN;
-                    const int k0 = s * SK_KC;
+                    const int per_slot = p.M * UPR;
                     stage_x_range<BITS, 64 / UN>(
-                        p.x, p.K, p.is_bf16, escale, MP, tid, SK_NISS * 32, p.M * UPR,
+                        p.x, p.K, p.is_bf16, escale, MP, tid, SK_NISS * 32, per_slot * p.nslots,
                         [&](int i, int& m, int& k, int& kk, uint8_t*& gd, uint32_t& sd) {
-                            m = i / UPR;
-                            kk = (i - m * UPR) * UN;
-                            k = k0 + kk;
+                            const int sl = i / per_slot, r = i - sl * per_slot;
+                            int st = s_a + sl;
+                            if (st >= p.S) st -= p.S;
+                            m = r / UPR;
+                            kk = (r - m * UPR) * UN;
+                            k = st * SK_KC + kk;
                             gd = nullptr;
-                            sd = xbase;
+                            sd = sbase + L.x_off + uint32_t(sl * MP * 512);
                         },
-                        [&](int, int m, int kk, float sum) {
-                            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xsbase + xsum_off(m, kk / 32)),
+                        [&](int i, int m, int kk, float sum) {
+                            const int sl = i / per_slot;
+                            asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbase + L.xs_off + uint32_t(sl * MP * 32) +
+                                                                          xsum_off(m, kk / 32)),
                                          "r"(xsum_pack(sum)));
                         });
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_xstage);
-                    sk_wait(bar_xstage, uint32_t(nstaged & 1), abort_flag, p.timeout);
-                    ++nstaged;
+                    sk_wait(bar_xstage, 0, abort_flag, p.timeout);
                 }
             } else {
                 xbase = sbase + L.x_off + uint32_t(sx * MP * 512);
@@ -923,7 +928,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                     if (dw == 0 && lane == 0) {
                         int last = 0;
                         if (sk_wait1(bar_gather, uint32_t(nsplit & 1), abort_flag, p.timeout)) {
-                            __threadfence();
+                            // every writer fenced its partial sums before the gather barrier
                             unsigned long long* word = p.counters + t;
                             unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(word);
                             for (int it = 0; it < 64; ++it) {
@@ -937,10 +942,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                                 }
                                 old = prev;
                             }
-                            if (last) {
-                                atomicExch(word, 0ull);  // ready for the next call that uses it
-                                __threadfence();
-                            }
+                            if (last) atomicExch(word, 0ull);  // ready for the next call that uses it
                         }
                         *verdict = last;
                         mbar_arrive(bar_verdict);
@@ -1078,7 +1080,7 @@ SkKernelFn pick_sk(int bits, int mp, bool xs) {
 
 constexpr int kNumSM = 148;
 constexpr size_t kSkMaxSmem = 227 * 1024;
-constexpr int kSkStagedMax = 6;  // x stages a block stages itself at most (default choice)
+constexpr int kSkStagedMax = 6;  // x stages a block stages itself at most (default choice, <= 16 tokens)
 
 size_t sk_smem(int bits, int mp, int sc, int xslots) {
     return size_t(sk_layout(bits, mp, sc, xslots).total) + 1024;  // + alignment slack
@@ -1257,7 +1259,7 @@ SkConfig sk_config(int64_t M, int64_t N, int64_t K, int bits, int group, int xmo
     // few stages of it and they fit beside a ring of at least 3 code stages; otherwise staged
     // once per call in the workspace by a small kernel and streamed per stage (ring of 3)
     auto fits = [&](int sc, int xslots) { return sk_smem(bits, c.mp, sc, xslots) <= kSkMaxSmem; };
-    bool xs = nst <= kSkStagedMax && fits(3, nst);
+    bool xs = c.mp == 16 && nst <= kSkStagedMax && fits(3, nst);
     if (xmode_req == 1) xs = true;
     if (xmode_req == 2) xs = false;
     if (c.mp > 64) xs = false;  // the wide variants take x from the workspace only
