@@ -95,6 +95,52 @@ __device__ __forceinline__ void dq6_triplet(uint32_t A, uint32_t B, uint32_t Cw,
     a[7] = scaled<SAFE>(((Cw >> 10) & 0x003F03F0u) | kM64_1024, kM64_1024, C.S, C.NB);
 }
 
+// ---------------------------------------------------------------- exact codes
+// The group-scaled kernels keep the codes exact in the MMA and apply each group's scale to
+// the group's fp32 partial sums instead, y = sum_g s_g (x . q)_g + b_g X_g: no rounding of
+// s*q to fp16 and no per-element scale arithmetic.
+//
+// 4-bit: a byte 0000qqqq read as FP8 E4M3 is exactly q * 2^-9 (exponent field 0 is the
+// subnormal range m * 2^-9, field 1 is 2^-6 + m * 2^-9 = (8 + m) * 2^-9: one linear scale
+// across both, and 0x7F, the only NaN below 0x80, is out of reach), so one conversion of two
+// such bytes gives the fp16 pair (q_a, q_b) * 2^-9 without any integer-to-float work.
+// Word v (nibble i = code i) -> pairs (0,2) (4,6) (1,3) (5,7), each times 2^-9.
+__device__ __forceinline__ uint32_t e4m3x2_lo(uint32_t v) {  // bytes 0, 1 -> fp16 pair
+    uint32_t d;
+    asm("{.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}" : "=r"(d) : "r"(v));
+    return d;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi(uint32_t v) {  // bytes 2, 3 -> fp16 pair
+    uint32_t d;
+    asm("{.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;\n\t}" : "=r"(d) : "r"(v));
+    return d;
+}
+__device__ __forceinline__ void dq4_exact(uint32_t v, uint32_t (&a)[4]) {
+    const uint32_t lo = v & 0x0F0F0F0Fu, hi = (v >> 4) & 0x0F0F0F0Fu;
+    a[0] = e4m3x2_lo(lo);
+    a[1] = e4m3x2_hi(lo);
+    a[2] = e4m3x2_lo(hi);
+    a[3] = e4m3x2_hi(hi);
+}
+
+// 8-bit word (byte i = code i) -> pairs (0,1) (2,3) of the exact codes: 1024 + q, then - 1024.
+__device__ __forceinline__ void dq8_exact(uint32_t v, uint32_t (&a)[2]) {
+    a[0] = hsub2(__byte_perm(v, 0x64646464u, 0x4140u), kM1024x2);
+    a[1] = hsub2(__byte_perm(v, 0x64646464u, 0x4342u), kM1024x2);
+}
+
+// Factor by which the exact-code MMA undercounts: the 4-bit values carry 2^-9.
+template <int BITS>
+__host__ __device__ constexpr float exact_code_unscale() { return BITS == 4 ? 512.f : 1.f; }
+
+// Order of the 8 codes of a word within its staged x chunk in the exact-code layout: the pair
+// order of dq4_exact (0 2 4 6 1 3 5 7) for 4-bit, natural for 8-bit.
+template <int BITS>
+__host__ __device__ constexpr int perm_nat(int i) {
+    if (BITS == 4) return i < 4 ? 2 * i : 2 * (i - 4) + 1;
+    return i;
+}
+
 // Position, within a lane's staged K-span, of each code of a staging unit (8 codes for 4/8-bit,
 // 16 for 6-bit): the pair order of the dequant.  4-bit: word pairs (i, i+4); 6-bit: the
 // triplet pairs (0,3) (1,4) (2,5) (6,9) (7,10) (8,11) (12,14) (13,15); 8-bit: natural order.
@@ -177,6 +223,10 @@ __device__ __forceinline__ void step_mma(const uint32_t (&w)[2][StepFmt<BITS>::N
 // ---------------------------------------------------------------- x staging
 constexpr int kXPad = 4;  // 16-byte chunks of padding after each staged x row
 
+// Padding of the exact-code layout: its 8-bit B fragments are 8-byte reads (4 lanes x 8 B a
+// token row), which a 32-byte row skew keeps free of bank conflicts; 16-byte reads take 64.
+__host__ __device__ constexpr int x_pad(int bits, bool nat) { return (nat && bits == 8) ? 2 : kXPad; }
+
 // Stage x[0:M, kc : kc + xchunk) as fp16 (zero past kend) in the lane
 // layout: row m, step s, lane span c, chunk j at 16-byte chunk m*RS + s*(KS/8) + 4j + c
 // (RS = xchunk/8 + kXPad, which keeps the B-fragment reads free of bank conflicts), codes in
@@ -187,7 +237,11 @@ constexpr int kXPad = 4;  // 16-byte chunks of padding after each staged x row
 // rows only reach accumulator columns that are never stored.
 // Run by `nthreads` threads (whole warps, threadIdx.x < nthreads); xchunk is a multiple of
 // the step and of the group.
-template <int BITS, int MT>
+//
+// NAT (the exact-code layout of the group-scaled kernels): each 8-code unit is one chunk at its
+// natural position (chunk kk of the row), its codes in perm_nat order, rows x_pad(BITS, true)
+// chunks apart past the data.
+template <int BITS, int MT, bool NAT = false>
 __device__ __forceinline__ void stage_x_tile(const uint16_t* __restrict__ x, int M, int K, int is_bf16, int group,
                                              int xchunk, int gpad, int nthreads, uint32_t xs, uint32_t xg, int kc,
                                              int kend, float xscale) {
@@ -198,7 +252,7 @@ __device__ __forceinline__ void stage_x_tile(const uint16_t* __restrict__ x, int
     const int rows = M < 8 * MT ? M : 8 * MT;              // token rows >= M are never read back
     const int total = rows * upr;
     const int totp = (total + 31) & ~31;                   // whole warps take part in the shuffles
-    const int RS = xchunk / 8 + kXPad;
+    const int RS = xchunk / 8 + x_pad(BITS, NAT);
     const int upg = group / UN;                            // units per group
     for (int u0 = 0; u0 < totp; u0 += nthreads) {
         if (u0 + int(threadIdx.x & ~31u) >= totp) break;   // whole warps only
@@ -243,17 +297,27 @@ __device__ __forceinline__ void stage_x_tile(const uint16_t* __restrict__ x, int
             asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(m * gpad + kk / upg) * 4u), "r"(pk));
         }
         // permuted fp16 chunks
-        const int s = kk / UPS, wu = kk - s * UPS;
-        const int c = wu / UPL, t = wu - c * UPL;
-#pragma unroll
-        for (int h = 0; h < UN / 8; ++h) {
-            const int j = t * (UN / 8) + h;
+        if constexpr (NAT) {
+            static_assert(UN == 8, "the exact-code layout stages one chunk per unit");
             uint4 o;
             uint32_t* ov = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                ov[i] = f32x2_to_f16x2(f[perm_src<BITS>(8 * h + 2 * i)], f[perm_src<BITS>(8 * h + 2 * i + 1)]);
-            sts_v4(xs + uint32_t(m * RS + s * (KS / 8) + 4 * j + c) * 16u, o);
+                ov[i] = f32x2_to_f16x2(f[perm_nat<BITS>(2 * i)], f[perm_nat<BITS>(2 * i + 1)]);
+            sts_v4(xs + uint32_t(m * RS + kk) * 16u, o);
+        } else {
+            const int s = kk / UPS, wu = kk - s * UPS;
+            const int c = wu / UPL, t = wu - c * UPL;
+#pragma unroll
+            for (int h = 0; h < UN / 8; ++h) {
+                const int j = t * (UN / 8) + h;
+                uint4 o;
+                uint32_t* ov = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    ov[i] = f32x2_to_f16x2(f[perm_src<BITS>(8 * h + 2 * i)], f[perm_src<BITS>(8 * h + 2 * i + 1)]);
+                sts_v4(xs + uint32_t(m * RS + s * (KS / 8) + 4 * j + c) * 16u, o);
+            }
         }
     }
     const int npg = xchunk / group;

@@ -13,11 +13,16 @@
 //     (double-buffered per tile) and, per K stage, one box of packed codes (128 rows x 128 B,
 //     192 B for 6-bit), each completing on an mbarrier; the ring runs across tiles, so a
 //     persistent block streams without gaps;
-//   * eight consumer warps own 16 rows each.  Per stage a lane reads its 64 codes (32 for
-//     8-bit) of two rows from shared memory, dequantizes them in registers to A = RN_fp16(s q)
-//     (qmm_dq.cuh) and runs mma.sync m16n8k16 against x held in shared memory for the whole
-//     K range of the block, staged once in the matching pair order.  The bias enters as b
-//     times the group sum of x, one more MMA per eight groups at the end of the tile;
+//   * sixteen consumer warps: eight 16-row groups times the two K halves of a stage.  At 4
+//     and 8 bits the codes go into the MMA exactly (y = sum_g s_g (x . q)_g + b_g X_g): a lane
+//     takes its code words by ldmatrix so that every m16n8k16 MMA covers 32 (4-bit) or 16
+//     (8-bit) consecutive codes, i.e. lies inside one group; 4-bit codes become fp16 through
+//     one FP8 (E4M3) conversion per pair (q * 2^-9, exact), 8-bit codes through a byte
+//     permute and a subtraction; a group's MMAs accumulate from zero and their sum is added
+//     into the row's fp32 total times the group's scale.  6-bit codes (24-byte lane spans)
+//     are dequantized per element to A = RN_fp16(s q) instead.  x sits in shared memory for
+//     the whole K range of the block, staged once in the matching order.  The bias enters as
+//     b times the group sum of x, one more MMA per eight groups at the end of the tile;
 //   * K is split across the blocks of a cluster when there are too few tiles to fill the
 //     GPU; partial sums are added over distributed shared memory in rank order, so results
 //     are deterministic.
@@ -96,7 +101,7 @@ __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int ks
     L.sb_slot = uint32_t(2 * ST_ROWS * (st_block_codes(bits, group) / group) * 2);  // scales + biases
     uint32_t off = L.sb_off + ST_SS * L.sb_slot;
     L.x_off = off;
-    L.xrs = uint32_t(kslice / 8 + kXPad);                     // 16-byte chunks per staged x row
+    L.xrs = uint32_t(kslice / 8 + x_pad(bits, bits != 6));    // 16-byte chunks per staged x row
     off += uint32_t(mrows) * L.xrs * 16;
     L.xg_off = off;
     L.gpad = uint32_t((kslice / group + 7) / 8 * 8);
@@ -143,6 +148,11 @@ __device__ __forceinline__ uint2 lds_v2(uint32_t a) {
     asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
 
 // Exponent E >= 0 such that max|x| * 2^-E < 2^15 over x[:, kb:ke] (bf16 activations only).
 template <int NCW>
@@ -168,7 +178,80 @@ __device__ __forceinline__ int bf16_exponent(const StParams& p, int kb, int ke, 
     return eb > 141 ? eb - 141 : 0;
 }
 
-template <int BITS, int MT, int NCW>
+// The MMAs of one step in the exact-code layout (4- and 8-bit): lane (g, c) holds, per row
+// (g, g+8), code word 4i + c of the step in w[r][i] (i = 0..3).  Block i (32 codes at 4 bits,
+// 16 at 8) is one MMA's K range for every lane, so each MMA lies inside one group: the
+// group's MMAs accumulate into tmp (from zero), and at the group's last block tmp is added
+// into acc times the group's scale (fa: row g, fb: row g+8).  `sj` = step within the half,
+// BPG = blocks per group, fa/fb = the fp16 scales of the half's groups, two to a word.
+template <int NGH>
+__device__ __forceinline__ float scale_at(const uint32_t (&f)[(NGH + 1) / 2], int i) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&f[i >> 1]);
+    return (i & 1) ? __high2float(h) : __low2float(h);
+}
+template <int BITS, int MT, int BPG, int NGH>
+__device__ __forceinline__ void step_exact(const uint32_t (&w)[2][4], const int sj, uint32_t xa, uint32_t xmt,
+                                           const uint32_t (&fa)[(NGH + 1) / 2], const uint32_t (&fb)[(NGH + 1) / 2],
+                                           float (&tmp)[MT][4], float (&acc)[MT][4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int bh = sj * 4 + i;  // block within the half
+        const bool first = bh % BPG == 0;
+        if constexpr (BITS == 4) {
+            uint32_t a0[4], a1[4];
+            dq4_exact(w[0][i], a0);
+            dq4_exact(w[1][i], a1);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const uint4 xb = lds_v4(xa + uint32_t(i * 64) + mt * xmt);
+                if (first) mma_16816_z(tmp[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
+                else mma_16816(tmp[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
+                mma_16816(tmp[mt], a0[2], a1[2], a0[3], a1[3], xb.z, xb.w);
+            }
+        } else {
+            uint32_t a0[2], a1[2];
+            dq8_exact(w[0][i], a0);
+            dq8_exact(w[1][i], a1);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const uint2 xb = lds_v2(xa + uint32_t(i * 32) + mt * xmt);
+                if (first) mma_16816_z(tmp[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
+                else mma_16816(tmp[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
+            }
+        }
+        if ((bh + 1) % BPG == 0) {
+            const float sa = scale_at<NGH>(fa, bh / BPG), sb = scale_at<NGH>(fb, bh / BPG);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                acc[mt][0] = fmaf(sa, tmp[mt][0], acc[mt][0]);
+                acc[mt][1] = fmaf(sa, tmp[mt][1], acc[mt][1]);
+                acc[mt][2] = fmaf(sb, tmp[mt][2], acc[mt][2]);
+                acc[mt][3] = fmaf(sb, tmp[mt][3], acc[mt][3]);
+            }
+        }
+    }
+}
+
+// The NGH fp16 scales starting at shared address a (2*NGH-byte aligned), two to a word.
+template <int NGH>
+__device__ __forceinline__ void load_scales(uint32_t a, uint32_t (&v)[(NGH + 1) / 2]) {
+    if constexpr (NGH == 1) {
+        v[0] = lds_u16(a);
+    } else if constexpr (NGH == 2) {
+        v[0] = lds_u32(a);
+    } else if constexpr (NGH == 4) {
+        const uint2 t = lds_v2(a);
+        v[0] = t.x; v[1] = t.y;
+    } else {
+        static_assert(NGH == 8, "a K half holds 1, 2, 4 or 8 groups");
+        const uint4 t = lds_v4(a);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    }
+}
+
+// G = the group size for the exact-code path (4- and 8-bit); 0 for 6-bit, whose codes are
+// dequantized to RN_fp16(s*q) per element (step_mma) and whose group size is a parameter.
+template <int BITS, int MT, int NCW, int G>
 __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     qmm_stream_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                       const __grid_constant__ CUtensorMap bmap, const StParams p) {
@@ -179,6 +262,11 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     constexpr int KS = SF::KSTG;               // codes per stage
     constexpr int NREG = F::NREG, U = F::U;
     constexpr int HPW = StWarps<NCW>::HPW;
+    constexpr bool NAT = BITS != 6;                       // exact codes, group-scaled partial sums
+    static_assert(NAT == (G != 0), "G is the group size of the exact-code path");
+    constexpr int BC = BITS == 4 ? 32 : 16;               // codes per MMA block (exact-code path)
+    constexpr int BPG = NAT ? G / BC : 1;                 // blocks per group
+    constexpr int NGH = NAT ? (KS / 2) / G : 1;           // groups per K half of a stage
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ float s_red[NCW];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -290,19 +378,23 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         const int g = lane >> 2, c = lane & 3;
         const int hbase = NCW == 16 ? (warp >> 3) : 0;         // first K half this warp takes
         const int rg = warp & 7;                                // 16-row group of the tile
-        const int rA = rg * 16 + ((g >> 1) | ((g & 1) << 2));  // rows of "g" and "g + 8": the
-        const int rB = rA + 8;                                  // permutation keeps the code reads conflict-free
+        // rows of "g" and "g + 8": natural for the ldmatrix reads of the exact-code path; the
+        // 6-bit reads (8-byte pieces of 24-byte lane spans) stay conflict-free under a permutation
+        const int rA = rg * 16 + (NAT ? g : ((g >> 1) | ((g & 1) << 2)));
+        const int rB = rA + 8;
         grid_dependency_wait();
         const int E = p.is_bf16 ? bf16_exponent<NCW>(p, kb, ke, s_red) : 0;
         const uint32_t xs = sbase + L.x_off, xg = sbase + L.xg_off;
-        stage_x_tile<BITS, MT>(p.x, p.M, p.K, p.is_bf16, p.group, p.kslice, int(L.gpad), NCW * 32, xs, xg, kb, ke,
-                               exp2i(-E));
+        stage_x_tile<BITS, MT, NAT>(p.x, p.M, p.K, p.is_bf16, p.group, p.kslice, int(L.gpad), NCW * 32, xs, xg, kb,
+                                    ke, exp2i(-E));
         consumer_sync<NCW>();
         grid_dependents_launch();
 
         const int tr0 = min(g, p.M - 1), tr1 = min(g + 8, p.M - 1);  // token rows of the two x tiles
         const uint32_t xmt = uint32_t(tr1 - tr0) * L.xrs * 16;
-        const uint32_t xlane = xs + uint32_t(tr0 * int(L.xrs) + c) * 16u + uint32_t(hbase * SPH * KSS * 2);
+        // the lane's B fragments: 16-byte chunk c of each 4-chunk block (8 bytes at 8-bit)
+        const uint32_t xlane = xs + uint32_t(tr0 * int(L.xrs)) * 16u + uint32_t(c * (BITS == 8 ? 8 : 16)) +
+                               uint32_t(hbase * SPH * KSS * 2);
         const uint32_t xgrow = xg + uint32_t(tr0 * int(L.gpad)) * 4u;
         const uint32_t xg_mt = uint32_t(tr1 - tr0) * L.gpad * 4;
         float* xf = reinterpret_cast<float*>(smem + L.xf_off) + (rg * 32 + lane) * 4 * MT;
@@ -315,15 +407,22 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 #pragma unroll
         for (int j = 0; j < HPW * SPH; ++j) lane_off[j] = (hbase * SPH + j) * KSS + c * U;
         const uint32_t rAg = uint32_t(rA * gbb) * 2u, rBg = uint32_t(rB * gbb) * 2u;
+        // exact-code path: the lane's ldmatrix row address within a code box, per step of the
+        // half (lanes 8i..8i+7 address rows 0..7 of the warp's 16 at chunk 4*step + i, under
+        // the 128-byte swizzle: chunk ^ (row & 7))
+        uint32_t ldm_off[SPH];
+#pragma unroll
+        for (int sj = 0; sj < SPH; ++sj)
+            ldm_off[sj] = uint32_t((rg * 16 + (lane & 7)) * 128 + ((((4 * sj + (lane >> 3)) ^ lane) & 7) << 4));
         for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++tc) {
             // After a timeout (abort flag set) every wait below returns at once and the work
             // is skipped, so all warps leave the loop together.
             const long long dl = clock64() + ST_TIMEOUT;
-            float acc[MT][4], tb[MT][4];
+            float acc[MT][4], tb[MT][4], tmp[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[mt][i] = tb[mt][i] = 0.f;
+                for (int i = 0; i < 4; ++i) acc[mt][i] = tb[mt][i] = tmp[mt][i] = 0.f;
             uint32_t sbuf = 0;
             bool sok = true;
             int sib = 0;             // stage within the scale block
@@ -335,7 +434,38 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                     sbuf = sbase + L.sb_off + ss * L.sb_slot;
                 }
                 const bool ok = sok && wait_or_abort(bar_full + 8 * s, ph, dl, abort_flag);
-                if (ok) {
+                if constexpr (NAT) {
+                  if (ok) {
+                    // the lane's code words 4i + c of rows rA and rB for each step of its K
+                    // half (halves), by ldmatrix; the ring slot is released once they are in
+                    // registers
+                    uint32_t w[HPW * SPH][2][4];
+                    const uint32_t stage = sbase + s * L.w_stage;
+#pragma unroll
+                    for (int hh = 0; hh < HPW; ++hh)
+#pragma unroll
+                        for (int sj = 0; sj < SPH; ++sj) {
+                            const uint32_t a = stage + uint32_t((hbase + hh) * (ST_ROWS * 128)) + ldm_off[sj];
+                            ldsm_x4(a, w[hh * SPH + sj][0]);
+                            ldsm_x4(a + 8 * 128, w[hh * SPH + sj][1]);
+                        }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+#pragma unroll
+                    for (int hh = 0; hh < HPW; ++hh) {
+                        // scales of the half's groups (a whole number of them: a half is 256
+                        // codes at 4-bit, 128 at 8-bit, and groups are at most 128)
+                        const uint32_t g0 = uint32_t((sib * KS + (hbase + hh) * (KS / 2)) / G) * 2u;
+                        uint32_t fa[(NGH + 1) / 2], fb[(NGH + 1) / 2];
+                        load_scales<NGH>(sbuf + rAg + g0, fa);
+                        load_scales<NGH>(sbuf + rBg + g0, fb);
+#pragma unroll
+                        for (int sj = 0; sj < SPH; ++sj)
+                            step_exact<BITS, MT, BPG, NGH>(w[hh * SPH + sj], sj, xst + uint32_t((hh * SPH + sj) * KSS * 2),
+                                                           xmt, fa, fb, tmp, acc);
+                    }
+                  }
+                } else if (ok) {  // 6-bit
                     // the lane's codes of rows rA and rB for the steps of its K half (halves);
                     // the ring slot is released as soon as they are in registers
                     uint32_t w[HPW * SPH][2][NREG];
@@ -346,21 +476,11 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 #pragma unroll
                         for (int r = 0; r < 2; ++r) {
                             const int row = r == 0 ? rA : rB;
-                            if constexpr (BITS == 6) {
 #pragma unroll
-                                for (int i = 0; i < 3; ++i) {
-                                    const uint2 v = lds_v2(stage + row * 192 + half * 96 + 24 * c + 8 * i);
-                                    w[hh][r][2 * i] = v.x;
-                                    w[hh][r][2 * i + 1] = v.y;
-                                }
-                            } else {  // box `half`, 128-byte swizzle: 16-byte chunk ^= row & 7
-#pragma unroll
-                                for (int j = 0; j < SPH; ++j) {
-                                    const uint4 v = lds_v4(stage + half * (ST_ROWS * 128) + row * 128 +
-                                                           ((((4 * j + c) ^ row) & 7) << 4));
-                                    w[hh * SPH + j][r][0] = v.x; w[hh * SPH + j][r][1] = v.y;
-                                    w[hh * SPH + j][r][2] = v.z; w[hh * SPH + j][r][3] = v.w;
-                                }
+                            for (int i = 0; i < 3; ++i) {
+                                const uint2 v = lds_v2(stage + row * 192 + half * 96 + 24 * c + 8 * i);
+                                w[hh][r][2 * i] = v.x;
+                                w[hh][r][2 * i + 1] = v.y;
                             }
                         }
                     }
@@ -444,7 +564,8 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[mt][i] = (acc[mt][i] + 128.f * tb[mt][i]) * yscale;
+                    for (int i = 0; i < 4; ++i)
+                        acc[mt][i] = ((NAT ? exact_code_unscale<BITS>() : 1.f) * acc[mt][i] + 128.f * tb[mt][i]) * yscale;
                 if (p.split == 1) {
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
@@ -515,15 +636,25 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 
 using StKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const StParams);
 
-template <int NCW>
-StKernelFn pick_stream_w(int bits, int mt) {
-    if (bits == 4) return mt == 1 ? qmm_stream_kernel<4, 1, NCW> : mt == 2 ? qmm_stream_kernel<4, 2, NCW> : nullptr;
-    if (bits == 6) return mt == 1 ? qmm_stream_kernel<6, 1, NCW> : mt == 2 ? qmm_stream_kernel<6, 2, NCW> : nullptr;
-    if (bits == 8) return mt == 1 ? qmm_stream_kernel<8, 1, NCW> : mt == 2 ? qmm_stream_kernel<8, 2, NCW> : nullptr;
-    return nullptr;
+template <int BITS, int MT>
+StKernelFn pick_stream_g(int group) {
+    if constexpr (BITS == 6) {
+        return qmm_stream_kernel<6, MT, 16, 0>;
+    } else {
+        if (group == 32) return qmm_stream_kernel<BITS, MT, 16, 32>;
+        if (group == 64) return qmm_stream_kernel<BITS, MT, 16, 64>;
+        if (group == 128) return qmm_stream_kernel<BITS, MT, 16, 128>;
+        return nullptr;
+    }
 }
-StKernelFn pick_stream(int bits, int mt, int ncw) {
-    return ncw == 8 ? pick_stream_w<8>(bits, mt) : pick_stream_w<16>(bits, mt);
+// 16 consumer warps (the 8-warp form of the kernel is not instantiated: it measured slower on
+// every configuration of the sweep)
+StKernelFn pick_stream(int bits, int mt, int ncw, int group) {
+    if (ncw != 16 || (mt != 1 && mt != 2)) return nullptr;
+    if (bits == 4) return mt == 1 ? pick_stream_g<4, 1>(group) : pick_stream_g<4, 2>(group);
+    if (bits == 6) return mt == 1 ? pick_stream_g<6, 1>(group) : pick_stream_g<6, 2>(group);
+    if (bits == 8) return mt == 1 ? pick_stream_g<8, 1>(group) : pick_stream_g<8, 2>(group);
+    return nullptr;
 }
 
 int ks_for(int bits) { return st_stage_codes(bits); }
@@ -685,7 +816,7 @@ cudaError_t ensure_smem_attr(StKernelFn fn, size_t smem) {
 
 cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream) {
     const int mt = int(a.M) > 8 ? 2 : 1;
-    StKernelFn fn = pick_stream(a.bits, mt, c.ncw);
+    StKernelFn fn = pick_stream(a.bits, mt, c.ncw, a.group);
     if (!fn || c.ring < 2) return cudaErrorNotSupported;
     // The three descriptors depend only on the weight arrays and the format; a call that
     // repeats them (the usual case: the same weights every step) reuses the encoded copies.
