@@ -72,12 +72,27 @@ struct StreamConfig {
     int stage_bytes;  // shared memory of one ring stage
     bool split_raised;  // K split beyond the tile-count choice only to make x fit
     int grid_x;    // blocks along N (persistent when split == 1)
+    // Persistent grids whose tile count is not a multiple of the grid: the last partial wave
+    // of tiles is cut into scale blocks dealt out evenly (tail), its tiles' partial sums added
+    // by the last block to finish each.  dp_tiles = tiles taken whole; tunits = scale blocks
+    // of the tail; tper = tail scale blocks per block (0: no tail).
+    int dp_tiles, tunits, tper;
+    // x streamed through the ring with the codes (x tiles written by a small x pass first)
+    // instead of staged whole per block: 9-16 tokens on persistent grids
+    bool xstream;
     int ncw;       // consumer warps per block (8 or 16)
     size_t smem;   // dynamic shared memory per block
     bool pdl;
     bool static_weights;
 };
 bool stream_supported(int64_t M, int64_t N, int64_t K, int bits, int group);
+
+// Device scratch of a stream (and of each graph capture in progress on it), grown on demand
+// and kept: the partial sums and arrival words of tiles that several blocks share.  Calls on
+// one stream run in order and may share it.
+cudaError_t split_workspace(cudaStream_t stream, size_t bytes, void** out);
+// A fresh 48-bit tag for the arrival words of one call (never 0).
+unsigned long long next_call_token();
 
 // Fully resolved launch configuration of the evenly split tensor-core kernel (qmm_sk.cu).
 struct SkConfig {

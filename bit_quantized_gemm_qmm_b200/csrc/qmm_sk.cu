@@ -31,6 +31,7 @@
 #include <cuda.h>
 
 #include <atomic>
+#include <chrono>
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
@@ -960,11 +961,20 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                                 for (int i = 0; i < 8; ++i) {
                                     const int m = 8 * ch + i;
                                     if (m < p.M) {
+                                        // in part order; eight loads in flight at a time
+                                        const float* src0 = p.partials + m * SK_ROWS + row;
                                         float sum = 0.f;
-                                        for (int k = 0; k < P; ++k) {
-                                            const float* src = p.partials + size_t(sk_slot(cf + k, t, p.per, p.S)) * MP * SK_ROWS;
-                                            sum += __ldcg(src + m * SK_ROWS + row);
+                                        int k = 0;
+                                        for (; k + 8 <= P; k += 8) {
+                                            float v[8];
+#pragma unroll
+                                            for (int j = 0; j < 8; ++j)
+                                                v[j] = __ldcg(src0 + size_t(sk_slot(cf + k + j, t, p.per, p.S)) * MP * SK_ROWS);
+#pragma unroll
+                                            for (int j = 0; j < 8; ++j) sum += v[j];
                                         }
+                                        for (; k < P; ++k)
+                                            sum += __ldcg(src0 + size_t(sk_slot(cf + k, t, p.per, p.S)) * MP * SK_ROWS);
                                         y[int64_t(m) * N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sum))
                                                                               : __half_as_ushort(__float2half_rn(sum));
                                     }
@@ -1086,6 +1096,8 @@ size_t sk_smem(int bits, int mp, int sc, int xslots) {
     return size_t(sk_layout(bits, mp, sc, xslots).total) + 1024;  // + alignment slack
 }
 
+}  // namespace
+
 // ---------------------------------------------------------------- host: workspace
 // Each stream has a workspace of its own (and each graph capture in progress on a stream
 // another one), grown on demand and never shrunk: the partial sums of split tiles, their
@@ -1093,6 +1105,7 @@ size_t sk_smem(int bits, int mp, int sc, int xslots) {
 // order, so they can share it; calls on different streams (or in different captured
 // graphs) never do.  The arrival words carry the tag of the call that last used them and
 // are reset by the last block to arrive, so the memory needs no clearing.
+namespace {
 struct WsKey {
     int dev;
     uintptr_t stream;
@@ -1113,7 +1126,9 @@ std::mutex g_ws_mu;
 std::unordered_map<WsKey, Ws, WsKeyHash> g_ws;
 std::vector<void*> g_ws_retired;  // outgrown workspaces: kernels in flight may still use them
 
-cudaError_t sk_workspace(cudaStream_t stream, size_t bytes, void** out) {
+}  // namespace
+
+cudaError_t split_workspace(cudaStream_t stream, size_t bytes, void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1149,7 +1164,18 @@ cudaError_t sk_workspace(cudaStream_t stream, size_t bytes, void** out) {
     return cudaSuccess;
 }
 
-std::atomic<unsigned long long> g_sk_token{1};
+// Call tags start at a value taken from the clock, so that arrival words left in reused
+// device memory by another process (whose tags started elsewhere) do not match this one's.
+unsigned long long next_call_token() {
+    static std::atomic<unsigned long long> next{
+        (static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count()) * 2654435761ull) &
+        0xFFFFFFFFFFFFull};
+    unsigned long long t = next.fetch_add(1) & 0xFFFFFFFFFFFFull;
+    if (t == 0) t = next.fetch_add(1) & 0xFFFFFFFFFFFFull;
+    return t;
+}
+
+namespace {
 
 // Per-thread cache of encoded weight descriptors, keyed by the arrays and the format.
 struct SkMaps {
@@ -1300,7 +1326,7 @@ cudaError_t launch_sk_items(const QmmArgs& a, const SkItem* items, int nitems, c
     if (tiles != c.T) return cudaErrorNotSupported;
     p.nitems = nitems;
     void* ws = nullptr;
-    cudaError_t e = sk_workspace(stream, sk_ws_bytes(c), &ws);
+    cudaError_t e = split_workspace(stream, sk_ws_bytes(c), &ws);
     if (e != cudaSuccess) return e;
     e = sk_smem_attr(fn, c.smem);
     if (e != cudaSuccess) return e;
@@ -1318,8 +1344,7 @@ cudaError_t launch_sk_items(const QmmArgs& a, const SkItem* items, int nitems, c
         off += size_t(c.S) * size_t(c.mp) * 512;
         p.xsum = reinterpret_cast<const uint32_t*>(w + off);
     }
-    p.token = g_sk_token.fetch_add(1) & 0xFFFFFFFFFFFFull;
-    if (p.token == 0) p.token = g_sk_token.fetch_add(1) & 0xFFFFFFFFFFFFull;
+    p.token = next_call_token();
     p.M = int(a.M);
     p.K = int(a.K);
     p.gshift = a.group == 32 ? 5 : a.group == 64 ? 6 : 7;

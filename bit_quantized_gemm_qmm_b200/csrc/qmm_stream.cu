@@ -32,6 +32,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <type_traits>
 #include <unordered_map>
 
 #include "qmm_common.cuh"
@@ -53,7 +54,7 @@ constexpr int ST_ROWS = 128;                  // weight rows per tile
 // Consumer warps: 16 (8 row groups x 2 K halves, the two halves' partial sums meet at the end
 // of a tile) or 8 (one warp takes both halves; smaller blocks, two fit on an SM).
 template <int NCW> struct StWarps {
-    static constexpr int THREADS = (NCW + 1) * 32;  // + the producer warp
+    static constexpr int THREADS = (NCW + 2) * 32;  // + the producer warp and the tail helper
     static constexpr int HPW = 16 / NCW;            // K halves per consumer warp
 };
 constexpr int ST_SS = 3;                      // scale / bias boxes in flight
@@ -85,24 +86,112 @@ struct StParams {
     int split;
     int ring;     // stages in the shared-memory ring
     int static_w;
+    // persistent grids: whole tiles below dp_tiles, then the tail's scale blocks (tunits in
+    // all, tper per block); a tail tile's partial sums go to `partials` (slot 2c for the first
+    // tile of block c's run, 2c + 1 for the second) and its arrivals to counters[tile -
+    // dp_tiles], tagged with `token`
+    int dp_tiles, tunits, tper;
+    float* partials;
+    unsigned long long* counters;
+    unsigned long long token;
+    // x streamed (xstream = 1): per-stage x tiles [stage][16][xrs chunks], group sums
+    // [M][gpad] and per-token exponents, written by st_xprep_kernel just before
+    int xstream;
+    const uint8_t* xt;
+    const uint32_t* xgw;
+    const int* xexp;
 };
 
+// This block's work as a list of items (tile t, stages [s0, s1)): first its run of tail scale
+// blocks (one piece per tile, at most two), then its whole tiles blockIdx.x, + gridDim.x, ...
+// below dp_tiles.  The tail goes first so that the hand-off of its partial sums overlaps the
+// whole tiles that follow.  The counts are worked out once per block, and only the (at most
+// two) tail items take divisions.
+struct StWork {
+    int n;   // items
+    int np;  // tail pieces among them (the first np)
+};
+
+// Item k of this block's work, from its definition.  False once there is no item k.
+__device__ __forceinline__ bool st_item(const StParams& p, int nst, int spb, int k, int& t, int& s0, int& s1) {
+    const int c = blockIdx.x, G = gridDim.x;
+    const int nsb = nst / spb;
+    int u = c * p.tper;
+    const int u1 = min(p.tunits, u + p.tper);
+    int npieces = 0, len0 = 0;
+    if (u < u1) {
+        len0 = min(nsb - u % nsb, u1 - u);
+        npieces = u + len0 < u1 ? 2 : 1;
+    }
+    if (k < npieces) {
+        int len = len0;
+        if (k == 1) {
+            u += len0;
+            len = u1 - u;
+        }
+        t = p.dp_tiles + u / nsb;
+        s0 = (u % nsb) * spb;
+        s1 = s0 + len * spb;
+        return true;
+    }
+    k -= npieces;
+    const int ndp = c < p.dp_tiles ? (p.dp_tiles - c + G - 1) / G : 0;
+    if (k >= ndp) return false;
+    t = c + k * G;
+    s0 = 0;
+    s1 = nst;
+    return true;
+}
+
+__device__ __forceinline__ StWork st_work(const StParams& p, int nst, int spb) {
+    StWork w;
+    int k = 0, t, a, b;
+    while (k < 2 && st_item(p, nst, spb, k, t, a, b) && t >= p.dp_tiles) ++k;
+    w.np = k;
+    const int c = blockIdx.x, G = gridDim.x;
+    w.n = k + (c < p.dp_tiles ? (p.dp_tiles - c + G - 1) / G : 0);
+    return w;
+}
+
+// Item k of the block's work: the tail pieces through st_item (two at most), the whole tiles
+// by a step of the grid.
+__device__ __forceinline__ void st_work_item(const StParams& p, const StWork& w, int nst, int spb, int k, int& t,
+                                             int& s0, int& s1) {
+    if (k < w.np) {
+        st_item(p, nst, spb, k, t, s0, s1);
+    } else {
+        t = int(blockIdx.x) + (k - w.np) * int(gridDim.x);
+        s0 = 0;
+        s1 = nst;
+    }
+}
+
+// Partial-sum slot of tail tile t (index ti past dp_tiles) from block c.
+__device__ __forceinline__ int st_slot(const StParams& p, int nsb, int c, int ti) {
+    return 2 * c + ((c * p.tper) / nsb == ti ? 0 : 1);
+}
+
 struct StLayout {
-    uint32_t w_stage, sb_off, sb_slot, x_off, xrs, xg_off, gpad, xf_off, red_off, bar_off, total;
+    uint32_t w_stage, slot, xtile, sb_off, sb_slot, x_off, xrs, xg_off, gpad, xf_off, red_off, bar_off, total;
 };
 
 // x and its group sums are staged for the M real token rows only (reads for token rows >= M
 // are redirected to row M-1: they feed accumulator columns that are never stored).
+// xs (x streamed): instead of x for the whole K range, each ring slot carries, after the
+// stage's codes, that stage's x tile [16 token rows][xrs chunks] (written once per call by
+// st_xprep_kernel and brought in by the same barrier as the codes).
 __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split, int ncw,
-                                              int mrows) {
+                                              int mrows, bool xs = false) {
     StLayout L;
     L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 256));  // 24 or 32 KB
-    L.sb_off = uint32_t(ring) * L.w_stage;
+    L.xrs = uint32_t((xs ? st_stage_codes(bits) : kslice) / 8 + x_pad(bits, bits != 6));  // chunks per x row
+    L.xtile = xs ? 16u * L.xrs * 16u : 0u;
+    L.slot = (L.w_stage + L.xtile + 1023) / 1024 * 1024;      // codes stay 1024-byte aligned (swizzle)
+    L.sb_off = uint32_t(ring) * L.slot;
     L.sb_slot = uint32_t(2 * ST_ROWS * (st_block_codes(bits, group) / group) * 2);  // scales + biases
     uint32_t off = L.sb_off + ST_SS * L.sb_slot;
     L.x_off = off;
-    L.xrs = uint32_t(kslice / 8 + x_pad(bits, bits != 6));    // 16-byte chunks per staged x row
-    off += uint32_t(mrows) * L.xrs * 16;
+    if (!xs) off += uint32_t(mrows) * L.xrs * 16;
     L.xg_off = off;
     L.gpad = uint32_t((kslice / group + 7) / 8 * 8);
     off += uint32_t(mrows) * L.gpad * 4;
@@ -112,7 +201,7 @@ __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int ks
     if (split > 1) off += uint32_t(split * ((ST_ROWS + split - 1) / split) * 8 * mt * 4);
     off = (off + 15) & ~15u;
     L.bar_off = off;
-    off += 8 * uint32_t(2 * ring + 2 * ST_SS + 16) + 16;
+    off += 8 * uint32_t(2 * ring + 2 * ST_SS + 18) + 16 + 64;  // + abort word; 2^E of 16 tokens
     L.total = off;
     return L;
 }
@@ -125,9 +214,11 @@ __device__ __forceinline__ void consumer_sync() {
 
 // Bounded mbarrier wait that gives up at once when the block is aborting, so that after a
 // timeout every warp runs through the rest of its loop without waiting (no warp is left
-// behind at a barrier).  A timeout sets the error bit and the block's abort flag.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, long long dl, volatile int* abort_flag) {
+// behind at a barrier).  A timeout (ST_TIMEOUT cycles from the first failed try) sets the
+// error bit and the block's abort flag.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
+    const long long dl = clock64() + ST_TIMEOUT;
     while (true) {
         if (*abort_flag) return false;
         if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
@@ -251,7 +342,9 @@ __device__ __forceinline__ void load_scales(uint32_t a, uint32_t (&v)[(NGH + 1) 
 
 // G = the group size for the exact-code path (4- and 8-bit); 0 for 6-bit, whose codes are
 // dequantized to RN_fp16(s*q) per element (step_mma) and whose group size is a parameter.
-template <int BITS, int MT, int NCW, int G>
+// XS: x streamed with the codes (p.xstream); a separate instance, so that the staged-x
+// instances carry none of its code.
+template <int BITS, int MT, int NCW, int G, bool XS>
 __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     qmm_stream_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                       const __grid_constant__ CUtensorMap bmap, const StParams p) {
@@ -270,7 +363,8 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ float s_red[NCW];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const StLayout L = st_layout(BITS, MT, p.ring, p.kslice, p.group, p.split, NCW, p.M);
+    static_assert(!XS || (BITS != 6 && MT == 2), "x is streamed for 9-16 tokens at 4 and 8 bits");
+    const StLayout L = st_layout(BITS, MT, p.ring, p.kslice, p.group, p.split, NCW, p.M, XS);
     const int S = p.ring;
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar_full = sbase + L.bar_off;
@@ -279,7 +373,9 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     const uint32_t bar_sempty = bar_sfull + 8 * ST_SS;  // [ST_SS]
     const uint32_t bar_xfull = bar_sempty + 8 * ST_SS;  // [8]: K-half partials written
     const uint32_t bar_xempty = bar_xfull + 8 * 8;      // [8]: ... and read
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bar_off + 8 * (2 * S + 2 * ST_SS + 16));
+    const uint32_t bar_tw = bar_xempty + 8 * 8;         // [2]: a tail piece's partial sums are out
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bar_off + 8 * (2 * S + 2 * ST_SS + 18));
+    float* ysc = const_cast<float*>(reinterpret_cast<volatile float*>(abort_flag + 4));  // 2^E per token
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kb = blockIdx.y * p.kslice;
@@ -302,6 +398,8 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
             mbar_init(bar_xfull + 8 * i, 1);
             mbar_init(bar_xempty + 8 * i, 1);
         }
+        mbar_init(bar_tw, 8);  // the eight row-group warps that hold a tile's sums
+        mbar_init(bar_tw + 8, 8);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -320,7 +418,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     if (warp == NCW) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            if (!p.static_w) grid_dependency_wait();
+            if (!p.static_w || XS) grid_dependency_wait();
             constexpr int BOXW = BITS == 6 ? 48 : 32;          // words per box row
             constexpr int NBOX = BITS == 6 ? 1 : 2;            // boxes per stage
             const int wcol0 = kb / 32 * BITS;  // kb * BITS / 32 (kb is a multiple of 256)
@@ -329,12 +427,14 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
             int s = 0, ss = 0;                 // their ring slots
             uint32_t ph = 0, sph = 0;          // ... and phases
             bool ok = true;
-            for (int t = blockIdx.x; t < p.T && ok; t += gridDim.x) {
-                const long long dl = clock64() + ST_TIMEOUT;
-                int sib = 0, gcol = gcol0, wcol = wcol0;
-                for (int st = 0; st < nst; ++st, ++it) {
+            const StWork wk = st_work(p, nst, spb);
+            for (int k = 0; ok && k < wk.n; ++k) {
+                int t, s0, s1;
+                st_work_item(p, wk, nst, spb, k, t, s0, s1);
+                int sib = 0, gcol = gcol0 + (s0 / spb) * gbb, wcol = wcol0 + s0 * (NBOX * BOXW);
+                for (int st = s0; st < s1; ++st, ++it) {
                     if (sib == 0) {  // scales and biases of the next block of groups
-                        if (blk >= ST_SS && !wait_or_abort(bar_sempty + 8 * ss, sph ^ 1u, dl, abort_flag)) {
+                        if (blk >= ST_SS && !wait_or_abort(bar_sempty + 8 * ss, sph ^ 1u, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -350,15 +450,18 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                         }
                     }
                     if (++sib == spb) sib = 0;
-                    if ((it >= S && !wait_or_abort(bar_empty + 8 * s, ph ^ 1u, dl, abort_flag)) || *abort_flag) {
+                    if ((it >= S && !wait_or_abort(bar_empty + 8 * s, ph ^ 1u, abort_flag)) || *abort_flag) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(bar_full + 8 * s, L.w_stage);
+                    mbar_arrive_expect_tx(bar_full + 8 * s, L.w_stage + L.xtile);
 #pragma unroll
                     for (int b = 0; b < NBOX; ++b)
-                        tma_load_2d(sbase + s * L.w_stage + b * (ST_ROWS * 128), &wmap, bar_full + 8 * s,
+                        tma_load_2d(sbase + s * L.slot + b * (ST_ROWS * 128), &wmap, bar_full + 8 * s,
                                     wcol + b * BOXW, t * ST_ROWS);
+                    if constexpr (XS)
+                        bulk_load(sbase + s * L.slot + L.w_stage, p.xt + size_t(kb / KS + st) * L.xtile, L.xtile,
+                                  bar_full + 8 * s);
                     wcol += NBOX * BOXW;
                     if (++s == S) {
                         s = 0;
@@ -373,7 +476,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
             for (int i = max(0, blk - ST_SS); i < blk; ++i)
                 if (!mbar_wait(bar_sfull + 8 * (i % ST_SS), (i / ST_SS) & 1, dl)) set_error(2u);
         }
-    } else {
+    } else if (warp < NCW) {
         // ------------------------------------------------------------ consumers
         const int g = lane >> 2, c = lane & 3;
         const int hbase = NCW == 16 ? (warp >> 3) : 0;         // first K half this warp takes
@@ -383,22 +486,32 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         const int rA = rg * 16 + (NAT ? g : ((g >> 1) | ((g & 1) << 2)));
         const int rB = rA + 8;
         grid_dependency_wait();
-        const int E = p.is_bf16 ? bf16_exponent<NCW>(p, kb, ke, s_red) : 0;
         const uint32_t xs = sbase + L.x_off, xg = sbase + L.xg_off;
-        stage_x_tile<BITS, MT, NAT>(p.x, p.M, p.K, p.is_bf16, p.group, p.kslice, int(L.gpad), NCW * 32, xs, xg, kb,
-                                    ke, exp2i(-E));
+        float yscale = 1.f;  // 2^E of the staged x (one exponent for the block's tokens)
+        if constexpr (XS) {
+            // the x tiles stream in with the codes; the group sums and exponents come from the
+            // x pass of this call
+            for (int e = threadIdx.x; e < p.M * int(L.gpad); e += NCW * 32)
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(e) * 4u), "r"(__ldg(p.xgw + e)));
+            if (threadIdx.x < 16) ysc[threadIdx.x] = int(threadIdx.x) < p.M ? exp2i(__ldg(p.xexp + threadIdx.x)) : 1.f;
+        } else {
+            const int E = p.is_bf16 ? bf16_exponent<NCW>(p, kb, ke, s_red) : 0;
+            stage_x_tile<BITS, MT, NAT>(p.x, p.M, p.K, p.is_bf16, p.group, p.kslice, int(L.gpad), NCW * 32, xs, xg,
+                                        kb, ke, exp2i(-E));
+            yscale = exp2i(E);
+        }
         consumer_sync<NCW>();
         grid_dependents_launch();
 
         const int tr0 = min(g, p.M - 1), tr1 = min(g + 8, p.M - 1);  // token rows of the two x tiles
         const uint32_t xmt = uint32_t(tr1 - tr0) * L.xrs * 16;
-        // the lane's B fragments: 16-byte chunk c of each 4-chunk block (8 bytes at 8-bit)
-        const uint32_t xlane = xs + uint32_t(tr0 * int(L.xrs)) * 16u + uint32_t(c * (BITS == 8 ? 8 : 16)) +
+        // the lane's B fragments: 16-byte chunk c of each 4-chunk block (8 bytes at 8-bit),
+        // relative to the x of its stage
+        const uint32_t xlane = uint32_t(tr0 * int(L.xrs)) * 16u + uint32_t(c * (BITS == 8 ? 8 : 16)) +
                                uint32_t(hbase * SPH * KSS * 2);
         const uint32_t xgrow = xg + uint32_t(tr0 * int(L.gpad)) * 4u;
         const uint32_t xg_mt = uint32_t(tr1 - tr0) * L.gpad * 4;
         float* xf = reinterpret_cast<float*>(smem + L.xf_off) + (rg * 32 + lane) * 4 * MT;
-        const float yscale = exp2i(E);
         // ring position (slot s, phase ph) and scale-block position (slot ss, phase sph) advance
         // incrementally; no division in the loop
         int s = 0, ss = 0, tc = 0;
@@ -414,10 +527,12 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 #pragma unroll
         for (int sj = 0; sj < SPH; ++sj)
             ldm_off[sj] = uint32_t((rg * 16 + (lane & 7)) * 128 + ((((4 * sj + (lane >> 3)) ^ lane) & 7) << 4));
-        for (int t = blockIdx.x; t < p.T; t += gridDim.x, ++tc) {
+        // One item (tile t, stages [s0, s1)); PARTIAL: a tail piece, which may hand partial
+        // sums to the tail helper.  Whole tiles take a copy of the body without that path.
+        auto run_item = [&](const int t, const int s0, const int s1, const int k, auto partial) {
+            constexpr bool PARTIAL = decltype(partial)::value;
             // After a timeout (abort flag set) every wait below returns at once and the work
             // is skipped, so all warps leave the loop together.
-            const long long dl = clock64() + ST_TIMEOUT;
             float acc[MT][4], tb[MT][4], tmp[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
@@ -425,32 +540,22 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                 for (int i = 0; i < 4; ++i) acc[mt][i] = tb[mt][i] = tmp[mt][i] = 0.f;
             uint32_t sbuf = 0;
             bool sok = true;
-            int sib = 0;             // stage within the scale block
-            uint32_t xblk = xgrow;   // group sums of the current block
-            uint32_t xst = xlane;    // staged x of the current stage
-            for (int st = 0; st < nst; ++st) {
+            int sib = 0;                                                 // stage within the scale block
+            uint32_t xblk = xgrow + uint32_t((s0 / spb) * gbb) * 4u;     // group sums of the current block
+            for (int st = s0; st < s1; ++st) {
+                // x of this stage: in the ring slot (streamed) or in the block's staged K range
+                const uint32_t xst = XS ? sbase + s * L.slot + L.w_stage + xlane : xs + xlane + uint32_t(st * KS * 2);
                 if (sib == 0) {
-                    sok = wait_or_abort(bar_sfull + 8 * ss, sph, dl, abort_flag);
+                    sok = wait_or_abort(bar_sfull + 8 * ss, sph, abort_flag);
                     sbuf = sbase + L.sb_off + ss * L.sb_slot;
                 }
-                const bool ok = sok && wait_or_abort(bar_full + 8 * s, ph, dl, abort_flag);
+                const bool ok = sok && wait_or_abort(bar_full + 8 * s, ph, abort_flag);
                 if constexpr (NAT) {
                   if (ok) {
                     // the lane's code words 4i + c of rows rA and rB for each step of its K
                     // half (halves), by ldmatrix; the ring slot is released once they are in
                     // registers
-                    uint32_t w[HPW * SPH][2][4];
-                    const uint32_t stage = sbase + s * L.w_stage;
-#pragma unroll
-                    for (int hh = 0; hh < HPW; ++hh)
-#pragma unroll
-                        for (int sj = 0; sj < SPH; ++sj) {
-                            const uint32_t a = stage + uint32_t((hbase + hh) * (ST_ROWS * 128)) + ldm_off[sj];
-                            ldsm_x4(a, w[hh * SPH + sj][0]);
-                            ldsm_x4(a + 8 * 128, w[hh * SPH + sj][1]);
-                        }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+                    const uint32_t stage = sbase + s * L.slot;
 #pragma unroll
                     for (int hh = 0; hh < HPW; ++hh) {
                         // scales of the half's groups (a whole number of them: a half is 256
@@ -460,16 +565,31 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                         load_scales<NGH>(sbuf + rAg + g0, fa);
                         load_scales<NGH>(sbuf + rBg + g0, fb);
 #pragma unroll
-                        for (int sj = 0; sj < SPH; ++sj)
-                            step_exact<BITS, MT, BPG, NGH>(w[hh * SPH + sj], sj, xst + uint32_t((hh * SPH + sj) * KSS * 2),
-                                                           xmt, fa, fb, tmp, acc);
+                        for (int sj = 0; sj < SPH; ++sj) {
+                            // the lane's code words 4i + c of rows rA and rB for this step, by
+                            // ldmatrix; the ring slot is released after the stage's last read
+                            uint32_t w[2][4];
+                            const uint32_t a = stage + uint32_t((hbase + hh) * (ST_ROWS * 128)) + ldm_off[sj];
+                            ldsm_x4(a, w[0]);
+                            ldsm_x4(a + 8 * 128, w[1]);
+                            if (hh == HPW - 1 && sj == SPH - 1 && !XS) {
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+                            }
+                            step_exact<BITS, MT, BPG, NGH>(w, sj, xst + uint32_t((hh * SPH + sj) * KSS * 2), xmt, fa, fb,
+                                                           tmp, acc);
+                        }
+                    }
+                    if constexpr (XS) {  // the slot's x tile was read up to the last step
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_empty + 8 * s);
                     }
                   }
                 } else if (ok) {  // 6-bit
                     // the lane's codes of rows rA and rB for the steps of its K half (halves);
                     // the ring slot is released as soon as they are in registers
                     uint32_t w[HPW * SPH][2][NREG];
-                    const uint32_t stage = sbase + s * L.w_stage;
+                    const uint32_t stage = sbase + s * L.slot;
 #pragma unroll
                     for (int hh = 0; hh < HPW; ++hh) {
                         const int half = hbase + hh;
@@ -516,15 +636,30 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                     s = 0;
                     ph ^= 1u;
                 }
-                xst += uint32_t(KS * 2);
                 if (++sib == spb) {
                     if (sok && hbase == 0) {  // bias term of the block's groups: y += b * X
                         const uint32_t bb = sbuf + L.sb_slot / 2;
+                        // exact-code path: into tmp (free between groups) and straight on into
+                        // acc, rescaled to its units; else into tb, added at the end
+                        float (&bt)[MT][4] = NAT ? tmp : tb;
+                        if (NAT) {
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) tmp[mt][i] = 0.f;
+                        }
                         for (int q = 0; q < gbb; q += 8)
                             bias_mma<MT>(lds_u16(bb + rAg + uint32_t(q + c) * 2u), lds_u16(bb + rBg + uint32_t(q + c) * 2u),
                                          lds_u16(bb + rAg + uint32_t(q + c + 4) * 2u),
                                          lds_u16(bb + rBg + uint32_t(q + c + 4) * 2u), xblk + uint32_t(q) * 4u, xg_mt, c,
-                                         tb);
+                                         bt);
+                        if (NAT) {
+                            constexpr float kb2acc = 128.f / exact_code_unscale<BITS>();
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) acc[mt][i] = fmaf(kb2acc, tmp[mt][i], acc[mt][i]);
+                        }
                     }
                     __syncwarp();
                     if (sok && lane == 0) mbar_arrive(bar_sempty + 8 * ss);
@@ -542,7 +677,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
             if constexpr (NCW == 16) {
                 own = false;
                 if (hbase == 1) {
-                    if (tc == 0 || wait_or_abort(bar_xempty + 8 * rg, ((tc - 1) & 1), dl, abort_flag)) {
+                    if (tc == 0 || wait_or_abort(bar_xempty + 8 * rg, ((tc - 1) & 1), abort_flag)) {
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -550,7 +685,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar_xfull + 8 * rg);
                     }
-                } else if (wait_or_abort(bar_xfull + 8 * rg, tc & 1, dl, abort_flag)) {
+                } else if (wait_or_abort(bar_xfull + 8 * rg, tc & 1, abort_flag)) {
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -564,9 +699,11 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        acc[mt][i] = ((NAT ? exact_code_unscale<BITS>() : 1.f) * acc[mt][i] + 128.f * tb[mt][i]) * yscale;
-                if (p.split == 1) {
+                    for (int i = 0; i < 4; ++i) {
+                        const float ys = XS ? ysc[8 * mt + 2 * c + (i & 1)] : yscale;
+                        acc[mt][i] = NAT ? exact_code_unscale<BITS>() * acc[mt][i] * ys : (acc[mt][i] + 128.f * tb[mt][i]) * ys;
+                    }
+                if (p.split == 1 && (!PARTIAL || s1 - s0 == nst)) {
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -578,6 +715,21 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                                                                 ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][i]))
                                                                 : __half_as_ushort(__float2half_rn(acc[mt][i]));
                         }
+                } else if (PARTIAL && p.split == 1) {
+                    // a piece of a tail tile (item k = 0 or 1: the tail comes first): its
+                    // partial sums go to this block's slot and the tail helper takes over
+                    float* part = p.partials +
+                                  size_t(st_slot(p, nst / spb, int(blockIdx.x), t - p.dp_tiles)) * (8 * MT * ST_ROWS);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int m = 8 * mt + 2 * c + (i & 1);
+                            if (m < p.M) part[m * ST_ROWS + (i < 2 ? rA : rB)] = acc[mt][i];
+                        }
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_tw + 8 * k);
                 } else {
                     // one tile per block when K is split: each partial goes straight into the
                     // shared memory of the block that sums its row (rows dealt out evenly over
@@ -601,6 +753,85 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                                 st_cluster_f32(red_la + uint32_t(((int(me) * 8 * MT + col) * rows_per + rl) * 4),
                                                uint32_t(owner), acc[mt][i]);
                         }
+                }
+            }
+                };
+        const StWork wk = st_work(p, nst, spb);
+        for (int k = 0; k < wk.np; ++k, ++tc) {
+            int t, s0, s1;
+            st_item(p, nst, spb, k, t, s0, s1);
+            run_item(t, s0, s1, k, std::true_type{});
+        }
+        for (int t = blockIdx.x; t < p.dp_tiles; t += gridDim.x, ++tc) run_item(t, 0, nst, 0, std::false_type{});
+
+    }
+    if (warp == NCW + 1 && p.split == 1 && p.tper > 0) {
+        // ------------------------------------------------------------ tail helper
+        // For each tail piece of this block (its first items): once the row-group warps have
+        // written and fenced its partial sums, count the block's arrival on the tile; the
+        // tile's last block to arrive adds the partial sums of the tile's blocks cf..cl in
+        // that order and writes y (the result does not depend on timing).  This warp does it
+        // while the consumers go on with their whole tiles, so none of its memory round trips
+        // (or the contention of the blocks arriving together) lands on the critical path.
+        const int nsb = nst / spb;
+        for (int k2 = 0; k2 < 2; ++k2) {
+            int t2, a2, b2;
+            if (!st_item(p, nst, spb, k2, t2, a2, b2) || t2 < p.dp_tiles) break;
+            if (b2 - a2 == nst) continue;  // a whole tile: written by the consumers
+            const int ti = t2 - p.dp_tiles;
+            const int cf = (ti * nsb) / p.tper, P = ((ti + 1) * nsb - 1) / p.tper - cf + 1;
+            int last = 0;
+            if (lane == 0 && wait_or_abort(bar_tw + 8 * k2, 0, abort_flag)) {
+                // arrival word: (call tag << 16) | arrivals; a word with another tag (left by
+                // an earlier call) counts as none
+                unsigned long long* word = p.counters + ti;
+                unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(word);
+                for (int it2 = 0; it2 < 256; ++it2) {
+                    const unsigned long long cnt = old & 0xFFFFull;
+                    const bool mine = (old >> 16) == p.token && cnt < unsigned(P);
+                    const unsigned long long nw = mine ? old + 1 : ((p.token << 16) | 1ull);
+                    const unsigned long long prev = atomicCAS(word, old, nw);
+                    if (prev == old) {
+                        last = int(nw & 0xFFFFull) == P;
+                        break;
+                    }
+                    old = prev;
+                }
+                if (last) atomicExch(word, 0ull);  // ready for the next call that uses it
+            }
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (!last) continue;
+            __threadfence();
+            // four rows a lane (16-byte loads), eight blocks' partial sums in flight at a time
+            const int ncols = min(8 * MT, p.M);
+            for (int u = lane; u < ncols * (ST_ROWS / 4); u += 32) {
+                const int col = u / (ST_ROWS / 4), r4 = (u - col * (ST_ROWS / 4)) * 4;
+                const float* src = p.partials + col * ST_ROWS + r4;
+                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                int q = 0;
+                for (; q + 8 <= P; q += 8) {
+                    float4 v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        v[j] = __ldcg(reinterpret_cast<const float4*>(
+                            src + size_t(st_slot(p, nsb, cf + q + j, ti)) * (8 * MT * ST_ROWS)));
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        sum.x += v[j].x; sum.y += v[j].y; sum.z += v[j].z; sum.w += v[j].w;
+                    }
+                }
+                for (; q < P; ++q) {
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                        src + size_t(st_slot(p, nsb, cf + q, ti)) * (8 * MT * ST_ROWS)));
+                    sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+                }
+                const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int n = t2 * ST_ROWS + r4 + i;
+                    if (n < p.N)
+                        p.y[int64_t(col) * p.N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sv[i]))
+                                                                : __half_as_ushort(__float2half_rn(sv[i]));
                 }
             }
         }
@@ -634,26 +865,115 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     }
 }
 
+// ---------------------------------------------------------------- x pass (streamed x)
+// One block per token row: the row's fp16 x tiles of every stage ([stage][16 rows][xrs
+// chunks]; each 8-code unit at its natural chunk, its codes in perm_nat order), its group
+// sums as (hi, lo) fp16 times 2^-7 ([row][gpad], zero past the last group) and its exponent:
+// bf16 rows are scaled by 2^-E with max|x| * 2^-E < 2^15 (E >= 0), fp16 rows are not.
+template <int BITS>
+__global__ void __launch_bounds__(256) st_xprep_kernel(const uint16_t* __restrict__ x, int K, int is_bf16, int group,
+                                                       int xrs, int gpad, uint8_t* __restrict__ xt,
+                                                       uint32_t* __restrict__ xgw, int* __restrict__ xexp) {
+    constexpr int CPS = (BITS == 4 ? 512 : 256) / 8;  // 16-byte chunks (8-code units) per stage
+    __shared__ float red[8];
+    grid_dependents_launch();
+    grid_dependency_wait();
+    const int m = blockIdx.x;
+    const uint16_t* xr = x + int64_t(m) * K;
+    int E = 0;
+    if (is_bf16) {
+        float amax = 0.f;
+        for (int k = threadIdx.x * 8; k < K; k += 256 * 8) {
+            const uint4 v = ldg_nc_v4(xr + k);
+            const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                amax = fmaxf(amax, fmaxf(fabsf(bf16lo_to_f32(r[i])), fabsf(bf16hi_to_f32(r[i]))));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+        __syncthreads();
+        float a = red[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
+        const int eb = int(__float_as_uint(a) >> 23) & 0xFF;  // a < 2^(eb-126)
+        E = eb > 141 ? eb - 141 : 0;
+    }
+    const float sc = exp2i(-E);
+    const int units = K / 8, upg = group / 8;
+    const int totp = (units + 31) & ~31;  // whole warps take part in the shuffles
+    for (int u = threadIdx.x; u < totp; u += 256) {
+        const bool valid = u < units;
+        float f[8];
+        if (valid) {
+            const uint4 v = ldg_nc_v4(xr + 8 * u);
+            const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (is_bf16) {
+                    f[2 * i] = bf16lo_to_f32(r[i]) * sc;
+                    f[2 * i + 1] = bf16hi_to_f32(r[i]) * sc;
+                } else {
+                    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
+                    f[2 * i] = t.x;
+                    f[2 * i + 1] = t.y;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = 0.f;
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum += f[i];
+        for (int o = 1; o < upg; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (!valid) continue;
+        if (u % upg == 0) {
+            const float X = sum * 0.0078125f;
+            const __half hi = __float2half_rn(X);
+            const __half lo = __float2half_rn(X - __half2float(hi));
+            xgw[m * gpad + u / upg] = uint32_t(__half_as_ushort(hi)) | (uint32_t(__half_as_ushort(lo)) << 16);
+        }
+        uint4 o;
+        uint32_t* ov = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ov[i] = f32x2_to_f16x2(f[perm_nat<BITS>(2 * i)], f[perm_nat<BITS>(2 * i + 1)]);
+        const int st = u / CPS, ch = u - st * CPS;
+        *reinterpret_cast<uint4*>(xt + ((size_t(st) * 16 + m) * xrs + ch) * 16) = o;
+    }
+    for (int gi = K / group + int(threadIdx.x); gi < gpad; gi += 256) xgw[m * gpad + gi] = 0u;
+    if (threadIdx.x == 0) xexp[m] = E;
+}
+
 using StKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const StParams);
 
-template <int BITS, int MT>
+template <int BITS, int MT, bool XS>
 StKernelFn pick_stream_g(int group) {
     if constexpr (BITS == 6) {
-        return qmm_stream_kernel<6, MT, 16, 0>;
+        return XS ? nullptr : qmm_stream_kernel<6, MT, 16, 0, false>;
+    } else if constexpr (XS && MT != 2) {
+        return nullptr;
     } else {
-        if (group == 32) return qmm_stream_kernel<BITS, MT, 16, 32>;
-        if (group == 64) return qmm_stream_kernel<BITS, MT, 16, 64>;
-        if (group == 128) return qmm_stream_kernel<BITS, MT, 16, 128>;
+        if (group == 32) return qmm_stream_kernel<BITS, MT, 16, 32, XS>;
+        if (group == 64) return qmm_stream_kernel<BITS, MT, 16, 64, XS>;
+        if (group == 128) return qmm_stream_kernel<BITS, MT, 16, 128, XS>;
         return nullptr;
     }
 }
 // 16 consumer warps (the 8-warp form of the kernel is not instantiated: it measured slower on
 // every configuration of the sweep)
-StKernelFn pick_stream(int bits, int mt, int ncw, int group) {
+StKernelFn pick_stream(int bits, int mt, int ncw, int group, bool xs) {
     if (ncw != 16 || (mt != 1 && mt != 2)) return nullptr;
-    if (bits == 4) return mt == 1 ? pick_stream_g<4, 1>(group) : pick_stream_g<4, 2>(group);
-    if (bits == 6) return mt == 1 ? pick_stream_g<6, 1>(group) : pick_stream_g<6, 2>(group);
-    if (bits == 8) return mt == 1 ? pick_stream_g<8, 1>(group) : pick_stream_g<8, 2>(group);
+    if (xs) {
+        if (mt != 2) return nullptr;
+        if (bits == 4) return pick_stream_g<4, 2, true>(group);
+        if (bits == 8) return pick_stream_g<8, 2, true>(group);
+        return nullptr;
+    }
+    if (bits == 4) return mt == 1 ? pick_stream_g<4, 1, false>(group) : pick_stream_g<4, 2, false>(group);
+    if (bits == 6) return mt == 1 ? pick_stream_g<6, 1, false>(group) : pick_stream_g<6, 2, false>(group);
+    if (bits == 8) return mt == 1 ? pick_stream_g<8, 1, false>(group) : pick_stream_g<8, 2, false>(group);
     return nullptr;
 }
 
@@ -668,10 +988,9 @@ int rup(int64_t a, int64_t b) { return int((a + b - 1) / b * b); }
 
 constexpr int kNumSM = 148;
 constexpr size_t kMaxSmem = 226 * 1024;  // dynamic, per block (static shared memory is tiny)
-constexpr size_t kSmSmem = 228 * 1024;   // per SM (including 1 KB reserved per block)
 
-size_t st_smem(int bits, int mt, int ring, int kslice, int group, int split, int ncw, int mrows) {
-    return size_t(st_layout(bits, mt, ring, kslice, group, split, ncw, mrows).total) + 1024;  // + alignment slack
+size_t st_smem(int bits, int mt, int ring, int kslice, int group, int split, int ncw, int mrows, bool xs) {
+    return size_t(st_layout(bits, mt, ring, kslice, group, split, ncw, mrows, xs).total) + 1024;  // + alignment slack
 }
 
 }  // namespace
@@ -709,6 +1028,9 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
     }
     split = std::max(1, std::min(8, split));
     const int split0 = split;
+    // 9-16 tokens on a persistent grid: x for the whole K range would take most of shared
+    // memory (64 KB per 2048 codes), so it streams with the codes instead (4- and 8-bit)
+    const bool xs_want = bits != 6 && M > 8 && split == 1 && T >= kNumSM;
     for (;; ++split) {
         const int kslice = rup(cdiv(K, split), unit);
         const int sp = cdiv(K, kslice);
@@ -720,8 +1042,9 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         // 16 consumer warps measured faster than 8 on every configuration of the sweep (the
         // 8-warp blocks fit two to an SM, but that bought no overlap between calls)
         const int ncw = 16;
-        while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M)) > kMaxSmem) --ring;
-        const bool fits = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M)) <= kMaxSmem;
+        const bool xs = xs_want && sp == 1;
+        while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M), xs) > kMaxSmem) --ring;
+        const bool fits = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M), xs) <= kMaxSmem;
         if (!fits || (ring < std::min(want, 3) && split < 8)) {
             if (split < 8) continue;
             c.ring = 0;  // does not fit: the caller uses another kernel
@@ -734,9 +1057,22 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         c.stage_bytes = ST_ROWS * KS * bits / 8;
         c.split_raised = split > split0;
         c.ncw = ncw;
-        c.smem = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M));
-        const int per_sm = std::max(1, int(kSmSmem / (c.smem + 1024)));
-        c.grid_x = sp > 1 ? T : std::min(T, kNumSM * per_sm);
+        c.smem = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M), xs);
+        c.xstream = xs;
+        // one block per SM: 17 warps at up to 96 registers leave no room for a second
+        c.grid_x = sp > 1 ? T : std::min(T, kNumSM);
+        c.dp_tiles = T;
+        c.tunits = c.tper = 0;
+        if (sp == 1 && T > c.grid_x && T % c.grid_x) {
+            // the last, partial wave of tiles would leave most SMs idle: deal its scale blocks
+            // out evenly instead (a block's run then spans at most two tiles, since the tail
+            // has fewer tiles than the grid has blocks)
+            const int G = c.grid_x;
+            c.dp_tiles = T / G * G;
+            const int nsb = nst / (st_block_codes(bits, group) / KS);
+            c.tunits = (T - c.dp_tiles) * nsb;
+            c.tper = cdiv(c.tunits, G);
+        }
         return c;
     }
 }
@@ -816,7 +1152,7 @@ cudaError_t ensure_smem_attr(StKernelFn fn, size_t smem) {
 
 cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream) {
     const int mt = int(a.M) > 8 ? 2 : 1;
-    StKernelFn fn = pick_stream(a.bits, mt, c.ncw, a.group);
+    StKernelFn fn = pick_stream(a.bits, mt, c.ncw, a.group, c.xstream);
     if (!fn || c.ring < 2) return cudaErrorNotSupported;
     // The three descriptors depend only on the weight arrays and the format; a call that
     // repeats them (the usual case: the same weights every step) reuses the encoded copies.
@@ -837,12 +1173,45 @@ cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t 
     p.split = c.split;
     p.ring = c.ring;
     p.static_w = c.static_weights ? 1 : 0;
+    p.dp_tiles = c.dp_tiles;
+    p.tunits = c.tunits;
+    p.tper = c.tper;
+    p.partials = nullptr;
+    p.counters = nullptr;
+    p.token = 0;
+    p.xstream = c.xstream ? 1 : 0;
+    p.xt = nullptr;
+    p.xgw = nullptr;
+    p.xexp = nullptr;
+    const StLayout L = st_layout(a.bits, mt, c.ring, c.kslice, a.group, c.split, c.ncw, int(a.M), c.xstream);
+    if (c.tper > 0 || c.xstream) {
+        // workspace: tail arrival words [T - dp_tiles], tail partial sums [2 * grid][8 * mt][128];
+        // streamed x: tiles [stages][16][xrs chunks], group sums [M][gpad], exponents [M]
+        const size_t cbytes = c.tper > 0 ? (size_t(p.T - c.dp_tiles) * 8 + 255) / 256 * 256 : 0;
+        const size_t pbytes = c.tper > 0 ? size_t(2 * c.grid_x) * 8 * mt * ST_ROWS * 4 : 0;
+        const size_t xtbytes = c.xstream ? size_t(a.K / ks_for(a.bits)) * L.xtile : 0;
+        const size_t xgbytes = c.xstream ? (size_t(a.M) * L.gpad * 4 + 255) / 256 * 256 : 0;
+        void* ws = nullptr;
+        cudaError_t e = split_workspace(stream, cbytes + pbytes + xtbytes + xgbytes + (c.xstream ? 256 : 0), &ws);
+        if (e != cudaSuccess) return e;
+        uint8_t* w = static_cast<uint8_t*>(ws);
+        if (c.tper > 0) {
+            p.counters = reinterpret_cast<unsigned long long*>(w);
+            p.partials = reinterpret_cast<float*>(w + cbytes);
+            p.token = next_call_token();
+        }
+        if (c.xstream) {
+            p.xt = w + cbytes + pbytes;
+            p.xgw = reinterpret_cast<const uint32_t*>(w + cbytes + pbytes + xtbytes);
+            p.xexp = reinterpret_cast<const int*>(w + cbytes + pbytes + xtbytes + xgbytes);
+        }
+    }
 
     cudaError_t e = ensure_smem_attr(fn, c.smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(c.grid_x), unsigned(c.split), 1);
-    cfg.blockDim = dim3(unsigned((c.ncw + 1) * 32), 1, 1);
+    cfg.blockDim = dim3(unsigned((c.ncw + 2) * 32), 1, 1);
     cfg.dynamicSmemBytes = c.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attrs[2];
@@ -861,6 +1230,26 @@ cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t 
     }
     cfg.attrs = attrs;
     cfg.numAttrs = unsigned(na);
+    if (c.xstream) {
+        // the x pass first (one block per token row); the main kernel waits for it
+        cudaLaunchConfig_t xc = {};
+        xc.gridDim = dim3(unsigned(a.M), 1, 1);
+        xc.blockDim = dim3(256, 1, 1);
+        xc.stream = stream;
+        cudaLaunchAttribute xa[1];
+        xa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        xa[0].val.programmaticStreamSerializationAllowed = 1;
+        xc.attrs = xa;
+        xc.numAttrs = c.pdl ? 1u : 0u;
+        uint8_t* xt = const_cast<uint8_t*>(p.xt);
+        uint32_t* xgw = const_cast<uint32_t*>(p.xgw);
+        int* xexp = const_cast<int*>(p.xexp);
+        e = a.bits == 4 ? cudaLaunchKernelEx(&xc, st_xprep_kernel<4>, a.x, int(a.K), a.is_bf16, a.group, int(L.xrs),
+                                             int(L.gpad), xt, xgw, xexp)
+                        : cudaLaunchKernelEx(&xc, st_xprep_kernel<8>, a.x, int(a.K), a.is_bf16, a.group, int(L.xrs),
+                                             int(L.gpad), xt, xgw, xexp);
+        if (e != cudaSuccess) return e;
+    }
     return cudaLaunchKernelEx(&cfg, fn, maps->w, maps->s, maps->b, p);
 }
 

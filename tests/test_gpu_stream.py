@@ -117,3 +117,77 @@ def test_deterministic_bitwise():
     y2 = q.qmm(x, P, S, B, 4, 64, plan=plan)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("N,K,bits,group,M,dtype", [
+    (31744, 2048, 4, 32, 1, torch.float16),   # 248 tiles: runs of 3 scale blocks over 4-block tiles
+    (19328, 4096, 4, 64, 5, torch.bfloat16),  # 151 tiles: a 3-tile tail, one scale block a block
+    (20000, 4096, 8, 128, 13, torch.bfloat16),  # ragged last tile inside the tail
+    (19100, 2048, 6, 64, 9, torch.float16),   # 150 tiles at 6 bits
+    (18960, 1024, 8, 32, 16, torch.float16),  # 149 tiles, one 8-bit stage a scale block
+])
+def test_tail_tiles(oracle_mod, N, K, bits, group, M, dtype):
+    """Persistent grids whose tile count is not a multiple of the grid: the last partial wave
+    is dealt out by scale blocks and each tail tile's partial sums are added by its last
+    block to finish."""
+    pd = q.plan_default(M, N, K, bits, group, dtype)
+    assert pd.kernel == q.KERNEL_STREAM and pd.split == 1
+    _run(oracle_mod, M, N, K, bits, group, dtype, 1.0 if dtype == torch.float16 else 0.02)
+
+
+def test_tail_tiles_repeatable_back_to_back_and_in_a_graph():
+    """The arrival words of the tail tiles are reset by each tile's last block and tagged per
+    call: calls issued back to back without a host sync, and replays of a captured graph,
+    give the same bits."""
+    M, N, K = 3, 19328, 4096
+    w = w_input(N, K, torch.float16, 7).cuda()
+    P, S, B = q.quantize(w, 4, 64)
+    xs = [x_input(M, K, torch.float16, seed=s).cuda() for s in range(3)]
+    ref = [q.qmm(x, P, S, B, 4, 64) for x in xs]
+    torch.cuda.synchronize()
+    outs = [q.qmm(xs[i % 3], P, S, B, 4, 64) for i in range(9)]
+    torch.cuda.synchronize()
+    for i, y in enumerate(outs):
+        assert torch.equal(y.view(torch.int16), ref[i % 3].view(torch.int16)), i
+    ys = [torch.empty_like(r) for r in ref]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(3):
+            q.qmm(xs[i], P, S, B, 4, 64, out=ys[i])
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(3):
+            q.qmm(xs[i], P, S, B, 4, 64, out=ys[i])
+    for _ in range(2):
+        for y in ys:
+            y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for i in range(3):
+            assert torch.equal(ys[i].view(torch.int16), ref[i].view(torch.int16)), i
+    assert q.device_errors() == 0
+
+
+@pytest.mark.parametrize("M", [9, 12, 16])
+@pytest.mark.parametrize("bits,group", [(4, 32), (4, 128), (8, 64)])
+def test_streamed_x(oracle_mod, M, bits, group):
+    """9-16 tokens on a persistent grid take x through the ring, one tile per stage written by
+    a separate x pass with a per-token exponent: rows of very different magnitudes (bf16)
+    each keep their precision."""
+    N, K = 19200, 3072  # 150 tiles: a persistent grid with a tail
+    x = randn((M, K), 1.0, torch.bfloat16, 11)
+    x[0] *= 3.0e5
+    x[M - 1] *= 1e-3
+    _run(oracle_mod, M, N, K, bits, group, torch.bfloat16, 0.02, x=x)
+    # each row on its own, against the oracle (a row's scale must not leak into another's)
+    w = w_input(N, K, torch.bfloat16, 0, 0.02)
+    op, os_, ob = oracle_quantize(oracle_mod, w, bits, group)
+    P, S, B = to_device_weights(op, os_, ob)
+    y = q.qmm(x.cuda(), P, S, B, bits, group, plan=q.make_plan(kernel=q.KERNEL_STREAM))
+    torch.cuda.synchronize()
+    ref = oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group)
+    for m in range(M):
+        check_close(y[m:m + 1], ref[m:m + 1], torch.bfloat16, f"streamed x, row {m}")
