@@ -124,10 +124,11 @@ def test_plans(L):
         assert p.kernel == q.KERNEL_STREAM and 1 <= p.split <= 8
     assert q.plan_default(4, 151936, 4096, 4, 64, f16).split == 1  # enough tiles: no split
     assert q.plan_default(17, 4096, 4096, 4, 64, f16).kernel != q.KERNEL_STREAM
-    # LM head (unsplit grid): x of up to 13 rows leaves a 3-stage ring, 14 does not
+    # LM head (persistent grid): 9-16 tokens stream x through the ring with the codes, so the
+    # streaming kernel keeps its ring at any M <= 16
     bf16 = __import__("torch").bfloat16
-    assert q.plan_default(13, 151936, 4096, 4, 64, bf16).kernel == q.KERNEL_STREAM
-    assert q.plan_default(14, 151936, 4096, 4, 64, bf16).kernel != q.KERNEL_STREAM
+    for M in (13, 14, 16):
+        assert q.plan_default(M, 151936, 4096, 4, 64, bf16).kernel == q.KERNEL_STREAM
     # 6-bit stages are smaller (24 KB): 4 of them are needed, so 6-bit gate/up leaves at M = 13
     assert q.plan_default(12, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_STREAM
     assert q.plan_default(13, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_TC
