@@ -119,10 +119,10 @@ qmm_status validate_qmm(const void* x, const uint32_t* packed, const uint16_t* s
 // whole number of its stages and scale blocks); above that the tensor-core kernel for wide N
 // and for large weight matrices, and the warp-tile kernel on the 4096-wide and narrower
 // projections up to M = 32.
-bool prefer_tc(int64_t M, int64_t N, int64_t K) {
+bool prefer_tc(int64_t M, int64_t N, int64_t K, int bits) {
     if (N >= 8192 && N * K <= (int64_t(1) << 27)) return true;  // gate/up-like: wide N, moderate size
     if (N * K >= (int64_t(1) << 25)) return M >= 9;             // >= 32M codes (down, LM head)
-    if (N * K < (int64_t(1) << 23)) return M >= 24;             // k/v-like: < 8M codes
+    if (N * K < (int64_t(1) << 23)) return M >= (bits == 8 ? 17 : 24);  // k/v-like: < 8M codes
     return M >= 28;  // q/o-like: the tensor-core kernel's time is flat over M = 17..32 (one
                      // 32-column tile) while the warp-tile kernel's grows; they cross near 28
 }
@@ -204,9 +204,12 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
         // to back, 96 KB in flight suffice (3 stages of 4- or 8-bit codes, 4 of 6-bit)
         const int ring_need =
             (st_ok && stc.split == 1) ? (96 * 1024 + stc.stage_bytes - 1) / std::max(1, stc.stage_bytes) : 4;
-        if (st_ok && (M <= 8 || (!stc.split_raised && stc.ring >= std::min(ring_need, stc.stages))))
+        // 6-bit codes are dequantized per element in the streaming kernel; with two token tiles
+        // that loses to the tensor-core kernel on the large matrices (measured)
+        const bool st_mt2_ok = !(bits == 6 && N * K >= (int64_t(1) << 25));
+        if (st_ok && (M <= 8 || (st_mt2_ok && !stc.split_raised && stc.ring >= std::min(ring_need, stc.stages))))
             p.kernel = QMM_KERNEL_STREAM;
-        else p.kernel = (tc_ok && prefer_tc(M, N, K)) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
+        else p.kernel = (tc_ok && prefer_tc(M, N, K, bits)) ? QMM_KERNEL_TC : QMM_KERNEL_MMA;
     }
     if (p.kernel == QMM_KERNEL_STREAM && !st_ok)
         return fail(QMM_ERR_UNSUPPORTED,

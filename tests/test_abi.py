@@ -129,9 +129,14 @@ def test_plans(L):
     bf16 = __import__("torch").bfloat16
     for M in (13, 14, 16):
         assert q.plan_default(M, 151936, 4096, 4, 64, bf16).kernel == q.KERNEL_STREAM
-    # 6-bit stages are smaller (24 KB): 4 of them are needed, so 6-bit gate/up leaves at M = 13
-    assert q.plan_default(12, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_STREAM
-    assert q.plan_default(13, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_TC
+    # 6-bit codes on the large matrices leave the streaming kernel above 8 tokens (one token
+    # tile); the small k/v ones keep it up to 16
+    assert q.plan_default(8, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_STREAM
+    assert q.plan_default(9, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_TC
+    assert q.plan_default(16, 1024, 4096, 6, 32, bf16).kernel == q.KERNEL_STREAM
+    # k/v size above 16 tokens: the tensor-core kernel at 8 bits, the warp-tile kernel at 6
+    assert q.plan_default(17, 1024, 4096, 8, 128, bf16).kernel == q.KERNEL_TC
+    assert q.plan_default(17, 1024, 4096, 6, 32, bf16).kernel == q.KERNEL_MMA
     # q/o size: the warp-tile kernel up to M = 27, the tensor-core kernel from 28
     assert q.plan_default(27, 4096, 4096, 4, 64, f16).kernel == q.KERNEL_MMA
     assert q.plan_default(28, 4096, 4096, 4, 64, f16).kernel == q.KERNEL_TC

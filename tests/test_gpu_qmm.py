@@ -210,6 +210,21 @@ FULL = [("qo", m) for m in WORKLOADS["qo"].Ms] + [("down", m) for m in WORKLOADS
        [("lmhead", m) for m in WORKLOADS["lmhead"].Ms]
 
 
+def _boundaries(name):
+    """The M on either side of each change of kernel in the default plan (M = 1..64), and
+    8/9 and 16/17, where the streaming kernel goes to two token tiles and runs out."""
+    wl = WORKLOADS[name]
+    ks = [q.plan_default(m, wl.N, wl.K, wl.bits, wl.group, wl.dtype).kernel for m in range(1, 66)]
+    out = {8, 9, 16, 17}
+    for i in range(64):
+        if ks[i] != ks[i + 1]:
+            out |= {i + 1, i + 2}
+    return sorted(m for m in out if m <= 64)
+
+
+FULL += [(n, m) for n in WORKLOADS for m in _boundaries(n) if (n, m) not in FULL]
+
+
 _FULL_CACHE = {}
 
 
@@ -224,8 +239,9 @@ def _full_weights(name):
 
 @pytest.mark.parametrize("name,M", FULL)
 def test_full_size_sampled(oracle_mod, name, M):
-    """Every configuration at full size, launched as the bench launches it; the oracle checks
-    256-row samples of the output (first, middle and last rows)."""
+    """Every configuration at full size, launched as the bench launches it, at the bench's M
+    and on both sides of every dispatch boundary; the oracle checks 256-row samples of the
+    output (first, middle and last rows)."""
     wl = WORKLOADS[name]
     N, K = wl.N, wl.K
     x = x_input(M, K, wl.dtype)
