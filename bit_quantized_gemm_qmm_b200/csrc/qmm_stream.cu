@@ -75,6 +75,41 @@ __host__ __device__ inline int st_block_codes(int bits, int group) {
     return a > b ? a : b;
 }
 
+struct StLayout {
+    uint32_t w_stage, slot, xtile, sb_off, sb_slot, x_off, xrs, xg_off, gpad, xf_off, red_off, bar_off, total;
+};
+
+// x and its group sums are staged for the M real token rows only (reads for token rows >= M
+// are redirected to row M-1: they feed accumulator columns that are never stored).
+// xs (x streamed): instead of x for the whole K range, each ring slot carries, after the
+// stage's codes, that stage's x tile [16 token rows][xrs chunks] (written once per call by
+// st_xprep_kernel and brought in by the same barrier as the codes).
+__host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split, int ncw,
+                                              int mrows, bool xs = false) {
+    StLayout L;
+    L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 256));  // 24 or 32 KB
+    L.xrs = uint32_t((xs ? st_stage_codes(bits) : kslice) / 8 + x_pad(bits, bits != 6));  // chunks per x row
+    L.xtile = xs ? 16u * L.xrs * 16u : 0u;
+    L.slot = (L.w_stage + L.xtile + 1023) / 1024 * 1024;      // codes stay 1024-byte aligned (swizzle)
+    L.sb_off = uint32_t(ring) * L.slot;
+    L.sb_slot = uint32_t(2 * ST_ROWS * (st_block_codes(bits, group) / group) * 2);  // scales + biases
+    uint32_t off = L.sb_off + ST_SS * L.sb_slot;
+    L.x_off = off;
+    if (!xs) off += uint32_t(mrows) * L.xrs * 16;
+    L.xg_off = off;
+    L.gpad = uint32_t((kslice / group + 7) / 8 * 8);
+    off += uint32_t(mrows) * L.gpad * 4;
+    L.xf_off = off;                                           // K-half partials: [8 warps][32][4*MT]
+    if (ncw == 16) off += uint32_t(8 * 32 * 4 * mt * 4);
+    L.red_off = off;
+    if (split > 1) off += uint32_t(split * ((ST_ROWS + split - 1) / split) * 8 * mt * 4);
+    off = (off + 15) & ~15u;
+    L.bar_off = off;
+    off += 8 * uint32_t(2 * ring + 2 * ST_SS + 18) + 16 + 64;  // + abort word; 2^E of 16 tokens
+    L.total = off;
+    return L;
+}
+
 struct StParams {
     const uint16_t* x;
     uint16_t* y;
@@ -100,6 +135,9 @@ struct StParams {
     const uint8_t* xt;
     const uint32_t* xgw;
     const int* xexp;
+    // the shared-memory layout, worked out on the host: in the kernel its fields are read
+    // from the parameter bank where used instead of living in registers
+    StLayout lay;
 };
 
 // This block's work as a list of items (tile t, stages [s0, s1)): first its run of tail scale
@@ -169,41 +207,6 @@ __device__ __forceinline__ void st_work_item(const StParams& p, const StWork& w,
 // Partial-sum slot of tail tile t (index ti past dp_tiles) from block c.
 __device__ __forceinline__ int st_slot(const StParams& p, int nsb, int c, int ti) {
     return 2 * c + ((c * p.tper) / nsb == ti ? 0 : 1);
-}
-
-struct StLayout {
-    uint32_t w_stage, slot, xtile, sb_off, sb_slot, x_off, xrs, xg_off, gpad, xf_off, red_off, bar_off, total;
-};
-
-// x and its group sums are staged for the M real token rows only (reads for token rows >= M
-// are redirected to row M-1: they feed accumulator columns that are never stored).
-// xs (x streamed): instead of x for the whole K range, each ring slot carries, after the
-// stage's codes, that stage's x tile [16 token rows][xrs chunks] (written once per call by
-// st_xprep_kernel and brought in by the same barrier as the codes).
-__host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split, int ncw,
-                                              int mrows, bool xs = false) {
-    StLayout L;
-    L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 256));  // 24 or 32 KB
-    L.xrs = uint32_t((xs ? st_stage_codes(bits) : kslice) / 8 + x_pad(bits, bits != 6));  // chunks per x row
-    L.xtile = xs ? 16u * L.xrs * 16u : 0u;
-    L.slot = (L.w_stage + L.xtile + 1023) / 1024 * 1024;      // codes stay 1024-byte aligned (swizzle)
-    L.sb_off = uint32_t(ring) * L.slot;
-    L.sb_slot = uint32_t(2 * ST_ROWS * (st_block_codes(bits, group) / group) * 2);  // scales + biases
-    uint32_t off = L.sb_off + ST_SS * L.sb_slot;
-    L.x_off = off;
-    if (!xs) off += uint32_t(mrows) * L.xrs * 16;
-    L.xg_off = off;
-    L.gpad = uint32_t((kslice / group + 7) / 8 * 8);
-    off += uint32_t(mrows) * L.gpad * 4;
-    L.xf_off = off;                                           // K-half partials: [8 warps][32][4*MT]
-    if (ncw == 16) off += uint32_t(8 * 32 * 4 * mt * 4);
-    L.red_off = off;
-    if (split > 1) off += uint32_t(split * ((ST_ROWS + split - 1) / split) * 8 * mt * 4);
-    off = (off + 15) & ~15u;
-    L.bar_off = off;
-    off += 8 * uint32_t(2 * ring + 2 * ST_SS + 18) + 16 + 64;  // + abort word; 2^E of 16 tokens
-    L.total = off;
-    return L;
 }
 
 __device__ __forceinline__ void set_error(unsigned bit) { atomicOr(&g_stream_error, bit); }
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     __shared__ float s_red[NCW];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     static_assert(!XS || (BITS != 6 && MT == 2), "x is streamed for 9-16 tokens at 4 and 8 bits");
-    const StLayout L = st_layout(BITS, MT, p.ring, p.kslice, p.group, p.split, NCW, p.M, XS);
+    const StLayout& L = p.lay;
     const int S = p.ring;
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar_full = sbase + L.bar_off;
@@ -381,9 +384,11 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     const int kb = blockIdx.y * p.kslice;
     const int ke = min(p.K, kb + p.kslice);
     const int nst = (ke - kb + KS - 1) / KS;
-    const int blkc = st_block_codes(BITS, p.group);
-    const int gbb = blkc >> p.gshift;            // groups per scale block (8 or 16)
-    const int spb = blkc / KS;                   // stages per scale block (1..4)
+    // codes per scale block (a whole number of stages and of 8 groups); compile-time constants
+    // on the exact-code path, whose group size is a template parameter
+    const int blkc = NAT ? (8 * G > KS ? 8 * G : KS) : st_block_codes(BITS, p.group);
+    const int gbb = NAT ? blkc / (G > 0 ? G : 1) : (blkc >> p.gshift);  // groups per scale block (8 or 16)
+    const int spb = blkc / KS;                                          // stages per scale block (1..4)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
@@ -1184,6 +1189,7 @@ cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t 
     p.xgw = nullptr;
     p.xexp = nullptr;
     const StLayout L = st_layout(a.bits, mt, c.ring, c.kslice, a.group, c.split, c.ncw, int(a.M), c.xstream);
+    p.lay = L;
     if (c.tper > 0 || c.xstream) {
         // workspace: tail arrival words [T - dp_tiles], tail partial sums [2 * grid][8 * mt][128];
         // streamed x: tiles [stages][16][xrs chunks], group sums [M][gpad], exponents [M]
