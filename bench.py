@@ -320,7 +320,7 @@ def run_grouped(q, dev, peak):
             plans = [q.plan_default(M, N, K, 4, 64, torch.float16) for N in Ns]
             for p_ in plans:
                 p_.flags |= q.PLAN_STATIC_WEIGHTS
-            gplan = q.make_plan(kernel=q.KERNEL_SK, flags=q.PLAN_PDL | q.PLAN_STATIC_WEIGHTS)
+            gplan = q.make_plan(kernel=q.KERNEL_AUTO, flags=q.PLAN_PDL | q.PLAN_STATIC_WEIGHTS)
 
             def grouped():
                 for mats in sets:

@@ -426,23 +426,18 @@ qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t 
             return fail(QMM_ERR_UNSUPPORTED, "item %d: grouped calls need 16-byte aligned packed/scales/biases", i);
         if (!sk_supported(M, live[i].N, K, bits, group))
             return fail(QMM_ERR_UNSUPPORTED,
-                        "item %d: grouped calls run on the even-split kernel, which needs a multiple of 8 groups "
-                        "per row and a 16-byte multiple of packed bytes per row", i);
+                        "item %d: grouped calls need a multiple of 8 groups per row and a 16-byte multiple of "
+                        "packed bytes per row", i);
     }
     qmm_plan pl;
     memset(&pl, 0, sizeof(pl));
     if (plan) pl = *plan;
-    if (pl.kernel != QMM_KERNEL_AUTO && pl.kernel != QMM_KERNEL_SK)
-        return fail(QMM_ERR_INVALID_ARG, "grouped calls run on the even-split kernel (kernel=%d)", pl.kernel);
-    if (pl.split < 0 || pl.split > 2) return fail(QMM_ERR_INVALID_ARG, "split=%d (x mode 0, 1 or 2)", pl.split);
+    if (pl.kernel != QMM_KERNEL_AUTO && pl.kernel != QMM_KERNEL_SK && pl.kernel != QMM_KERNEL_STREAM)
+        return fail(QMM_ERR_INVALID_ARG, "grouped calls run on the streaming or the even-split kernel (kernel=%d)",
+                    pl.kernel);
     if (pl.flags & ~uint32_t(QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS))
         return fail(QMM_ERR_INVALID_ARG, "unknown or unsupported plan flags 0x%x", pl.flags);
     if (tiles * 128 > (int64_t(1) << 30)) return fail(QMM_ERR_UNSUPPORTED, "too many rows in one grouped call");
-    SkConfig c = sk_config(M, tiles * 128, K, bits, group, pl.split);
-    if (!c.ok) return fail(QMM_ERR_UNSUPPORTED, "even-split plan does not fit shared memory");
-    c.pdl = plan ? (pl.flags & QMM_PLAN_PDL) != 0 : true;
-    c.static_weights = plan ? (pl.flags & QMM_PLAN_STATIC_WEIGHTS) != 0 : false;
-    c.test_timeout = false;
     QmmArgs a;
     memset(&a, 0, sizeof(a));
     a.x = static_cast<const uint16_t*>(x);
@@ -452,6 +447,45 @@ qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t 
     a.bits = bits;
     a.group = group;
     a.is_bf16 = dtype == QMM_BF16;
+    // up to 16 tokens: the streaming kernel over the matrices' tiles, numbered one after
+    // another (the measured choice: it beats separate calls, whose launches do not overlap);
+    // above, or when forced, the even-split kernel
+    if (pl.kernel == QMM_KERNEL_STREAM || (pl.kernel == QMM_KERNEL_AUTO && M <= 16)) {
+        if (pl.kernel == QMM_KERNEL_STREAM && (pl.split < 0 || pl.split > 8))
+            return fail(QMM_ERR_INVALID_ARG, "split=%d (the streaming kernel splits K 1..8 ways, 0 = auto)", pl.split);
+        StreamConfig sc = {};
+        if (stream_supported(M, tiles * 128, K, bits, group))
+            sc = stream_config(M, tiles * 128, K, bits, group, pl.kernel == QMM_KERNEL_STREAM ? pl.split : 0);
+        if (sc.ring >= 2) {
+            sc.pdl = plan ? (pl.flags & QMM_PLAN_PDL) != 0 : true;
+            sc.static_weights = plan ? (pl.flags & QMM_PLAN_STATIC_WEIGHTS) != 0 : false;
+            return launch_result(launch_stream_items(a, live, n, sc, st), "qmm_grouped launch");
+        }
+        if (pl.kernel == QMM_KERNEL_STREAM)
+            return fail(QMM_ERR_UNSUPPORTED, "the streaming kernel takes 1 <= M <= 16 and whole stages and scale "
+                        "blocks of K");
+    }
+    if (pl.kernel == QMM_KERNEL_AUTO && M > 16) {
+        // above 16 tokens one even-split launch over the group measured slower than the
+        // matrices' own default plans back to back (the tensor-core and warp-tile kernels
+        // are not grouped), so the default takes those
+        qmm_plan one;
+        memset(&one, 0, sizeof(one));
+        one.kernel = QMM_KERNEL_AUTO;
+        one.flags = plan ? (pl.flags & (QMM_PLAN_PDL | QMM_PLAN_STATIC_WEIGHTS)) : QMM_PLAN_PDL;
+        for (int i = 0; i < n; ++i) {
+            qmm_status r = qmm_ex(x, live[i].packed, live[i].scales, live[i].biases, live[i].y, M, live[i].N, K, bits,
+                                  group, dtype, &one, stream);
+            if (r != QMM_OK) return r;
+        }
+        return QMM_OK;
+    }
+    if (pl.split < 0 || pl.split > 2) return fail(QMM_ERR_INVALID_ARG, "split=%d (x mode 0, 1 or 2)", pl.split);
+    SkConfig c = sk_config(M, tiles * 128, K, bits, group, pl.split);
+    if (!c.ok) return fail(QMM_ERR_UNSUPPORTED, "even-split plan does not fit shared memory");
+    c.pdl = plan ? (pl.flags & QMM_PLAN_PDL) != 0 : true;
+    c.static_weights = plan ? (pl.flags & QMM_PLAN_STATIC_WEIGHTS) != 0 : false;
+    c.test_timeout = false;
     return launch_result(launch_sk_items(a, live, n, c, st), "qmm_grouped launch");
 }
 

@@ -110,10 +110,22 @@ __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int ks
     return L;
 }
 
+constexpr int ST_MAX_ITEMS = 4;  // weight matrices one launch may cover (they share x)
+
+// The weight matrices of one launch (one, or up to four that share x: a layer's q/k/v or
+// gate/up projections).  Their 128-row tiles are numbered one after another: matrix i owns
+// tiles [tile0[i], tile0[i + 1]).
+struct StMapSet {
+    CUtensorMap w[ST_MAX_ITEMS], s[ST_MAX_ITEMS], b[ST_MAX_ITEMS];
+};
+
 struct StParams {
     const uint16_t* x;
-    uint16_t* y;
-    int M, N, K;
+    uint16_t* y[ST_MAX_ITEMS];      // outputs [M, Ns[i]]
+    int Ns[ST_MAX_ITEMS];           // rows of each matrix
+    int tile0[ST_MAX_ITEMS + 1];    // first tile of each matrix (tile0[nitems] = T)
+    int nitems;
+    int M, K;
     int group, gshift;
     int is_bf16;
     int T;        // 128-row tiles
@@ -202,6 +214,23 @@ __device__ __forceinline__ void st_work_item(const StParams& p, const StWork& w,
         s0 = 0;
         s1 = nst;
     }
+}
+
+// Which matrix tile t belongs to.
+__device__ __forceinline__ int st_mat(const StParams& p, int t) {
+    int i = 0;
+    while (i + 1 < p.nitems && t >= p.tile0[i + 1]) ++i;
+    return i;
+}
+
+// y[m, n] of the matrix tile t belongs to, n = its row r within the tile; rows past the
+// matrix's N are not stored.
+__device__ __forceinline__ void st_store_y(const StParams& p, int t, int m, int r, float v) {
+    const int i = st_mat(p, t);
+    const int n = (t - p.tile0[i]) * ST_ROWS + r, N = p.Ns[i];
+    if (n < N)
+        p.y[i][int64_t(m) * N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v))
+                                               : __half_as_ushort(__float2half_rn(v));
 }
 
 // Partial-sum slot of tail tile t (index ti past dp_tiles) from block c.
@@ -349,8 +378,7 @@ __device__ __forceinline__ void load_scales(uint32_t a, uint32_t (&v)[(NGH + 1) 
 // instances carry none of its code.
 template <int BITS, int MT, int NCW, int G, bool XS>
 __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
-    qmm_stream_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
-                      const __grid_constant__ CUtensorMap bmap, const StParams p) {
+    qmm_stream_kernel(const __grid_constant__ StMapSet maps, const StParams p) {
     using F = StepFmt<BITS>;
     using SF = SFmt<BITS>;
     constexpr int KSS = F::KS;                 // codes per step
@@ -414,9 +442,11 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     if (p.split > 1) asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
     bool cl_waited = false;
     if (threadIdx.x == 32 * NCW) {
-        prefetch_tensormap(&wmap);
-        prefetch_tensormap(&smap);
-        prefetch_tensormap(&bmap);
+        for (int i = 0; i < p.nitems; ++i) {
+            prefetch_tensormap(&maps.w[i]);
+            prefetch_tensormap(&maps.s[i]);
+            prefetch_tensormap(&maps.b[i]);
+        }
     }
     __syncthreads();
 
@@ -436,6 +466,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
             for (int k = 0; ok && k < wk.n; ++k) {
                 int t, s0, s1;
                 st_work_item(p, wk, nst, spb, k, t, s0, s1);
+                const int mi = st_mat(p, t), row0 = (t - p.tile0[mi]) * ST_ROWS;  // matrix, first row
                 int sib = 0, gcol = gcol0 + (s0 / spb) * gbb, wcol = wcol0 + s0 * (NBOX * BOXW);
                 for (int st = s0; st < s1; ++st, ++it) {
                     if (sib == 0) {  // scales and biases of the next block of groups
@@ -445,8 +476,8 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                         }
                         const uint32_t dst = sbase + L.sb_off + ss * L.sb_slot;
                         mbar_arrive_expect_tx(bar_sfull + 8 * ss, L.sb_slot);
-                        tma_load_2d(dst, &smap, bar_sfull + 8 * ss, gcol, t * ST_ROWS);
-                        tma_load_2d(dst + L.sb_slot / 2, &bmap, bar_sfull + 8 * ss, gcol, t * ST_ROWS);
+                        tma_load_2d(dst, &maps.s[mi], bar_sfull + 8 * ss, gcol, row0);
+                        tma_load_2d(dst + L.sb_slot / 2, &maps.b[mi], bar_sfull + 8 * ss, gcol, row0);
                         gcol += gbb;
                         ++blk;
                         if (++ss == ST_SS) {
@@ -462,8 +493,8 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                     mbar_arrive_expect_tx(bar_full + 8 * s, L.w_stage + L.xtile);
 #pragma unroll
                     for (int b = 0; b < NBOX; ++b)
-                        tma_load_2d(sbase + s * L.slot + b * (ST_ROWS * 128), &wmap, bar_full + 8 * s,
-                                    wcol + b * BOXW, t * ST_ROWS);
+                        tma_load_2d(sbase + s * L.slot + b * (ST_ROWS * 128), &maps.w[mi], bar_full + 8 * s,
+                                    wcol + b * BOXW, row0);
                     if constexpr (XS)
                         bulk_load(sbase + s * L.slot + L.w_stage, p.xt + size_t(kb / KS + st) * L.xtile, L.xtile,
                                   bar_full + 8 * s);
@@ -714,11 +745,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const int m = 8 * mt + 2 * c + (i & 1);
-                            const int n = t * ST_ROWS + (i < 2 ? rA : rB);
-                            if (m < p.M && n < p.N)
-                                p.y[int64_t(m) * p.N + n] = p.is_bf16
-                                                                ? __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][i]))
-                                                                : __half_as_ushort(__float2half_rn(acc[mt][i]));
+                            if (m < p.M) st_store_y(p, t, m, i < 2 ? rA : rB, acc[mt][i]);
                         }
                 } else if (PARTIAL && p.split == 1) {
                     // a piece of a tail tile (item k = 0 or 1: the tail comes first): its
@@ -832,12 +859,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                 }
                 const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int n = t2 * ST_ROWS + r4 + i;
-                    if (n < p.N)
-                        p.y[int64_t(col) * p.N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sv[i]))
-                                                                : __half_as_ushort(__float2half_rn(sv[i]));
-                }
+                for (int i = 0; i < 4; ++i) st_store_y(p, t2, col, r4 + i, sv[i]);
             }
         }
     }
@@ -860,12 +882,9 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         const bool ok = *abort_flag == 0;
         for (int e = threadIdx.x; e < nrows * ncols; e += StWarps<NCW>::THREADS) {
             const int col = e / nrows, rl = e - col * nrows;
-            const int n = t * ST_ROWS + rlo + rl;
             float sum = 0.f;
             for (int q = 0; q < p.split; ++q) sum += red[(q * 8 * MT + col) * rows_per + rl];
-            if (n < p.N && ok)
-                p.y[int64_t(col) * p.N + n] = p.is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(sum))
-                                                        : __half_as_ushort(__float2half_rn(sum));
+            if (ok) st_store_y(p, t, col, rlo + rl, sum);
         }
     }
 }
@@ -951,7 +970,7 @@ __global__ void __launch_bounds__(256) st_xprep_kernel(const uint16_t* __restric
     if (threadIdx.x == 0) xexp[m] = E;
 }
 
-using StKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const StParams);
+using StKernelFn = void (*)(const StMapSet, const StParams);
 
 template <int BITS, int MT, bool XS>
 StKernelFn pick_stream_g(int group) {
@@ -1155,25 +1174,49 @@ cudaError_t ensure_smem_attr(StKernelFn fn, size_t smem) {
 
 }  // namespace
 
-cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream) {
+cudaError_t launch_stream_items(const QmmArgs& a, const SkItem* items, int nitems, const StreamConfig& c,
+                                cudaStream_t stream) {
     const int mt = int(a.M) > 8 ? 2 : 1;
     StKernelFn fn = pick_stream(a.bits, mt, c.ncw, a.group, c.xstream);
-    if (!fn || c.ring < 2) return cudaErrorNotSupported;
-    // The three descriptors depend only on the weight arrays and the format; a call that
-    // repeats them (the usual case: the same weights every step) reuses the encoded copies.
-    const StMaps* maps = weight_maps(a);
-    if (!maps) return cudaErrorNotSupported;
+    if (!fn || c.ring < 2 || nitems < 1 || nitems > ST_MAX_ITEMS) return cudaErrorNotSupported;
 
     StParams p;
+    StMapSet maps;
+    std::memset(&maps, 0, sizeof(maps));
+    int tiles = 0;
+    for (int i = 0; i < nitems; ++i) {
+        // The three descriptors depend only on the weight arrays and the format; a call that
+        // repeats them (the usual case: the same weights every step) reuses the encoded copies.
+        QmmArgs ai = a;
+        ai.packed = items[i].packed;
+        ai.scales = items[i].scales;
+        ai.biases = items[i].biases;
+        ai.N = items[i].N;
+        const StMaps* m = weight_maps(ai);
+        if (!m) return cudaErrorNotSupported;
+        maps.w[i] = m->w;
+        maps.s[i] = m->s;
+        maps.b[i] = m->b;
+        p.y[i] = items[i].y;
+        p.Ns[i] = int(items[i].N);
+        p.tile0[i] = tiles;
+        tiles += cdiv(items[i].N, ST_ROWS);
+    }
+    for (int i = nitems; i <= ST_MAX_ITEMS; ++i) p.tile0[i] = tiles;
+    for (int i = nitems; i < ST_MAX_ITEMS; ++i) {
+        p.y[i] = nullptr;
+        p.Ns[i] = 0;
+    }
+    p.nitems = nitems;
     p.x = a.x;
-    p.y = a.y;
     p.M = int(a.M);
-    p.N = int(a.N);
     p.K = int(a.K);
     p.group = a.group;
     p.gshift = ilog2(a.group);
     p.is_bf16 = a.is_bf16;
-    p.T = cdiv(a.N, ST_ROWS);
+    p.T = tiles;
+    // the configuration must be the one stream_config gave for N = 128 * tiles
+    if (c.split > 1 ? c.grid_x != tiles : c.dp_tiles > tiles) return cudaErrorNotSupported;
     p.kslice = c.kslice;
     p.split = c.split;
     p.ring = c.ring;
@@ -1256,7 +1299,12 @@ cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t 
                                              int(L.gpad), xt, xgw, xexp);
         if (e != cudaSuccess) return e;
     }
-    return cudaLaunchKernelEx(&cfg, fn, maps->w, maps->s, maps->b, p);
+    return cudaLaunchKernelEx(&cfg, fn, maps, p);
+}
+
+cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream) {
+    const SkItem it{a.packed, a.scales, a.biases, a.y, a.N};
+    return launch_stream_items(a, &it, 1, c, stream);
 }
 
 cudaError_t stream_read_and_clear_errors(unsigned* out) {

@@ -170,19 +170,24 @@ typedef struct {
 /*
  * qmm_grouped -- y_i = x . dequant(items[i])^T for 1 <= count <= 4 weight matrices that share
  * x, K and the format (bits, group, dtype): a decoder layer's q, k and v projections, or its
- * gate and up projections, in ONE launch of the even-split kernel (two when x is staged in
- * the workspace).  "How the NAX Verify Kernel Path Improves Decode Performance in MTPLX",
+ * gate and up projections, in ONE launch over all their 128-row tiles (numbered one matrix
+ * after another).  "How the NAX Verify Kernel Path Improves Decode Performance in MTPLX",
  * section "Architectural Differences: Stock MLX vs. NAX Verify", puts the small verify
  * calls' cost in per-call dispatch overhead; one launch over the layer's matrices pays it
- * once and splits all their weight bytes evenly over the SMs.
- * Each item must meet the even-split kernel's shape rules (1 <= M <= 64, a multiple of 8
- * groups per row, a 16-byte multiple of packed bytes per row; packed, scales, biases, x and
- * y 16-byte aligned), else QMM_ERR_UNSUPPORTED and nothing is launched.  `plan` may be NULL
- * or name QMM_KERNEL_AUTO / QMM_KERNEL_SK with its x mode in `split` and the QMM_PLAN_PDL /
- * QMM_PLAN_STATIC_WEIGHTS flags (NULL = PDL, weights not static).  Each y_i meets the same
- * tolerance as a qmm() call and is bitwise reproducible run to run (the split points, and so
- * the order partial sums meet in, depend on the whole group).  M == 0 is a no-op; K == 0
- * writes zeros to every y.  Stream, scratch memory and errors as for qmm().
+ * once and spreads all their weight bytes over the SMs.  Up to 16 tokens the launch is the
+ * streaming kernel's (plus its x pass for 9-16 tokens on a persistent grid).  Above 16 tokens
+ * QMM_KERNEL_AUTO runs each matrix's own default plan instead (separate launches: one
+ * even-split launch over the group measured slower there), and QMM_KERNEL_SK forces the one
+ * even-split launch (plus its x pass when x is staged in the workspace).
+ * Each item must have a multiple of 8 groups per row and a 16-byte multiple of packed bytes
+ * per row, with packed, scales, biases, x and y 16-byte aligned; 1 <= M <= 64; else
+ * QMM_ERR_UNSUPPORTED and nothing is launched.  `plan` may be NULL or name QMM_KERNEL_AUTO,
+ * QMM_KERNEL_STREAM (M <= 16; `split` = its K split, 0 = auto) or QMM_KERNEL_SK (`split` =
+ * its x mode), with the QMM_PLAN_PDL / QMM_PLAN_STATIC_WEIGHTS flags (NULL = PDL, weights not
+ * static).  Each y_i meets the same tolerance as a qmm() call and is bitwise reproducible run
+ * to run (how the work is split, and so the order partial sums meet in, depends on the whole
+ * group).  M == 0 is a no-op; K == 0 writes zeros to every y.  Stream, scratch memory and
+ * errors as for qmm().
  */
 qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t M, int64_t K,
                        int bits, int group, qmm_dtype dtype, const qmm_plan* plan, void* stream);

@@ -73,6 +73,35 @@ def test_grouped_matches_separate_calls(oracle_mod):
         check_close(ys[i], q.qmm(x, P, S, B, 4, 64).double().cpu().numpy(), dtype, f"grouped vs separate {i}")
 
 
+@pytest.mark.parametrize("M", [1, 4, 8, 9, 16])
+@pytest.mark.parametrize("shape", ["qkv", "gate_up", "ragged"])
+def test_grouped_streaming(oracle_mod, M, shape):
+    """Up to 16 tokens the default grouped call runs on the streaming kernel: q/k/v (48 tiles)
+    on a K-split grid, gate/up (224 tiles) on a persistent grid whose tail tiles are all in
+    the second matrix's range, ragged matrices whose last tiles are partly past their N; 9-16
+    tokens stream x on the persistent grid."""
+    if shape == "qkv":
+        K, Ns, bits, group, dtype = 2048, (4096, 1024, 1024), 4, 64, torch.float16
+    elif shape == "gate_up":
+        K, Ns, bits, group, dtype = 1024, (14336, 14336), 8, 64, torch.bfloat16
+    else:
+        K, Ns, bits, group, dtype = 1024, (1000, 333, 17), 6, 32, torch.float16
+    mats = _mats(oracle_mod, Ns, K, bits, group, dtype)
+    x = x_input(M, K, dtype)
+    ys = q.qmm_grouped(x.cuda(), [d for _, d in mats], bits, group)
+    torch.cuda.synchronize()
+    assert q.device_errors() == 0
+    for i, ((op, os_, ob), _) in enumerate(mats):
+        check_close(ys[i], oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group), dtype, f"{shape} item {i} M={M}")
+    # forced onto the streaming kernel with an explicit K split: the same bits as before for
+    # the K-split grid (the split it chose), and within tolerance for any other
+    plan = q.make_plan(kernel=q.KERNEL_STREAM, split=2)
+    ys2 = q.qmm_grouped(x.cuda(), [d for _, d in mats], bits, group, plan=plan)
+    torch.cuda.synchronize()
+    for i, ((op, os_, ob), _) in enumerate(mats):
+        check_close(ys2[i], oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group), dtype, f"{shape} item {i} split 2")
+
+
 def test_grouped_rejects():
     L = q.lib()
     items = (q.Item * 5)()
@@ -85,5 +114,14 @@ def test_grouped_rejects():
     x = torch.zeros((4, 512), dtype=torch.float16, device="cuda")
     items[0] = q.Item(P.data_ptr(), S.data_ptr() + 2, S.data_ptr(), y.data_ptr(), 256)
     assert L.qmm_grouped(x.data_ptr(), items, 1, 4, 512, 4, 64, 0, None, None) == q.QMM_ERR_UNSUPPORTED
+    # grouped plans name the streaming or the even-split kernel; the streaming one takes M <= 16
+    items[0] = q.Item(P.data_ptr(), S.data_ptr(), S.data_ptr(), y.data_ptr(), 256)
+    tc = q.make_plan(kernel=q.KERNEL_TC)
+    assert L.qmm_grouped(x.data_ptr(), items, 1, 4, 512, 4, 64, 0, ctypes.byref(tc), None) == q.QMM_ERR_INVALID_ARG
+    y17 = torch.zeros((17, 256), dtype=torch.float16, device="cuda")
+    x17 = torch.zeros((17, 512), dtype=torch.float16, device="cuda")
+    items[0] = q.Item(P.data_ptr(), S.data_ptr(), S.data_ptr(), y17.data_ptr(), 256)
+    stp = q.make_plan(kernel=q.KERNEL_STREAM)
+    assert L.qmm_grouped(x17.data_ptr(), items, 1, 17, 512, 4, 64, 0, ctypes.byref(stp), None) == q.QMM_ERR_UNSUPPORTED
     # M == 0 and all-empty groups are no-ops
     assert L.qmm_grouped(0, items, 1, 0, 512, 4, 64, 0, None, None) == q.QMM_OK
