@@ -117,6 +117,27 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+FALLBACK_TENSOR_TFLOPS = 1400.0  # dense bf16/fp16, sustained under the power cap (earlier measurement)
+
+
+def tensor_peak():
+    """Sustained dense fp16/bf16 tensor rate (TFLOP/s): the measured one, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d.get("bf16_tflops_sustained") or d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_TENSOR_TFLOPS, "fallback"
+
+
+def roofline_gbs(wl, M: int, hbm_gbs: float, tflops: float) -> float:
+    """The cell's roofline in weight GB/s: the HBM rate, or the tensor rate over the call's
+    intensity (2*M*N*K flops per weight byte) where that is lower (4-bit, M >= ~60)."""
+    flops_per_byte = 2.0 * M * wl.N * wl.K / wl.weight_bytes()
+    return min(hbm_gbs, tflops * 1e3 / flops_per_byte)
+
+
 def host_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -260,6 +281,7 @@ def run_breakdown(q, dev, peak):
     three 4-bit shapes, M in {4, 16, 64} on the mixed-precision ones."""
     from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS
     out = {}
+    tflops, _ = tensor_peak()
     for name in GATED + MIXED:
         wl = WORKLOADS[name]
         weights = make_weights(q, wl, dev)
@@ -271,8 +293,10 @@ def run_breakdown(q, dev, peak):
             plan = default_plan(q, wl, M)
             t = time_cell(q, wl, weights, M, dev, plan)
             gbs = wbytes / t / 1e9
+            bound = roofline_gbs(wl, M, peak, tflops)
             cells[str(M)] = {"gbs": round(gbs, 1), "us": round(t * 1e6, 3), "frac_of_measured": round(gbs / peak, 4),
                              "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                             "roofline_gbs": round(bound, 1), "frac_of_roofline": round(gbs / bound, 4),
                              "kernel": KERNEL_NAMES.get(plan.kernel, "?"), "plan": plan.as_dict()}
         g = [c["gbs"] for c in cells.values()]
         drops = [(int(a), round(1 - cells[b]["gbs"] / cells[a]["gbs"], 4)) for a, b in zip(list(cells)[:-1], list(cells)[1:])]
@@ -479,6 +503,7 @@ def run_ours(args, rank, world):
         out["clocks"] = clk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=12.0)
+        out["cpu_baseline"]["single_thread"] = oracle_single_thread()
     if rank == 0:
         if args.breakdown_out:
             with open(args.breakdown_out, "w") as f:
@@ -573,6 +598,34 @@ def _oracle_pass(wl, pq, xs, rows: int) -> float:
     for M in BENCH_MS:
         oracle.qmm(xs[M], p[:rows], s[:rows], b[:rows], wl.K, wl.bits, wl.group, wl.dtype == torch.bfloat16)
     return time.perf_counter() - t0
+
+
+def oracle_single_thread():
+    """Seconds of one oracle call on one host thread (a separate process with OMP_NUM_THREADS=1),
+    at M = 4 on the tiny and the q/o configurations, whole matrices."""
+    import subprocess
+    code = (
+        "import json, time, sys\n"
+        "sys.path.insert(0, %r)\n"
+        "import torch, oracle\n"
+        "from bit_quantized_gemm_qmm_b200.inputs import WORKLOADS, w_input, x_input\n"
+        "from bench import _oracle_inputs\n"
+        "oracle.build()\n"
+        "out = {}\n"
+        "for name in ('tiny', 'qo'):\n"
+        "    wl = WORKLOADS[name]\n"
+        "    (p, s, b), xs = _oracle_inputs(wl, wl.N)\n"
+        "    x = xs[4]\n"
+        "    t0 = time.perf_counter()\n"
+        "    oracle.qmm(x, p, s, b, wl.K, wl.bits, wl.group, wl.dtype == torch.bfloat16)\n"
+        "    out[name + '_m4_s'] = round(time.perf_counter() - t0, 4)\n"
+        "print(json.dumps(out))\n") % ROOT
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT, timeout=600)
+        return json.loads(r.stdout.strip().splitlines()[-1])
+    except Exception as e:  # reported, never fatal: the single-thread time is context only
+        return {"error": str(e)[:200]}
 
 
 def cpu_baseline(wl, budget_s: float = 12.0, rows: int = 8192):
