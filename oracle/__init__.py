@@ -70,6 +70,8 @@ def _load():
         lib.oracle_round_f32.argtypes = [P, I64, I, P]
         lib.oracle_round_f32.restype = None
         lib.oracle_qmm.argtypes = [P, I, I64, P, P, P, I64, I64, I, I, P]
+        lib.oracle_qmm_nt.restype = I
+        lib.oracle_qmm_nt.argtypes = [P, I, I64, P, P, P, I64, I64, I, I, P]
         lib.oracle_qmm.restype = I
         _lib = lib
     return _lib
@@ -189,6 +191,22 @@ def qmm(x, packed, scales, biases, K: int, bits: int, group: int, x_is_bf16: boo
     y = np.empty((M, N), dtype=np.float64)
     _check(_load().oracle_qmm(_ptr(x), int(x_is_bf16), M, _ptr(packed), _ptr(scales), _ptr(biases),
                               N, K, bits, group, _ptr(y)), "qmm")
+    return y
+
+
+def qmm_nt(x, packed, scales, biases, N: int, bits: int, group: int, x_is_bf16: bool) -> np.ndarray:
+    """y[M,N] float64 = x[M,K] . dequant(W') for W' [K,N] quantized along N (packed
+    [K, N*bits/32], scales/biases [K, N/group]): the transpose=False form of the MLX issue #4720
+    call, fp64 accumulation with k ascending."""
+    x = _as_u16(x)
+    M, K = x.shape
+    packed = np.ascontiguousarray(packed, dtype=np.uint32)
+    scales = _as_u16(scales)
+    biases = _as_u16(biases)
+    assert packed.shape[0] == K and packed.shape[1] * 32 == N * bits
+    y = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_qmm_nt(_ptr(x), int(x_is_bf16), M, _ptr(packed), _ptr(scales), _ptr(biases),
+                                 K, N, bits, group, _ptr(y)), "qmm_nt")
     return y
 
 

@@ -27,6 +27,10 @@
  * [bits*k, bits*k + bits); 32-bit word j holds stream bits [32j, 32j + 32).
  * Dequantization: d = RN_fp32(s*q + b), the exact value rounded once to fp32.
  * Matmul: y[m,n] = sum_k x[m,k] * d[n,k], accumulated in fp64 with k ascending.
+ * Non-transposed matmul (oracle_qmm_nt): quantized_matmul(x, *w, transpose=False) of the same
+ * page, "Describe the bug" (the reported dispatch is specific to transposed, non-batched calls,
+ * so the others exist): W'[K,N] is quantized along its rows (groups of `group` consecutive
+ * elements along N) and y[m,n] = sum_k x[m,k] * d'[k,n], fp64, k ascending.
  *
  * fp16 / bf16 rounding is written here from the IEEE-754 binary16 definition and from the
  * definition of bfloat16 as the upper half of a binary32 (round to nearest, ties to even).
@@ -252,6 +256,42 @@ int oracle_qmm(const uint16_t *x, int x_is_bf16, int64_t M, const uint32_t *pack
                 for (int64_t k = 0; k < K; ++k)
                     acc += (double)load_w(x, x_is_bf16, m * K + k) * (double)d[k];
                 y[m * N + n] = acc;
+            }
+        }
+        free(d);
+    }
+    return failed ? -2 : 0;
+}
+
+/* y[M,N] (fp64) = x[M,K] (fp16/bf16 bits) . dequant(W'), W' = [K,N] quantized along N
+ * (packed [K, N*bits/32], scales/biases [K, N/group]); k ascending, fp64 accumulation.  Each
+ * column of W' is dequantized once into d[0..K) and then dotted with every x row. */
+int oracle_qmm_nt(const uint16_t *x, int x_is_bf16, int64_t M, const uint32_t *packed,
+                  const uint16_t *scales, const uint16_t *biases, int64_t K, int64_t N, int bits,
+                  int group, double *y) {
+    if (!(bits == 4 || bits == 6 || bits == 8)) return -1;
+    if (!(group == 32 || group == 64 || group == 128)) return -1;
+    if (M < 0 || N < 0 || K < 0 || N % group != 0) return -1;
+    int64_t G = N / group, nw = N * bits / 32;
+    int failed = 0;
+#pragma omp parallel
+    {
+        float *d = (float *)malloc((size_t)(K > 0 ? K : 1) * sizeof(float));
+        if (!d) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(static)
+        for (int64_t n = 0; n < N; ++n) {
+            if (!d) continue;
+            for (int64_t kk = 0; kk < K; ++kk)
+                d[kk] = dequant_one(scales[kk * G + n / group], biases[kk * G + n / group],
+                                    unpack_one(packed + kk * nw, n, bits));
+            for (int64_t m = 0; m < M; ++m) {
+                double sum = 0.0;
+                for (int64_t kk = 0; kk < K; ++kk)
+                    sum += (double)load_w(x, x_is_bf16, m * K + kk) * (double)d[kk];
+                y[m * N + n] = sum;
             }
         }
         free(d);

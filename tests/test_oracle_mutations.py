@@ -48,6 +48,14 @@ MUTANTS = [
      "                for (int64_t k = 1; k < K; ++k)\n                    acc +="),
     ("x read transposed",
      "load_w(x, x_is_bf16, m * K + k)", "load_w(x, x_is_bf16, k * M + m)"),
+    ("non-transposed matmul: scale and bias swapped",
+     "d[kk] = dequant_one(scales[kk * G + n / group], biases[kk * G + n / group],",
+     "d[kk] = dequant_one(biases[kk * G + n / group], scales[kk * G + n / group],"),
+    ("non-transposed matmul drops the first term",
+     "for (int64_t kk = 0; kk < K; ++kk)\n                    sum +=",
+     "for (int64_t kk = 1; kk < K; ++kk)\n                    sum +="),
+    ("non-transposed matmul reads x transposed",
+     "load_w(x, x_is_bf16, m * K + kk)", "load_w(x, x_is_bf16, kk * M + m)"),
 ]
 
 

@@ -366,3 +366,55 @@ def test_brute_force_tiny(oracle_mod, bits, group):
                 dv = float(np.float32(float(ss[n][k // group]) * qs[n][k] + float(bs[n][k // group])))
                 acc += xl[m][k] * dv
             assert y[m, n] == acc
+
+
+# ------------------------------------------------------------------------ non-transposed matmul
+# quantized_matmul(x, *w, transpose=False) (MLX issue #4720, "Describe the bug": the reported
+# dispatch concerns transposed, non-batched calls, so this form exists): W' [K, N] quantized
+# along N, y = x . dequant(W').
+
+@pytest.mark.parametrize("bits,group", [(4, 64), (6, 32), (8, 128)])
+@pytest.mark.parametrize("is_bf16", [False, True])
+def test_qmm_nt_matches_blas_matmul(oracle_mod, bits, group, is_bf16):
+    dtype = torch.bfloat16 if is_bf16 else torch.float16
+    M, K, N = 5, 96, 768
+    _, packed, s, b = _quantize_cfg(oracle_mod, K, N, bits, group, dtype, 1.0, 25)  # W' [K, N]
+    x = randn((M, K), 1.0, dtype, 26)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    y = oracle_mod.qmm_nt(xb, packed, s, b, N, bits, group, is_bf16)
+    d = oracle_mod.dequantize_f32(packed, s, b, N, bits, group).astype(np.float64)  # [K, N]
+    ref = x.double().numpy() @ d
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("bits,group", [(4, 64), (6, 32), (8, 128)])
+def test_qmm_nt_one_hot_reproduces_rows(oracle_mod, bits, group):
+    K, N = 40, 256
+    _, packed, s, b = _quantize_cfg(oracle_mod, K, N, bits, group, torch.float16, 1.0, 27)
+    ks = [0, 1, 17, 38, 39]
+    x = np.zeros((len(ks), K), dtype=np.float16)
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    y = oracle_mod.qmm_nt(x, packed, s, b, N, bits, group, False)
+    d = oracle_mod.dequantize_f32(packed, s, b, N, bits, group)
+    for i, k in enumerate(ks):
+        assert np.array_equal(y[i], d[k].astype(np.float64))
+
+
+@pytest.mark.parametrize("bits,group", [(4, 32), (6, 32), (8, 64)])
+def test_qmm_nt_brute_force_tiny(oracle_mod, bits, group):
+    """The definition in plain Python loops over the pure-Python quantization of W'."""
+    M, K, N = 3, 5, 2 * group
+    w = randn((K, N), 1.0, torch.float16, 28)
+    x = randn((M, K), 1.0, torch.float16, 29)
+    qs, ss, bs = _py_quantize(w.float().tolist(), bits, group)  # rows of W' = K
+    packed, s, b = oracle_mod.quantize(w.numpy(), bits, group, False)
+    y = oracle_mod.qmm_nt(x.numpy(), packed, s, b, N, bits, group, False)
+    xl = x.float().tolist()
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                dv = float(np.float32(float(ss[k][n // group]) * qs[k][n] + float(bs[k][n // group])))
+                acc += xl[m][k] * dv
+            assert y[m, n] == acc
