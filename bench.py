@@ -319,6 +319,58 @@ GROUPS = {  # one decoder layer's projections that share x (Qwen3-8B-like widths
 GROUP_MS = (1, 4, 16, 64)
 
 
+NT_SHAPES = {  # the non-transposed form on the q/o and LM-head sizes: W' [K, N] quantized along N
+    "qo_nt": {"K": 4096, "N": 4096, "dtype": torch.float16, "sets": 27},
+    "lmhead_nt": {"K": 4096, "N": 151936, "dtype": torch.bfloat16, "sets": 1},
+}
+NT_MS = (1, 4, 16)
+
+
+def run_nt(q, dev, peak):
+    """GB/s of the non-transposed form (qmm_nt), 4-bit g64, per M; weight sets rotated
+    (>= 2x L2), one CUDA graph of one call per set."""
+    from bit_quantized_gemm_qmm_b200.inputs import w_input, x_input
+    out = {}
+    for name, c in NT_SHAPES.items():
+        K, N, dt = c["K"], c["N"], c["dtype"]
+        weights = []
+        for i in range(c["sets"]):
+            w = w_input(K, N, dt, i, 0.02 if dt is torch.bfloat16 else 1.0).to(dev)
+            weights.append(q.quantize(w, 4, 64))
+            del w
+        wbytes = K * N // 2 + K * (N // 64) * 4
+        cells = {}
+        for M in NT_MS:
+            x = x_input(M, K, dt).to(dev)
+            y = torch.empty((M, N), dtype=dt, device=dev)
+            for (P, S, B) in weights:
+                q.qmm_nt(x, P, S, B, 4, 64, out=y)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for (P, S, B) in weights:
+                    q.qmm_nt(x, P, S, B, 4, 64, out=y)
+            g.replay()
+            torch.cuda.synchronize()
+            reps = max(3, int(1e9 / (wbytes * len(weights))))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            e1.synchronize()
+            t = e0.elapsed_time(e1) * 1e-3 / reps / len(weights)
+            cells[str(M)] = {"gbs": round(wbytes / t / 1e9, 1), "us": round(t * 1e6, 3),
+                             "frac_of_measured": round(wbytes / t / 1e9 / peak, 4)}
+            del g
+        out[name] = {"shape": f"W' [K={K}, N={N}] 4-bit g64 {str(dt).replace('torch.', '')}", "weight_sets": len(weights),
+                     "kernel": "qmm_nt_kernel (CUDA cores)", "M": cells}
+        del weights
+        torch.cuda.empty_cache()
+        print(f"[nt] {name}: " + " ".join(f"{m}:{v['gbs']:.0f}" for m, v in cells.items()), file=sys.stderr, flush=True)
+    return out
+
+
 def run_grouped(q, dev, peak):
     """One launch over a layer's matrices (qmm_grouped) against the same matrices as separate
     calls: GB/s of the group's weight bytes per M, weight sets rotated (>= 2x L2)."""
@@ -467,12 +519,13 @@ def run_ours(args, rank, world):
     e2e = run_e2e(wl, weights, plans, dev, max(5, args.steps // 10))
     del g
     torch.cuda.synchronize()
-    breakdown = grouped = None
+    breakdown = grouped = nt = None
     if not args.no_breakdown:
         del weights
         torch.cuda.empty_cache()
         breakdown = run_breakdown(q, dev, peak)
         grouped = run_grouped(q, dev, peak)
+        nt = run_nt(q, dev, peak)
 
     kernel = KERNEL_NAMES.get(plans[BENCH_MS[0]].kernel, "?")
     out = {
@@ -498,6 +551,7 @@ def run_ours(args, rank, world):
     if breakdown is not None:
         out["breakdown"] = breakdown
         out["grouped"] = grouped
+        out["non_transposed"] = nt
     if clk:
         clk["window"] = f"{CLOCK_SOAK_S:.1f} s of the same replays immediately before the timed region, and the timed region"
         out["clocks"] = clk

@@ -91,6 +91,10 @@ def lib() -> ctypes.CDLL:
     L.qmm_noalloc.restype = I
     L.qmm_grouped.argtypes = [P, ctypes.POINTER(Item), I, I64, I64, I, I, U, ctypes.POINTER(Plan), P]
     L.qmm_grouped.restype = I
+    L.qmm_nt.argtypes = [P, P, P, P, P, I64, I64, I64, I, I, U, P]
+    L.qmm_nt.restype = I
+    L.qmm_batched.argtypes = [P, I64, P, I64, P, P, I64, P, I64, I64, I64, I64, I64, I, I, U, I, P]
+    L.qmm_batched.restype = I
     _lib = L
     return L
 
@@ -294,6 +298,77 @@ def qmm_grouped(x: torch.Tensor, weights, bits: int, group: int, outs=None, plan
         _check(lib().qmm_grouped(x.data_ptr(), items, len(weights), M, K, bits, group, _dtype_code(x.dtype),
                                  None if plan is None else ctypes.byref(plan), _current_stream(dev)))
     return outs
+
+
+def qmm_nt(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+           bits: int, group: int, out: torch.Tensor | None = None):
+    """y[M,N] = x[M,K] . dequant(W') for W' [K, N] quantized along N (the transpose=False form):
+    packed [K, N*bits/32], scales and biases [K, N/group] (what quantize(W') returns)."""
+    for t in (x, packed, scales, biases):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("x, packed, scales and biases must be contiguous CUDA tensors")
+    dev = x.get_device()
+    if packed.get_device() != dev or scales.get_device() != dev or biases.get_device() != dev:
+        raise ValueError("all tensors must be on the same CUDA device")
+    if x.dim() != 2 or packed.dim() != 2 or packed.element_size() != 4:
+        raise ValueError("x must be [M, K] and packed [K, N*bits/32] 32-bit words")
+    M, K = x.shape
+    if packed.shape[0] != K:
+        raise ValueError(f"packed has {packed.shape[0]} rows; W' needs K={K}")
+    N = packed.shape[1] * 32 // bits
+    if scales.dtype is not torch.float16 or biases.dtype is not torch.float16 or group <= 0 \
+            or scales.numel() != K * (N // group) or biases.numel() != K * (N // group):
+        raise ValueError(f"scales and biases must be fp16 [K, N/group] = [{K}, {N // max(group, 1)}]")
+    if out is None:
+        out = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    elif not (out.is_cuda and out.get_device() == dev and out.is_contiguous() and out.dtype is x.dtype
+              and tuple(out.shape) == (M, N)):
+        raise ValueError("out must be a contiguous [M, N] CUDA tensor with x's dtype on x's device")
+    with torch.cuda.device(dev):
+        _check(lib().qmm_nt(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
+                            M, N, K, bits, group, _dtype_code(x.dtype), _current_stream(dev)))
+    return out
+
+
+def qmm_batched(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+                bits: int, group: int, transpose: bool = True, out: torch.Tensor | None = None):
+    """A batch of independent calls: x [B, M, K]; weights shared (packed 2-D) or one per problem
+    (packed 3-D, [B, ...]); transpose=True takes W [N, K] (qmm), False W' [K, N] (qmm_nt).
+    Returns y [B, M, N]."""
+    for t in (x, packed, scales, biases):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("x, packed, scales and biases must be contiguous CUDA tensors")
+    if x.dim() != 3:
+        raise ValueError("x must be [B, M, K]")
+    Bn, M, K = x.shape
+    batched_w = packed.dim() == 3
+    if batched_w and (packed.shape[0] != Bn or scales.shape[0] != Bn or biases.shape[0] != Bn):
+        raise ValueError("batched weights must have the batch as their first dimension")
+    P2 = packed[0] if batched_w else packed
+    S2 = scales[0] if batched_w else scales
+    if transpose:
+        N = P2.shape[0]
+        if P2.shape[1] * 32 != K * bits:
+            raise ValueError("packed must be [N, K*bits/32]")
+        groups = N * (K // group)
+    else:
+        N = P2.shape[1] * 32 // bits
+        if P2.shape[0] != K:
+            raise ValueError("packed must be [K, N*bits/32]")
+        groups = K * (N // group)
+    if S2.numel() != groups or scales.dtype is not torch.float16 or biases.dtype is not torch.float16:
+        raise ValueError("scales and biases must be fp16 with one value per group")
+    if out is None:
+        out = torch.empty((Bn, M, N), dtype=x.dtype, device=x.device)
+    elif not (out.is_contiguous() and out.dtype is x.dtype and tuple(out.shape) == (Bn, M, N)):
+        raise ValueError("out must be a contiguous [B, M, N] tensor with x's dtype")
+    dev = x.get_device()
+    with torch.cuda.device(dev):
+        _check(lib().qmm_batched(x.data_ptr(), M * K, packed.data_ptr(), P2.numel() if batched_w else 0,
+                                 scales.data_ptr(), biases.data_ptr(), S2.numel() if batched_w else 0,
+                                 out.data_ptr(), M * N, Bn, M, N, K, bits, group, _dtype_code(x.dtype),
+                                 int(transpose), _current_stream(dev)))
+    return out
 
 
 def device_errors() -> int:

@@ -389,6 +389,69 @@ qmm_status qmm(const void* x, const uint32_t* packed, const uint16_t* scales,
     return qmm_ex(x, packed, scales, biases, y, M, N, K, bits, group, dtype, nullptr, stream);
 }
 
+qmm_status qmm_nt(const void* x, const uint32_t* packed, const uint16_t* scales, const uint16_t* biases,
+                  void* y, int64_t M, int64_t N, int64_t K, int bits, int group, qmm_dtype dtype,
+                  void* stream) {
+    // W' [K, N] is a K-row matrix quantized along its N columns: the format rules of a
+    // [rows = K, length = N] matrix
+    qmm_status s = check_format(K, N, bits, group);
+    if (s != QMM_OK) return s;
+    if (dtype != QMM_F16 && dtype != QMM_BF16) return fail(QMM_ERR_INVALID_ARG, "dtype=%d", int(dtype));
+    if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M=%lld", (long long)M);
+    if (M > kMaxTotalM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %lld", (long long)M, (long long)kMaxTotalM);
+    if (M == 0 || N == 0) return QMM_OK;
+    if (!y || !aligned(y, 2)) return fail(QMM_ERR_INVALID_ARG, "y must be a 2-byte aligned pointer");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) {
+        cudaError_t e = cudaMemsetAsync(y, 0, size_t(M) * size_t(N) * 2, st);
+        return e == cudaSuccess ? QMM_OK : cuda_fail(e, "qmm_nt zero fill");
+    }
+    if (!x || !packed || !scales || !biases) return fail(QMM_ERR_INVALID_ARG, "null input pointer");
+    if (!aligned(x, 2) || !aligned(packed, 4) || !aligned(scales, 2) || !aligned(biases, 2))
+        return fail(QMM_ERR_INVALID_ARG, "misaligned pointer (x, scales, biases 2-byte; packed 4-byte)");
+    QmmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = static_cast<const uint16_t*>(x);
+    a.packed = packed;
+    a.scales = scales;
+    a.biases = biases;
+    a.y = static_cast<uint16_t*>(y);
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.bits = bits;
+    a.group = group;
+    a.is_bf16 = dtype == QMM_BF16;
+    return launch_result(launch_nt(a, st), "qmm_nt launch");
+}
+
+qmm_status qmm_batched(const void* x, int64_t x_stride, const uint32_t* packed, int64_t w_stride,
+                       const uint16_t* scales, const uint16_t* biases, int64_t s_stride, void* y,
+                       int64_t y_stride, int64_t batch, int64_t M, int64_t N, int64_t K, int bits,
+                       int group, qmm_dtype dtype, int transpose, void* stream) {
+    if (batch < 0) return fail(QMM_ERR_INVALID_ARG, "negative batch=%lld", (long long)batch);
+    if (x_stride < 0 || w_stride < 0 || s_stride < 0 || y_stride < 0)
+        return fail(QMM_ERR_INVALID_ARG, "negative stride");
+    if (batch == 0) return QMM_OK;
+    auto one = [&](int64_t i0, int64_t m) -> qmm_status {
+        const void* xi = static_cast<const uint16_t*>(x) + i0 * x_stride;
+        void* yi = static_cast<uint16_t*>(y) + i0 * y_stride;
+        const uint32_t* pi = packed + i0 * w_stride;
+        const uint16_t* si = scales + i0 * s_stride;
+        const uint16_t* bi = biases + i0 * s_stride;
+        return transpose ? qmm_ex(xi, pi, si, bi, yi, m, N, K, bits, group, dtype, nullptr, stream)
+                         : qmm_nt(xi, pi, si, bi, yi, m, N, K, bits, group, dtype, stream);
+    };
+    // shared weights over contiguous x and y: one call over all the batch's tokens
+    if (w_stride == 0 && s_stride == 0 && x_stride == M * K && y_stride == M * N && batch * M <= kMaxTotalM)
+        return one(0, batch * M);
+    for (int64_t i = 0; i < batch; ++i) {
+        qmm_status s = one(i, M);
+        if (s != QMM_OK) return s;
+    }
+    return QMM_OK;
+}
+
 qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t M, int64_t K,
                        int bits, int group, qmm_dtype dtype, const qmm_plan* plan, void* stream) {
     if (count < 1 || count > kSkMaxItems) return fail(QMM_ERR_INVALID_ARG, "count=%d (1..%d)", count, kSkMaxItems);

@@ -129,6 +129,8 @@ cudaError_t launch_sk_items(const QmmArgs& a, const SkItem* items, int nitems, c
 cudaError_t sk_read_and_clear_errors(unsigned* out);
 StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group, int split_req);
 cudaError_t launch_stream(const QmmArgs& a, const StreamConfig& c, cudaStream_t stream);
+// The non-transposed form (qmm_nt.cu): a's N and K are those of y = x . dequant(W'), W' [K, N].
+cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream);
 // The streaming kernel over up to four matrices that share x (a's packed/scales/biases/y/N are
 // ignored); c must come from stream_config with N = 128 * the total of the matrices' tiles.
 cudaError_t launch_stream_items(const QmmArgs& a, const SkItem* items, int nitems, const StreamConfig& c,

@@ -1,0 +1,211 @@
+// qmm_nt.cu -- the non-transposed quantized matmul y = x . dequant(W'), W' [K, N] quantized
+// along N (sm_100a).
+//
+// quantized_matmul(x, *w, transpose=False) (MLX issue #4720, "Describe the bug": the reported
+// dispatch concerns transposed, non-batched calls, so this form and batched calls exist).
+// W' is stored like any quantized matrix, its rows being the K rows: packed [K, N*bits/32],
+// scales and biases [K, N/group].  So
+//
+//     y[m, n] = sum_k x[m,k] * (s[k, n/g] * q[k,n] + b[k, n/g])
+//             = sum_k (x[m,k] * s[k, n/g]) * q[k,n]  +  sum_k x[m,k] * b[k, n/g].
+//
+// A thread owns the codes of one packed unit of a row (8 codes of a 4-bit word, 4 of an 8-bit
+// word, 16 of a 6-bit word triple) for a range of K rows.  Per row it forms x[m,k] * s once per
+// token (exact in fp32: an 11-bit times an 11-bit significand) and adds that times each code
+// into its fp32 sums; the bias term sum_k x[m,k] * b[k, j] is the same for all the thread's
+// codes (they lie in one group) and is added at the end.  Tokens are taken TM at a time; K is
+// split over grid.y so the grid fills the GPU, and the split sums are added in split order
+// by a second kernel (deterministic).  Coalescing: consecutive threads read consecutive units
+// of a row.  This is the CUDA-core path of the less common form; it does not use the tensor
+// cores.
+#include <algorithm>
+#include <cstring>
+
+#include "qmm_common.cuh"
+#include "qmm_internal.h"
+
+namespace qmm_impl {
+namespace {
+
+constexpr int NT_THREADS = 128;
+
+template <int BITS> struct NtFmt {
+    static constexpr int CPU = BITS == 6 ? 16 : 32 / BITS;  // codes per packed unit
+    static constexpr int WPU = BITS == 6 ? 3 : 1;          // words per packed unit
+    static constexpr int TM = BITS == 6 ? 4 : 8;           // tokens a pass
+    static constexpr int RU = BITS == 6 ? 4 : 8;           // rows whose loads are in flight together
+};
+
+template <int BITS>
+__device__ __forceinline__ uint32_t nt_code(const uint32_t (&w)[NtFmt<BITS>::WPU], int i) {
+    if constexpr (BITS == 4) {
+        return (w[0] >> (4 * i)) & 0xFu;
+    } else if constexpr (BITS == 8) {
+        return (w[0] >> (8 * i)) & 0xFFu;
+    } else {  // code i at bits 6i..6i+5 of the 96-bit little-endian unit
+        const int b = 6 * i, wi = b >> 5, o = b & 31;
+        const uint32_t lo = w[wi] >> o;
+        const uint32_t hi = (o > 26 && wi < 2) ? (w[wi + 1] << (32 - o)) : 0u;
+        return (lo | hi) & 0x3Fu;
+    }
+}
+
+__device__ __forceinline__ float nt_load_x(const uint16_t* x, int is_bf16, int64_t i) {
+    const uint16_t v = x[i];
+    return is_bf16 ? __uint_as_float(uint32_t(v) << 16) : __half2float(__ushort_as_half(v));
+}
+
+__device__ __forceinline__ uint16_t nt_round(float v, int is_bf16) {
+    return is_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v)) : __half_as_ushort(__float2half_rn(v));
+}
+
+// grid.x: column blocks of NT_THREADS units; grid.y: K slices of `krange` rows.  With one
+// slice y is written directly, else part[slice][m][n] (fp32).
+template <int BITS>
+__global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __restrict__ x,
+                                                            const uint32_t* __restrict__ packed,
+                                                            const uint16_t* __restrict__ scales,
+                                                            const uint16_t* __restrict__ biases,
+                                                            uint16_t* __restrict__ y, float* __restrict__ part,
+                                                            int M, int K, int N, int gshift, int is_bf16,
+                                                            int krange) {
+    using F = NtFmt<BITS>;
+    constexpr int CPU = F::CPU, WPU = F::WPU, TM = F::TM, RU = F::RU;
+    __shared__ float xs[TM][64];  // x of the current tokens, 64 rows of K at a time
+    const int units = N / CPU;
+    const int u = blockIdx.x * NT_THREADS + threadIdx.x;  // this thread's unit of every row
+    const bool live = u < units;
+    const int n0 = u * CPU;
+    const int G = N >> gshift;
+    const int j = live ? (n0 >> gshift) : 0;  // the unit's group
+    const int64_t rw = int64_t(N) * BITS / 32;  // words per row of W'
+    const int k0 = blockIdx.y * krange, k1 = min(K, k0 + krange);
+    grid_dependency_wait();
+    for (int m0 = 0; m0 < M; m0 += TM) {
+        float acc[TM][CPU], accb[TM];
+#pragma unroll
+        for (int t = 0; t < TM; ++t) {
+            accb[t] = 0.f;
+#pragma unroll
+            for (int i = 0; i < CPU; ++i) acc[t][i] = 0.f;
+        }
+        for (int kb = k0; kb < k1; kb += 64) {
+            const int kn = min(64, k1 - kb);
+            __syncthreads();  // the previous rows' x are no longer read
+            for (int e = threadIdx.x; e < TM * 64; e += NT_THREADS) {
+                const int t = e / 64, kk = e - t * 64;
+                xs[t][kk] = (m0 + t < M && kk < kn) ? nt_load_x(x, is_bf16, int64_t(m0 + t) * K + kb + kk) : 0.f;
+            }
+            __syncthreads();
+            if (live) {
+                // RU rows at a time: all their loads are issued before any of them is used, so
+                // that a thread keeps RU independent loads in flight
+                for (int kk0 = 0; kk0 < kn; kk0 += RU) {
+                    uint32_t w[RU][WPU];
+                    uint16_t sh[RU], bh[RU];
+#pragma unroll
+                    for (int r = 0; r < RU; ++r) {
+                        const int k = kb + min(kk0 + r, kn - 1);  // rows past kn repeat the last (unused)
+#pragma unroll
+                        for (int i = 0; i < WPU; ++i) w[r][i] = __ldg(packed + int64_t(k) * rw + int64_t(u) * WPU + i);
+                        sh[r] = __ldg(scales + int64_t(k) * G + j);
+                        bh[r] = __ldg(biases + int64_t(k) * G + j);
+                    }
+#pragma unroll
+                    for (int r = 0; r < RU; ++r) {
+                        if (kk0 + r >= kn) break;
+                        const float s = __half2float(__ushort_as_half(sh[r]));
+                        const float b = __half2float(__ushort_as_half(bh[r]));
+                        float q[CPU];
+#pragma unroll
+                        for (int i = 0; i < CPU; ++i) q[i] = float(nt_code<BITS>(w[r], i));
+#pragma unroll
+                        for (int t = 0; t < TM; ++t) {
+                            const float xv = xs[t][kk0 + r];
+                            const float xsv = xv * s;  // exact: 11-bit by 11-bit significands
+                            accb[t] = fmaf(xv, b, accb[t]);
+#pragma unroll
+                            for (int i = 0; i < CPU; ++i) acc[t][i] = fmaf(xsv, q[i], acc[t][i]);
+                        }
+                    }
+                }
+            }
+        }
+        if (live) {
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+                const int m = m0 + t;
+                if (m >= M) break;
+#pragma unroll
+                for (int i = 0; i < CPU; ++i) {
+                    const float v = acc[t][i] + accb[t];
+                    if (part) part[(int64_t(blockIdx.y) * M + m) * N + n0 + i] = v;
+                    else y[int64_t(m) * N + n0 + i] = nt_round(v, is_bf16);
+                }
+            }
+        }
+    }
+}
+
+// y[m, n] = sum over the S K slices of part[s][m][n], in slice order.
+__global__ void __launch_bounds__(256) qmm_nt_reduce(const float* __restrict__ part, uint16_t* __restrict__ y,
+                                                     int64_t MN, int S, int is_bf16) {
+    for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < MN; i += int64_t(gridDim.x) * 256) {
+        // in slice order; eight loads in flight at a time
+        float v = 0.f;
+        int s = 0;
+        for (; s + 8 <= S; s += 8) {
+            float t[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t[j] = __ldcg(part + int64_t(s + j) * MN + i);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v += t[j];
+        }
+        for (; s < S; ++s) v += __ldcg(part + int64_t(s) * MN + i);
+        y[i] = nt_round(v, is_bf16);
+    }
+}
+
+constexpr int kNtSMs = 148;
+
+}  // namespace
+
+cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
+    const int cpu = a.bits == 6 ? 16 : 32 / a.bits;
+    const int units = int(a.N / cpu);
+    const int cblocks = (units + NT_THREADS - 1) / NT_THREADS;
+    // K slices: about eight blocks per SM, at least 64 rows a slice, and the fp32 split sums
+    // kept under 256 MB
+    int S = std::max(1, (8 * kNtSMs + cblocks - 1) / cblocks);
+    S = std::min<int64_t>(S, std::max<int64_t>(1, a.K / 64));
+    while (S > 1 && int64_t(S) * a.M * a.N * 4 > (int64_t(256) << 20)) --S;
+    const int krange = int((a.K + S - 1) / S + 63) / 64 * 64;
+    S = int((a.K + krange - 1) / krange);
+    float* part = nullptr;
+    if (S > 1) {
+        void* ws = nullptr;
+        cudaError_t e = split_workspace(stream, size_t(S) * size_t(a.M) * size_t(a.N) * 4, &ws);
+        if (e != cudaSuccess) return e;
+        part = static_cast<float*>(ws);
+    }
+    int gshift = 0;
+    while ((1 << gshift) < a.group) ++gshift;
+    const dim3 grid(unsigned(cblocks), unsigned(S), 1);
+    if (a.bits == 4)
+        qmm_nt_kernel<4><<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M),
+                                                          int(a.K), int(a.N), gshift, a.is_bf16, krange);
+    else if (a.bits == 6)
+        qmm_nt_kernel<6><<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M),
+                                                          int(a.K), int(a.N), gshift, a.is_bf16, krange);
+    else
+        qmm_nt_kernel<8><<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M),
+                                                          int(a.K), int(a.N), gshift, a.is_bf16, krange);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || S == 1) return e;
+    const int64_t MN = a.M * a.N;
+    const int rblocks = int(std::min<int64_t>((MN + 255) / 256, 4 * kNtSMs));
+    qmm_nt_reduce<<<rblocks, 256, 0, stream>>>(part, a.y, MN, S, a.is_bf16);
+    return cudaGetLastError();
+}
+
+}  // namespace qmm_impl

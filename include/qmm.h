@@ -217,6 +217,39 @@ qmm_status qmm_noalloc(const void* x, const uint32_t* packed, const uint16_t* sc
                        const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                        int group, qmm_dtype dtype, void* stream);
 
+/*
+ * qmm_nt -- the non-transposed form, y = x . dequant(W') with W' [K, N] quantized along N:
+ * quantized_matmul(x, *w, transpose=False) of MLX issue #4720 ("Describe the bug" names the
+ * reported dispatch as specific to transposed, non-batched calls, so this form exists).
+ *   y[m,n] = sum_k x[m,k] * (s[k, n/group] * q[k,n] + b[k, n/group])
+ * Layouts: x [M, K] and y [M, N] row-major fp16/bf16 (dtype); packed [K, N*bits/32] uint32
+ * (each row of W' packed as qmm_quantize packs a row: qmm_quantize(W', ..., N = K, K = N)
+ * makes these arrays); scales, biases [K, N/group] fp16.  N must be a multiple of `group`.
+ * Pointers: device memory, owned by the caller; x, y, scales, biases 2-byte and packed 4-byte
+ * aligned.  Arithmetic: fp32, x*s exact per row, the split sums added in a fixed order, y
+ * rounded once (same tolerance as qmm, bitwise repeatable).  Runs on CUDA cores (this form is
+ * not on the tensor-core path); M up to 2^20; may use the stream's workspace (as qmm).
+ * M == 0 or N == 0 is a no-op; K == 0 writes zeros.  Errors as for qmm().
+ */
+qmm_status qmm_nt(const void* x, const uint32_t* packed, const uint16_t* scales, const uint16_t* biases,
+                  void* y, int64_t M, int64_t N, int64_t K, int bits, int group, qmm_dtype dtype,
+                  void* stream);
+
+/*
+ * qmm_batched -- `batch` independent calls of qmm() (transpose != 0) or qmm_nt()
+ * (transpose == 0), problem i taking x + i*x_stride, y + i*y_stride and the weights at
+ * packed + i*w_stride, scales + i*s_stride, biases + i*s_stride.  Strides are in elements
+ * of each array (16-bit for x, y, scales, biases; 32-bit words for packed); a weight stride
+ * of 0 shares one weight matrix, and when x and y are then contiguous ([batch*M, K] and
+ * [batch*M, N]) the batch runs as one call over batch*M tokens.  Shapes, formats, alignment
+ * and errors as for qmm() / qmm_nt() per problem; the first failing problem's status is
+ * returned and later problems are not launched.
+ */
+qmm_status qmm_batched(const void* x, int64_t x_stride, const uint32_t* packed, int64_t w_stride,
+                       const uint16_t* scales, const uint16_t* biases, int64_t s_stride, void* y,
+                       int64_t y_stride, int64_t batch, int64_t M, int64_t N, int64_t K, int bits,
+                       int group, qmm_dtype dtype, int transpose, void* stream);
+
 /* Read and clear the current device's kernel error word (synchronizes with the device).
  * Bit 0: a tensor-core kernel block gave up waiting on one of its pipeline barriers (a wait
  * that should finish in microseconds ran for about two seconds).  That block then dropped
