@@ -51,6 +51,9 @@ namespace {
 using namespace sm100;
 
 constexpr int SK_ROWS = 128;                        // weight rows per tile (MMA M)
+constexpr int SK_MAXM = 128;                        // tokens of one pass at most (MMA N)
+constexpr int SK_XEXP_BYTES = SK_MAXM * 4;          // workspace: one exponent per token of a pass
+static_assert(SK_MAXM >= kSkMaxTokens, "per-token tables must cover a whole launch");
 constexpr int SK_KC = 256;                          // codes per stage and row
 constexpr int SK_NISS = 3;                          // MMA issuer warps (1..3)
 constexpr int SK_DQ0 = 1 + SK_NISS;                 // first dequantizer warp
@@ -143,7 +146,8 @@ __host__ __device__ inline SkLayout sk_layout(int bits, int mp, int sc, int xslo
     // verdict, MMAs drained
     off = L.bar_off + 8u * uint32_t(2 * 8 + 2 * SK_SS + 2 * 8 + 2 * 4 + 8);
     L.misc_off = align_up(off, 16);
-    off = L.misc_off + 3 * 64 * 4 + 16;  // amax[64], pow2E[64], escale[64], tmem holder, abort, verdict
+    // amax, pow2E and escale for every token of a pass (128 at most), tmem holder, abort, verdict
+    off = L.misc_off + 3 * SK_MAXM * 4 + 16;
     L.total = off;
     return L;
 }
@@ -423,6 +427,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     using F = SkFmt<BITS>;
     using TM = SkTm<MP>;
     constexpr int NACC = TM::NACC, NA = TM::NA;
+    static_assert(MP <= SK_MAXM, "the per-token tables hold SK_MAXM tokens");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int SC = p.sc, SX = p.sx;
@@ -445,9 +450,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     const uint32_t bar_verdict = bar_gather + 8;       // ... and this block's arrival is counted
     const uint32_t bar_mdone = bar_verdict + 8;        // every MMA issued has completed
     int* amax = reinterpret_cast<int*>(smem + L.misc_off);        // max|x_m| (float bits)
-    float* pow2E = reinterpret_cast<float*>(amax + 64);           // 2^E_m (epilogue)
-    float* escale = pow2E + 64;                                   // 2^-E_m (x staging)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(escale + 64);
+    float* pow2E = reinterpret_cast<float*>(amax + SK_MAXM);      // 2^E_m (epilogue)
+    float* escale = pow2E + SK_MAXM;                              // 2^-E_m (x staging)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(escale + SK_MAXM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* verdict = abort_flag + 1;
 
@@ -484,7 +489,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         mbar_init(bar_gather, SK_NDQ);
         mbar_init(bar_verdict, 1);
         mbar_init(bar_mdone, NACC);
-        for (int m = 0; m < 64; ++m) amax[m] = 0;
+        for (int m = 0; m < SK_MAXM; ++m) amax[m] = 0;
         *abort_flag = 0;
         *verdict = 0;
         fence_mbar_init();
@@ -634,7 +639,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         if (lane == 0) mbar_arrive(bar_emax);
         sk_wait(bar_emax, 0, abort_flag, p.timeout);
         if (j == 0) {
-            for (int m = lane; m < 64; m += 32) {
+            for (int m = lane; m < MP; m += 32) {  // every token column of the pass
                 float e2 = 1.f, es = 1.f;
                 if (m < p.M && p.is_bf16) {
                     int E;
@@ -1014,7 +1019,7 @@ __global__ void __launch_bounds__(256) sk_xprep_kernel(const uint16_t* __restric
                                                        uint8_t* __restrict__ xsum, int* __restrict__ xexp) {
     constexpr int UN = SkFmt<BITS>::UN, UPR = SK_KC / UN;
     __shared__ float red[8];
-    __shared__ float scl[64];
+    __shared__ float scl[SK_MAXM];  // 2^-E of each token row, indexed by the row (grid = M <= SK_MAXM)
     grid_dependents_launch();
     grid_dependency_wait();
     const int m = blockIdx.x;
@@ -1252,7 +1257,7 @@ size_t sk_ws_bytes(const SkConfig& c) {
     b = (b + 255) / 256 * 256;
     b += size_t(2 * c.grid) * size_t(c.mp) * SK_ROWS * 4;
     if (!c.x_staged) {
-        b += 256;                                            // exponents
+        b += SK_XEXP_BYTES;                                  // exponents
         b += size_t(c.S) * size_t(c.mp) * (512 + 32);        // x tiles and sums
     }
     return b;
@@ -1339,7 +1344,7 @@ cudaError_t launch_sk_items(const QmmArgs& a, const SkItem* items, int nitems, c
     off += size_t(2 * c.grid) * size_t(c.mp) * SK_ROWS * 4;
     if (!c.x_staged) {
         p.xexp = reinterpret_cast<const int*>(w + off);
-        off += 256;
+        off += SK_XEXP_BYTES;
         p.xt = reinterpret_cast<const uint16_t*>(w + off);
         off += size_t(c.S) * size_t(c.mp) * 512;
         p.xsum = reinterpret_cast<const uint32_t*>(w + off);

@@ -44,6 +44,16 @@ def check_close(y_gpu: torch.Tensor, y_ref: np.ndarray, dtype: torch.dtype, what
     amax = float(np.max(np.abs(y_ref))) if y_ref.size else 0.0
     worst = float(np.max(np.abs(diff))) if diff.size else 0.0
     bound = 1e-2 * amax + 1e-3
-    assert rel <= REL_FRO[dtype], f"{what}: rel Frobenius {rel:.3e} > {REL_FRO[dtype]:.1e}"
-    assert worst <= bound, f"{what}: max |diff| {worst:.3e} > {bound:.3e}"
+    if rel > REL_FRO[dtype] or worst > bound:
+        # where the error sits (a few elements, a token, a row block) tells a race from a
+        # rounding difference
+        bad = np.argwhere(np.abs(diff) > bound)
+        top = np.argsort(np.abs(diff), axis=None)[::-1][:5]
+        where = [(int(i // diff.shape[-1]), int(i % diff.shape[-1]), float(diff.flat[i]), float(y_ref.flat[i]))
+                 for i in top] if diff.ndim == 2 else []
+        detail = f"; {len(bad)} elements over the bound; worst (m, n, diff, ref): {where}"
+    else:
+        detail = ""
+    assert rel <= REL_FRO[dtype], f"{what}: rel Frobenius {rel:.3e} > {REL_FRO[dtype]:.1e}{detail}"
+    assert worst <= bound, f"{what}: max |diff| {worst:.3e} > {bound:.3e}{detail}"
     return {"rel_fro": rel, "max_abs": worst}
