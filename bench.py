@@ -568,8 +568,9 @@ def run_ours(args, rank, world):
 def run_e2e(wl, weights, plans, dev, steps):
     """Each step through the Python API: the step's inputs (x for each M) go from pinned host
     memory to the device, every call of the step runs, and every output comes back to pinned
-    host memory; the weights stay resident, as a model's do.  The output of one M goes back on
-    a copy stream while the calls of the next M run."""
+    host memory before the step ends; the weights stay resident, as a model's do.  The output
+    of one M goes back on a copy stream while the calls of the next M run, largest M first, so
+    that only the smallest output's copy is left after the last call."""
     import bit_quantized_gemm_qmm_b200 as q
     from bit_quantized_gemm_qmm_b200.inputs import x_input
     S = len(weights)
@@ -585,7 +586,7 @@ def run_e2e(wl, weights, plans, dev, steps):
     def one_step():
         for M in BENCH_MS:
             dx[M].copy_(hx[M], non_blocking=True)
-        for M in BENCH_MS:
+        for M in sorted(BENCH_MS, reverse=True):
             for (P, S_, B), y in zip(weights, outs[M]):
                 q.qmm(dx[M], P, S_, B, wl.bits, wl.group, out=y, plan=plans[M])
             done[M].record(stream)

@@ -201,9 +201,11 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
         // the streaming kernel up to M = 8, and up to 16 while staging x still leaves room
         // for a 4-stage ring (or for all the stages a block streams) without splitting K
         // further than the tile count asks for; on an unsplit grid, whose blocks stream back
-        // to back, 96 KB in flight suffice (3 stages of 4- or 8-bit codes, 4 of 6-bit)
-        const int ring_need =
-            (st_ok && stc.split == 1) ? (96 * 1024 + stc.stage_bytes - 1) / std::max(1, stc.stage_bytes) : 4;
+        // to back, and wherever x streams with the codes, 96 KB in flight suffice (3 stages of
+        // 4- or 8-bit codes, 4 of 6-bit)
+        const int ring_need = (st_ok && (stc.split == 1 || stc.xstream))
+                                  ? (96 * 1024 + stc.stage_bytes - 1) / std::max(1, stc.stage_bytes)
+                                  : 4;
         // 6-bit codes are dequantized per element in the streaming kernel; with two token tiles
         // that loses to the tensor-core kernel on the large matrices (measured)
         const bool st_mt2_ok = !(bits == 6 && N * K >= (int64_t(1) << 25));
@@ -511,9 +513,12 @@ qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t 
     a.group = group;
     a.is_bf16 = dtype == QMM_BF16;
     // up to 16 tokens: the streaming kernel over the matrices' tiles, numbered one after
-    // another (the measured choice: it beats separate calls, whose launches do not overlap);
-    // above, or when forced, the even-split kernel
-    if (pl.kernel == QMM_KERNEL_STREAM || (pl.kernel == QMM_KERNEL_AUTO && M <= 16)) {
+    // another (the measured choice: it beats separate calls, whose launches do not overlap),
+    // except at 9-16 tokens over at least one tile per SM (a persistent grid with two token
+    // tiles and a long tail lost to the matrices' own calls: gate/up at 16 tokens, 1455
+    // against 1838 GB/s); above, or when forced, the even-split kernel
+    const bool own_calls = pl.kernel == QMM_KERNEL_AUTO && (M > 16 || (M > 8 && tiles >= kNumSM));
+    if (pl.kernel == QMM_KERNEL_STREAM || (pl.kernel == QMM_KERNEL_AUTO && !own_calls)) {
         if (pl.kernel == QMM_KERNEL_STREAM && (pl.split < 0 || pl.split > 8))
             return fail(QMM_ERR_INVALID_ARG, "split=%d (the streaming kernel splits K 1..8 ways, 0 = auto)", pl.split);
         StreamConfig sc = {};
@@ -528,7 +533,7 @@ qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t 
             return fail(QMM_ERR_UNSUPPORTED, "the streaming kernel takes 1 <= M <= 16 and whole stages and scale "
                         "blocks of K");
     }
-    if (pl.kernel == QMM_KERNEL_AUTO && M > 16) {
+    if (own_calls) {
         // above 16 tokens one even-split launch over the group measured slower than the
         // matrices' own default plans back to back (the tensor-core and warp-tile kernels
         // are not grouped), so the default takes those

@@ -82,14 +82,14 @@ struct StLayout {
 // x and its group sums are staged for the M real token rows only (reads for token rows >= M
 // are redirected to row M-1: they feed accumulator columns that are never stored).
 // xs (x streamed): instead of x for the whole K range, each ring slot carries, after the
-// stage's codes, that stage's x tile [16 token rows][xrs chunks] (written once per call by
+// stage's codes, that stage's x tile [8 * mt token rows][xrs chunks] (written once per call by
 // st_xprep_kernel and brought in by the same barrier as the codes).
 __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split, int ncw,
                                               int mrows, bool xs = false) {
     StLayout L;
     L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 256));  // 24 or 32 KB
     L.xrs = uint32_t((xs ? st_stage_codes(bits) : kslice) / 8 + x_pad(bits, bits != 6));  // chunks per x row
-    L.xtile = xs ? 16u * L.xrs * 16u : 0u;
+    L.xtile = xs ? uint32_t(8 * mt) * L.xrs * 16u : 0u;  // 8 token rows per token tile
     L.slot = (L.w_stage + L.xtile + 1023) / 1024 * 1024;      // codes stay 1024-byte aligned (swizzle)
     L.sb_off = uint32_t(ring) * L.slot;
     L.sb_slot = uint32_t(2 * ST_ROWS * (st_block_codes(bits, group) / group) * 2);  // scales + biases
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ float s_red[NCW];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    static_assert(!XS || (BITS != 6 && MT == 2), "x is streamed for 9-16 tokens at 4 and 8 bits");
+    static_assert(!XS || BITS != 6, "x is streamed at 4 and 8 bits");
     const StLayout& L = p.lay;
     const int S = p.ring;
     const uint32_t sbase = smem_addr(smem);
@@ -527,8 +527,14 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         if constexpr (XS) {
             // the x tiles stream in with the codes; the group sums and exponents come from the
             // x pass of this call
-            for (int e = threadIdx.x; e < p.M * int(L.gpad); e += NCW * 32)
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(e) * 4u), "r"(__ldg(p.xgw + e)));
+            // the x pass's rows of group sums span the whole K range (stride gst); this block's
+            // groups start at kb / group
+            const int gst = (p.K / p.group + 7) / 8 * 8, g0 = kb >> p.gshift, gpad = int(L.gpad);
+            for (int e = threadIdx.x; e < p.M * gpad; e += NCW * 32) {
+                const int m = e / gpad, gi = g0 + (e - m * gpad);
+                const uint32_t v = gi < gst ? __ldg(p.xgw + m * gst + gi) : 0u;
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(e) * 4u), "r"(v));
+            }
             if (threadIdx.x < 16) ysc[threadIdx.x] = int(threadIdx.x) < p.M ? exp2i(__ldg(p.xexp + threadIdx.x)) : 1.f;
         } else {
             const int E = p.is_bf16 ? bf16_exponent<NCW>(p, kb, ke, s_red) : 0;
@@ -890,13 +896,14 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 }
 
 // ---------------------------------------------------------------- x pass (streamed x)
-// One block per token row: the row's fp16 x tiles of every stage ([stage][16 rows][xrs
+// One block per token row: the row's fp16 x tiles of every stage ([stage][rows = 8 * MT][xrs
 // chunks]; each 8-code unit at its natural chunk, its codes in perm_nat order), its group
-// sums as (hi, lo) fp16 times 2^-7 ([row][gpad], zero past the last group) and its exponent:
+// sums as (hi, lo) fp16 times 2^-7 ([row][gst], gst = the groups of the whole K range rounded
+// up to 8, zero past the last group) and its exponent:
 // bf16 rows are scaled by 2^-E with max|x| * 2^-E < 2^15 (E >= 0), fp16 rows are not.
 template <int BITS>
 __global__ void __launch_bounds__(256) st_xprep_kernel(const uint16_t* __restrict__ x, int K, int is_bf16, int group,
-                                                       int xrs, int gpad, uint8_t* __restrict__ xt,
+                                                       int rows, int xrs, int gst, uint8_t* __restrict__ xt,
                                                        uint32_t* __restrict__ xgw, int* __restrict__ xexp) {
     constexpr int CPS = (BITS == 4 ? 512 : 256) / 8;  // 16-byte chunks (8-code units) per stage
     __shared__ float red[8];
@@ -957,16 +964,16 @@ __global__ void __launch_bounds__(256) st_xprep_kernel(const uint16_t* __restric
             const float X = sum * 0.0078125f;
             const __half hi = __float2half_rn(X);
             const __half lo = __float2half_rn(X - __half2float(hi));
-            xgw[m * gpad + u / upg] = uint32_t(__half_as_ushort(hi)) | (uint32_t(__half_as_ushort(lo)) << 16);
+            xgw[m * gst + u / upg] = uint32_t(__half_as_ushort(hi)) | (uint32_t(__half_as_ushort(lo)) << 16);
         }
         uint4 o;
         uint32_t* ov = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
         for (int i = 0; i < 4; ++i) ov[i] = f32x2_to_f16x2(f[perm_nat<BITS>(2 * i)], f[perm_nat<BITS>(2 * i + 1)]);
         const int st = u / CPS, ch = u - st * CPS;
-        *reinterpret_cast<uint4*>(xt + ((size_t(st) * 16 + m) * xrs + ch) * 16) = o;
+        *reinterpret_cast<uint4*>(xt + ((size_t(st) * rows + m) * xrs + ch) * 16) = o;
     }
-    for (int gi = K / group + int(threadIdx.x); gi < gpad; gi += 256) xgw[m * gpad + gi] = 0u;
+    for (int gi = K / group + int(threadIdx.x); gi < gst; gi += 256) xgw[m * gst + gi] = 0u;
     if (threadIdx.x == 0) xexp[m] = E;
 }
 
@@ -976,8 +983,6 @@ template <int BITS, int MT, bool XS>
 StKernelFn pick_stream_g(int group) {
     if constexpr (BITS == 6) {
         return XS ? nullptr : qmm_stream_kernel<6, MT, 16, 0, false>;
-    } else if constexpr (XS && MT != 2) {
-        return nullptr;
     } else {
         if (group == 32) return qmm_stream_kernel<BITS, MT, 16, 32, XS>;
         if (group == 64) return qmm_stream_kernel<BITS, MT, 16, 64, XS>;
@@ -990,9 +995,8 @@ StKernelFn pick_stream_g(int group) {
 StKernelFn pick_stream(int bits, int mt, int ncw, int group, bool xs) {
     if (ncw != 16 || (mt != 1 && mt != 2)) return nullptr;
     if (xs) {
-        if (mt != 2) return nullptr;
-        if (bits == 4) return pick_stream_g<4, 2, true>(group);
-        if (bits == 8) return pick_stream_g<8, 2, true>(group);
+        if (bits == 4) return mt == 1 ? pick_stream_g<4, 1, true>(group) : pick_stream_g<4, 2, true>(group);
+        if (bits == 8) return mt == 1 ? pick_stream_g<8, 1, true>(group) : pick_stream_g<8, 2, true>(group);
         return nullptr;
     }
     if (bits == 4) return mt == 1 ? pick_stream_g<4, 1, false>(group) : pick_stream_g<4, 2, false>(group);
@@ -1011,6 +1015,7 @@ int cdiv(int64_t a, int64_t b) { return int((a + b - 1) / b); }
 int rup(int64_t a, int64_t b) { return int((a + b - 1) / b * b); }
 
 constexpr int kNumSM = 148;
+constexpr int64_t kXsStagedMax = 64 * 1024;  // staged x (bytes) above which 9-16 tokens stream x
 constexpr size_t kMaxSmem = 226 * 1024;  // dynamic, per block (static shared memory is tiny)
 
 size_t st_smem(int bits, int mt, int ring, int kslice, int group, int split, int ncw, int mrows, bool xs) {
@@ -1052,9 +1057,14 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
     }
     split = std::max(1, std::min(8, split));
     const int split0 = split;
-    // 9-16 tokens on a persistent grid: x for the whole K range would take most of shared
-    // memory (64 KB per 2048 codes), so it streams with the codes instead (4- and 8-bit)
-    const bool xs_want = bits != 6 && M > 8 && split == 1 && T >= kNumSM;
+    // x streams with the codes instead of being staged whole per block (4- and 8-bit): at
+    // 9-16 tokens on a persistent grid, or wherever x for a block's K range would take more
+    // than 64 KB of shared memory; at 1-8 tokens on an unsplit grid of fewer tiles than SMs
+    // (each block takes one whole tile) where its x would take more than 32 KB, an
+    // unamortized prologue otherwise (measured: 8-bit gate/up +15-23% at 6-8 tokens; at 4
+    // tokens, 32 KB, even at 8 bits and 5% slower at 4; on K-split grids the x pass costs
+    // more than it saves, down -8-13%)
+    const bool xs_bits = bits != 6;
     for (;; ++split) {
         const int kslice = rup(cdiv(K, split), unit);
         const int sp = cdiv(K, kslice);
@@ -1066,7 +1076,9 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         // 16 consumer warps measured faster than 8 on every configuration of the sweep (the
         // 8-warp blocks fit two to an SM, but that bought no overlap between calls)
         const int ncw = 16;
-        const bool xs = xs_want && sp == 1;
+        const int64_t xbytes = int64_t(M) * kslice * 2;  // x of a block's K range, staged whole
+        const bool xs = xs_bits && (M > 8 ? ((sp == 1 && T >= kNumSM) || xbytes > kXsStagedMax)
+                                          : (sp == 1 && T < kNumSM && xbytes > kXsStagedMax / 2));
         while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M), xs) > kMaxSmem) --ring;
         const bool fits = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M), xs) <= kMaxSmem;
         if (!fits || (ring < std::min(want, 3) && split < 8)) {
@@ -1233,13 +1245,14 @@ cudaError_t launch_stream_items(const QmmArgs& a, const SkItem* items, int nitem
     p.xexp = nullptr;
     const StLayout L = st_layout(a.bits, mt, c.ring, c.kslice, a.group, c.split, c.ncw, int(a.M), c.xstream);
     p.lay = L;
+    const int gst = int((a.K / a.group + 7) / 8 * 8);  // streamed x: group sums a row (the whole K range)
     if (c.tper > 0 || c.xstream) {
         // workspace: tail arrival words [T - dp_tiles], tail partial sums [2 * grid][8 * mt][128];
-        // streamed x: tiles [stages][16][xrs chunks], group sums [M][gpad], exponents [M]
+        // streamed x: tiles [stages][8 * mt][xrs chunks], group sums [M][gst], exponents [M]
         const size_t cbytes = c.tper > 0 ? (size_t(p.T - c.dp_tiles) * 8 + 255) / 256 * 256 : 0;
         const size_t pbytes = c.tper > 0 ? size_t(2 * c.grid_x) * 8 * mt * ST_ROWS * 4 : 0;
         const size_t xtbytes = c.xstream ? size_t(a.K / ks_for(a.bits)) * L.xtile : 0;
-        const size_t xgbytes = c.xstream ? (size_t(a.M) * L.gpad * 4 + 255) / 256 * 256 : 0;
+        const size_t xgbytes = c.xstream ? (size_t(a.M) * gst * 4 + 255) / 256 * 256 : 0;
         void* ws = nullptr;
         cudaError_t e = split_workspace(stream, cbytes + pbytes + xtbytes + xgbytes + (c.xstream ? 256 : 0), &ws);
         if (e != cudaSuccess) return e;
@@ -1293,10 +1306,10 @@ cudaError_t launch_stream_items(const QmmArgs& a, const SkItem* items, int nitem
         uint8_t* xt = const_cast<uint8_t*>(p.xt);
         uint32_t* xgw = const_cast<uint32_t*>(p.xgw);
         int* xexp = const_cast<int*>(p.xexp);
-        e = a.bits == 4 ? cudaLaunchKernelEx(&xc, st_xprep_kernel<4>, a.x, int(a.K), a.is_bf16, a.group, int(L.xrs),
-                                             int(L.gpad), xt, xgw, xexp)
-                        : cudaLaunchKernelEx(&xc, st_xprep_kernel<8>, a.x, int(a.K), a.is_bf16, a.group, int(L.xrs),
-                                             int(L.gpad), xt, xgw, xexp);
+        e = a.bits == 4 ? cudaLaunchKernelEx(&xc, st_xprep_kernel<4>, a.x, int(a.K), a.is_bf16, a.group, 8 * mt,
+                                             int(L.xrs), gst, xt, xgw, xexp)
+                        : cudaLaunchKernelEx(&xc, st_xprep_kernel<8>, a.x, int(a.K), a.is_bf16, a.group, 8 * mt,
+                                             int(L.xrs), gst, xt, xgw, xexp);
         if (e != cudaSuccess) return e;
     }
     return cudaLaunchKernelEx(&cfg, fn, maps, p);

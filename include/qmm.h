@@ -175,10 +175,12 @@ typedef struct {
  * section "Architectural Differences: Stock MLX vs. NAX Verify", puts the small verify
  * calls' cost in per-call dispatch overhead; one launch over the layer's matrices pays it
  * once and spreads all their weight bytes over the SMs.  Up to 16 tokens the launch is the
- * streaming kernel's (plus its x pass for 9-16 tokens on a persistent grid).  Above 16 tokens
- * QMM_KERNEL_AUTO runs each matrix's own default plan instead (separate launches: one
- * even-split launch over the group measured slower there), and QMM_KERNEL_SK forces the one
- * even-split launch (plus its x pass when x is staged in the workspace).
+ * streaming kernel's (plus its x pass where x streams), except that at 9-16 tokens over at
+ * least 148 tiles in all (a persistent grid) QMM_KERNEL_AUTO runs each matrix's own default
+ * plan (separate launches measured faster there).  Above 16 tokens QMM_KERNEL_AUTO runs each
+ * matrix's own default plan too (one even-split launch over the group measured slower), and
+ * QMM_KERNEL_SK forces the one even-split launch (plus its x pass when x is staged in the
+ * workspace).
  * Each item must have a multiple of 8 groups per row and a 16-byte multiple of packed bytes
  * per row, with packed, scales, biases, x and y 16-byte aligned; 1 <= M <= 64; else
  * QMM_ERR_UNSUPPORTED and nothing is launched.  `plan` may be NULL or name QMM_KERNEL_AUTO,

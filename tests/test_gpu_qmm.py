@@ -170,6 +170,33 @@ def test_bf16_large_activations_do_not_overflow(oracle_mod):
         check_close(y[m:m + 1], ref[m:m + 1], torch.bfloat16, f"row {m}")
 
 
+@pytest.mark.parametrize("N,K,bits,group,M,kernel,spread", [
+    (4096, 4096, 4, 64, 20, q.KERNEL_TC, (2.0e5, 1e-3)),     # per-token exponents (x kernel)
+    (4096, 4096, 4, 64, 40, q.KERNEL_TC, (2.0e5, 1e-3)),
+    (19200, 2048, 4, 64, 12, q.KERNEL_STREAM, (2.0e5, 1e-3)),  # streamed x: per-token exponents
+    (14336, 4096, 8, 128, 6, q.KERNEL_STREAM, (2.0e5, 1e-3)),
+    (4096, 4096, 4, 64, 5, q.KERNEL_STREAM, (1.0e3, 1e-2)),   # staged x: one exponent a block
+    (4096, 4096, 4, 64, 20, q.KERNEL_MMA, (1.0e3, 1e-2)),
+])
+def test_bf16_rows_of_very_different_magnitude(oracle_mod, N, K, bits, group, M, kernel, spread):
+    """One bf16 row far larger than the others, one far smaller, each row checked on its own.
+    Paths that scale x per token (the tensor-core kernel's x kernel, streamed x) keep every
+    row's fp16 precision even 2e8 apart; paths that stage x whole take one exponent for the
+    block's tokens, which holds rows 1e5 apart (a row more than about 2^24 below the block's
+    largest would reach fp16's subnormals there)."""
+    w = w_input(N, K, torch.bfloat16, 4, 0.02)
+    x = randn((M, K), 1.0, torch.bfloat16, 6)
+    x[0] *= spread[0]
+    x[M - 1] *= spread[1]
+    op, os_, ob = oracle_quantize(oracle_mod, w, bits, group)
+    P, S, B = to_device_weights(op, os_, ob)
+    y = q.qmm(x.cuda(), P, S, B, bits, group, plan=q.make_plan(kernel=kernel))
+    torch.cuda.synchronize()
+    ref = oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group)
+    for m in range(M):
+        check_close(y[m:m + 1], ref[m:m + 1], torch.bfloat16, f"kernel {kernel} M={M} row {m}")
+
+
 @pytest.mark.parametrize("split", [1, 2, 3, 5, 8, 16])
 @pytest.mark.parametrize("warps", [4, 8])
 def test_forced_plans(oracle_mod, split, warps):

@@ -192,3 +192,34 @@ def test_streamed_x(oracle_mod, M, bits, group):
     ref = oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group)
     for m in range(M):
         check_close(y[m:m + 1], ref[m:m + 1], torch.bfloat16, f"streamed x, row {m}")
+
+
+@pytest.mark.parametrize("N,K,bits,group,M", [
+    (4096, 14336, 4, 64, 9),    # down: 32 tiles, K split over clusters of 4; x for a block's K
+    (4096, 14336, 4, 64, 16),   # range would take more than 64 KB, so it streams
+    (4096, 14336, 8, 128, 12),
+    (14336, 4096, 8, 128, 5),   # gate/up: 112 tiles, unsplit, fewer blocks than SMs: x streams
+    (14336, 4096, 8, 128, 8),   # from 3 tokens (one token tile up to 8)
+    (14336, 4096, 8, 128, 9),
+    (14336, 4096, 8, 128, 16),
+])
+def test_streamed_x_split_and_partial_grids(oracle_mod, N, K, bits, group, M):
+    """x streams wherever staging it whole would crowd the ring (9-16 tokens) or be a long
+    prologue of a one-tile block (3-8 tokens on unsplit grids, one token tile): on K-split
+    grids (each block reads its K range's x tiles and group sums from the x pass's whole-K
+    rows, partial sums added over the cluster) and on unsplit grids of fewer tiles than SMs.
+    bf16 rows of very different magnitudes (per-token exponents), each checked on its own."""
+    pd = q.plan_default(M, N, K, bits, group, torch.bfloat16)
+    assert pd.kernel == q.KERNEL_STREAM, pd.as_dict()
+    x = randn((M, K), 1.0, torch.bfloat16, 12)
+    x[1] *= 2.0e5
+    x[M - 1] *= 1e-3
+    w = w_input(N, K, torch.bfloat16, 3, 0.02)
+    op, os_, ob = oracle_quantize(oracle_mod, w, bits, group)
+    P, S, B = to_device_weights(op, os_, ob)
+    y = q.qmm(x.cuda(), P, S, B, bits, group)
+    torch.cuda.synchronize()
+    assert q.device_errors() == 0
+    ref = oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group)
+    for m in range(M):
+        check_close(y[m:m + 1], ref[m:m + 1], torch.bfloat16, f"streamed x split={pd.split}, row {m}")
