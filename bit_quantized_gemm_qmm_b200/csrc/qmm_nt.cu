@@ -13,7 +13,9 @@
 // word, 16 of a 6-bit word triple) for a range of K rows.  Per row it forms x[m,k] * s once per
 // token (exact in fp32: an 11-bit times an 11-bit significand) and adds that times each code
 // into its fp32 sums; the bias term sum_k x[m,k] * b[k, j] is the same for all the thread's
-// codes (they lie in one group) and is added at the end.  Tokens are taken TM at a time; K is
+// codes (they lie in one group) and is added at the end.  Tokens are taken TM at a time (TM
+// the smallest of 1, 2, 4, 8 that covers M, at most 8, 4 at 6 bits: FMAs on padded tokens would
+// make small-M calls FMA-bound); K is
 // split over grid.y so the grid fills the GPU, and the split sums are added in split order
 // by a second kernel (deterministic).  Coalescing: consecutive threads read consecutive units
 // of a row.  This is the CUDA-core path of the less common form; it does not use the tensor
@@ -29,15 +31,15 @@ namespace {
 
 constexpr int NT_THREADS = 128;
 
-template <int BITS> struct NtFmt {
+template <int BITS, int TM_> struct NtFmt {
     static constexpr int CPU = BITS == 6 ? 16 : 32 / BITS;  // codes per packed unit
     static constexpr int WPU = BITS == 6 ? 3 : 1;          // words per packed unit
-    static constexpr int TM = BITS == 6 ? 4 : 8;           // tokens a pass
-    static constexpr int RU = BITS == 6 ? 4 : 8;           // rows whose loads are in flight together
+    static constexpr int TM = TM_;                         // tokens a pass
+    static constexpr int RU = BITS == 6 ? 4 : 8;            // rows whose loads are in flight together
 };
 
 template <int BITS>
-__device__ __forceinline__ uint32_t nt_code(const uint32_t (&w)[NtFmt<BITS>::WPU], int i) {
+__device__ __forceinline__ uint32_t nt_code(const uint32_t (&w)[BITS == 6 ? 3 : 1], int i) {
     if constexpr (BITS == 4) {
         return (w[0] >> (4 * i)) & 0xFu;
     } else if constexpr (BITS == 8) {
@@ -61,7 +63,7 @@ __device__ __forceinline__ uint16_t nt_round(float v, int is_bf16) {
 
 // grid.x: column blocks of NT_THREADS units; grid.y: K slices of `krange` rows.  With one
 // slice y is written directly, else part[slice][m][n] (fp32).
-template <int BITS>
+template <int BITS, int TM_>
 __global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __restrict__ x,
                                                             const uint32_t* __restrict__ packed,
                                                             const uint16_t* __restrict__ scales,
@@ -69,7 +71,7 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __re
                                                             uint16_t* __restrict__ y, float* __restrict__ part,
                                                             int M, int K, int N, int gshift, int is_bf16,
                                                             int krange) {
-    using F = NtFmt<BITS>;
+    using F = NtFmt<BITS, TM_>;
     constexpr int CPU = F::CPU, WPU = F::WPU, TM = F::TM, RU = F::RU;
     __shared__ float xs[TM][64];  // x of the current tokens, 64 rows of K at a time
     const int units = N / CPU;
@@ -168,6 +170,19 @@ __global__ void __launch_bounds__(256) qmm_nt_reduce(const float* __restrict__ p
 
 constexpr int kNtSMs = 148;
 
+template <int BITS>
+void launch_nt_tm(int tm, dim3 grid, cudaStream_t stream, const QmmArgs& a, float* part, int gshift, int krange) {
+#define QMM_NT_LAUNCH(T)                                                                                   \
+    qmm_nt_kernel<BITS, T><<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, \
+                                                           int(a.M), int(a.K), int(a.N), gshift, a.is_bf16, krange)
+    if (tm == 1) QMM_NT_LAUNCH(1);
+    else if (tm == 2) QMM_NT_LAUNCH(2);
+    else if constexpr (BITS == 6) QMM_NT_LAUNCH(4);
+    else if (tm == 4) QMM_NT_LAUNCH(4);
+    else QMM_NT_LAUNCH(8);
+#undef QMM_NT_LAUNCH
+}
+
 }  // namespace
 
 cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
@@ -191,15 +206,15 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     int gshift = 0;
     while ((1 << gshift) < a.group) ++gshift;
     const dim3 grid(unsigned(cblocks), unsigned(S), 1);
+    // tokens a pass: the smallest of 1, 2, 4, 8 (4 at 6 bits) that covers M
+    const int tmax = a.bits == 6 ? 4 : 8;
+    const int tm = a.M >= tmax ? tmax : (a.M > 2 ? 4 : int(a.M));
     if (a.bits == 4)
-        qmm_nt_kernel<4><<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M),
-                                                          int(a.K), int(a.N), gshift, a.is_bf16, krange);
+        launch_nt_tm<4>(tm, grid, stream, a, part, gshift, krange);
     else if (a.bits == 6)
-        qmm_nt_kernel<6><<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M),
-                                                          int(a.K), int(a.N), gshift, a.is_bf16, krange);
+        launch_nt_tm<6>(tm, grid, stream, a, part, gshift, krange);
     else
-        qmm_nt_kernel<8><<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M),
-                                                          int(a.K), int(a.N), gshift, a.is_bf16, krange);
+        launch_nt_tm<8>(tm, grid, stream, a, part, gshift, krange);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || S == 1) return e;
     const int64_t MN = a.M * a.N;
