@@ -204,12 +204,10 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- our arm
-def launches_per_call(plan) -> int:
-    """Kernels one call launches: the tensor-core kernels with x staged in the workspace run a
-    small x kernel first."""
-    if plan.kernel == 2 or (plan.kernel == 4 and plan.split == 2):
-        return 2
-    return 1
+def launches_per_call(q, wl, M: int, plan) -> int:
+    """Kernels one call launches, from the library (C ABI qmm_plan_launches): the main kernel
+    and the small x kernel where x is prepared in the workspace."""
+    return q.plan_launches(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype, plan)
 
 
 def make_weights(q, wl, dev):
@@ -449,7 +447,7 @@ def run_ours(args, rank, world):
     calls_per_step = len(BENCH_MS) * nsets
     step_wbytes = wbytes * calls_per_step
     step_algo_bytes = sum((wbytes + 2 * M * wl.K + 2 * M * wl.N) * len(weights) for M in BENCH_MS)
-    launches_per_step = sum(launches_per_call(plans[M]) * len(weights) for M in BENCH_MS)
+    launches_per_step = sum(launches_per_call(q, wl, M, plans[M]) * len(weights) for M in BENCH_MS)
 
     def step(Ms=BENCH_MS):
         for M in Ms:

@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.qmm_ex.restype = I
     L.qmm_plan_default.argtypes = [I64, I64, I64, I, I, U, ctypes.POINTER(Plan)]
     L.qmm_plan_default.restype = I
+    L.qmm_plan_launches.argtypes = [I64, I64, I64, I, I, U, ctypes.POINTER(Plan), ctypes.POINTER(ctypes.c_int32)]
+    L.qmm_plan_launches.restype = I
     L.qmm_status_string.argtypes = [I]
     L.qmm_status_string.restype = ctypes.c_char_p
     L.qmm_last_error.argtypes = []
@@ -186,6 +188,15 @@ def plan_default(M: int, N: int, K: int, bits: int, group: int, dtype: torch.dty
     p = Plan()
     _check(lib().qmm_plan_default(M, N, K, bits, group, _dtype_code(dtype), ctypes.byref(p)))
     return p
+
+
+def plan_launches(M: int, N: int, K: int, bits: int, group: int, dtype: torch.dtype, plan: Plan | None = None) -> int:
+    """Kernel launches one qmm() call of this shape makes (C ABI qmm_plan_launches): the main
+    kernel, plus the x kernel where x is prepared in the workspace, over every chunk of M."""
+    n = ctypes.c_int32(0)
+    _check(lib().qmm_plan_launches(M, N, K, bits, group, _dtype_code(dtype), ctypes.byref(plan) if plan else None,
+                                   ctypes.byref(n)))
+    return n.value
 
 
 def make_plan(kernel: int = KERNEL_AUTO, split: int = 0, warps: int = 0, flags: int = PLAN_PDL) -> Plan:

@@ -338,6 +338,36 @@ qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group
                         reinterpret_cast<const void*>(16), plan, nullptr);
 }
 
+qmm_status qmm_plan_launches(int64_t M, int64_t N, int64_t K, int bits, int group, qmm_dtype dtype,
+                             const qmm_plan* plan, int32_t* launches) {
+    qmm_status s = check_format(N, K, bits, group);
+    if (s != QMM_OK) return s;
+    if (dtype != QMM_F16 && dtype != QMM_BF16) return fail(QMM_ERR_INVALID_ARG, "dtype=%d", int(dtype));
+    if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M");
+    if (M > kMaxTotalM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %lld", (long long)M, (long long)kMaxTotalM);
+    if (!launches) return fail(QMM_ERR_INVALID_ARG, "launches is null");
+    *launches = 0;
+    if (M == 0 || N == 0 || K == 0) return QMM_OK;  // nothing, or a memset
+    // the chunks qmm_ex cuts M into, each with its own plan
+    const int64_t nch = (M + kSkMaxTokens - 1) / kSkMaxTokens;
+    int64_t m0 = 0;
+    int32_t n = 0;
+    for (int64_t i = 0; i < nch; ++i) {
+        const int64_t mc = (M - m0) / (nch - i);
+        Resolved r;
+        s = resolve_plan(mc, N, K, bits, group, plan, reinterpret_cast<const void*>(16),
+                         reinterpret_cast<const void*>(16), nullptr, &r);
+        if (s != QMM_OK) return s;
+        n += r.kernel == QMM_KERNEL_STREAM ? 1 + (r.st.xstream ? 1 : 0)
+             : r.kernel == QMM_KERNEL_TC   ? 2
+             : r.kernel == QMM_KERNEL_SK   ? 1 + (r.sk.x_staged ? 0 : 1)
+                                           : 1;
+        m0 += mc;
+    }
+    *launches = n;
+    return QMM_OK;
+}
+
 qmm_status qmm_ex(const void* x, const uint32_t* packed, const uint16_t* scales,
                   const uint16_t* biases, void* y, int64_t M, int64_t N, int64_t K, int bits,
                   int group, qmm_dtype dtype, const qmm_plan* plan, void* stream) {

@@ -151,6 +151,17 @@ typedef struct {
 qmm_status qmm_plan_default(int64_t M, int64_t N, int64_t K, int bits, int group,
                             qmm_dtype dtype, qmm_plan* plan);
 
+/*
+ * qmm_plan_launches -- how many kernel launches a qmm()/qmm_ex() call of this shape makes with
+ * `plan` (NULL = the default plan), for 16-byte aligned scales and biases: the main kernel,
+ * plus the small x kernel where x is prepared in the workspace (streamed x, the tensor-core
+ * kernel, the even-split kernel above its shared-memory x), over every chunk of M > 128.
+ * 0 for M == 0, N == 0 or K == 0 (a zero fill).  *launches is written on QMM_OK; the status
+ * and errors are those of qmm_plan_default / qmm_ex for the same arguments.
+ */
+qmm_status qmm_plan_launches(int64_t M, int64_t N, int64_t K, int bits, int group, qmm_dtype dtype,
+                             const qmm_plan* plan, int32_t* launches);
+
 /* qmm() with an explicit plan (NULL = the default plan).  Fields left at 0 take the default
  * (kernel AUTO, split chosen by the table, ...).  An invalid plan returns
  * QMM_ERR_INVALID_ARG and launches nothing. */

@@ -181,3 +181,22 @@ def test_default_plan_for_every_workload_and_m(L):
             assert 1 <= p.split <= 16, (name, M, p.as_dict())
             assert p.kernel != q.KERNEL_STREAM or M <= 16, (name, M)
             assert q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype).as_dict() == p.as_dict()
+
+
+def test_plan_launches(L):
+    """Kernel launches per call, as the library counts them: the main kernel and the x kernel
+    where x is prepared in the workspace, summed over the chunks of M > 128."""
+    torch = __import__("torch")
+    bf16, f16 = torch.bfloat16, torch.float16
+    assert q.plan_launches(1, 151936, 4096, 4, 64, bf16) == 1    # streaming, x staged
+    assert q.plan_launches(16, 151936, 4096, 4, 64, bf16) == 2   # + the x pass (x streamed)
+    assert q.plan_launches(32, 151936, 4096, 4, 64, bf16) == 2   # tensor-core kernel + its x kernel
+    assert q.plan_launches(32, 4096, 14336, 4, 64, bf16) == 2
+    assert q.plan_launches(1, 4096, 4096, 4, 64, f16) == 1
+    assert q.plan_launches(6, 14336, 4096, 8, 128, bf16) == 2    # one tile a block: x streamed
+    assert q.plan_launches(4, 14336, 4096, 8, 128, bf16) == 1    # 32 KB of x: staged
+    assert q.plan_launches(200, 4096, 4096, 4, 64, f16) == 4     # two chunks of 100, x kernel each
+    assert q.plan_launches(0, 4096, 4096, 4, 64, f16) == 0
+    assert q.plan_launches(4, 4096, 0, 4, 64, f16) == 0
+    st = q.make_plan(kernel=q.KERNEL_STREAM)
+    assert q.plan_launches(4, 4096, 4096, 4, 64, f16, st) == 1
