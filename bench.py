@@ -564,17 +564,26 @@ def run_ours(args, rank, world):
 
 
 def run_e2e(wl, weights, plans, dev, steps):
-    """Each step through the Python API: the step's inputs (x for each M) go from pinned host
-    memory to the device, every call of the step runs, and every output comes back to pinned
-    host memory before the step ends; the weights stay resident, as a model's do.  The output
-    of one M goes back on a copy stream while the calls of the next M run, largest M first, so
-    that only the smallest output's copy is left after the last call."""
+    """Each step through the Python API: the step's inputs (x for each M, one pinned buffer, one
+    copy) go from pinned host memory to the device, every call of the step runs, and every
+    output comes back to pinned host memory before the step ends; the weights stay resident,
+    as a model's do.  The output of one M goes back on a copy stream while the calls of the
+    next M run, largest M first, so that only the smallest output's copy is left after the
+    last call."""
     import bit_quantized_gemm_qmm_b200 as q
     from bit_quantized_gemm_qmm_b200.inputs import x_input
     S = len(weights)
-    hx = {M: x_input(M, wl.K, wl.dtype).pin_memory() for M in BENCH_MS}
+    # the step's inputs (x of every M) in one pinned buffer, so one copy brings them over
+    rows = sum(BENCH_MS)
+    hx_all = torch.empty((rows, wl.K), dtype=wl.dtype).pin_memory()
+    dx_all = torch.empty((rows, wl.K), dtype=wl.dtype, device=dev)
+    hx, dx, r0 = {}, {}, 0
+    for M in BENCH_MS:
+        hx[M] = hx_all[r0:r0 + M]
+        hx[M].copy_(x_input(M, wl.K, wl.dtype))
+        dx[M] = dx_all[r0:r0 + M]
+        r0 += M
     hy = {M: torch.empty((S, M, wl.N), dtype=wl.dtype).pin_memory() for M in BENCH_MS}
-    dx = {M: torch.empty((M, wl.K), dtype=wl.dtype, device=dev) for M in BENCH_MS}
     dy = {M: torch.empty((S, M, wl.N), dtype=wl.dtype, device=dev) for M in BENCH_MS}
     outs = {M: list(dy[M].unbind(0)) for M in BENCH_MS}  # each call's own output slice
     stream = torch.cuda.current_stream(dev)
@@ -582,8 +591,7 @@ def run_e2e(wl, weights, plans, dev, steps):
     done = {M: torch.cuda.Event() for M in BENCH_MS}
 
     def one_step():
-        for M in BENCH_MS:
-            dx[M].copy_(hx[M], non_blocking=True)
+        dx_all.copy_(hx_all, non_blocking=True)
         for M in sorted(BENCH_MS, reverse=True):
             for (P, S_, B), y in zip(weights, outs[M]):
                 q.qmm(dx[M], P, S_, B, wl.bits, wl.group, out=y, plan=plans[M])
