@@ -215,7 +215,8 @@ qmm_status resolve_plan(int64_t M, int64_t N, int64_t K, int bits, int group, co
     }
     if (p.kernel == QMM_KERNEL_STREAM && !st_ok)
         return fail(QMM_ERR_UNSUPPORTED,
-                    "streaming kernel needs 1 <= M <= 16, K a multiple of 8 groups, a 16-byte "
+                    "streaming kernel needs 1 <= M <= 16 (17..24: 4/8-bit, >= 148 row tiles, no split), "
+                    "K a multiple of 8 groups, a 16-byte "
                     "multiple of packed bytes per row and 16-byte aligned scales/biases");
     if (p.kernel == QMM_KERNEL_SK && !sk_ok)
         return fail(QMM_ERR_UNSUPPORTED,

@@ -64,7 +64,7 @@ cudaError_t launch_tc(const QmmArgs& a, const TcConfig& c, cudaStream_t stream);
 
 // Fully resolved launch configuration of the TMA-fed streaming kernel (qmm_stream.cu).
 struct StreamConfig {
-    int mt;        // 8-token column tiles (1 or 2)
+    int mt;        // 8-token column tiles (1, 2 or 3)
     int split;     // K slices = cluster size along grid.y
     int kslice;    // K codes per slice
     int ring;      // shared-memory stages (0: the shape does not fit this kernel)
@@ -80,7 +80,8 @@ struct StreamConfig {
     // x streamed through the ring with the codes (x tiles written by a small x pass first)
     // instead of staged whole per block: 9-16 tokens on persistent grids
     bool xstream;
-    int ncw;       // consumer warps per block (8 or 16)
+    int ncw;       // consumer warps per block (16, or 8 for 17-24 tokens)
+    int rw;        // 16-row tiles per consumer warp (1, or 2 for 17-24 tokens)
     size_t smem;   // dynamic shared memory per block
     bool pdl;
     bool static_weights;

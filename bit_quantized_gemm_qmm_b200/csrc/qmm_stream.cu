@@ -4,7 +4,7 @@
 // quantized_matmul(x, *w, transpose=True); formats from "What Are NAX Verify Kernels ...",
 // "Supported Data Formats and Quantization Schemes").
 //
-// At M <= 16 the matmul streams the packed weights once and does little arithmetic per byte,
+// At small M the matmul streams the packed weights once and does little arithmetic per byte,
 // so the kernel is built around keeping HBM busy.  The warp-tile kernel (qmm_mma.cu) holds
 // its codes in flight in registers, which caps the warps per SM and with them the bytes in
 // flight; here the tensor memory accelerator (TMA) moves the codes into a shared-memory ring
@@ -21,8 +21,12 @@
 //     permute and a subtraction; a group's MMAs accumulate from zero and their sum is added
 //     into the row's fp32 total times the group's scale.  6-bit codes (24-byte lane spans)
 //     are dequantized per element to A = RN_fp16(s q) instead.  x sits in shared memory for
-//     the whole K range of the block, staged once in the matching order.  The bias enters as
-//     b times the group sum of x, one more MMA per eight groups at the end of the tile;
+//     the whole K range of the block, staged once in the matching order, or streams through
+//     the ring with the codes (one tile per stage, written by a small x pass) where staging
+//     it would crowd shared memory or be a long prologue.  The bias enters as b times the
+//     group sum of x, one more MMA per eight groups at the end of the tile.  17-24 tokens (on
+//     grids of at least one tile per SM) take eight consumer warps of two 16-row tiles each,
+//     so that every x fragment feeds two row tiles;
 //   * K is split across the blocks of a cluster when there are too few tiles to fill the
 //     GPU; partial sums are added over distributed shared memory in rank order, so results
 //     are deterministic.
@@ -51,11 +55,17 @@ namespace {
 using namespace sm100;
 
 constexpr int ST_ROWS = 128;                  // weight rows per tile
-// Consumer warps: 16 (8 row groups x 2 K halves, the two halves' partial sums meet at the end
-// of a tile) or 8 (one warp takes both halves; smaller blocks, two fit on an SM).
-template <int NCW> struct StWarps {
+// Consumer warps: 16 (8 row groups of 16 rows x 2 K halves, the two halves' partial sums meet
+// at the end of a tile), 8 with RW = 1 (one warp takes both halves of 16 rows; smaller blocks,
+// two fit on an SM), or 8 with RW = 2 (4 row groups of 32 rows x 2 K halves: every x fragment
+// feeds the MMAs of two 16-row tiles, which halves the shared-memory reads of x per code; the
+// form for 17-24 tokens, one block per SM).
+template <int NCW, int RW = 1> struct StWarps {
     static constexpr int THREADS = (NCW + 2) * 32;  // + the producer warp and the tail helper
-    static constexpr int HPW = 16 / NCW;            // K halves per consumer warp
+    static constexpr int NRG = 8 / RW;              // row groups (16 * RW rows each)
+    static constexpr int NKH = NCW / NRG;           // K-half groups (1: a warp takes both halves)
+    static constexpr int HPW = 2 / NKH;             // K halves per consumer warp
+    static_assert(NKH * NRG == NCW && (NKH == 1 || NKH == 2), "consumer warp shape");
 };
 constexpr int ST_SS = 3;                      // scale / bias boxes in flight
 constexpr long long ST_TIMEOUT = 4000000000LL;  // cycles (about 2 s)
@@ -83,9 +93,9 @@ struct StLayout {
 // are redirected to row M-1: they feed accumulator columns that are never stored).
 // xs (x streamed): instead of x for the whole K range, each ring slot carries, after the
 // stage's codes, that stage's x tile [8 * mt token rows][xrs chunks] (written once per call by
-// st_xprep_kernel and brought in by the same barrier as the codes).
+// st_xprep_kernel, rows past M zero, and brought in by the same barrier as the codes).
 __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int kslice, int group, int split, int ncw,
-                                              int mrows, bool xs = false) {
+                                              int mrows, bool xs = false, int rw = 1) {
     StLayout L;
     L.w_stage = uint32_t(ST_ROWS * (bits == 6 ? 192 : 256));  // 24 or 32 KB
     L.xrs = uint32_t((xs ? st_stage_codes(bits) : kslice) / 8 + x_pad(bits, bits != 6));  // chunks per x row
@@ -99,13 +109,13 @@ __host__ __device__ inline StLayout st_layout(int bits, int mt, int ring, int ks
     L.xg_off = off;
     L.gpad = uint32_t((kslice / group + 7) / 8 * 8);
     off += uint32_t(mrows) * L.gpad * 4;
-    L.xf_off = off;                                           // K-half partials: [8 warps][32][4*MT]
-    if (ncw == 16) off += uint32_t(8 * 32 * 4 * mt * 4);
+    L.xf_off = off;  // K-half partials, one 16-row tile at a time: [row groups][32][4*MT]
+    if (ncw * rw == 16) off += uint32_t((8 / rw) * 32 * 4 * mt * 4);
     L.red_off = off;
     if (split > 1) off += uint32_t(split * ((ST_ROWS + split - 1) / split) * 8 * mt * 4);
     off = (off + 15) & ~15u;
     L.bar_off = off;
-    off += 8 * uint32_t(2 * ring + 2 * ST_SS + 18) + 16 + 64;  // + abort word; 2^E of 16 tokens
+    off += 8 * uint32_t(2 * ring + 2 * ST_SS + 18) + 16 + 128;  // + abort word; 2^E of 32 tokens
     L.total = off;
     return L;
 }
@@ -301,55 +311,72 @@ __device__ __forceinline__ int bf16_exponent(const StParams& p, int kb, int ke, 
     return eb > 141 ? eb - 141 : 0;
 }
 
-// The MMAs of one step in the exact-code layout (4- and 8-bit): lane (g, c) holds, per row
-// (g, g+8), code word 4i + c of the step in w[r][i] (i = 0..3).  Block i (32 codes at 4 bits,
-// 16 at 8) is one MMA's K range for every lane, so each MMA lies inside one group: the
-// group's MMAs accumulate into tmp (from zero), and at the group's last block tmp is added
-// into acc times the group's scale (fa: row g, fb: row g+8).  `sj` = step within the half,
-// BPG = blocks per group, fa/fb = the fp16 scales of the half's groups, two to a word.
+// The MMAs of one step in the exact-code layout (4- and 8-bit), for RW 16-row tiles: lane
+// (g, c) holds, per tile r and row (g, g+8), code word 4i + c of the step in w[r][h][i]
+// (i = 0..3).  Block i (32 codes at 4 bits, 16 at 8) is one MMA's K range for every lane, so
+// each MMA lies inside one group: the group's MMAs accumulate into tmp (from zero), and at the
+// group's last block tmp is added into acc times the group's scale (fa: row g, fb: row g+8).
+// Each x fragment is read once and feeds the MMAs of all RW tiles.  `sj` = step within the
+// half, BPG = blocks per group, fa/fb = the fp16 scales of the half's groups, two to a word.
 template <int NGH>
 __device__ __forceinline__ float scale_at(const uint32_t (&f)[(NGH + 1) / 2], int i) {
     const __half2 h = *reinterpret_cast<const __half2*>(&f[i >> 1]);
     return (i & 1) ? __high2float(h) : __low2float(h);
 }
-template <int BITS, int MT, int BPG, int NGH>
-__device__ __forceinline__ void step_exact(const uint32_t (&w)[2][4], const int sj, uint32_t xa, uint32_t xmt,
-                                           const uint32_t (&fa)[(NGH + 1) / 2], const uint32_t (&fb)[(NGH + 1) / 2],
-                                           float (&tmp)[MT][4], float (&acc)[MT][4]) {
+template <int BITS, int MT, int BPG, int NGH, int RW>
+__device__ __forceinline__ void step_exact(const uint32_t (&w)[RW][2][4], const int sj, uint32_t xa, uint32_t xmt,
+                                           const uint32_t (&fa)[RW][(NGH + 1) / 2],
+                                           const uint32_t (&fb)[RW][(NGH + 1) / 2], float (&tmp)[RW][MT][4],
+                                           float (&acc)[RW][MT][4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int bh = sj * 4 + i;  // block within the half
         const bool first = bh % BPG == 0;
         if constexpr (BITS == 4) {
-            uint32_t a0[4], a1[4];
-            dq4_exact(w[0][i], a0);
-            dq4_exact(w[1][i], a1);
+            uint32_t a0[RW][4], a1[RW][4];
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                dq4_exact(w[r][0][i], a0[r]);
+                dq4_exact(w[r][1][i], a1[r]);
+            }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const uint4 xb = lds_v4(xa + uint32_t(i * 64) + mt * xmt);
-                if (first) mma_16816_z(tmp[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
-                else mma_16816(tmp[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
-                mma_16816(tmp[mt], a0[2], a1[2], a0[3], a1[3], xb.z, xb.w);
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    if (first) mma_16816_z(tmp[r][mt], a0[r][0], a1[r][0], a0[r][1], a1[r][1], xb.x, xb.y);
+                    else mma_16816(tmp[r][mt], a0[r][0], a1[r][0], a0[r][1], a1[r][1], xb.x, xb.y);
+                    mma_16816(tmp[r][mt], a0[r][2], a1[r][2], a0[r][3], a1[r][3], xb.z, xb.w);
+                }
             }
         } else {
-            uint32_t a0[2], a1[2];
-            dq8_exact(w[0][i], a0);
-            dq8_exact(w[1][i], a1);
+            uint32_t a0[RW][2], a1[RW][2];
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                dq8_exact(w[r][0][i], a0[r]);
+                dq8_exact(w[r][1][i], a1[r]);
+            }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const uint2 xb = lds_v2(xa + uint32_t(i * 32) + mt * xmt);
-                if (first) mma_16816_z(tmp[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
-                else mma_16816(tmp[mt], a0[0], a1[0], a0[1], a1[1], xb.x, xb.y);
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    if (first) mma_16816_z(tmp[r][mt], a0[r][0], a1[r][0], a0[r][1], a1[r][1], xb.x, xb.y);
+                    else mma_16816(tmp[r][mt], a0[r][0], a1[r][0], a0[r][1], a1[r][1], xb.x, xb.y);
+                }
             }
         }
         if ((bh + 1) % BPG == 0) {
-            const float sa = scale_at<NGH>(fa, bh / BPG), sb = scale_at<NGH>(fb, bh / BPG);
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                acc[mt][0] = fmaf(sa, tmp[mt][0], acc[mt][0]);
-                acc[mt][1] = fmaf(sa, tmp[mt][1], acc[mt][1]);
-                acc[mt][2] = fmaf(sb, tmp[mt][2], acc[mt][2]);
-                acc[mt][3] = fmaf(sb, tmp[mt][3], acc[mt][3]);
+            for (int r = 0; r < RW; ++r) {
+                const float sa = scale_at<NGH>(fa[r], bh / BPG), sb = scale_at<NGH>(fb[r], bh / BPG);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    acc[r][mt][0] = fmaf(sa, tmp[r][mt][0], acc[r][mt][0]);
+                    acc[r][mt][1] = fmaf(sa, tmp[r][mt][1], acc[r][mt][1]);
+                    acc[r][mt][2] = fmaf(sb, tmp[r][mt][2], acc[r][mt][2]);
+                    acc[r][mt][3] = fmaf(sb, tmp[r][mt][3], acc[r][mt][3]);
+                }
             }
         }
     }
@@ -375,9 +402,9 @@ __device__ __forceinline__ void load_scales(uint32_t a, uint32_t (&v)[(NGH + 1) 
 // G = the group size for the exact-code path (4- and 8-bit); 0 for 6-bit, whose codes are
 // dequantized to RN_fp16(s*q) per element (step_mma) and whose group size is a parameter.
 // XS: x streamed with the codes (p.xstream); a separate instance, so that the staged-x
-// instances carry none of its code.
-template <int BITS, int MT, int NCW, int G, bool XS>
-__global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
+// instances carry none of its code.  RW: 16-row tiles per consumer warp (StWarps).
+template <int BITS, int MT, int NCW, int G, bool XS, int RW = 1>
+__global__ void __launch_bounds__(StWarps<NCW, RW>::THREADS, (NCW == 8 && RW == 1) ? 2 : 1)
     qmm_stream_kernel(const __grid_constant__ StMapSet maps, const StParams p) {
     using F = StepFmt<BITS>;
     using SF = SFmt<BITS>;
@@ -385,7 +412,8 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     constexpr int SPH = SF::SPH;               // steps per K half of a stage
     constexpr int KS = SF::KSTG;               // codes per stage
     constexpr int NREG = F::NREG, U = F::U;
-    constexpr int HPW = StWarps<NCW>::HPW;
+    using WS = StWarps<NCW, RW>;
+    constexpr int HPW = WS::HPW, NRG = WS::NRG, NKH = WS::NKH;
     constexpr bool NAT = BITS != 6;                       // exact codes, group-scaled partial sums
     static_assert(NAT == (G != 0), "G is the group size of the exact-code path");
     constexpr int BC = BITS == 4 ? 32 : 16;               // codes per MMA block (exact-code path)
@@ -395,6 +423,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     __shared__ float s_red[NCW];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     static_assert(!XS || BITS != 6, "x is streamed at 4 and 8 bits");
+    static_assert(RW == 1 || (NAT && XS && NCW == 8), "two 16-row tiles a warp: the 8-warp streamed-x form");
     const StLayout& L = p.lay;
     const int S = p.ring;
     const uint32_t sbase = smem_addr(smem);
@@ -431,8 +460,8 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
             mbar_init(bar_xfull + 8 * i, 1);
             mbar_init(bar_xempty + 8 * i, 1);
         }
-        mbar_init(bar_tw, 8);  // the eight row-group warps that hold a tile's sums
-        mbar_init(bar_tw + 8, 8);
+        mbar_init(bar_tw, NRG);  // the row-group warps that hold a tile's sums
+        mbar_init(bar_tw + 8, NRG);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -515,11 +544,11 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
     } else if (warp < NCW) {
         // ------------------------------------------------------------ consumers
         const int g = lane >> 2, c = lane & 3;
-        const int hbase = NCW == 16 ? (warp >> 3) : 0;         // first K half this warp takes
-        const int rg = warp & 7;                                // 16-row group of the tile
+        const int hbase = NKH == 2 ? warp / NRG : 0;           // first K half this warp takes
+        const int rg = warp % NRG;                             // row group (16 * RW rows) of the tile
         // rows of "g" and "g + 8": natural for the ldmatrix reads of the exact-code path; the
         // 6-bit reads (8-byte pieces of 24-byte lane spans) stay conflict-free under a permutation
-        const int rA = rg * 16 + (NAT ? g : ((g >> 1) | ((g & 1) << 2)));
+        const int rA = rg * 16 * RW + (NAT ? g : ((g >> 1) | ((g & 1) << 2)));  // (+ 16 r: tile r)
         const int rB = rA + 8;
         grid_dependency_wait();
         const uint32_t xs = sbase + L.x_off, xg = sbase + L.xg_off;
@@ -530,12 +559,13 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
             // the x pass's rows of group sums span the whole K range (stride gst); this block's
             // groups start at kb / group
             const int gst = (p.K / p.group + 7) / 8 * 8, g0 = kb >> p.gshift, gpad = int(L.gpad);
-            for (int e = threadIdx.x; e < p.M * gpad; e += NCW * 32) {
+            for (int e = threadIdx.x; e < 8 * MT * gpad; e += NCW * 32) {  // (rows past M: zeros)
                 const int m = e / gpad, gi = g0 + (e - m * gpad);
                 const uint32_t v = gi < gst ? __ldg(p.xgw + m * gst + gi) : 0u;
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(xg + uint32_t(e) * 4u), "r"(v));
             }
-            if (threadIdx.x < 16) ysc[threadIdx.x] = int(threadIdx.x) < p.M ? exp2i(__ldg(p.xexp + threadIdx.x)) : 1.f;
+            if (threadIdx.x < 8 * MT)
+                ysc[threadIdx.x] = int(threadIdx.x) < p.M ? exp2i(__ldg(p.xexp + threadIdx.x)) : 1.f;
         } else {
             const int E = p.is_bf16 ? bf16_exponent<NCW>(p, kb, ke, s_red) : 0;
             stage_x_tile<BITS, MT, NAT>(p.x, p.M, p.K, p.is_bf16, p.group, p.kslice, int(L.gpad), NCW * 32, xs, xg,
@@ -545,7 +575,9 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         consumer_sync<NCW>();
         grid_dependents_launch();
 
-        const int tr0 = min(g, p.M - 1), tr1 = min(g + 8, p.M - 1);  // token rows of the two x tiles
+        // token rows of the lane's first two x tiles (streamed x holds all 8 * MT rows, zero past
+        // M, so its tiles are evenly spaced; staged x only M rows, MT <= 2)
+        const int tr0 = XS ? g : min(g, p.M - 1), tr1 = XS ? g + 8 : min(g + 8, p.M - 1);
         const uint32_t xmt = uint32_t(tr1 - tr0) * L.xrs * 16;
         // the lane's B fragments: 16-byte chunk c of each 4-chunk block (8 bytes at 8-bit),
         // relative to the x of its stage
@@ -568,18 +600,20 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         uint32_t ldm_off[SPH];
 #pragma unroll
         for (int sj = 0; sj < SPH; ++sj)
-            ldm_off[sj] = uint32_t((rg * 16 + (lane & 7)) * 128 + ((((4 * sj + (lane >> 3)) ^ lane) & 7) << 4));
+            ldm_off[sj] = uint32_t((rg * 16 * RW + (lane & 7)) * 128 + ((((4 * sj + (lane >> 3)) ^ lane) & 7) << 4));
         // One item (tile t, stages [s0, s1)); PARTIAL: a tail piece, which may hand partial
         // sums to the tail helper.  Whole tiles take a copy of the body without that path.
         auto run_item = [&](const int t, const int s0, const int s1, const int k, auto partial) {
             constexpr bool PARTIAL = decltype(partial)::value;
             // After a timeout (abort flag set) every wait below returns at once and the work
             // is skipped, so all warps leave the loop together.
-            float acc[MT][4], tb[MT][4], tmp[MT][4];
+            float acc[RW][MT][4], tb[RW][MT][4], tmp[RW][MT][4];
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
+            for (int r = 0; r < RW; ++r)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[mt][i] = tb[mt][i] = tmp[mt][i] = 0.f;
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[r][mt][i] = tb[r][mt][i] = tmp[r][mt][i] = 0.f;
             uint32_t sbuf = 0;
             bool sok = true;
             int sib = 0;                                                 // stage within the scale block
@@ -594,32 +628,37 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                 const bool ok = sok && wait_or_abort(bar_full + 8 * s, ph, abort_flag);
                 if constexpr (NAT) {
                   if (ok) {
-                    // the lane's code words 4i + c of rows rA and rB for each step of its K
-                    // half (halves), by ldmatrix; the ring slot is released once they are in
-                    // registers
+                    // the lane's code words 4i + c of rows rA and rB (+ 16 r) for each step of
+                    // its K half (halves), by ldmatrix
                     const uint32_t stage = sbase + s * L.slot;
 #pragma unroll
                     for (int hh = 0; hh < HPW; ++hh) {
                         // scales of the half's groups (a whole number of them: a half is 256
                         // codes at 4-bit, 128 at 8-bit, and groups are at most 128)
                         const uint32_t g0 = uint32_t((sib * KS + (hbase + hh) * (KS / 2)) / G) * 2u;
-                        uint32_t fa[(NGH + 1) / 2], fb[(NGH + 1) / 2];
-                        load_scales<NGH>(sbuf + rAg + g0, fa);
-                        load_scales<NGH>(sbuf + rBg + g0, fb);
+                        uint32_t fa[RW][(NGH + 1) / 2], fb[RW][(NGH + 1) / 2];
+#pragma unroll
+                        for (int r = 0; r < RW; ++r) {
+                            load_scales<NGH>(sbuf + rAg + uint32_t(r * 16 * gbb) * 2u + g0, fa[r]);
+                            load_scales<NGH>(sbuf + rBg + uint32_t(r * 16 * gbb) * 2u + g0, fb[r]);
+                        }
 #pragma unroll
                         for (int sj = 0; sj < SPH; ++sj) {
                             // the lane's code words 4i + c of rows rA and rB for this step, by
                             // ldmatrix; the ring slot is released after the stage's last read
-                            uint32_t w[2][4];
+                            uint32_t w[RW][2][4];
                             const uint32_t a = stage + uint32_t((hbase + hh) * (ST_ROWS * 128)) + ldm_off[sj];
-                            ldsm_x4(a, w[0]);
-                            ldsm_x4(a + 8 * 128, w[1]);
+#pragma unroll
+                            for (int r = 0; r < RW; ++r) {
+                                ldsm_x4(a + uint32_t(r * 16 * 128), w[r][0]);
+                                ldsm_x4(a + uint32_t(r * 16 * 128 + 8 * 128), w[r][1]);
+                            }
                             if (hh == HPW - 1 && sj == SPH - 1 && !XS) {
                                 __syncwarp();
                                 if (lane == 0) mbar_arrive(bar_empty + 8 * s);
                             }
-                            step_exact<BITS, MT, BPG, NGH>(w, sj, xst + uint32_t((hh * SPH + sj) * KSS * 2), xmt, fa, fb,
-                                                           tmp, acc);
+                            step_exact<BITS, MT, BPG, NGH, RW>(w, sj, xst + uint32_t((hh * SPH + sj) * KSS * 2), xmt,
+                                                               fa, fb, tmp, acc);
                         }
                     }
                     if constexpr (XS) {  // the slot's x tile was read up to the last step
@@ -627,7 +666,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                         if (lane == 0) mbar_arrive(bar_empty + 8 * s);
                     }
                   }
-                } else if (ok) {  // 6-bit
+                } else if (ok) {  // 6-bit (one 16-row tile a warp)
                     // the lane's codes of rows rA and rB for the steps of its K half (halves);
                     // the ring slot is released as soon as they are in registers
                     uint32_t w[HPW * SPH][2][NREG];
@@ -664,13 +703,13 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 #pragma unroll
                         for (int j = 0; j < HPW * SPH; ++j) {
                             const RowConst C[2] = {row_const<BITS>(sv[j][0]), row_const<BITS>(sv[j][1])};
-                            step_mma<BITS, MT, true>(w[j], C, xst + uint32_t(j * KSS * 2), xmt, acc);
+                            step_mma<BITS, MT, true>(w[j], C, xst + uint32_t(j * KSS * 2), xmt, acc[0]);
                         }
                     } else {
 #pragma unroll
                         for (int j = 0; j < HPW * SPH; ++j) {
                             const RowConst C[2] = {row_const<BITS>(sv[j][0]), row_const<BITS>(sv[j][1])};
-                            step_mma<BITS, MT, false>(w[j], C, xst + uint32_t(j * KSS * 2), xmt, acc);
+                            step_mma<BITS, MT, false>(w[j], C, xst + uint32_t(j * KSS * 2), xmt, acc[0]);
                         }
                     }
                 }
@@ -683,24 +722,33 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                         const uint32_t bb = sbuf + L.sb_slot / 2;
                         // exact-code path: into tmp (free between groups) and straight on into
                         // acc, rescaled to its units; else into tb, added at the end
-                        float (&bt)[MT][4] = NAT ? tmp : tb;
+                        float (&bt)[RW][MT][4] = NAT ? tmp : tb;
                         if (NAT) {
 #pragma unroll
-                            for (int mt = 0; mt < MT; ++mt)
+                            for (int r = 0; r < RW; ++r)
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) tmp[mt][i] = 0.f;
+                                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) tmp[r][mt][i] = 0.f;
                         }
-                        for (int q = 0; q < gbb; q += 8)
-                            bias_mma<MT>(lds_u16(bb + rAg + uint32_t(q + c) * 2u), lds_u16(bb + rBg + uint32_t(q + c) * 2u),
-                                         lds_u16(bb + rAg + uint32_t(q + c + 4) * 2u),
-                                         lds_u16(bb + rBg + uint32_t(q + c + 4) * 2u), xblk + uint32_t(q) * 4u, xg_mt, c,
-                                         bt);
+#pragma unroll
+                        for (int r = 0; r < RW; ++r) {
+                            const uint32_t ra = bb + rAg + uint32_t(r * 16 * gbb) * 2u;
+                            const uint32_t rb = bb + rBg + uint32_t(r * 16 * gbb) * 2u;
+                            for (int q = 0; q < gbb; q += 8)
+                                bias_mma<MT>(lds_u16(ra + uint32_t(q + c) * 2u), lds_u16(rb + uint32_t(q + c) * 2u),
+                                             lds_u16(ra + uint32_t(q + c + 4) * 2u),
+                                             lds_u16(rb + uint32_t(q + c + 4) * 2u), xblk + uint32_t(q) * 4u, xg_mt, c,
+                                             bt[r]);
+                        }
                         if (NAT) {
                             constexpr float kb2acc = 128.f / exact_code_unscale<BITS>();
 #pragma unroll
-                            for (int mt = 0; mt < MT; ++mt)
+                            for (int r = 0; r < RW; ++r)
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) acc[mt][i] = fmaf(kb2acc, tmp[mt][i], acc[mt][i]);
+                                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) acc[r][mt][i] = fmaf(kb2acc, tmp[r][mt][i], acc[r][mt][i]);
                         }
                     }
                     __syncwarp();
@@ -713,58 +761,74 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                     }
                 }
             }
-            // with 16 warps the two K halves meet: half 1 hands its partial sums to half 0
-            // (mbarrier handshake); with 8 warps each warp already holds the whole sum
+            // with two K-half groups the halves meet: half 1 hands its partial sums to half 0
+            // (mbarrier handshake), one 16-row tile at a time; with one each warp already holds
+            // the whole sum
             bool own = true;
-            if constexpr (NCW == 16) {
-                own = false;
-                if (hbase == 1) {
-                    if (tc == 0 || wait_or_abort(bar_xempty + 8 * rg, ((tc - 1) & 1), abort_flag)) {
+            if constexpr (NKH == 2) {
+                bool hok = true;
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    const int q = tc * RW + r;  // hand-offs of this row group so far
+                    if (hbase == 1) {
+                        if (hok && (q == 0 || wait_or_abort(bar_xempty + 8 * rg, ((q - 1) & 1), abort_flag))) {
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) xf[4 * mt + i] = acc[r][mt][i];
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar_xfull + 8 * rg);
+                        } else {
+                            hok = false;
+                        }
+                    } else if (hok && wait_or_abort(bar_xfull + 8 * rg, q & 1, abort_flag)) {
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) xf[4 * mt + i] = acc[mt][i];
+                            for (int i = 0; i < 4; ++i) acc[r][mt][i] += xf[4 * mt + i];
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(bar_xfull + 8 * rg);
+                        if (lane == 0) mbar_arrive(bar_xempty + 8 * rg);
+                    } else {
+                        hok = false;
                     }
-                } else if (wait_or_abort(bar_xfull + 8 * rg, tc & 1, abort_flag)) {
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) acc[mt][i] += xf[4 * mt + i];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_xempty + 8 * rg);
-                    own = true;
                 }
+                own = hbase == 0 && hok;
             }
             if (own) {
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float ys = XS ? ysc[8 * mt + 2 * c + (i & 1)] : yscale;
-                        acc[mt][i] = NAT ? exact_code_unscale<BITS>() * acc[mt][i] * ys : (acc[mt][i] + 128.f * tb[mt][i]) * ys;
-                    }
-                if (p.split == 1 && (!PARTIAL || s1 - s0 == nst)) {
+                for (int r = 0; r < RW; ++r)
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const int m = 8 * mt + 2 * c + (i & 1);
-                            if (m < p.M) st_store_y(p, t, m, i < 2 ? rA : rB, acc[mt][i]);
+                            const float ys = XS ? ysc[8 * mt + 2 * c + (i & 1)] : yscale;
+                            acc[r][mt][i] = NAT ? exact_code_unscale<BITS>() * acc[r][mt][i] * ys
+                                                : (acc[r][mt][i] + 128.f * tb[r][mt][i]) * ys;
                         }
+                if (p.split == 1 && (!PARTIAL || s1 - s0 == nst)) {
+#pragma unroll
+                    for (int r = 0; r < RW; ++r)
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int m = 8 * mt + 2 * c + (i & 1);
+                                if (m < p.M) st_store_y(p, t, m, (i < 2 ? rA : rB) + 16 * r, acc[r][mt][i]);
+                            }
                 } else if (PARTIAL && p.split == 1) {
                     // a piece of a tail tile (item k = 0 or 1: the tail comes first): its
                     // partial sums go to this block's slot and the tail helper takes over
                     float* part = p.partials +
                                   size_t(st_slot(p, nst / spb, int(blockIdx.x), t - p.dp_tiles)) * (8 * MT * ST_ROWS);
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
+                    for (int r = 0; r < RW; ++r)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int m = 8 * mt + 2 * c + (i & 1);
-                            if (m < p.M) part[m * ST_ROWS + (i < 2 ? rA : rB)] = acc[mt][i];
-                        }
+                        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int m = 8 * mt + 2 * c + (i & 1);
+                                if (m < p.M) part[m * ST_ROWS + (i < 2 ? rA : rB) + 16 * r] = acc[r][mt][i];
+                            }
                     __threadfence();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_tw + 8 * k);
@@ -779,18 +843,21 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
                     const int rows_per = (ST_ROWS + p.split - 1) / p.split;
                     const uint32_t me = cluster_ctarank();
                     const uint32_t red_la = sbase + L.red_off;
-                    const int oA = rA / rows_per, oB = rB / rows_per;
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
+                    for (int r = 0; r < RW; ++r) {
+                        const int oA = (rA + 16 * r) / rows_per, oB = (rB + 16 * r) / rows_per;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int col = 8 * mt + 2 * c + (i & 1);
-                            const int owner = i < 2 ? oA : oB;
-                            const int rl = (i < 2 ? rA : rB) - owner * rows_per;
-                            if (col < p.M)
-                                st_cluster_f32(red_la + uint32_t(((int(me) * 8 * MT + col) * rows_per + rl) * 4),
-                                               uint32_t(owner), acc[mt][i]);
-                        }
+                        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int col = 8 * mt + 2 * c + (i & 1);
+                                const int owner = i < 2 ? oA : oB;
+                                const int rl = (i < 2 ? rA : rB) + 16 * r - owner * rows_per;
+                                if (col < p.M)
+                                    st_cluster_f32(red_la + uint32_t(((int(me) * 8 * MT + col) * rows_per + rl) * 4),
+                                                   uint32_t(owner), acc[r][mt][i]);
+                            }
+                    }
                 }
             }
                 };
@@ -886,7 +953,7 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
         const int ncols = min(8 * MT, p.M);
         const float* red = reinterpret_cast<const float*>(smem + L.red_off);
         const bool ok = *abort_flag == 0;
-        for (int e = threadIdx.x; e < nrows * ncols; e += StWarps<NCW>::THREADS) {
+        for (int e = threadIdx.x; e < nrows * ncols; e += WS::THREADS) {
             const int col = e / nrows, rl = e - col * nrows;
             float sum = 0.f;
             for (int q = 0; q < p.split; ++q) sum += red[(q * 8 * MT + col) * rows_per + rl];
@@ -896,23 +963,25 @@ __global__ void __launch_bounds__(StWarps<NCW>::THREADS, NCW == 8 ? 2 : 1)
 }
 
 // ---------------------------------------------------------------- x pass (streamed x)
-// One block per token row: the row's fp16 x tiles of every stage ([stage][rows = 8 * MT][xrs
+// One block per token row of the tiles (rows = 8 * MT; rows past M are zeros): the row's
+// fp16 x tiles of every stage ([stage][rows][xrs
 // chunks]; each 8-code unit at its natural chunk, its codes in perm_nat order), its group
 // sums as (hi, lo) fp16 times 2^-7 ([row][gst], gst = the groups of the whole K range rounded
 // up to 8, zero past the last group) and its exponent:
 // bf16 rows are scaled by 2^-E with max|x| * 2^-E < 2^15 (E >= 0), fp16 rows are not.
 template <int BITS>
-__global__ void __launch_bounds__(256) st_xprep_kernel(const uint16_t* __restrict__ x, int K, int is_bf16, int group,
-                                                       int rows, int xrs, int gst, uint8_t* __restrict__ xt,
+__global__ void __launch_bounds__(256) st_xprep_kernel(const uint16_t* __restrict__ x, int M, int K, int is_bf16,
+                                                       int group, int rows, int xrs, int gst, uint8_t* __restrict__ xt,
                                                        uint32_t* __restrict__ xgw, int* __restrict__ xexp) {
     constexpr int CPS = (BITS == 4 ? 512 : 256) / 8;  // 16-byte chunks (8-code units) per stage
     __shared__ float red[8];
     grid_dependents_launch();
     grid_dependency_wait();
     const int m = blockIdx.x;
-    const uint16_t* xr = x + int64_t(m) * K;
+    const bool real = m < M;  // the block's row holds a token (uniform over the block)
+    const uint16_t* xr = x + int64_t(real ? m : 0) * K;
     int E = 0;
-    if (is_bf16) {
+    if (is_bf16 && real) {
         float amax = 0.f;
         for (int k = threadIdx.x * 8; k < K; k += 256 * 8) {
             const uint4 v = ldg_nc_v4(xr + k);
@@ -937,7 +1006,7 @@ __global__ void __launch_bounds__(256) st_xprep_kernel(const uint16_t* __restric
     for (int u = threadIdx.x; u < totp; u += 256) {
         const bool valid = u < units;
         float f[8];
-        if (valid) {
+        if (valid && real) {
             const uint4 v = ldg_nc_v4(xr + 8 * u);
             const uint32_t r[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -990,10 +1059,25 @@ StKernelFn pick_stream_g(int group) {
         return nullptr;
     }
 }
-// 16 consumer warps (the 8-warp form of the kernel is not instantiated: it measured slower on
-// every configuration of the sweep)
-StKernelFn pick_stream(int bits, int mt, int ncw, int group, bool xs) {
-    if (ncw != 16 || (mt != 1 && mt != 2)) return nullptr;
+// 17-24 tokens: three token tiles, 8 consumer warps of two 16-row tiles each, x streamed
+template <int BITS>
+StKernelFn pick_stream_wide(int group) {
+    if (group == 32) return qmm_stream_kernel<BITS, 3, 8, 32, true, 2>;
+    if (group == 64) return qmm_stream_kernel<BITS, 3, 8, 64, true, 2>;
+    if (group == 128) return qmm_stream_kernel<BITS, 3, 8, 128, true, 2>;
+    return nullptr;
+}
+// 16 consumer warps up to 16 tokens (the 8-warp form with one 16-row tile a warp is not
+// instantiated: it measured slower on every configuration of the sweep); 17-24 tokens the
+// 8-warp form with two
+StKernelFn pick_stream(int bits, int mt, int ncw, int group, bool xs, int rw) {
+    if (mt == 3) {
+        if (ncw != 8 || rw != 2 || !xs) return nullptr;
+        if (bits == 4) return pick_stream_wide<4>(group);
+        if (bits == 8) return pick_stream_wide<8>(group);
+        return nullptr;
+    }
+    if (ncw != 16 || rw != 1 || (mt != 1 && mt != 2)) return nullptr;
     if (xs) {
         if (bits == 4) return mt == 1 ? pick_stream_g<4, 1, true>(group) : pick_stream_g<4, 2, true>(group);
         if (bits == 8) return mt == 1 ? pick_stream_g<8, 1, true>(group) : pick_stream_g<8, 2, true>(group);
@@ -1018,15 +1102,17 @@ constexpr int kNumSM = 148;
 constexpr int64_t kXsStagedMax = 64 * 1024;  // staged x (bytes) above which 9-16 tokens stream x
 constexpr size_t kMaxSmem = 226 * 1024;  // dynamic, per block (static shared memory is tiny)
 
-size_t st_smem(int bits, int mt, int ring, int kslice, int group, int split, int ncw, int mrows, bool xs) {
-    return size_t(st_layout(bits, mt, ring, kslice, group, split, ncw, mrows, xs).total) + 1024;  // + alignment slack
+size_t st_smem(int bits, int mt, int ring, int kslice, int group, int split, int ncw, int mrows, bool xs, int rw) {
+    return size_t(st_layout(bits, mt, ring, kslice, group, split, ncw, mrows, xs, rw).total) + 1024;  // + alignment slack
 }
 
 }  // namespace
 
 bool stream_supported(int64_t M, int64_t N, int64_t K, int bits, int group) {
-    if (M < 1 || M > 16 || N < 1) return false;
+    if (M < 1 || M > 24 || N < 1) return false;
     if (bits != 4 && bits != 6 && bits != 8) return false;
+    // 17-24 tokens: 4- and 8-bit codes on grids of at least one tile per SM (x streamed)
+    if (M > 16 && (bits == 6 || (N + ST_ROWS - 1) / ST_ROWS < kNumSM)) return false;
     if ((K * bits / 8) % 16) return false;       // code rows must be 16-byte pitched for TMA
     if (K % (8 * int64_t(group))) return false;  // scale / bias rows too (groups per row % 8)
     return K % st_block_codes(bits, group) == 0;  // whole stages and scale blocks
@@ -1034,7 +1120,8 @@ bool stream_supported(int64_t M, int64_t N, int64_t K, int bits, int group) {
 
 StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group, int split_req) {
     StreamConfig c = {};
-    c.mt = M > 8 ? 2 : 1;
+    c.mt = M > 16 ? 3 : (M > 8 ? 2 : 1);
+    const bool wide = M > 16;  // 8 consumer warps of two 16-row tiles, x streamed, no K split
     const int KS = ks_for(bits);
     const int T = cdiv(N, ST_ROWS);
     const int unit = st_block_codes(bits, group);  // kslice granularity: whole stages and scale blocks
@@ -1056,6 +1143,7 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         }
     }
     split = std::max(1, std::min(8, split));
+    if (wide && split != 1) return c;  // ring 0: not this kernel
     const int split0 = split;
     // x streams with the codes instead of being staged whole per block (4- and 8-bit): at
     // 9-16 tokens on a persistent grid, or wherever x for a block's K range would take more
@@ -1074,13 +1162,20 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         const int want = std::min(sp > 1 ? nst : 6, 6);
         int ring = std::max(want, 2);
         // 16 consumer warps measured faster than 8 on every configuration of the sweep (the
-        // 8-warp blocks fit two to an SM, but that bought no overlap between calls)
-        const int ncw = 16;
+        // 8-warp blocks fit two to an SM, but that bought no overlap between calls); 17-24
+        // tokens take 8 warps of two 16-row tiles (one block per SM)
+        const int ncw = wide ? 8 : 16, rw = wide ? 2 : 1;
         const int64_t xbytes = int64_t(M) * kslice * 2;  // x of a block's K range, staged whole
         const bool xs = xs_bits && (M > 8 ? ((sp == 1 && T >= kNumSM) || xbytes > kXsStagedMax)
                                           : (sp == 1 && T < kNumSM && xbytes > kXsStagedMax / 2));
-        while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M), xs) > kMaxSmem) --ring;
-        const bool fits = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M), xs) <= kMaxSmem;
+        if (wide && !(xs && sp == 1 && T >= kNumSM)) return c;  // ring 0: persistent grids only
+        const int mrows = xs ? 8 * c.mt : int(M);  // token rows of x (and its group sums) held
+        while (ring > 2 && st_smem(bits, c.mt, ring, kslice, group, sp, ncw, mrows, xs, rw) > kMaxSmem) --ring;
+        const bool fits = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, mrows, xs, rw) <= kMaxSmem;
+        if (wide && (!fits || ring < 3)) {
+            c.ring = 0;  // no K split to make room: the caller uses another kernel
+            return c;
+        }
         if (!fits || (ring < std::min(want, 3) && split < 8)) {
             if (split < 8) continue;
             c.ring = 0;  // does not fit: the caller uses another kernel
@@ -1093,7 +1188,8 @@ StreamConfig stream_config(int64_t M, int64_t N, int64_t K, int bits, int group,
         c.stage_bytes = ST_ROWS * KS * bits / 8;
         c.split_raised = split > split0;
         c.ncw = ncw;
-        c.smem = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, int(M), xs);
+        c.rw = rw;
+        c.smem = st_smem(bits, c.mt, ring, kslice, group, sp, ncw, mrows, xs, rw);
         c.xstream = xs;
         // one block per SM: 17 warps at up to 96 registers leave no room for a second
         c.grid_x = sp > 1 ? T : std::min(T, kNumSM);
@@ -1188,8 +1284,9 @@ cudaError_t ensure_smem_attr(StKernelFn fn, size_t smem) {
 
 cudaError_t launch_stream_items(const QmmArgs& a, const SkItem* items, int nitems, const StreamConfig& c,
                                 cudaStream_t stream) {
-    const int mt = int(a.M) > 8 ? 2 : 1;
-    StKernelFn fn = pick_stream(a.bits, mt, c.ncw, a.group, c.xstream);
+    const int mt = c.mt;
+    if (mt != (a.M > 16 ? 3 : (a.M > 8 ? 2 : 1))) return cudaErrorNotSupported;
+    StKernelFn fn = pick_stream(a.bits, mt, c.ncw, a.group, c.xstream, c.rw);
     if (!fn || c.ring < 2 || nitems < 1 || nitems > ST_MAX_ITEMS) return cudaErrorNotSupported;
 
     StParams p;
@@ -1243,16 +1340,18 @@ cudaError_t launch_stream_items(const QmmArgs& a, const SkItem* items, int nitem
     p.xt = nullptr;
     p.xgw = nullptr;
     p.xexp = nullptr;
-    const StLayout L = st_layout(a.bits, mt, c.ring, c.kslice, a.group, c.split, c.ncw, int(a.M), c.xstream);
+    const int mrows = c.xstream ? 8 * mt : int(a.M);  // token rows of x held (streamed: all 8 * mt)
+    const StLayout L = st_layout(a.bits, mt, c.ring, c.kslice, a.group, c.split, c.ncw, mrows, c.xstream, c.rw);
     p.lay = L;
     const int gst = int((a.K / a.group + 7) / 8 * 8);  // streamed x: group sums a row (the whole K range)
     if (c.tper > 0 || c.xstream) {
         // workspace: tail arrival words [T - dp_tiles], tail partial sums [2 * grid][8 * mt][128];
-        // streamed x: tiles [stages][8 * mt][xrs chunks], group sums [M][gst], exponents [M]
+        // streamed x: tiles [stages][8 * mt][xrs chunks], group sums [8 * mt][gst], exponents
+        // [8 * mt] (rows past M zero)
         const size_t cbytes = c.tper > 0 ? (size_t(p.T - c.dp_tiles) * 8 + 255) / 256 * 256 : 0;
         const size_t pbytes = c.tper > 0 ? size_t(2 * c.grid_x) * 8 * mt * ST_ROWS * 4 : 0;
         const size_t xtbytes = c.xstream ? size_t(a.K / ks_for(a.bits)) * L.xtile : 0;
-        const size_t xgbytes = c.xstream ? (size_t(a.M) * gst * 4 + 255) / 256 * 256 : 0;
+        const size_t xgbytes = c.xstream ? (size_t(mrows) * gst * 4 + 255) / 256 * 256 : 0;
         void* ws = nullptr;
         cudaError_t e = split_workspace(stream, cbytes + pbytes + xtbytes + xgbytes + (c.xstream ? 256 : 0), &ws);
         if (e != cudaSuccess) return e;
@@ -1293,9 +1392,9 @@ cudaError_t launch_stream_items(const QmmArgs& a, const SkItem* items, int nitem
     cfg.attrs = attrs;
     cfg.numAttrs = unsigned(na);
     if (c.xstream) {
-        // the x pass first (one block per token row); the main kernel waits for it
+        // the x pass first (one block per token row of the tiles); the main kernel waits for it
         cudaLaunchConfig_t xc = {};
-        xc.gridDim = dim3(unsigned(a.M), 1, 1);
+        xc.gridDim = dim3(unsigned(mrows), 1, 1);
         xc.blockDim = dim3(256, 1, 1);
         xc.stream = stream;
         cudaLaunchAttribute xa[1];
@@ -1306,9 +1405,9 @@ cudaError_t launch_stream_items(const QmmArgs& a, const SkItem* items, int nitem
         uint8_t* xt = const_cast<uint8_t*>(p.xt);
         uint32_t* xgw = const_cast<uint32_t*>(p.xgw);
         int* xexp = const_cast<int*>(p.xexp);
-        e = a.bits == 4 ? cudaLaunchKernelEx(&xc, st_xprep_kernel<4>, a.x, int(a.K), a.is_bf16, a.group, 8 * mt,
+        e = a.bits == 4 ? cudaLaunchKernelEx(&xc, st_xprep_kernel<4>, a.x, int(a.M), int(a.K), a.is_bf16, a.group, 8 * mt,
                                              int(L.xrs), gst, xt, xgw, xexp)
-                        : cudaLaunchKernelEx(&xc, st_xprep_kernel<8>, a.x, int(a.K), a.is_bf16, a.group, 8 * mt,
+                        : cudaLaunchKernelEx(&xc, st_xprep_kernel<8>, a.x, int(a.M), int(a.K), a.is_bf16, a.group, 8 * mt,
                                              int(L.xrs), gst, xt, xgw, xexp);
         if (e != cudaSuccess) return e;
     }

@@ -113,7 +113,9 @@ enum {
     QMM_KERNEL_MMA = 1,    /* warp-per-16-row tile, register-streamed codes, mma.sync       */
     QMM_KERNEL_TC = 2,     /* swap-AB tcgen05 tile: 128 weight rows x M tokens, TMEM accum   */
     QMM_KERNEL_STREAM = 3, /* M <= 16: TMA-staged codes, mma.sync consumer warps; K split over
-                              a cluster only when the 128-row tiles cannot fill the GPU      */
+                              a cluster only when the 128-row tiles cannot fill the GPU.
+                              17 <= M <= 24: 4- and 8-bit codes on matrices of at least 148
+                              row tiles (one per SM), x streamed with the codes, no K split  */
     QMM_KERNEL_SK = 4,     /* 1 <= M <= 64: tcgen05 tile of 128 weight rows x M tokens with the
                               weight stream split evenly over at most one block per SM; the
                               partial sums of a tile split between blocks are added by the last

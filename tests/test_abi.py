@@ -129,6 +129,15 @@ def test_plans(L):
     bf16 = __import__("torch").bfloat16
     for M in (13, 14, 16):
         assert q.plan_default(M, 151936, 4096, 4, 64, bf16).kernel == q.KERNEL_STREAM
+    # ... and 17-24 tokens (three token tiles, warps of two 16-row tiles) at 4 and 8 bits; not
+    # 6-bit codes, not past 24 tokens, not below one tile per SM
+    for M in (17, 20, 24):
+        assert q.plan_default(M, 151936, 4096, 4, 64, bf16).kernel == q.KERNEL_STREAM
+        assert q.plan_default(M, 151936, 4096, 8, 128, bf16).kernel == q.KERNEL_STREAM
+    assert q.plan_default(25, 151936, 4096, 4, 64, bf16).kernel == q.KERNEL_TC
+    assert q.plan_default(17, 151936, 4096, 6, 64, bf16).kernel != q.KERNEL_STREAM
+    assert q.plan_default(17, 147 * 128, 4096, 4, 64, bf16).kernel != q.KERNEL_STREAM
+    assert q.plan_default(17, 148 * 128, 4096, 4, 64, bf16).kernel == q.KERNEL_STREAM
     # 6-bit codes on the large matrices leave the streaming kernel above 8 tokens (one token
     # tile); the small k/v ones keep it up to 16
     assert q.plan_default(8, 14336, 4096, 6, 32, bf16).kernel == q.KERNEL_STREAM
@@ -179,7 +188,7 @@ def test_default_plan_for_every_workload_and_m(L):
             p = q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype)
             assert p.kernel in (q.KERNEL_MMA, q.KERNEL_TC, q.KERNEL_STREAM), (name, M, p.as_dict())
             assert 1 <= p.split <= 16, (name, M, p.as_dict())
-            assert p.kernel != q.KERNEL_STREAM or M <= 16, (name, M)
+            assert p.kernel != q.KERNEL_STREAM or M <= 16 or (M <= 24 and p.split == 1), (name, M)
             assert q.plan_default(M, wl.N, wl.K, wl.bits, wl.group, wl.dtype).as_dict() == p.as_dict()
 
 
@@ -191,6 +200,7 @@ def test_plan_launches(L):
     assert q.plan_launches(1, 151936, 4096, 4, 64, bf16) == 1    # streaming, x staged
     assert q.plan_launches(16, 151936, 4096, 4, 64, bf16) == 2   # + the x pass (x streamed)
     assert q.plan_launches(32, 151936, 4096, 4, 64, bf16) == 2   # tensor-core kernel + its x kernel
+    assert q.plan_launches(20, 151936, 4096, 4, 64, bf16) == 2   # streaming, x streamed
     assert q.plan_launches(32, 4096, 14336, 4, 64, bf16) == 2
     assert q.plan_launches(1, 4096, 4096, 4, 64, f16) == 1
     assert q.plan_launches(6, 14336, 4096, 8, 128, bf16) == 2    # one tile a block: x streamed

@@ -125,6 +125,8 @@ def test_deterministic_bitwise():
     (20000, 4096, 8, 128, 13, torch.bfloat16),  # ragged last tile inside the tail
     (19100, 2048, 6, 64, 9, torch.float16),   # 150 tiles at 6 bits
     (18960, 1024, 8, 32, 16, torch.float16),  # 149 tiles, one 8-bit stage a scale block
+    (19328, 4096, 4, 64, 20, torch.bfloat16),  # 17-24 tokens: warps of two 16-row tiles
+    (20000, 2048, 8, 128, 24, torch.float16),  # ... at 8 bits, ragged last tile in the tail
 ])
 def test_tail_tiles(oracle_mod, N, K, bits, group, M, dtype):
     """Persistent grids whose tile count is not a multiple of the grid: the last partial wave
@@ -172,12 +174,12 @@ def test_tail_tiles_repeatable_back_to_back_and_in_a_graph():
     assert q.device_errors() == 0
 
 
-@pytest.mark.parametrize("M", [9, 12, 16])
+@pytest.mark.parametrize("M", [9, 12, 16, 17, 20, 24])
 @pytest.mark.parametrize("bits,group", [(4, 32), (4, 128), (8, 64)])
 def test_streamed_x(oracle_mod, M, bits, group):
-    """9-16 tokens on a persistent grid take x through the ring, one tile per stage written by
-    a separate x pass with a per-token exponent: rows of very different magnitudes (bf16)
-    each keep their precision."""
+    """9-24 tokens on a persistent grid take x through the ring, one tile per stage written by
+    a separate x pass with a per-token exponent (17-24: three token tiles, warps of two 16-row
+    tiles): rows of very different magnitudes (bf16) each keep their precision."""
     N, K = 19200, 3072  # 150 tiles: a persistent grid with a tail
     x = randn((M, K), 1.0, torch.bfloat16, 11)
     x[0] *= 3.0e5
@@ -223,3 +225,39 @@ def test_streamed_x_split_and_partial_grids(oracle_mod, N, K, bits, group, M):
     ref = oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group)
     for m in range(M):
         check_close(y[m:m + 1], ref[m:m + 1], torch.bfloat16, f"streamed x split={pd.split}, row {m}")
+
+
+@pytest.mark.parametrize("M", [17, 24])
+def test_wide_form_repeatable_and_in_a_graph(M):
+    """The 17-24 token form: the same bits back to back without a host sync and in graph
+    replays (tail arrival words, per-call x tiles in the stream's workspace)."""
+    N, K = 19328, 2048
+    w = w_input(N, K, torch.bfloat16, 8, 0.02).cuda()
+    P, S, B = q.quantize(w, 4, 64)
+    assert q.plan_default(M, N, K, 4, 64, torch.bfloat16).kernel == q.KERNEL_STREAM
+    xs = [x_input(M, K, torch.bfloat16, seed=s).cuda() for s in range(2)]
+    ref = [q.qmm(x, P, S, B, 4, 64) for x in xs]
+    torch.cuda.synchronize()
+    outs = [q.qmm(xs[i % 2], P, S, B, 4, 64) for i in range(6)]
+    torch.cuda.synchronize()
+    for i, y in enumerate(outs):
+        assert torch.equal(y.view(torch.int16), ref[i % 2].view(torch.int16)), i
+    ys = [torch.empty_like(r) for r in ref]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(2):
+            q.qmm(xs[i], P, S, B, 4, 64, out=ys[i])
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(2):
+            q.qmm(xs[i], P, S, B, 4, 64, out=ys[i])
+    for y in ys:
+        y.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    for i in range(2):
+        assert torch.equal(ys[i].view(torch.int16), ref[i].view(torch.int16)), i
+    assert q.device_errors() == 0
