@@ -561,8 +561,8 @@ qmm_status qmm_grouped(const void* x, const qmm_item* items, int count, int64_t 
             return launch_result(launch_stream_items(a, live, n, sc, st), "qmm_grouped launch");
         }
         if (pl.kernel == QMM_KERNEL_STREAM)
-            return fail(QMM_ERR_UNSUPPORTED, "the streaming kernel takes 1 <= M <= 16 and whole stages and scale "
-                        "blocks of K");
+            return fail(QMM_ERR_UNSUPPORTED, "the streaming kernel takes 1 <= M <= 16 (17..24: 4/8-bit, >= 148 "
+                        "tiles in all) and whole stages and scale blocks of K");
     }
     if (own_calls) {
         // above 16 tokens one even-split launch over the group measured slower than the

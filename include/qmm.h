@@ -197,7 +197,8 @@ typedef struct {
  * Each item must have a multiple of 8 groups per row and a 16-byte multiple of packed bytes
  * per row, with packed, scales, biases, x and y 16-byte aligned; 1 <= M <= 64; else
  * QMM_ERR_UNSUPPORTED and nothing is launched.  `plan` may be NULL or name QMM_KERNEL_AUTO,
- * QMM_KERNEL_STREAM (M <= 16; `split` = its K split, 0 = auto) or QMM_KERNEL_SK (`split` =
+ * QMM_KERNEL_STREAM (M <= 16, or 17-24 on at least 148 tiles at 4/8 bits; `split` = its K
+ * split, 0 = auto) or QMM_KERNEL_SK (`split` =
  * its x mode), with the QMM_PLAN_PDL / QMM_PLAN_STATIC_WEIGHTS flags (NULL = PDL, weights not
  * static).  Each y_i meets the same tolerance as a qmm() call and is bitwise reproducible run
  * to run (how the work is split, and so the order partial sums meet in, depends on the whole

@@ -125,3 +125,20 @@ def test_grouped_rejects():
     assert L.qmm_grouped(x17.data_ptr(), items, 1, 17, 512, 4, 64, 0, ctypes.byref(stp), None) == q.QMM_ERR_UNSUPPORTED
     # M == 0 and all-empty groups are no-ops
     assert L.qmm_grouped(0, items, 1, 0, 512, 4, 64, 0, None, None) == q.QMM_OK
+
+
+@pytest.mark.parametrize("M", [17, 24])
+def test_grouped_streaming_wide_form(oracle_mod, M):
+    """Forced onto the streaming kernel at 17-24 tokens, a group of at least 148 tiles (gate/up,
+    224) runs the eight-warp three-tile form over both matrices' tiles (x streamed, tail tiles in
+    the second matrix's range); the default grouped call takes the matrices' own plans there."""
+    K, Ns, bits, group, dtype = 1024, (14336, 14336), 4, 64, torch.bfloat16
+    mats = _mats(oracle_mod, Ns, K, bits, group, dtype)
+    x = x_input(M, K, dtype)
+    for plan in (q.make_plan(kernel=q.KERNEL_STREAM), None):
+        ys = q.qmm_grouped(x.cuda(), [d for _, d in mats], bits, group, plan=plan)
+        torch.cuda.synchronize()
+        assert q.device_errors() == 0
+        for i, ((op, os_, ob), _) in enumerate(mats):
+            check_close(ys[i], oracle_qmm(oracle_mod, x, op, os_, ob, K, bits, group), dtype,
+                        f"gate_up item {i} M={M} plan={'stream' if plan else 'auto'}")
