@@ -22,6 +22,8 @@
 // cores.
 #include <algorithm>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "qmm_common.cuh"
 #include "qmm_internal.h"
@@ -170,17 +172,34 @@ __global__ void __launch_bounds__(256) qmm_nt_reduce(const float* __restrict__ p
 
 constexpr int kNtSMs = 148;
 
-template <int BITS>
-void launch_nt_tm(int tm, dim3 grid, cudaStream_t stream, const QmmArgs& a, float* part, int gshift, int krange) {
-#define QMM_NT_LAUNCH(T)                                                                                   \
-    qmm_nt_kernel<BITS, T><<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, \
-                                                           int(a.M), int(a.K), int(a.N), gshift, a.is_bf16, krange)
-    if (tm == 1) QMM_NT_LAUNCH(1);
-    else if (tm == 2) QMM_NT_LAUNCH(2);
-    else if constexpr (BITS == 6) QMM_NT_LAUNCH(4);
-    else if (tm == 4) QMM_NT_LAUNCH(4);
-    else QMM_NT_LAUNCH(8);
-#undef QMM_NT_LAUNCH
+using NtKernelFn = void (*)(const uint16_t*, const uint32_t*, const uint16_t*, const uint16_t*, uint16_t*, float*, int,
+                            int, int, int, int, int);
+
+// The instance for the format and tokens a pass (tm = 1, 2, 4, or 8 at 4 and 8 bits).
+NtKernelFn nt_kernel(int bits, int tm) {
+    if (bits == 4) return tm == 1 ? qmm_nt_kernel<4, 1> : tm == 2 ? qmm_nt_kernel<4, 2> : tm == 4 ? qmm_nt_kernel<4, 4> : qmm_nt_kernel<4, 8>;
+    if (bits == 8) return tm == 1 ? qmm_nt_kernel<8, 1> : tm == 2 ? qmm_nt_kernel<8, 2> : tm == 4 ? qmm_nt_kernel<8, 4> : qmm_nt_kernel<8, 8>;
+    return tm == 1 ? qmm_nt_kernel<6, 1> : tm == 2 ? qmm_nt_kernel<6, 2> : qmm_nt_kernel<6, 4>;
+}
+
+// Resident blocks per SM of an instance (its registers decide), cached per device and
+// instance; 8 if the query fails (no device to ask).
+int nt_blocks_per_sm(NtKernelFn fn) {
+    static std::mutex mu;
+    static std::unordered_map<uint64_t, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 8;
+    const uint64_t key = (uint64_t(dev) << 48) ^ uint64_t(reinterpret_cast<uintptr_t>(fn));
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, NT_THREADS, 0) != cudaSuccess || n < 1) {
+        cudaGetLastError();  // a failed query must not leave a sticky error behind
+        n = 8;
+    }
+    cache[key] = n;
+    return n;
 }
 
 }  // namespace
@@ -189,10 +208,27 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     const int cpu = a.bits == 6 ? 16 : 32 / a.bits;
     const int units = int(a.N / cpu);
     const int cblocks = (units + NT_THREADS - 1) / NT_THREADS;
-    // K slices: about eight blocks per SM, at least 64 rows a slice, and the fp32 split sums
+    // tokens a pass: the smallest of 1, 2, 4, 8 (4 at 6 bits) that covers M
+    const int tmax = a.bits == 6 ? 4 : 8;
+    const int tm = a.M >= tmax ? tmax : (a.M > 2 ? 4 : int(a.M));
+    const NtKernelFn fn = nt_kernel(a.bits, tm);
+    // K slices (at least 64 rows each): the fewest whose blocks fill at least 85% of the
+    // resident-block slots of the waves they take (else the best filling), so that neither a
+    // nearly empty last wave nor an under-filled single wave is left; the fp32 split sums are
     // kept under 256 MB
-    int S = std::max(1, (8 * kNtSMs + cblocks - 1) / cblocks);
-    S = std::min<int64_t>(S, std::max<int64_t>(1, a.K / 64));
+    const int64_t slots = int64_t(nt_blocks_per_sm(fn)) * kNtSMs;
+    const int smax = int(std::max<int64_t>(1, std::min<int64_t>(64, a.K / 64)));
+    int S = 1;
+    double best = 0.0;
+    for (int sc = 1; sc <= smax; ++sc) {
+        const int64_t nb = int64_t(cblocks) * sc;
+        const double fill = double(nb) / double((nb + slots - 1) / slots * slots);
+        if (fill > best + 1e-9) {
+            best = fill;
+            S = sc;
+        }
+        if (fill >= 0.85) break;
+    }
     while (S > 1 && int64_t(S) * a.M * a.N * 4 > (int64_t(256) << 20)) --S;
     const int krange = int((a.K + S - 1) / S + 63) / 64 * 64;
     S = int((a.K + krange - 1) / krange);
@@ -206,15 +242,8 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     int gshift = 0;
     while ((1 << gshift) < a.group) ++gshift;
     const dim3 grid(unsigned(cblocks), unsigned(S), 1);
-    // tokens a pass: the smallest of 1, 2, 4, 8 (4 at 6 bits) that covers M
-    const int tmax = a.bits == 6 ? 4 : 8;
-    const int tm = a.M >= tmax ? tmax : (a.M > 2 ? 4 : int(a.M));
-    if (a.bits == 4)
-        launch_nt_tm<4>(tm, grid, stream, a, part, gshift, krange);
-    else if (a.bits == 6)
-        launch_nt_tm<6>(tm, grid, stream, a, part, gshift, krange);
-    else
-        launch_nt_tm<8>(tm, grid, stream, a, part, gshift, krange);
+    fn<<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M), int(a.K), int(a.N),
+                                        gshift, a.is_bf16, krange);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || S == 1) return e;
     const int64_t MN = a.M * a.N;
