@@ -347,8 +347,10 @@ qmm_status qmm_plan_launches(int64_t M, int64_t N, int64_t K, int bits, int grou
     if (M < 0) return fail(QMM_ERR_INVALID_ARG, "negative M");
     if (M > kMaxTotalM) return fail(QMM_ERR_UNSUPPORTED, "M=%lld > %lld", (long long)M, (long long)kMaxTotalM);
     if (!launches) return fail(QMM_ERR_INVALID_ARG, "launches is null");
-    *launches = 0;
-    if (M == 0 || N == 0 || K == 0) return QMM_OK;  // nothing, or a memset
+    if (M == 0 || N == 0 || K == 0) {  // nothing, or a memset
+        *launches = 0;
+        return QMM_OK;
+    }
     // the chunks qmm_ex cuts M into, each with its own plan
     const int64_t nch = (M + kSkMaxTokens - 1) / kSkMaxTokens;
     int64_t m0 = 0;

@@ -210,3 +210,18 @@ def test_plan_launches(L):
     assert q.plan_launches(4, 4096, 0, 4, 64, f16) == 0
     st = q.make_plan(kernel=q.KERNEL_STREAM)
     assert q.plan_launches(4, 4096, 4096, 4, 64, f16, st) == 1
+
+
+def test_plan_launches_rejects(L):
+    """qmm_plan_launches checks its arguments like qmm_plan_default: a null result pointer, a
+    bad dtype, negative or oversized M, an unsupported format; nothing is written then."""
+    n = ctypes.c_int32(-7)
+    assert L.qmm_plan_launches(4, 4096, 4096, 4, 64, 0, None, None) == q.QMM_ERR_INVALID_ARG
+    assert L.qmm_plan_launches(4, 4096, 4096, 4, 64, 9, None, ctypes.byref(n)) == q.QMM_ERR_INVALID_ARG
+    assert L.qmm_plan_launches(-1, 4096, 4096, 4, 64, 0, None, ctypes.byref(n)) == q.QMM_ERR_INVALID_ARG
+    assert L.qmm_plan_launches((1 << 20) + 1, 4096, 4096, 4, 64, 0, None, ctypes.byref(n)) == q.QMM_ERR_UNSUPPORTED
+    assert L.qmm_plan_launches(4, 4096, 4096, 5, 64, 0, None, ctypes.byref(n)) != q.QMM_OK
+    assert n.value == -7
+    bad = q.make_plan(kernel=9)
+    assert L.qmm_plan_launches(4, 4096, 4096, 4, 64, 0, ctypes.byref(bad), ctypes.byref(n)) == q.QMM_ERR_INVALID_ARG
+    assert n.value == -7
