@@ -16,7 +16,7 @@
 // codes (they lie in one group) and is added at the end.  Tokens are taken TM at a time (TM
 // the smallest of 1, 2, 4, 8 that covers M, at most 8, 4 at 6 bits: FMAs on padded tokens would
 // make small-M calls FMA-bound); K is
-// split over grid.y so the grid fills the GPU, and the split sums are added in split order
+// split over grid.y so the grid fills the GPU, and the split sums are added in a fixed order
 // by a second kernel (deterministic).  Coalescing: consecutive threads read consecutive units
 // of a row.  This is the CUDA-core path of the less common form; it does not use the tensor
 // cores.
@@ -151,22 +151,36 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __re
     }
 }
 
-// y[m, n] = sum over the S K slices of part[s][m][n], in slice order.
+// y[m, n] = sum over the S K slices of part[s][m][n].  GL lanes (a power of two, 1..16) share
+// an output: lane l adds the slices of its contiguous run in order (eight loads in flight at a
+// time), then the GL partial sums meet through a shuffle tree, so the order is fixed and the
+// result repeatable; few outputs (the q/o shape) get many lanes each, so that the slices'
+// loads are not a long chain of round trips.
+template <int GL>
 __global__ void __launch_bounds__(256) qmm_nt_reduce(const float* __restrict__ part, uint16_t* __restrict__ y,
                                                      int64_t MN, int S, int is_bf16) {
-    for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < MN; i += int64_t(gridDim.x) * 256) {
-        // in slice order; eight loads in flight at a time
+    const int l = int(threadIdx.x) & (GL - 1);
+    const int per = (S + GL - 1) / GL;
+    const int s0 = min(S, l * per), s1 = min(S, s0 + per);
+    const int64_t step = int64_t(gridDim.x) * (256 / GL);
+    // (every lane of a group runs the same iterations: the shuffles below take whole groups)
+    for (int64_t i0 = int64_t(blockIdx.x) * (256 / GL); i0 < MN; i0 += step) {
+        const int64_t i = i0 + int(threadIdx.x) / GL;
         float v = 0.f;
-        int s = 0;
-        for (; s + 8 <= S; s += 8) {
-            float t[8];
+        if (i < MN) {
+            int s = s0;
+            for (; s + 8 <= s1; s += 8) {
+                float t[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) t[j] = __ldcg(part + int64_t(s + j) * MN + i);
+                for (int j = 0; j < 8; ++j) t[j] = __ldcg(part + int64_t(s + j) * MN + i);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v += t[j];
+                for (int j = 0; j < 8; ++j) v += t[j];
+            }
+            for (; s < s1; ++s) v += __ldcg(part + int64_t(s) * MN + i);
         }
-        for (; s < S; ++s) v += __ldcg(part + int64_t(s) * MN + i);
-        y[i] = nt_round(v, is_bf16);
+#pragma unroll
+        for (int o = GL / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, GL);
+        if (l == 0 && i < MN) y[i] = nt_round(v, is_bf16);
     }
 }
 
@@ -247,8 +261,18 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || S == 1) return e;
     const int64_t MN = a.M * a.N;
-    const int rblocks = int(std::min<int64_t>((MN + 255) / 256, 4 * kNtSMs));
-    qmm_nt_reduce<<<rblocks, 256, 0, stream>>>(part, a.y, MN, S, a.is_bf16);
+    // lanes per output: more while the outputs alone fill fewer than four blocks per SM and
+    // each lane keeps at least four slices
+    int gl = 1;
+    while (gl < 16 && MN * gl < int64_t(4) * kNtSMs * 256 && S >= 8 * gl) gl *= 2;
+    const int rblocks = int(std::min<int64_t>((MN * gl + 255) / 256, 4 * kNtSMs));
+    switch (gl) {
+        case 1: qmm_nt_reduce<1><<<rblocks, 256, 0, stream>>>(part, a.y, MN, S, a.is_bf16); break;
+        case 2: qmm_nt_reduce<2><<<rblocks, 256, 0, stream>>>(part, a.y, MN, S, a.is_bf16); break;
+        case 4: qmm_nt_reduce<4><<<rblocks, 256, 0, stream>>>(part, a.y, MN, S, a.is_bf16); break;
+        case 8: qmm_nt_reduce<8><<<rblocks, 256, 0, stream>>>(part, a.y, MN, S, a.is_bf16); break;
+        default: qmm_nt_reduce<16><<<rblocks, 256, 0, stream>>>(part, a.y, MN, S, a.is_bf16); break;
+    }
     return cudaGetLastError();
 }
 
