@@ -83,7 +83,11 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __re
     const int G = N >> gshift;
     const int j = live ? (n0 >> gshift) : 0;  // the unit's group
     const int64_t rw = int64_t(N) * BITS / 32;  // words per row of W'
-    const int k0 = blockIdx.y * krange, k1 = min(K, k0 + krange);
+    // this block's K slice takes rows y0, y0 + S, y0 + 2S, ... (interleaved: the slices' loads
+    // at any moment are a few rows apart, not a slice apart, which spreads them over the DRAM
+    // channels); krange (rows of a contiguous slice) is an upper bound on their number
+    const int S = int(gridDim.y), y0 = int(blockIdx.y);
+    const int nj = y0 < K ? min(krange, (K - y0 + S - 1) / S) : 0;
     grid_dependency_wait();
     for (int m0 = 0; m0 < M; m0 += TM) {
         float acc[TM][CPU], accb[TM];
@@ -93,12 +97,14 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __re
 #pragma unroll
             for (int i = 0; i < CPU; ++i) acc[t][i] = 0.f;
         }
-        for (int kb = k0; kb < k1; kb += 64) {
-            const int kn = min(64, k1 - kb);
+        for (int jb = 0; jb < nj; jb += 64) {
+            const int kn = min(64, nj - jb);
             __syncthreads();  // the previous rows' x are no longer read
             for (int e = threadIdx.x; e < TM * 64; e += NT_THREADS) {
                 const int t = e / 64, kk = e - t * 64;
-                xs[t][kk] = (m0 + t < M && kk < kn) ? nt_load_x(x, is_bf16, int64_t(m0 + t) * K + kb + kk) : 0.f;
+                xs[t][kk] = (m0 + t < M && kk < kn)
+                                ? nt_load_x(x, is_bf16, int64_t(m0 + t) * K + y0 + int64_t(S) * (jb + kk))
+                                : 0.f;
             }
             __syncthreads();
             if (live) {
@@ -109,7 +115,8 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __re
                     uint16_t sh[RU], bh[RU];
 #pragma unroll
                     for (int r = 0; r < RU; ++r) {
-                        const int k = kb + min(kk0 + r, kn - 1);  // rows past kn repeat the last (unused)
+                        // rows past kn repeat the last (unused)
+                        const int k = y0 + S * (jb + min(kk0 + r, kn - 1));
 #pragma unroll
                         for (int i = 0; i < WPU; ++i) w[r][i] = __ldg(packed + int64_t(k) * rw + int64_t(u) * WPU + i);
                         sh[r] = __ldg(scales + int64_t(k) * G + j);
