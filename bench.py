@@ -362,7 +362,7 @@ def run_nt(q, dev, peak):
                              "frac_of_measured": round(wbytes / t / 1e9 / peak, 4)}
             del g
         out[name] = {"shape": f"W' [K={K}, N={N}] 4-bit g64 {str(dt).replace('torch.', '')}", "weight_sets": len(weights),
-                     "kernel": "qmm_nt_kernel (CUDA cores)", "M": cells}
+                     "kernel": "qmm_nta_kernel (CUDA cores, rows staged by cp.async)", "M": cells}
         del weights
         torch.cuda.empty_cache()
         print(f"[nt] {name}: " + " ".join(f"{m}:{v['gbs']:.0f}" for m, v in cells.items()), file=sys.stderr, flush=True)

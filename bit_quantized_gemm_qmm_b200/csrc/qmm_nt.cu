@@ -19,8 +19,10 @@
 // split over grid.y so the grid fills the GPU, and the split sums are added in a fixed order
 // by a second kernel (deterministic).  Coalescing: consecutive threads read consecutive units
 // of a row.  This is the CUDA-core path of the less common form; it does not use the tensor
-// cores.
+// cores.  Where every copy can be aligned, the pipelined form below (qmm_nta_kernel) runs
+// instead: the same sums, with the rows staged through shared memory by asynchronous copies.
 #include <algorithm>
+#include <utility>
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
@@ -158,6 +160,203 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __re
     }
 }
 
+// ---- the pipelined form: rows staged in shared memory by asynchronous copies --------------
+//
+// The form above keeps RU rows of loads in flight per thread, a few KB per SM: every batch
+// of rows costs a full memory round trip, so small matrices and wide ones alike run far
+// below the copy rate.  Here the block's rows go through a ring of NTA_STAGES slots in shared
+// memory, filled by cp.async (16-byte copies of the codes, 4-byte copies of the scale, bias
+// and x pairs); NTA_STAGES - 1 stages of R rows are in flight while one is summed, tens of
+// KB per block.  The arithmetic is that of the form above (codes exact in fp32, x*s exact, a
+// thread's sums in row order); K slices are contiguous row ranges, so a slice's x is a
+// contiguous run of each token row.  Requirements (the host checks them, else the form
+// above runs): packed 16-byte aligned with 16-byte rows, K even, scales/biases/x 4-byte
+// aligned and N/group even, so that every copy is aligned.
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t n) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t n) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// exact float of a code below 2^23: its bits under the exponent of 2^23, minus 2^23
+__device__ __forceinline__ float code_f32(uint32_t q) { return __uint_as_float(q | 0x4B000000u) - 8388608.0f; }
+
+// Code i of a 4- or 8-bit word as the float 1 + q/2^BITS (exact): the code shifted to the top
+// of the significand under the exponent of 1.0, one shift and one logic operation.  Sums of
+// xs * (1 + q/2^BITS) minus the sum of xs, times 2^BITS, give the sums of xs * q.
+template <int BITS, int I> __device__ __forceinline__ float code_1p(uint32_t w) {
+    constexpr int SH = 23 - BITS - BITS * I;
+    constexpr uint32_t MASK = ((1u << BITS) - 1u) << (23 - BITS);
+    const uint32_t v = SH >= 0 ? (w << (SH >= 0 ? SH : 0)) : (w >> (SH < 0 ? -SH : 0));
+    return __uint_as_float((v & MASK) | 0x3F800000u);
+}
+template <int BITS, int... I>
+__device__ __forceinline__ void codes_1p(uint32_t w, float* f, std::integer_sequence<int, I...>) {
+    ((f[I] = code_1p<BITS, I>(w)), ...);
+}
+
+template <int BITS, int TM_> struct NtaFmt {
+    static constexpr int CPU = NtFmt<BITS, TM_>::CPU, WPU = NtFmt<BITS, TM_>::WPU, TM = TM_;
+    static constexpr int CW = NT_THREADS * WPU;             // code words of a row of the block's strip
+    static constexpr int R = BITS == 6 ? 8 : 16;            // rows a stage
+    static constexpr int STAGES = 4;                        // ring slots (41-57 KB a block)
+    static constexpr int SBH = NT_THREADS * CPU / 32 / 2;   // scale words a row at most (group 32)
+    static constexpr int SBW = 2 * SBH;                     // scale then bias words a row
+    static constexpr int XW = TM * R / 2;                   // x words (pairs of rows) a stage
+    static constexpr int STAGE_WORDS = R * CW + R * SBW + XW;
+    static constexpr int SMEM = STAGES * STAGE_WORDS * 4;
+};
+
+template <int BITS, int TM_>
+__global__ void __launch_bounds__(NT_THREADS) qmm_nta_kernel(const uint16_t* __restrict__ x,
+                                                             const uint32_t* __restrict__ packed,
+                                                             const uint16_t* __restrict__ scales,
+                                                             const uint16_t* __restrict__ biases,
+                                                             uint16_t* __restrict__ y, float* __restrict__ part,
+                                                             int M, int K, int N, int gshift, int is_bf16,
+                                                             int krange) {
+    using F = NtaFmt<BITS, TM_>;
+    constexpr int CPU = F::CPU, WPU = F::WPU, TM = F::TM, CW = F::CW, R = F::R, NS = F::STAGES;
+    constexpr int SBH = F::SBH, SBW = F::SBW, XW = F::XW, SW = F::STAGE_WORDS;
+    constexpr bool ONEP = BITS != 6;  // codes as 1 + q/2^BITS (4 and 8 bits)
+    extern __shared__ __align__(16) uint32_t nta_smem[];
+    const int tid = int(threadIdx.x);
+    const int units = N / CPU;
+    const int u = blockIdx.x * NT_THREADS + tid;
+    const bool live = u < units;
+    const int n0 = u * CPU;
+    const int G = N >> gshift;
+    const int jl = (tid * CPU) >> gshift;                        // the unit's group within the block
+    const int gb = (NT_THREADS * CPU >> gshift) / 2;             // scale words of a row of the block
+    const int j0 = blockIdx.x * (NT_THREADS * CPU >> gshift);   // the block's first group (even)
+    const int64_t rw = int64_t(N) * BITS / 32;                   // words per row of W'
+    const int64_t cw0 = int64_t(blockIdx.x) * CW;                // the strip's first word of a row
+    const int k0 = int(blockIdx.y) * krange;
+    const int kend = min(K, k0 + krange);
+    const int nj = max(0, kend - k0);
+    const int nchunk = (nj + R - 1) / R;
+    const uint32_t sbase = smem_addr(nta_smem);
+    grid_dependency_wait();
+    for (int m0 = 0; m0 < M; m0 += TM) {
+        // stage c of this pass into slot c % NS (an empty group past the last, so that the
+        // wait counts stay uniform)
+        auto issue = [&](int c) {
+            if (c < nchunk) {
+                const int kb = k0 + c * R;
+                const uint32_t slot = sbase + uint32_t((c % NS) * SW) * 4u;
+                for (int e = tid; e < R * CW / 4; e += NT_THREADS) {
+                    const int r = e / (CW / 4), c4 = (e - r * (CW / 4)) * 4;
+                    const int k = kb + r;
+                    const bool ok = k < kend && cw0 + c4 < rw;
+                    const uint32_t* src = ok ? packed + int64_t(k) * rw + cw0 + c4 : packed;
+                    cp_async16(slot + uint32_t(r * CW + c4) * 4u, src, ok ? 16u : 0u);
+                }
+                const uint32_t sslot = slot + uint32_t(R * CW) * 4u;
+                for (int e = tid; e < R * 2 * gb; e += NT_THREADS) {
+                    const int r = e / (2 * gb), w = e - r * (2 * gb);
+                    const int which = w >= gb, wi = w - which * gb;
+                    const int k = kb + r, j = j0 + 2 * wi;
+                    const bool ok = k < kend && j < G;
+                    const uint16_t* base = which ? biases : scales;
+                    const uint16_t* src = ok ? base + int64_t(k) * G + j : base;
+                    cp_async4(sslot + uint32_t(r * SBW + which * SBH + wi) * 4u, src, ok ? 4u : 0u);
+                }
+                const uint32_t xslot = sslot + uint32_t(R * SBW) * 4u;
+                for (int e = tid; e < XW; e += NT_THREADS) {
+                    const int t = e / (R / 2), p = e - t * (R / 2);
+                    const int k = kb + 2 * p, m = m0 + t;
+                    const bool ok = m < M && k < kend;
+                    const uint16_t* src = ok ? x + int64_t(m) * K + k : x;
+                    cp_async4(xslot + uint32_t(e) * 4u, src, ok ? 4u : 0u);
+                }
+            }
+            cp_async_commit();
+        };
+        float acc[TM][CPU], accb[TM], accx[TM];
+#pragma unroll
+        for (int t = 0; t < TM; ++t) {
+            accb[t] = 0.f;
+            accx[t] = 0.f;
+#pragma unroll
+            for (int i = 0; i < CPU; ++i) acc[t][i] = 0.f;
+        }
+        __syncthreads();  // the previous pass has finished reading every slot
+#pragma unroll
+        for (int c = 0; c < NS - 1; ++c) issue(c);
+        for (int c = 0; c < nchunk; ++c) {
+            cp_async_wait<NS - 2>();
+            __syncthreads();  // stage c has landed for all threads; slot (c - 1) % NS is free
+            issue(c + NS - 1);
+            const uint32_t* cs = nta_smem + (c % NS) * SW;
+            const uint32_t* sb = cs + R * CW;
+            const uint16_t* xh = reinterpret_cast<const uint16_t*>(sb + R * SBW);
+            const int kn = min(R, kend - (k0 + c * R));
+            if (live) {
+                const uint32_t* cst = cs + tid * WPU;
+                const uint32_t* sbt = sb + (jl >> 1);
+                const int hs = (jl & 1) * 16;
+                auto row = [&](int r) {
+                    uint32_t w[WPU];
+#pragma unroll
+                    for (int i = 0; i < WPU; ++i) w[i] = cst[r * CW + i];
+                    const float s = __half2float(__ushort_as_half(uint16_t(sbt[r * SBW] >> hs)));
+                    const float b = __half2float(__ushort_as_half(uint16_t(sbt[r * SBW + SBH] >> hs)));
+                    float qf[CPU];
+                    if constexpr (ONEP) {
+                        codes_1p<BITS>(w[0], qf, std::make_integer_sequence<int, CPU>{});
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < CPU; ++i) qf[i] = code_f32(nt_code<BITS>(w, i));
+                    }
+#pragma unroll
+                    for (int t = 0; t < TM; ++t) {
+                        const uint16_t xv16 = xh[t * R + r];
+                        const float xv = is_bf16 ? __uint_as_float(uint32_t(xv16) << 16)
+                                                 : __half2float(__ushort_as_half(xv16));
+                        const float xsv = xv * s;  // exact: 11-bit by 11-bit significands
+                        accb[t] = fmaf(xv, b, accb[t]);
+                        if constexpr (ONEP) accx[t] += xsv;
+#pragma unroll
+                        for (int i = 0; i < CPU; ++i) acc[t][i] = fmaf(xsv, qf[i], acc[t][i]);
+                    }
+                };
+                if (kn == R) {
+                    // a whole stage: unrolled in runs of UR rows (all of it for one token; fewer
+                    // rows for more tokens, whose longer bodies would outgrow the instruction cache)
+                    constexpr int UR = TM == 1 ? R : 2;
+#pragma unroll 1
+                    for (int r0 = 0; r0 < R; r0 += UR) {
+#pragma unroll
+                        for (int r = 0; r < UR; ++r) row(r0 + r);
+                    }
+                } else {
+                    for (int r = 0; r < kn; ++r) row(r);
+                }
+            }
+        }
+        cp_async_wait<0>();  // the trailing empty groups
+        if (live) {
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+                const int m = m0 + t;
+                if (m >= M) break;
+#pragma unroll
+                for (int i = 0; i < CPU; ++i) {
+                    const float v = (ONEP ? (acc[t][i] - accx[t]) * float(1 << BITS) : acc[t][i]) + accb[t];
+                    if (part) part[(int64_t(blockIdx.y) * M + m) * N + n0 + i] = v;
+                    else y[int64_t(m) * N + n0 + i] = nt_round(v, is_bf16);
+                }
+            }
+        }
+    }
+}
+
 // y[m, n] = sum over the S K slices of part[s][m][n].  GL lanes (a power of two, 1..16) share
 // an output: lane l adds the slices of its contiguous run in order (eight loads in flight at a
 // time), then the GL partial sums meet through a shuffle tree, so the order is fixed and the
@@ -203,24 +402,57 @@ NtKernelFn nt_kernel(int bits, int tm) {
     return tm == 1 ? qmm_nt_kernel<6, 1> : tm == 2 ? qmm_nt_kernel<6, 2> : qmm_nt_kernel<6, 4>;
 }
 
-// Resident blocks per SM of an instance (its registers decide), cached per device and
-// instance; 8 if the query fails (no device to ask).
-int nt_blocks_per_sm(NtKernelFn fn) {
+template <int BITS, int TM> NtKernelFn nta_instance() {
+    static_assert(NtaFmt<BITS, TM>::SMEM <= 227 * 1024, "ring larger than a block's shared memory");
+    return qmm_nta_kernel<BITS, TM>;
+}
+
+// The pipelined instance for the format and tokens a pass, and its shared memory.
+NtKernelFn nta_kernel(int bits, int tm, int* smem) {
+    if (bits == 4) {
+        *smem = tm == 1 ? NtaFmt<4, 1>::SMEM : tm == 2 ? NtaFmt<4, 2>::SMEM : tm == 4 ? NtaFmt<4, 4>::SMEM : NtaFmt<4, 8>::SMEM;
+        return tm == 1 ? nta_instance<4, 1>() : tm == 2 ? nta_instance<4, 2>() : tm == 4 ? nta_instance<4, 4>() : nta_instance<4, 8>();
+    }
+    if (bits == 8) {
+        *smem = tm == 1 ? NtaFmt<8, 1>::SMEM : tm == 2 ? NtaFmt<8, 2>::SMEM : tm == 4 ? NtaFmt<8, 4>::SMEM : NtaFmt<8, 8>::SMEM;
+        return tm == 1 ? nta_instance<8, 1>() : tm == 2 ? nta_instance<8, 2>() : tm == 4 ? nta_instance<8, 4>() : nta_instance<8, 8>();
+    }
+    *smem = tm == 1 ? NtaFmt<6, 1>::SMEM : tm == 2 ? NtaFmt<6, 2>::SMEM : NtaFmt<6, 4>::SMEM;
+    return tm == 1 ? nta_instance<6, 1>() : tm == 2 ? nta_instance<6, 2>() : nta_instance<6, 4>();
+}
+
+// Resident blocks per SM of an instance with `smem` bytes of dynamic shared memory (the
+// attribute is raised to it first), cached per device and instance; 8 if the query fails (no
+// device to ask), and a failed attribute call is returned.
+cudaError_t nt_blocks_per_sm(NtKernelFn fn, int smem, int* blocks) {
     static std::mutex mu;
     static std::unordered_map<uint64_t, int> cache;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 8;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        *blocks = 8;
+        return cudaSuccess;
+    }
     const uint64_t key = (uint64_t(dev) << 48) ^ uint64_t(reinterpret_cast<uintptr_t>(fn));
     std::lock_guard<std::mutex> lk(mu);
     auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
+    if (it != cache.end()) {
+        *blocks = it->second;
+        return cudaSuccess;
+    }
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, NT_THREADS, 0) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, NT_THREADS, size_t(smem)) != cudaSuccess || n < 1) {
         cudaGetLastError();  // a failed query must not leave a sticky error behind
         n = 8;
     }
     cache[key] = n;
-    return n;
+    *blocks = n;
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -232,12 +464,21 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     // tokens a pass: the smallest of 1, 2, 4, 8 (4 at 6 bits) that covers M
     const int tmax = a.bits == 6 ? 4 : 8;
     const int tm = a.M >= tmax ? tmax : (a.M > 2 ? 4 : int(a.M));
-    const NtKernelFn fn = nt_kernel(a.bits, tm);
+    // the pipelined form wherever every copy it makes is aligned
+    const int64_t rbytes = a.N * a.bits / 8;
+    auto al = [](const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0; };
+    const bool pipelined = rbytes % 16 == 0 && a.K % 2 == 0 && (a.N / a.group) % 2 == 0 && al(a.packed, 16) &&
+                           al(a.x, 4) && al(a.scales, 4) && al(a.biases, 4);
+    int smem = 0;
+    const NtKernelFn fn = pipelined ? nta_kernel(a.bits, tm, &smem) : nt_kernel(a.bits, tm);
+    int bps = 0;
+    cudaError_t e0 = nt_blocks_per_sm(fn, smem, &bps);
+    if (e0 != cudaSuccess) return e0;
     // K slices (at least 64 rows each): the fewest whose blocks fill at least 85% of the
     // resident-block slots of the waves they take (else the best filling), so that neither a
     // nearly empty last wave nor an under-filled single wave is left; the fp32 split sums are
     // kept under 256 MB
-    const int64_t slots = int64_t(nt_blocks_per_sm(fn)) * kNtSMs;
+    const int64_t slots = int64_t(bps) * kNtSMs;
     const int smax = int(std::max<int64_t>(1, std::min<int64_t>(64, a.K / 64)));
     int S = 1;
     double best = 0.0;
@@ -263,7 +504,7 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     int gshift = 0;
     while ((1 << gshift) < a.group) ++gshift;
     const dim3 grid(unsigned(cblocks), unsigned(S), 1);
-    fn<<<grid, NT_THREADS, 0, stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M), int(a.K), int(a.N),
+    fn<<<grid, NT_THREADS, size_t(smem), stream>>>(a.x, a.packed, a.scales, a.biases, a.y, part, int(a.M), int(a.K), int(a.N),
                                         gshift, a.is_bf16, krange);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || S == 1) return e;

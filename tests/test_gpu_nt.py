@@ -51,6 +51,29 @@ def test_shapes(oracle_mod, M, K, N):
     _run(oracle_mod, M, K, N, 4, 64, torch.float16)
 
 
+@pytest.mark.parametrize("M,K,N,bits,group", [(2, 99, 512, 4, 64), (3, 256, 96, 4, 32), (5, 128, 96, 6, 32),
+                                                (9, 200, 224, 8, 32)])
+def test_forms_without_aligned_copies(oracle_mod, M, K, N, bits, group):
+    """Shapes whose rows or pointers cannot be copied in aligned 4/16-byte pieces (odd K, an
+    odd number of groups a row, rows not a multiple of 16 bytes) take the per-thread form."""
+    _run(oracle_mod, M, K, N, bits, group, torch.float16)
+
+
+@pytest.mark.parametrize("M", [1, 6])
+def test_x_not_4_byte_aligned(oracle_mod, M):
+    K, N = 512, 1024
+    wp = w_input(K, N, torch.float16, 7)
+    op, os_, ob = oracle_quantize(oracle_mod, wp, 4, 64)
+    P, S, B = to_device_weights(op, os_, ob)
+    x = x_input(M, K, torch.float16)
+    buf = torch.zeros(M * K + 1, dtype=torch.float16, device="cuda")
+    xo = buf[1:].view(M, K)  # 2-byte aligned only
+    xo.copy_(x.cuda())
+    y = q.qmm_nt(xo, P, S, B, 4, 64)
+    torch.cuda.synchronize()
+    check_close(y, _nt_ref(oracle_mod, x, op, os_, ob, N, 4, 64), torch.float16, f"qmm_nt x+2B M={M}")
+
+
 def test_bf16_large_activations(oracle_mod):
     M, K, N = 3, 1024, 256
     x = randn((M, K), 1.0, torch.bfloat16, 5)
