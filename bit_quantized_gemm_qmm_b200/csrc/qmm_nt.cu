@@ -201,19 +201,24 @@ __device__ __forceinline__ void codes_1p(uint32_t w, float* f, std::integer_sequ
     ((f[I] = code_1p<BITS, I>(w)), ...);
 }
 
-template <int BITS, int TM_> struct NtaFmt {
+template <int BITS, int TM_, int UPT_> struct NtaFmt {
     static constexpr int CPU = NtFmt<BITS, TM_>::CPU, WPU = NtFmt<BITS, TM_>::WPU, TM = TM_;
-    static constexpr int CW = NT_THREADS * WPU;             // code words of a row of the block's strip
-    static constexpr int R = BITS == 6 ? 8 : 16;            // rows a stage
+    // packed units a thread (1 or 2; 2 only at 4 and 8 bits: the per-row scale, bias and x
+    // handling is then shared by the 16 or 8 codes of one group)
+    static constexpr int UPT = UPT_;
+    static_assert(UPT == 1 || (UPT == 2 && BITS != 6), "two units a thread at 4 and 8 bits only");
+    static constexpr int CPT = CPU * UPT;                   // codes a thread
+    static constexpr int CW = NT_THREADS * WPU * UPT;       // code words of a row of the block's strip
+    static constexpr int R = (BITS == 6 || UPT == 2) ? 8 : 16;  // rows a stage (16 KB of codes at 4/8 bits)
     static constexpr int STAGES = 4;                        // ring slots (41-57 KB a block)
-    static constexpr int SBH = NT_THREADS * CPU / 32 / 2;   // scale words a row at most (group 32)
+    static constexpr int SBH = NT_THREADS * CPT / 32 / 2;   // scale words a row at most (group 32)
     static constexpr int SBW = 2 * SBH;                     // scale then bias words a row
     static constexpr int XW = TM * R / 2;                   // x words (pairs of rows) a stage
     static constexpr int STAGE_WORDS = R * CW + R * SBW + XW;
     static constexpr int SMEM = STAGES * STAGE_WORDS * 4;
 };
 
-template <int BITS, int TM_>
+template <int BITS, int TM_, int UPT_>
 __global__ void __launch_bounds__(NT_THREADS) qmm_nta_kernel(const uint16_t* __restrict__ x,
                                                              const uint32_t* __restrict__ packed,
                                                              const uint16_t* __restrict__ scales,
@@ -221,20 +226,23 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nta_kernel(const uint16_t* __r
                                                              uint16_t* __restrict__ y, float* __restrict__ part,
                                                              int M, int K, int N, int gshift, int is_bf16,
                                                              int krange) {
-    using F = NtaFmt<BITS, TM_>;
-    constexpr int CPU = F::CPU, WPU = F::WPU, TM = F::TM, CW = F::CW, R = F::R, NS = F::STAGES;
+    using F = NtaFmt<BITS, TM_, UPT_>;
+    constexpr int CPU = F::CPU, WPU = F::WPU, UPT = F::UPT, CPT = F::CPT, TM = F::TM, CW = F::CW, R = F::R;
+    constexpr int NS = F::STAGES;
     constexpr int SBH = F::SBH, SBW = F::SBW, XW = F::XW, SW = F::STAGE_WORDS;
     constexpr bool ONEP = BITS != 6;  // codes as 1 + q/2^BITS (4 and 8 bits)
     extern __shared__ __align__(16) uint32_t nta_smem[];
     const int tid = int(threadIdx.x);
     const int units = N / CPU;
-    const int u = blockIdx.x * NT_THREADS + tid;
-    const bool live = u < units;
+    const int u = (blockIdx.x * NT_THREADS + tid) * UPT;          // the thread's first unit
+    const bool live = u < units;                                 // (units is a multiple of UPT)
     const int n0 = u * CPU;
     const int G = N >> gshift;
-    const int jl = (tid * CPU) >> gshift;                        // the unit's group within the block
-    const int gb = (NT_THREADS * CPU >> gshift) / 2;             // scale words of a row of the block
-    const int j0 = blockIdx.x * (NT_THREADS * CPU >> gshift);   // the block's first group (even)
+    const int jl = (tid * CPT) >> gshift;                        // the thread's group within the block
+    const int gbl = NT_THREADS * CPT >> gshift;                  // groups of the block: a power of two
+    const int gb = gbl / 2;                                      // scale words of a row of the block
+    const int lg = 31 - __clz(gbl);                              // log2 of the scale+bias words a row
+    const int j0 = blockIdx.x * gbl;                             // the block's first group (even)
     const int64_t rw = int64_t(N) * BITS / 32;                   // words per row of W'
     const int64_t cw0 = int64_t(blockIdx.x) * CW;                // the strip's first word of a row
     const int k0 = int(blockIdx.y) * krange;
@@ -259,7 +267,7 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nta_kernel(const uint16_t* __r
                 }
                 const uint32_t sslot = slot + uint32_t(R * CW) * 4u;
                 for (int e = tid; e < R * 2 * gb; e += NT_THREADS) {
-                    const int r = e / (2 * gb), w = e - r * (2 * gb);
+                    const int r = e >> lg, w = e & (gbl - 1);
                     const int which = w >= gb, wi = w - which * gb;
                     const int k = kb + r, j = j0 + 2 * wi;
                     const bool ok = k < kend && j < G;
@@ -278,13 +286,13 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nta_kernel(const uint16_t* __r
             }
             cp_async_commit();
         };
-        float acc[TM][CPU], accb[TM], accx[TM];
+        float acc[TM][CPT], accb[TM], accx[TM];
 #pragma unroll
         for (int t = 0; t < TM; ++t) {
             accb[t] = 0.f;
             accx[t] = 0.f;
 #pragma unroll
-            for (int i = 0; i < CPU; ++i) acc[t][i] = 0.f;
+            for (int i = 0; i < CPT; ++i) acc[t][i] = 0.f;
         }
         __syncthreads();  // the previous pass has finished reading every slot
 #pragma unroll
@@ -298,18 +306,26 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nta_kernel(const uint16_t* __r
             const uint16_t* xh = reinterpret_cast<const uint16_t*>(sb + R * SBW);
             const int kn = min(R, kend - (k0 + c * R));
             if (live) {
-                const uint32_t* cst = cs + tid * WPU;
+                const uint32_t* cst = cs + tid * WPU * UPT;
                 const uint32_t* sbt = sb + (jl >> 1);
                 const int hs = (jl & 1) * 16;
                 auto row = [&](int r) {
-                    uint32_t w[WPU];
+                    uint32_t w[WPU * UPT];
+                    if constexpr (UPT == 2) {
+                        const uint2 w2 = *reinterpret_cast<const uint2*>(cst + r * CW);
+                        w[0] = w2.x;
+                        w[1] = w2.y;
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < WPU; ++i) w[i] = cst[r * CW + i];
+                        for (int i = 0; i < WPU; ++i) w[i] = cst[r * CW + i];
+                    }
                     const float s = __half2float(__ushort_as_half(uint16_t(sbt[r * SBW] >> hs)));
                     const float b = __half2float(__ushort_as_half(uint16_t(sbt[r * SBW + SBH] >> hs)));
-                    float qf[CPU];
+                    float qf[CPT];
                     if constexpr (ONEP) {
-                        codes_1p<BITS>(w[0], qf, std::make_integer_sequence<int, CPU>{});
+#pragma unroll
+                        for (int v = 0; v < UPT; ++v)
+                            codes_1p<BITS>(w[v], qf + v * CPU, std::make_integer_sequence<int, CPU>{});
                     } else {
 #pragma unroll
                         for (int i = 0; i < CPU; ++i) qf[i] = code_f32(nt_code<BITS>(w, i));
@@ -323,7 +339,7 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nta_kernel(const uint16_t* __r
                         accb[t] = fmaf(xv, b, accb[t]);
                         if constexpr (ONEP) accx[t] += xsv;
 #pragma unroll
-                        for (int i = 0; i < CPU; ++i) acc[t][i] = fmaf(xsv, qf[i], acc[t][i]);
+                        for (int i = 0; i < CPT; ++i) acc[t][i] = fmaf(xsv, qf[i], acc[t][i]);
                     }
                 };
                 if (kn == R) {
@@ -347,7 +363,7 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nta_kernel(const uint16_t* __r
                 const int m = m0 + t;
                 if (m >= M) break;
 #pragma unroll
-                for (int i = 0; i < CPU; ++i) {
+                for (int i = 0; i < CPT; ++i) {
                     const float v = (ONEP ? (acc[t][i] - accx[t]) * float(1 << BITS) : acc[t][i]) + accb[t];
                     if (part) part[(int64_t(blockIdx.y) * M + m) * N + n0 + i] = v;
                     else y[int64_t(m) * N + n0 + i] = nt_round(v, is_bf16);
@@ -402,23 +418,24 @@ NtKernelFn nt_kernel(int bits, int tm) {
     return tm == 1 ? qmm_nt_kernel<6, 1> : tm == 2 ? qmm_nt_kernel<6, 2> : qmm_nt_kernel<6, 4>;
 }
 
-template <int BITS, int TM> NtKernelFn nta_instance() {
-    static_assert(NtaFmt<BITS, TM>::SMEM <= 227 * 1024, "ring larger than a block's shared memory");
-    return qmm_nta_kernel<BITS, TM>;
+template <int BITS, int TM, int UPT> NtKernelFn nta_instance(int* smem) {
+    static_assert(NtaFmt<BITS, TM, UPT>::SMEM <= 227 * 1024, "ring larger than a block's shared memory");
+    *smem = NtaFmt<BITS, TM, UPT>::SMEM;
+    return qmm_nta_kernel<BITS, TM, UPT>;
 }
 
-// The pipelined instance for the format and tokens a pass, and its shared memory.
-NtKernelFn nta_kernel(int bits, int tm, int* smem) {
+// The pipelined instance for the format, tokens a pass and units a thread, and its shared
+// memory.
+NtKernelFn nta_kernel(int bits, int tm, int upt, int* smem) {
     if (bits == 4) {
-        *smem = tm == 1 ? NtaFmt<4, 1>::SMEM : tm == 2 ? NtaFmt<4, 2>::SMEM : tm == 4 ? NtaFmt<4, 4>::SMEM : NtaFmt<4, 8>::SMEM;
-        return tm == 1 ? nta_instance<4, 1>() : tm == 2 ? nta_instance<4, 2>() : tm == 4 ? nta_instance<4, 4>() : nta_instance<4, 8>();
+        if (tm == 2) return upt == 2 ? nta_instance<4, 2, 2>(smem) : nta_instance<4, 2, 1>(smem);
+        return tm == 1 ? nta_instance<4, 1, 1>(smem) : tm == 4 ? nta_instance<4, 4, 1>(smem) : nta_instance<4, 8, 1>(smem);
     }
     if (bits == 8) {
-        *smem = tm == 1 ? NtaFmt<8, 1>::SMEM : tm == 2 ? NtaFmt<8, 2>::SMEM : tm == 4 ? NtaFmt<8, 4>::SMEM : NtaFmt<8, 8>::SMEM;
-        return tm == 1 ? nta_instance<8, 1>() : tm == 2 ? nta_instance<8, 2>() : tm == 4 ? nta_instance<8, 4>() : nta_instance<8, 8>();
+        if (tm == 2) return upt == 2 ? nta_instance<8, 2, 2>(smem) : nta_instance<8, 2, 1>(smem);
+        return tm == 1 ? nta_instance<8, 1, 1>(smem) : tm == 4 ? nta_instance<8, 4, 1>(smem) : nta_instance<8, 8, 1>(smem);
     }
-    *smem = tm == 1 ? NtaFmt<6, 1>::SMEM : tm == 2 ? NtaFmt<6, 2>::SMEM : NtaFmt<6, 4>::SMEM;
-    return tm == 1 ? nta_instance<6, 1>() : tm == 2 ? nta_instance<6, 2>() : nta_instance<6, 4>();
+    return tm == 1 ? nta_instance<6, 1, 1>(smem) : tm == 2 ? nta_instance<6, 2, 1>(smem) : nta_instance<6, 4, 1>(smem);
 }
 
 // Resident blocks per SM of an instance with `smem` bytes of dynamic shared memory (the
@@ -460,7 +477,6 @@ cudaError_t nt_blocks_per_sm(NtKernelFn fn, int smem, int* blocks) {
 cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     const int cpu = a.bits == 6 ? 16 : 32 / a.bits;
     const int units = int(a.N / cpu);
-    const int cblocks = (units + NT_THREADS - 1) / NT_THREADS;
     // tokens a pass: the smallest of 1, 2, 4, 8 (4 at 6 bits) that covers M
     const int tmax = a.bits == 6 ? 4 : 8;
     const int tm = a.M >= tmax ? tmax : (a.M > 2 ? 4 : int(a.M));
@@ -469,8 +485,14 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     auto al = [](const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0; };
     const bool pipelined = rbytes % 16 == 0 && a.K % 2 == 0 && (a.N / a.group) % 2 == 0 && al(a.packed, 16) &&
                            al(a.x, 4) && al(a.scales, 4) && al(a.biases, 4);
+    // units a thread: two in the pipelined form at 4 and 8 bits for two tokens a pass on wide
+    // matrices (the LM-head shape +7%, bound by instruction issue); one for one token (two
+    // measured -5%: half the column blocks, twice the stages) and on narrow matrices (q/o -10%:
+    // half as many blocks, which are bound by latency)
+    const int upt = (pipelined && a.bits != 6 && tm == 2 && units >= 16 * 2 * NT_THREADS) ? 2 : 1;
+    const int cblocks = (units + NT_THREADS * upt - 1) / (NT_THREADS * upt);
     int smem = 0;
-    const NtKernelFn fn = pipelined ? nta_kernel(a.bits, tm, &smem) : nt_kernel(a.bits, tm);
+    const NtKernelFn fn = pipelined ? nta_kernel(a.bits, tm, upt, &smem) : nt_kernel(a.bits, tm);
     int bps = 0;
     cudaError_t e0 = nt_blocks_per_sm(fn, smem, &bps);
     if (e0 != cudaSuccess) return e0;
@@ -492,7 +514,11 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
         if (fill >= 0.85) break;
     }
     while (S > 1 && int64_t(S) * a.M * a.N * 4 > (int64_t(256) << 20)) --S;
-    const int krange = int((a.K + S - 1) / S + 63) / 64 * 64;
+    // slice rows: a multiple of 64 in the per-thread form, of 16 (a stage) in the pipelined one,
+    // whose slice count then stays the one chosen (LM-head shape: 9 slices, 0.91 of two waves,
+    // not 8 at 0.81)
+    const int gran = pipelined ? 16 : 64;
+    const int krange = int((a.K + S - 1) / S + gran - 1) / gran * gran;
     S = int((a.K + krange - 1) / krange);
     float* part = nullptr;
     if (S > 1) {

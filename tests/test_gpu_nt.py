@@ -59,6 +59,37 @@ def test_forms_without_aligned_copies(oracle_mod, M, K, N, bits, group):
     _run(oracle_mod, M, K, N, bits, group, torch.float16)
 
 
+@pytest.mark.parametrize("bits,N,group", [(4, 33024, 64), (4, 32768, 32), (8, 16640, 128)])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_wide_two_tokens(oracle_mod, bits, N, group, dtype):
+    """Two tokens on a wide matrix: two packed units a thread (a partial last column block at
+    N = 33024 and 16640)."""
+    _run(oracle_mod, 2, 320, N, bits, group, dtype, 1.0 if dtype == torch.float16 else 0.02)
+
+
+_NT_FULL = {}
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 16])
+def test_lmhead_shape_full_size_sampled(oracle_mod, M):
+    """The LM-head size in the non-transposed form (W' [K=4096, N=151936] 4-bit g64, bf16),
+    launched as the bench launches it; the oracle checks 256-column samples (first, middle,
+    last) of y, their weights quantized by the oracle from the same columns of W'."""
+    K, N = 4096, 151936
+    if "w" not in _NT_FULL:
+        _NT_FULL["w"] = w_input(K, N, torch.bfloat16, 0, 0.02)  # W' [K, N]
+        _NT_FULL["q"] = q.quantize(_NT_FULL["w"].cuda(), 4, 64)
+    wp = _NT_FULL["w"]
+    P, S, B = _NT_FULL["q"]
+    x = x_input(M, K, torch.bfloat16)
+    y = q.qmm_nt(x.cuda(), P, S, B, 4, 64)
+    torch.cuda.synchronize()
+    for c0 in sorted({0, (N // 2) // 256 * 256, N - 256}):
+        op, os_, ob = oracle_quantize(oracle_mod, wp[:, c0:c0 + 256].contiguous(), 4, 64)
+        ref = _nt_ref(oracle_mod, x, op, os_, ob, 256, 4, 64)
+        check_close(y[:, c0:c0 + 256], ref, torch.bfloat16, f"qmm_nt LM-head shape M={M} columns {c0}:{c0 + 256}")
+
+
 @pytest.mark.parametrize("M", [1, 6])
 def test_x_not_4_byte_aligned(oracle_mod, M):
     K, N = 512, 1024
