@@ -429,11 +429,13 @@ template <int BITS, int TM, int UPT> NtKernelFn nta_instance(int* smem) {
 NtKernelFn nta_kernel(int bits, int tm, int upt, int* smem) {
     if (bits == 4) {
         if (tm == 2) return upt == 2 ? nta_instance<4, 2, 2>(smem) : nta_instance<4, 2, 1>(smem);
-        return tm == 1 ? nta_instance<4, 1, 1>(smem) : tm == 4 ? nta_instance<4, 4, 1>(smem) : nta_instance<4, 8, 1>(smem);
+        if (tm == 4) return upt == 2 ? nta_instance<4, 4, 2>(smem) : nta_instance<4, 4, 1>(smem);
+        return tm == 1 ? nta_instance<4, 1, 1>(smem) : nta_instance<4, 8, 1>(smem);
     }
     if (bits == 8) {
         if (tm == 2) return upt == 2 ? nta_instance<8, 2, 2>(smem) : nta_instance<8, 2, 1>(smem);
-        return tm == 1 ? nta_instance<8, 1, 1>(smem) : tm == 4 ? nta_instance<8, 4, 1>(smem) : nta_instance<8, 8, 1>(smem);
+        if (tm == 4) return upt == 2 ? nta_instance<8, 4, 2>(smem) : nta_instance<8, 4, 1>(smem);
+        return tm == 1 ? nta_instance<8, 1, 1>(smem) : nta_instance<8, 8, 1>(smem);
     }
     return tm == 1 ? nta_instance<6, 1, 1>(smem) : tm == 2 ? nta_instance<6, 2, 1>(smem) : nta_instance<6, 4, 1>(smem);
 }
@@ -485,11 +487,12 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     auto al = [](const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0; };
     const bool pipelined = rbytes % 16 == 0 && a.K % 2 == 0 && (a.N / a.group) % 2 == 0 && al(a.packed, 16) &&
                            al(a.x, 4) && al(a.scales, 4) && al(a.biases, 4);
-    // units a thread: two in the pipelined form at 4 and 8 bits for two tokens a pass on wide
-    // matrices (the LM-head shape +7%, bound by instruction issue); one for one token (two
-    // measured -5%: half the column blocks, twice the stages) and on narrow matrices (q/o -10%:
-    // half as many blocks, which are bound by latency)
-    const int upt = (pipelined && a.bits != 6 && tm == 2 && units >= 16 * 2 * NT_THREADS) ? 2 : 1;
+    // units a thread: two in the pipelined form at 4 and 8 bits for two or four tokens a pass
+    // on wide matrices (the LM-head shape +7% at two tokens, +13% at four: bound by instruction
+    // issue); one for one token (two measured -5%: half the column blocks, twice the stages),
+    // for eight (the accumulators would not fit) and on narrow matrices (q/o -10%: half as many
+    // blocks, which are bound by latency)
+    const int upt = (pipelined && a.bits != 6 && (tm == 2 || tm == 4) && units >= 16 * 2 * NT_THREADS) ? 2 : 1;
     const int cblocks = (units + NT_THREADS * upt - 1) / (NT_THREADS * upt);
     int smem = 0;
     const NtKernelFn fn = pipelined ? nta_kernel(a.bits, tm, upt, &smem) : nt_kernel(a.bits, tm);

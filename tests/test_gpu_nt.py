@@ -61,10 +61,11 @@ def test_forms_without_aligned_copies(oracle_mod, M, K, N, bits, group):
 
 @pytest.mark.parametrize("bits,N,group", [(4, 33024, 64), (4, 32768, 32), (8, 16640, 128)])
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
-def test_wide_two_tokens(oracle_mod, bits, N, group, dtype):
-    """Two tokens on a wide matrix: two packed units a thread (a partial last column block at
-    N = 33024 and 16640)."""
-    _run(oracle_mod, 2, 320, N, bits, group, dtype, 1.0 if dtype == torch.float16 else 0.02)
+@pytest.mark.parametrize("M", [2, 3, 4])
+def test_wide_two_units(oracle_mod, bits, N, group, dtype, M):
+    """Two to four tokens on a wide matrix: two packed units a thread (a partial last column
+    block at N = 33024 and 16640; M = 3 pads the four-token pass)."""
+    _run(oracle_mod, M, 320, N, bits, group, dtype, 1.0 if dtype == torch.float16 else 0.02)
 
 
 _NT_FULL = {}
