@@ -504,7 +504,11 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     // nearly empty last wave nor an under-filled single wave is left; the fp32 split sums are
     // kept under 256 MB
     const int64_t slots = int64_t(bps) * kNtSMs;
-    const int smax = int(std::max<int64_t>(1, std::min<int64_t>(64, a.K / 64)));
+    // (the pipelined form may go to 128 slices of 32 rows while the split sums stay within the
+    // weights' bytes: q/o +4-6% at 1-4 tokens; past that, -2-3% at 8-16)
+    const int64_t smax64 = std::min<int64_t>(64, a.K / 64);
+    const int64_t smaxf = std::min<int64_t>(std::min<int64_t>(128, a.K / 32), a.K * a.bits / (32 * std::max<int64_t>(1, a.M)));
+    const int smax = int(std::max<int64_t>(1, pipelined ? std::max(smax64, smaxf) : smax64));
     int S = 1;
     double best = 0.0;
     for (int sc = 1; sc <= smax; ++sc) {
