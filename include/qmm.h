@@ -242,9 +242,13 @@ qmm_status qmm_noalloc(const void* x, const uint32_t* packed, const uint16_t* sc
  * (each row of W' packed as qmm_quantize packs a row: qmm_quantize(W', ..., N = K, K = N)
  * makes these arrays); scales, biases [K, N/group] fp16.  N must be a multiple of `group`.
  * Pointers: device memory, owned by the caller; x, y, scales, biases 2-byte and packed 4-byte
- * aligned.  Arithmetic: fp32, x*s exact per row, the split sums added in a fixed order, y
- * rounded once (same tolerance as qmm, bitwise repeatable).  Runs on CUDA cores (this form is
- * not on the tensor-core path); M up to 2^20; may use the stream's workspace (as qmm).
+ * aligned.  Performance: the rows are staged through shared memory by asynchronous copies
+ * when packed is 16-byte aligned with rows a multiple of 16 bytes, x, scales and biases are
+ * 4-byte aligned, K is even and N/group is even; other calls take a slower kernel with the
+ * same results within rounding.  Arithmetic: fp32, x*s exact per row, the split sums added
+ * in a fixed order, y rounded once (same tolerance as qmm, bitwise repeatable).  Runs on CUDA
+ * cores (this form is not on the tensor-core path); M up to 2^20; may use the stream's
+ * workspace (as qmm).
  * M == 0 or N == 0 is a no-op; K == 0 writes zeros.  Errors as for qmm().
  */
 qmm_status qmm_nt(const void* x, const uint32_t* packed, const uint16_t* scales, const uint16_t* biases,
