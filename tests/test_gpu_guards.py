@@ -1,6 +1,6 @@
 """Guard regions around the output: every kernel path writes exactly y[0:M, 0:N] and nothing
 around it.  Each output lives inside a larger buffer whose bytes before and after it hold a
-known pattern that must survive the call (the safety aid the survey lists beside the
+known pattern that must survive the call (a canary check, the companion of the kernels'
 bounded waits).  Shapes are chosen with a ragged last row tile, so an off-by-one in a tile's
 row limit would land in the guard."""
 import pytest
