@@ -499,10 +499,11 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
     int bps = 0;
     cudaError_t e0 = nt_blocks_per_sm(fn, smem, &bps);
     if (e0 != cudaSuccess) return e0;
-    // K slices (at least 64 rows each): the fewest whose blocks fill at least 85% of the
-    // resident-block slots of the waves they take (else the best filling), so that neither a
-    // nearly empty last wave nor an under-filled single wave is left; the fp32 split sums are
-    // kept under 256 MB
+    // K slices: the fewest whose blocks fill at least 93% of the resident-block slots of the
+    // waves they take (else the best filling), so that neither a nearly empty last wave nor an
+    // under-filled single wave is left (on the LM-head shape 14 slices at 0.94 of three waves
+    // measured 3-5% faster at 1, 8 and 16 tokens than 9 at 0.91 of two, and 1% slower at 4);
+    // the fp32 split sums are kept under 256 MB
     const int64_t slots = int64_t(bps) * kNtSMs;
     // (the pipelined form may go to 128 slices of 32 rows while the split sums stay within the
     // weights' bytes: q/o +4-6% at 1-4 tokens; past that, -2-3% at 8-16)
@@ -518,12 +519,11 @@ cudaError_t launch_nt(const QmmArgs& a, cudaStream_t stream) {
             best = fill;
             S = sc;
         }
-        if (fill >= 0.85) break;
+        if (fill >= 0.93) break;
     }
     while (S > 1 && int64_t(S) * a.M * a.N * 4 > (int64_t(256) << 20)) --S;
     // slice rows: a multiple of 64 in the per-thread form, of 16 (a stage) in the pipelined one,
-    // whose slice count then stays the one chosen (LM-head shape: 9 slices, 0.91 of two waves,
-    // not 8 at 0.81)
+    // whose slice count then stays the one chosen (LM-head shape: 14 slices, not 13 at 0.87)
     const int gran = pipelined ? 16 : 64;
     const int krange = int((a.K + S - 1) / S + gran - 1) / gran * gran;
     S = int((a.K + krange - 1) / krange);
