@@ -164,14 +164,17 @@ __global__ void __launch_bounds__(NT_THREADS) qmm_nt_kernel(const uint16_t* __re
 //
 // The form above keeps RU rows of loads in flight per thread, a few KB per SM: every batch
 // of rows costs a full memory round trip, so small matrices and wide ones alike run far
-// below the copy rate.  Here the block's rows go through a ring of NTA_STAGES slots in shared
-// memory, filled by cp.async (16-byte copies of the codes, 4-byte copies of the scale, bias
-// and x pairs); NTA_STAGES - 1 stages of R rows are in flight while one is summed, tens of
-// KB per block.  The arithmetic is that of the form above (codes exact in fp32, x*s exact, a
-// thread's sums in row order); K slices are contiguous row ranges, so a slice's x is a
-// contiguous run of each token row.  Requirements (the host checks them, else the form
-// above runs): packed 16-byte aligned with 16-byte rows, K even, scales/biases/x 4-byte
-// aligned and N/group even, so that every copy is aligned.
+// below the copy rate.  Here the block's rows go through a ring of four slots in shared
+// memory (NtaFmt::STAGES), filled by cp.async (16-byte copies of the codes, 4-byte copies of
+// the scale, bias and x pairs); three stages of 16 rows (8 at 6 bits or with two units a
+// thread) are in flight while one is summed, tens of KB per block.  The arithmetic is that of
+// the form above (x*s exact, a thread's sums in row order), except that 4- and 8-bit codes
+// enter as 1 + q/2^BITS (code_1p below).  A thread takes one packed unit, or two adjacent ones
+// of one group (UPT = 2, chosen by the host for two or four tokens on wide matrices).  K
+// slices are contiguous row ranges, so a slice's x is a contiguous run of each token row.
+// Requirements (the host checks them, else the form above runs): packed 16-byte aligned with
+// 16-byte rows, K even, scales/biases/x 4-byte aligned and N/group even, so that every copy
+// is aligned.
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t n) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n) : "memory");
